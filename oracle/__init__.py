@@ -1,0 +1,200 @@
+"""CPU oracle for tile-routed mixed-precision prefill attention -- TEST INFRASTRUCTURE.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may use
+this package.  It shares no code with the CUDA library: the arithmetic lives in
+``oracle.cpp`` (plain C++17 loops, fp64 softmax, exact integer / exact fp64 8-bit dot
+products), built here with g++ and called through ctypes on numpy arrays.
+
+What it computes, with the pages' passages it follows:
+  * ``quantize``      -- per-block INT8 / E4M3 quantisation (TileMix page, section 2, "The
+                         Dual-Path Engine", item 2; LampAttention abstract, "8-bit formats").
+  * ``build_mask``    -- the packed routing bitmask, one bit per group of key tiles, 0 = FP16,
+                         1 = INT8 (TileMix page, section 2, "Packed Bitmasks").
+  * ``attention``     -- routed scores, shared softmax and 16-bit-routed tiles (TileMix page,
+                         section 2, "The Dual-Path Engine"; LampAttention abstract for the
+                         adaptive 8-bit -> 16-bit recomputation).
+Every function is pinned by CPU tests against closed forms, brute force and invariants.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.cpp")
+_LIB_PATH = os.path.join(_HERE, "_build", "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+CXXFLAGS = ["-O2", "-std=c++17", "-ffp-contract=off", "-fno-fast-math", "-shared", "-fPIC",
+            "-pthread"]
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.cpp into oracle/_build/liboracle.so (g++)."""
+    os.makedirs(os.path.dirname(_LIB_PATH), exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["g++", *CXXFLAGS, _SRC, "-o", tmp])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+class _Args(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("Hkv", ctypes.c_int), ("Lq", ctypes.c_int),
+        ("Lk", ctypes.c_int), ("D", ctypes.c_int), ("bm", ctypes.c_int), ("bn", ctypes.c_int),
+        ("causal", ctypes.c_int), ("window", ctypes.c_int),
+        ("scale", ctypes.c_double),
+        ("mask", ctypes.c_void_p), ("mask_words", ctypes.c_int), ("group_tiles", ctypes.c_int),
+        ("adaptive", ctypes.c_int), ("fmt", ctypes.c_int), ("tau", ctypes.c_double),
+        ("rows", ctypes.c_void_p), ("nrows", ctypes.c_int), ("threads", ctypes.c_int),
+        ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("route", ctypes.c_void_p),
+        ("margin", ctypes.c_void_p), ("route_hint", ctypes.c_void_p),
+        ("hint_margin", ctypes.c_double),
+        ("q_codes", ctypes.c_void_p), ("q_scales", ctypes.c_void_p),
+        ("k_codes", ctypes.c_void_p), ("k_scales", ctypes.c_void_p),
+    ]
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = build()
+            L = ctypes.CDLL(path)
+            L.orc_e4m3_decode.restype = ctypes.c_double
+            L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+            L.orc_e4m3_encode.restype = ctypes.c_uint8
+            L.orc_e4m3_encode.argtypes = [ctypes.c_float]
+            L.orc_splitmix64_next.restype = ctypes.c_uint64
+            L.orc_splitmix64_next.argtypes = [ctypes.c_uint64]
+            L.orc_quantize.restype = None
+            L.orc_quantize.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                       ctypes.c_void_p]
+            L.orc_build_mask.restype = None
+            L.orc_build_mask.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                         ctypes.c_uint64]
+            L.orc_attention.restype = ctypes.c_int
+            L.orc_attention.argtypes = [ctypes.POINTER(_Args)]
+            _lib = L
+    return _lib
+
+
+FMT = {"int8": 0, "e4m3": 1}
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def e4m3_decode(code: int) -> float:
+    return lib().orc_e4m3_decode(int(code) & 0xFF)
+
+
+def e4m3_encode(x: float) -> int:
+    return int(lib().orc_e4m3_encode(float(x)))
+
+
+def splitmix64_next(state: int) -> int:
+    return int(lib().orc_splitmix64_next(int(state) & 0xFFFFFFFFFFFFFFFF))
+
+
+def quantize(x: np.ndarray, blk: int, fmt: str = "int8"):
+    """Per-block quantisation of x [..., L, D] (fp32 values) in blocks of ``blk`` rows.
+
+    Returns (codes uint8 [..., L, D] -- int8 two's complement or e4m3 bits --,
+    scales float32 [..., ceil(L/blk)]).
+    """
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    *lead, L, D = x.shape
+    outer = int(np.prod(lead)) if lead else 1
+    nb = -(-L // blk)
+    codes = np.empty(x.shape, dtype=np.uint8)
+    scales = np.empty((*lead, nb), dtype=np.float32)
+    lib().orc_quantize(_ptr(x), outer, L, D, blk, FMT[fmt], _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def mask_words(nkt: int, group_tiles: int) -> int:
+    ng = -(-nkt // group_tiles)
+    return max(1, -(-ng // 64))
+
+
+def build_mask(B: int, H: int, nqt: int, nkt: int, group_tiles: int, p_fp16: float,
+               seed: int) -> np.ndarray:
+    """uint64 [B, H, nQT, W] routing mask drawn from the seeded SplitMix64 template."""
+    ng = -(-nkt // group_tiles)
+    W = mask_words(nkt, group_tiles)
+    m = np.empty((B, H, nqt, W), dtype=np.uint64)
+    lib().orc_build_mask(_ptr(m), B, H, nqt, ng, W, float(p_fp16), int(seed) & (2**64 - 1))
+    return m
+
+
+def attention(q, k, v, *, bm, bn, causal=False, window=0, scale=None, mask=None, group_tiles=1,
+              route="bitmask", fmt="int8", tau=0.0, rows=None, threads=0, want_codes=False,
+              route_hint=None, hint_margin=0.0):
+    """Routed attention on fp32 values of 16-bit inputs.
+
+    q [B,H,Lq,D], k/v [B,Hkv,Lk,D].  ``mask`` uint64 [B,H,nQT,W] or None (all 8-bit) in
+    bitmask routing.  ``rows`` int64 [B,H,n] (sorted per head) restricts the output rows.
+    Returns a dict with o (fp64 [B,H,R,D]), lse (fp64 [B,H,R]), route (uint8 [B,H,nQT,nKT]:
+    0 dead, 1 8-bit, 2 16-bit by mask, 3 16-bit flagged), margin (fp64, adaptive decisions).
+    """
+    q = np.ascontiguousarray(q, dtype=np.float32)
+    k = np.ascontiguousarray(k, dtype=np.float32)
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    B, H, Lq, D = q.shape
+    _, Hkv, Lk, _ = k.shape
+    nqt, nkt = -(-Lq // bm), -(-Lk // bn)
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    if rows is not None:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        R = rows.shape[-1]
+    else:
+        R = Lq
+    o = np.empty((B, H, R, D), dtype=np.float64)
+    lse = np.empty((B, H, R), dtype=np.float64)
+    rmap = np.empty((B, H, nqt, nkt), dtype=np.uint8)
+    margin = np.empty((B, H, nqt, nkt), dtype=np.float64)
+    if mask is not None:
+        mask = np.ascontiguousarray(mask, dtype=np.uint64)
+    if route_hint is not None:
+        route_hint = np.ascontiguousarray(route_hint, dtype=np.uint8)
+    a = _Args()
+    a.q, a.k, a.v = _ptr(q), _ptr(k), _ptr(v)
+    a.B, a.H, a.Hkv, a.Lq, a.Lk, a.D, a.bm, a.bn = B, H, Hkv, Lq, Lk, D, bm, bn
+    a.causal, a.window = int(bool(causal)), int(window)
+    a.scale = float(scale)
+    a.mask = _ptr(mask)
+    a.mask_words = mask.shape[-1] if mask is not None else 0
+    a.group_tiles = int(group_tiles)
+    a.adaptive = 1 if route == "adaptive" else 0
+    a.fmt = FMT[fmt]
+    a.tau = float(tau)
+    a.rows = _ptr(rows)
+    a.nrows = R if rows is not None else 0
+    a.threads = int(threads) if threads else (os.cpu_count() or 1)
+    a.o, a.lse, a.route, a.margin = _ptr(o), _ptr(lse), _ptr(rmap), _ptr(margin)
+    a.route_hint = _ptr(route_hint)
+    a.hint_margin = float(hint_margin)
+    out = {"o": o, "lse": lse, "route": rmap, "margin": margin}
+    if want_codes:
+        qc = np.empty(q.shape, np.uint8)
+        qs = np.empty((B, H, nqt), np.float32)
+        kc = np.empty(k.shape, np.uint8)
+        ks = np.empty((B, Hkv, nkt), np.float32)
+        a.q_codes, a.q_scales, a.k_codes, a.k_scales = _ptr(qc), _ptr(qs), _ptr(kc), _ptr(ks)
+        out.update(q_codes=qc, q_scales=qs, k_codes=kc, k_scales=ks)
+    rc = lib().orc_attention(ctypes.byref(a))
+    if rc != 0:
+        raise ValueError(f"oracle rejected the arguments (code {rc})")
+    return out

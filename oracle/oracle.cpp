@@ -1,0 +1,404 @@
+// CPU oracle for tile-routed mixed-precision attention (prefill forward).
+//
+// TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or load this file;
+// only the tests, the smoke check and the benchmark's CPU-baseline leg use it.  It shares no
+// code, header, table or constant with the CUDA library.
+//
+// Plain and slow on purpose: loops over rows, keys and channels; exact integer dot products
+// for INT8 tiles, exact fp64 sums for E4M3 tiles (every product of two e4m3 codes is exact in
+// fp64 and the sums stay far below 2^53), fp64 dot products on the 16-bit inputs for 16-bit
+// tiles, and a two-pass fp64 softmax.  Sources:
+//   * TileMix page, section 2 "How It Works", "The Dual-Path Engine": INT8 path = per-block
+//     quantised Q and K, tensor-core product, rescale with per-block scale factors; FP16 path =
+//     plain floating-point product; both feed one shared online-softmax state.
+//   * TileMix page, section 2, "Packed Bitmasks": one bit per group of adjacent key tiles,
+//     0 = FP16, 1 = INT8, one mask per query row (read here: per query routing tile).
+//   * LampAttention page, abstract: 8-bit key-query products, sensitive sub-blocks found
+//     adaptively and recomputed in 16 bits.  The rule used: a tile is recomputed when, for some
+//     row, its 8-bit tile max reaches the running row max minus tau.
+// Readings of the pages that they leave open are listed with each function below.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <thread>
+#include <vector>
+
+namespace {
+
+// ---------------------------------------------------------------------------------------
+// E4M3 (OCP "e4m3fn"): 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits, no infinities,
+// S.1111.111 is NaN, largest finite 448, subnormals 2^-6 * m/8.
+// ---------------------------------------------------------------------------------------
+double e4m3_decode(uint8_t c) {
+  int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  if (e == 15 && m == 7) return std::numeric_limits<double>::quiet_NaN();
+  double mag = (e == 0) ? std::ldexp(m / 8.0, -6) : std::ldexp(1.0 + m / 8.0, e - 7);
+  return s ? -mag : mag;
+}
+
+// Round to nearest representable e4m3 value, ties to even mantissa, saturating to +-448.
+uint8_t e4m3_encode(float xf) {
+  double x = xf;
+  if (std::isnan(x)) return 0x7F;
+  uint8_t sign = std::signbit(x) ? 0x80 : 0x00;
+  double a = std::fabs(x);
+  if (a >= 448.0) return sign | 0x7E;  // satfinite (RNE of [448,464) is 448 as well)
+  const double min_normal = std::ldexp(1.0, -6);
+  if (a < min_normal) {
+    // subnormal grid: multiples of 2^-9
+    double qm = std::nearbyint(a * 512.0);  // exact scaling, RNE
+    int m = (int)qm;                        // 0..8; 8 is the smallest normal (code 0x08)
+    return sign | (uint8_t)m;
+  }
+  int E;
+  std::frexp(a, &E);          // a = f * 2^E, f in [0.5, 1)
+  int e = E - 1;              // a = mant * 2^e, mant in [1, 2)
+  double mant = std::ldexp(a, -e);
+  double qm = std::nearbyint((mant - 1.0) * 8.0);  // exact, RNE
+  int m = (int)qm;
+  if (m == 8) { m = 0; e += 1; }
+  int code = ((e + 7) << 3) | m;
+  if (code > 0x7E) code = 0x7E;
+  return sign | (uint8_t)code;
+}
+
+// ---------------------------------------------------------------------------------------
+// Per-block quantisation (TileMix "Dual-Path Engine", INT8 path; LampAttention 8-bit formats).
+// Block = `blk` consecutive rows x all D channels of one (batch, head).  Reading: the block
+// is the routing tile's extent on that operand; scale = absmax / 127 (INT8, symmetric, codes
+// in [-127, 127]) or absmax / 448 (E4M3); codes = round-to-nearest-even of x / scale, both the
+// scale and the quotient rounded to fp32 (IEEE divide); an all-zero block has scale 0, codes 0.
+// ---------------------------------------------------------------------------------------
+void quantize_block(const float* x, int rows, int D, int fmt, uint8_t* codes, float* scale) {
+  float a = 0.0f;
+  for (int r = 0; r < rows; ++r)
+    for (int d = 0; d < D; ++d) a = std::fmax(a, std::fabs(x[(size_t)r * D + d]));
+  if (a == 0.0f) {
+    *scale = 0.0f;
+    std::memset(codes, 0, (size_t)rows * D);
+    return;
+  }
+  const float denom = (fmt == 0) ? 127.0f : 448.0f;
+  float s = a / denom;  // IEEE fp32 divide (the build forbids contraction and fast-math)
+  *scale = s;
+  for (int r = 0; r < rows; ++r)
+    for (int d = 0; d < D; ++d) {
+      float y = x[(size_t)r * D + d] / s;
+      if (fmt == 0) {
+        float c = std::nearbyint(y);
+        if (c > 127.0f) c = 127.0f;
+        if (c < -127.0f) c = -127.0f;
+        codes[(size_t)r * D + d] = (uint8_t)(int8_t)(int)c;
+      } else {
+        codes[(size_t)r * D + d] = e4m3_encode(y);
+      }
+    }
+}
+
+// SplitMix64 (Steele, Lea and Flood, OOPSLA 2014): one step of the generator from state x:
+// add the golden gamma, then the variant-13 finaliser.
+uint64_t splitmix64_next(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+struct Geometry {
+  int B, H, Hkv, Lq, Lk, D, bm, bn, causal, window;
+  int nqt() const { return (Lq + bm - 1) / bm; }
+  int nkt() const { return (Lk + bn - 1) / bn; }
+  // Reading (causal, bottom-right aligned; window of W keys including the diagonal):
+  // query i sees key j iff j <= i + (Lk - Lq) and, when W > 0, j > i + (Lk - Lq) - W.
+  void visible(int i, long* lo, long* hi) const {
+    if (!causal) { *lo = 0; *hi = Lk - 1; return; }
+    long h = (long)i + (Lk - Lq);
+    if (h > Lk - 1) h = Lk - 1;
+    long l = 0;
+    if (window > 0) { l = (long)i + (Lk - Lq) - window + 1; if (l < 0) l = 0; }
+    *lo = l; *hi = h;
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+struct orc_args {
+  const float* q;      // [B,H,Lq,D]   exact values of the 16-bit inputs
+  const float* k;      // [B,Hkv,Lk,D]
+  const float* v;      // [B,Hkv,Lk,D]
+  int B, H, Hkv, Lq, Lk, D, bm, bn;
+  int causal, window;
+  double scale;            // softmax scale applied to q.k
+  const uint64_t* mask;    // bitmask routing [B,H,nQT,W] (NULL: every tile 8-bit)
+  int mask_words;          // W
+  int group_tiles;
+  int adaptive;            // 0: bitmask routing, 1: look-ahead rule
+  int fmt;                 // 0: INT8, 1: E4M3
+  double tau;
+  const int64_t* rows;     // optional [B,H,nrows] sorted query rows; NULL = every row
+  int nrows;
+  int threads;
+  double* o;               // [B,H,R,D]  R = nrows or Lq
+  double* lse;             // [B,H,R]
+  uint8_t* route;          // optional [B,H,nQT,nKT]: 0 dead, 1 8-bit, 2 16-bit by mask, 3 16-bit flagged
+  double* margin;          // optional [B,H,nQT,nKT]: adaptive decision margin (inf elsewhere)
+  const uint8_t* route_hint;  // optional [B,H,nQT,nKT]: decisions to follow where margin < hint_margin
+  double hint_margin;
+  uint8_t* q_codes;        // optional [B,H,Lq,D] output of the Q quantiser (all blocks)
+  float* q_scales;         // optional [B,H,nQT]
+  uint8_t* k_codes;        // optional [B,Hkv,Lk,D]
+  float* k_scales;         // optional [B,Hkv,nKT]
+};
+
+double orc_e4m3_decode(uint8_t c) { return e4m3_decode(c); }
+uint8_t orc_e4m3_encode(float x) { return e4m3_encode(x); }
+uint64_t orc_splitmix64_next(uint64_t x) { return splitmix64_next(x); }
+
+// Quantise x [outer, L, D] in blocks of `blk` rows: codes [outer, L, D], scales [outer, ceil(L/blk)].
+void orc_quantize(const float* x, int outer, int L, int D, int blk, int fmt, uint8_t* codes,
+                  float* scales) {
+  int nb = (L + blk - 1) / blk;
+  for (int o = 0; o < outer; ++o)
+    for (int b = 0; b < nb; ++b) {
+      int r0 = b * blk, rows = (L - r0 < blk) ? (L - r0) : blk;
+      size_t off = ((size_t)o * L + r0) * D;
+      quantize_block(x + off, rows, D, fmt, codes + off, scales + (size_t)o * nb + b);
+    }
+}
+
+// Seeded Bernoulli routing template (the pages' routing policy is a static, data-free
+// template; the exact template shape is not given, so each group bit is drawn i.i.d.):
+// bit g of the mask of (b, h, qt) is 0 (16-bit) iff u53 * 2^-53 < p_fp16, where
+// u = splitmix64_next(seed XOR idx * 0x9E3779B97F4A7C15), idx = ((b*H + h)*nQT + qt)*nG + g
+// and u53 = u >> 11.  Bits at g >= nG are zero.
+void orc_build_mask(uint64_t* mask, int B, int H, int nqt, int ng, int W, double p_fp16,
+                    uint64_t seed) {
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h)
+      for (int qt = 0; qt < nqt; ++qt) {
+        uint64_t* row = mask + (((size_t)b * H + h) * nqt + qt) * W;
+        for (int w = 0; w < W; ++w) row[w] = 0;
+        for (int g = 0; g < ng; ++g) {
+          uint64_t idx = (((uint64_t)b * H + h) * nqt + qt) * (uint64_t)ng + g;
+          uint64_t u = splitmix64_next(seed ^ (idx * 0x9E3779B97F4A7C15ull));
+          double r = (double)(u >> 11) * 0x1.0p-53;
+          int eight_bit = (r < p_fp16) ? 0 : 1;
+          if (eight_bit) row[g >> 6] |= (1ull << (g & 63));
+        }
+      }
+}
+
+int orc_attention(const orc_args* a) {
+  Geometry g{a->B, a->H, a->Hkv, a->Lq, a->Lk, a->D, a->bm, a->bn, a->causal, a->window};
+  if (g.H % g.Hkv != 0 || g.D <= 0 || g.bm <= 0 || g.bn <= 0) return 1;
+  const int G = g.H / g.Hkv, D = g.D, nqt = g.nqt(), nkt = g.nkt();
+  const double NEG_INF = -std::numeric_limits<double>::infinity();
+  const double INF = std::numeric_limits<double>::infinity();
+
+  // Quantise K for every (b, kv head) block of bn rows.
+  std::vector<uint8_t> kc((size_t)g.B * g.Hkv * g.Lk * D);
+  std::vector<float> ks((size_t)g.B * g.Hkv * nkt);
+  orc_quantize(a->k, g.B * g.Hkv, g.Lk, D, g.bn, a->fmt, kc.data(), ks.data());
+  if (a->k_codes) std::memcpy(a->k_codes, kc.data(), kc.size());
+  if (a->k_scales) std::memcpy(a->k_scales, ks.data(), ks.size() * sizeof(float));
+  if (a->q_codes || a->q_scales) {
+    std::vector<uint8_t> qc((size_t)g.B * g.H * g.Lq * D);
+    std::vector<float> qs((size_t)g.B * g.H * nqt);
+    orc_quantize(a->q, g.B * g.H, g.Lq, D, g.bm, a->fmt, qc.data(), qs.data());
+    if (a->q_codes) std::memcpy(a->q_codes, qc.data(), qc.size());
+    if (a->q_scales) std::memcpy(a->q_scales, qs.data(), qs.size() * sizeof(float));
+  }
+
+  // Work items: (b, h, qt) tiles that hold at least one requested row.
+  const int R = a->rows ? a->nrows : g.Lq;
+  struct Item { int b, h, qt, r_begin, r_end; };  // [r_begin, r_end) into the requested rows
+  std::vector<Item> items;
+  for (int b = 0; b < g.B; ++b)
+    for (int h = 0; h < g.H; ++h) {
+      if (!a->rows) {
+        for (int qt = 0; qt < nqt; ++qt) {
+          int r0 = qt * g.bm, r1 = std::min(g.Lq, r0 + g.bm);
+          items.push_back({b, h, qt, r0, r1});
+        }
+      } else {
+        const int64_t* rr = a->rows + ((size_t)b * g.H + h) * R;
+        int s = 0;
+        while (s < R) {
+          int qt = (int)(rr[s] / g.bm), e = s;
+          while (e < R && rr[e] / g.bm == qt) ++e;
+          items.push_back({b, h, qt, s, e});
+          s = e;
+        }
+      }
+    }
+  if (a->route) std::memset(a->route, 0, (size_t)g.B * g.H * nqt * nkt);
+  if (a->margin)
+    for (size_t i = 0; i < (size_t)g.B * g.H * nqt * nkt; ++i) a->margin[i] = INF;
+
+  std::atomic<size_t> next{0};
+  auto worker = [&]() {
+    std::vector<uint8_t> qcode((size_t)g.bm * D);
+    std::vector<double> m_run(g.bm), s8row(g.bn), s16row(g.bn);
+    std::vector<uint8_t> tile_route(nkt);
+    std::vector<double> srow(g.Lk);
+    for (;;) {
+      size_t it = next.fetch_add(1);
+      if (it >= items.size()) break;
+      const Item& I = items[it];
+      const int b = I.b, h = I.h, qt = I.qt, kvh = h / G;
+      const int r0 = qt * g.bm, rows_in_tile = std::min(g.Lq, r0 + g.bm) - r0;
+      const float* qh = a->q + ((size_t)b * g.H + h) * g.Lq * D;
+      const float* kh = a->k + ((size_t)b * g.Hkv + kvh) * g.Lk * D;
+      const float* vh = a->v + ((size_t)b * g.Hkv + kvh) * g.Lk * D;
+      const uint8_t* kch = kc.data() + ((size_t)b * g.Hkv + kvh) * g.Lk * D;
+      const float* ksh = ks.data() + ((size_t)b * g.Hkv + kvh) * nkt;
+      float qscale;
+      quantize_block(qh + (size_t)r0 * D, rows_in_tile, D, a->fmt, qcode.data(), &qscale);
+
+      // 8-bit score of (query row r0+r, key j): exact code dot product times the scales.
+      auto score8 = [&](int r, long j) -> double {
+        const uint8_t* cq = qcode.data() + (size_t)r * D;
+        const uint8_t* ck = kch + (size_t)j * D;
+        double dot;
+        if (a->fmt == 0) {
+          int64_t acc = 0;
+          for (int d = 0; d < D; ++d) acc += (int64_t)(int8_t)cq[d] * (int64_t)(int8_t)ck[d];
+          dot = (double)acc;
+        } else {
+          double acc = 0.0;
+          for (int d = 0; d < D; ++d) acc += e4m3_decode(cq[d]) * e4m3_decode(ck[d]);
+          dot = acc;
+        }
+        int kt = (int)(j / g.bn);
+        return dot * (double)qscale * (double)ksh[kt] * a->scale;
+      };
+      // 16-bit score: fp64 dot product of the 16-bit input values.
+      auto score16 = [&](int r, long j) -> double {
+        const float* x = qh + (size_t)(r0 + r) * D;
+        const float* y = kh + (size_t)j * D;
+        double acc = 0.0;
+        for (int d = 0; d < D; ++d) acc += (double)x[d] * (double)y[d];
+        return acc * a->scale;
+      };
+
+      // Live key tiles of this query tile: some row of the tile sees some key of the tile.
+      std::vector<long> lo(rows_in_tile), hi(rows_in_tile);
+      for (int r = 0; r < rows_in_tile; ++r) g.visible(r0 + r, &lo[r], &hi[r]);
+      auto tile_live = [&](int kt) {
+        long c0 = (long)kt * g.bn, c1 = std::min<long>(g.Lk, c0 + g.bn) - 1;
+        for (int r = 0; r < rows_in_tile; ++r)
+          if (lo[r] <= hi[r] && lo[r] <= c1 && hi[r] >= c0) return true;
+        return false;
+      };
+
+      // Routing of every key tile of this query tile.
+      for (int kt = 0; kt < nkt; ++kt) tile_route[kt] = 0;
+      if (!a->adaptive) {
+        const uint64_t* mrow =
+            a->mask ? a->mask + (((size_t)b * g.H + h) * nqt + qt) * a->mask_words : nullptr;
+        for (int kt = 0; kt < nkt; ++kt) {
+          if (!tile_live(kt)) continue;
+          int gi = kt / a->group_tiles;
+          int bit = mrow ? (int)((mrow[gi >> 6] >> (gi & 63)) & 1ull) : 1;
+          tile_route[kt] = bit ? 1 : 2;
+        }
+      } else {
+        // Look-ahead rule, ascending key tiles: t_r = 8-bit max of row r over its visible
+        // keys in the tile; m_r = running max of the scores used so far (before this tile);
+        // the tile is recomputed in 16 bits iff some row has t_r >= m_r - tau.
+        for (int r = 0; r < rows_in_tile; ++r) m_run[r] = NEG_INF;
+        const uint8_t* hint =
+            a->route_hint ? a->route_hint + (((size_t)b * g.H + h) * nqt + qt) * nkt : nullptr;
+        std::vector<double> t(rows_in_tile);
+        for (int kt = 0; kt < nkt; ++kt) {
+          if (!tile_live(kt)) continue;
+          long c0 = (long)kt * g.bn, c1 = std::min<long>(g.Lk, c0 + g.bn) - 1;
+          // Decision and its margin: the distance the deciding quantity is from the
+          // threshold.  Flagged: the largest t_r - (m_r - tau) over voting rows (infinite
+          // when some voting row has no running max yet).  Not flagged: the smallest
+          // (m_r - tau) - t_r.
+          bool flagged = false;
+          double pass_margin = NEG_INF, fail_margin = INF;
+          for (int r = 0; r < rows_in_tile; ++r) {
+            t[r] = NEG_INF;
+            long jl = std::max(lo[r], c0), jh = std::min(hi[r], c1);
+            if (jl > jh) continue;
+            for (long j = jl; j <= jh; ++j) t[r] = std::max(t[r], score8(r, j));
+            double thr = m_run[r] - a->tau;
+            if (t[r] >= thr) {
+              flagged = true;
+              pass_margin = std::max(pass_margin, m_run[r] == NEG_INF ? INF : t[r] - thr);
+            } else {
+              fail_margin = std::min(fail_margin, thr - t[r]);
+            }
+          }
+          double margin = flagged ? pass_margin : fail_margin;
+          // Where the decision is within `hint_margin` of flipping, two correct
+          // implementations may disagree; follow the supplied routing map there.
+          if (hint && margin < a->hint_margin && (hint[kt] == 1 || hint[kt] == 3))
+            flagged = (hint[kt] == 3);
+          tile_route[kt] = flagged ? 3 : 1;
+          size_t ti = (((size_t)b * g.H + h) * nqt + qt) * nkt + kt;
+          if (a->margin) a->margin[ti] = margin;
+          for (int r = 0; r < rows_in_tile; ++r) {
+            long jl = std::max(lo[r], c0), jh = std::min(hi[r], c1);
+            if (jl > jh) continue;
+            double mx = NEG_INF;
+            if (flagged)
+              for (long j = jl; j <= jh; ++j) mx = std::max(mx, score16(r, j));
+            else
+              mx = t[r];
+            m_run[r] = std::max(m_run[r], mx);
+          }
+        }
+      }
+      if (a->route)
+        std::memcpy(a->route + (((size_t)b * g.H + h) * nqt + qt) * nkt, tile_route.data(), nkt);
+
+      // Outputs of the requested rows: two-pass fp64 softmax over the routed scores.
+      for (int s = I.r_begin; s < I.r_end; ++s) {
+        int i = a->rows ? (int)a->rows[((size_t)b * g.H + h) * R + s] : s;
+        int r = i - r0;
+        double* orow = a->o + (((size_t)b * g.H + h) * R + s) * D;
+        double* lrow = a->lse + ((size_t)b * g.H + h) * R + s;
+        long jl = lo[r], jh = hi[r];
+        if (jl > jh) {
+          for (int d = 0; d < D; ++d) orow[d] = 0.0;
+          *lrow = NEG_INF;
+          continue;
+        }
+        double M = NEG_INF;
+        for (long j = jl; j <= jh; ++j) {
+          int rt = tile_route[j / g.bn];
+          double sc = (rt == 1) ? score8(r, j) : score16(r, j);
+          srow[j] = sc;
+          M = std::max(M, sc);
+        }
+        double l = 0.0;
+        for (int d = 0; d < D; ++d) orow[d] = 0.0;
+        for (long j = jl; j <= jh; ++j) {
+          double p = std::exp(srow[j] - M);
+          l += p;
+          const float* vj = vh + (size_t)j * D;
+          for (int d = 0; d < D; ++d) orow[d] += p * (double)vj[d];
+        }
+        for (int d = 0; d < D; ++d) orow[d] /= l;
+        *lrow = M + std::log(l);
+      }
+    }
+  };
+  int nt = a->threads > 0 ? a->threads : (int)std::thread::hardware_concurrency();
+  if (nt < 1) nt = 1;
+  std::vector<std::thread> pool;
+  for (int t = 1; t < nt; ++t) pool.emplace_back(worker);
+  worker();
+  for (auto& th : pool) th.join();
+  return 0;
+}
+
+}  // extern "C"
