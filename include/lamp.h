@@ -1,0 +1,145 @@
+/*
+ * lamp.h -- C ABI of the tile-routed mixed-precision prefill attention library (B200, sm_100a).
+ *
+ * The operation (TileMix page, section 2 "How It Works"; LampAttention abstract):
+ *   softmax attention O = softmax(scale * Q K^T) V, computed tile by tile over the score
+ *   matrix.  Each (query tile, key tile) score tile is computed either from 8-bit per-block
+ *   quantised Q and K (INT8 with fp32 block scales, or FP8 E4M3), then rescaled, or from the
+ *   16-bit inputs.  The choice comes from a packed per-query-tile bitmask in which one bit
+ *   governs a group of adjacent key tiles (0 = 16-bit, 1 = 8-bit; TileMix "Packed
+ *   Bitmasks"), or from a look-ahead rule: a tile is recomputed in 16 bits when, for some row,
+ *   its 8-bit tile max reaches the running row max minus tau (LampAttention).  Both paths
+ *   update one online-softmax state per row; P.V is always 16-bit.
+ *
+ * Conventions for every call:
+ *   - Pointers named q, k, v, o, lse, q8, k8, q_scale, k_scale, mask_bits, route_out are
+ *     DEVICE pointers owned by the caller; the library keeps none of them after the call
+ *     returns.  All device work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and is asynchronous.
+ *   - Layouts are contiguous row-major: q, o [B][H][Lq][D]; k, v [B][Hkv][Lk][D]; lse
+ *     [B][H][Lq]; q8 like q, k8 like k (one byte per element); q_scale [B][H][nQT];
+ *     k_scale [B][Hkv][nKT]; mask_bits [B][H][nQT][W] uint64 words, bit g of a row at word
+ *     g>>6, bit g&63 (LSB first).  nQT = ceil(Lq/BM), nKT = ceil(Lk/BN), W = ceil(nG/64),
+ *     nG = ceil(nKT/group_tiles), with (BM, BN) from lamp_tile_shape(D).
+ *   - q, k, v, q8, k8 must be 16-byte aligned (TMA); D must be 64, 128 or 256.
+ *   - Return value: LAMP_OK or an error code.  Arguments are checked synchronously before
+ *     anything is launched; on error nothing is enqueued and lamp_last_error() describes the
+ *     problem (thread-local string).  Device-side failures (a bounded wait in a kernel that
+ *     gave up) are reported by lamp_check().
+ */
+#ifndef LAMP_H
+#define LAMP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  LAMP_OK = 0,
+  LAMP_ERR_INVALID = 1,      /* bad argument (null pointer, size, alignment, H % Hkv)      */
+  LAMP_ERR_UNSUPPORTED = 2,  /* valid but not implemented here (D, window without causal) */
+  LAMP_ERR_CUDA = 3,         /* a CUDA runtime call failed                                */
+  LAMP_ERR_TIMEOUT = 4       /* a device-side bounded wait gave up (see lamp_check)       */
+};
+
+/* mode bit field */
+#define LAMP_ROUTE_BITMASK 0x0u  /* bit 0: routing from mask_bits (TileMix)               */
+#define LAMP_ROUTE_ADAPTIVE 0x1u /* bit 0: look-ahead rule with threshold tau (Lamp)      */
+#define LAMP_FMT_INT8 0x0u       /* bit 1: 8-bit format INT8, scale = absmax/127          */
+#define LAMP_FMT_E4M3 0x2u       /* bit 1: 8-bit format FP8 E4M3, scale = absmax/448      */
+#define LAMP_IN_FP16 0x0u        /* bit 2: q, k, v are fp16                               */
+#define LAMP_IN_BF16 0x4u        /* bit 2: q, k, v are bf16                               */
+#define LAMP_OUT_F32 0x0u        /* bit 3: o is fp32                                      */
+#define LAMP_OUT_INDTYPE 0x8u    /* bit 3: o has the input dtype                          */
+
+/* Routing tile (BM x BN) for head dimension D: 64 -> 64x64, 128 -> 128x128, 256 -> 64x128
+ * (TileMix "The Tile Architecture": hardware-aligned score tiles of 128x128 or 64x64).
+ * Returns LAMP_OK, or LAMP_ERR_UNSUPPORTED for any other D.  bm/bn may not be NULL. */
+int lamp_tile_shape(int D, int* bm, int* bn);
+
+/* Number W of uint64 mask words per query tile (TileMix "Packed Bitmasks", grouping of
+ * adjacent key tiles): W = ceil(ceil(nKT / group_tiles) / 64).  Returns W > 0, or -1 when the
+ * arguments are invalid (Lk < 1, group_tiles < 1, unsupported D). */
+int lamp_mask_words(int Lk, int D, int group_tiles);
+
+/* Per-block quantisation of Q and K to 8 bits (TileMix "The Dual-Path Engine", item 2;
+ * LampAttention "8-bit formats").  For every (batch, head) block of BM query rows (Q) or BN
+ * key rows (K) over all D channels: a = max |x|; scale = fl32(a / 127) (INT8) or
+ * fl32(a / 448) (E4M3); code = RNE(fl32(x / scale)), clamped to [-127, 127] (INT8) or
+ * saturated to +-448 (E4M3); an all-zero block gets scale 0 and zero codes.
+ * q8/k8 receive int8 two's complement or e4m3 bytes; q_scale/k_scale the fp32 scales.
+ * mode: LAMP_FMT_* | LAMP_IN_*; other bits ignored.  k/k8/k_scale may all be NULL to
+ * quantise Q only (and q/q8/q_scale NULL for K only). */
+int lamp_quant_qk(const void* q, const void* k, void* q8, void* k8, float* q_scale,
+                  float* k_scale, int B, int H, int Hkv, int Lq, int Lk, int D, int mode,
+                  void* stream);
+
+/* Seeded routing template (TileMix: routing policies are static, data-free templates; the
+ * template's shape is not given, so each group bit is an independent draw).  Bit g of the
+ * mask of (b, h, qt) is 0 (16-bit) with probability fp16_fraction:
+ *   u = splitmix64(seed XOR idx * 0x9E3779B97F4A7C15), idx = ((b*H + h)*nQT + qt)*nG + g,
+ *   bit = ((u >> 11) * 2^-53 < fp16_fraction) ? 0 : 1; bits g >= nG are 0.
+ * splitmix64(x) is one step of Steele-Lea-Flood SplitMix64 from state x.
+ * mask_bits: device buffer of B*H*nQT*W uint64 words, fully written. */
+int lamp_build_mask(uint64_t* mask_bits, int B, int H, int Lq, int Lk, int D, int group_tiles,
+                    float fp16_fraction, uint64_t seed, void* stream);
+
+/* Routed attention forward, end to end: quantises Q and K into the library workspace
+ * (lamp_set_workspace, or a cached allocation made on first use with cudaMalloc), then runs
+ * the routed attention kernel.  Arguments as lamp_attn_fwd_q8 without the 8-bit operands.
+ * o receives O (fp32, or the input dtype with LAMP_OUT_INDTYPE); lse receives the natural-log
+ * row log-sum-exp of the scaled, routed scores (may be NULL).  Rows that see no key get
+ * O = 0 and lse = -inf.  Calls that share the library workspace must not overlap on the GPU. */
+int lamp_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                  int H, int Hkv, int Lq, int Lk, int D, int causal, int window, float scale,
+                  const uint64_t* mask_bits, int group_tiles, int mode, float tau, void* stream);
+
+/* Routed attention forward on already-quantised operands (the attention kernel alone).
+ *   causal: 0/1, bottom-right aligned (query i sees key j iff j <= i + Lk - Lq);
+ *   window: > 0 keeps only the `window` most recent keys (j > i + Lk - Lq - window); needs
+ *           causal = 1, else LAMP_ERR_UNSUPPORTED;
+ *   scale:  softmax scale applied to q.k; <= 0 means 1/sqrt(D);
+ *   mask_bits/group_tiles: bitmask routing; mask_bits NULL = every tile 8-bit; ignored in
+ *           adaptive mode;
+ *   tau:    adaptive threshold in natural-log units of the scaled score; ignored in bitmask
+ *           mode;
+ *   route_out: optional device buffer uint8 [B][H][nQT][nKT] receiving the routing decision
+ *           of every tile: 0 = no visible pair, 1 = 8-bit, 2 = 16-bit by mask, 3 = 16-bit by
+ *           the look-ahead rule.  NULL to skip.
+ * GQA: query head h reads KV head h / (H / Hkv). */
+int lamp_attn_fwd_q8(const void* q, const void* k, const void* v, const void* q8,
+                     const void* k8, const float* q_scale, const float* k_scale, void* o,
+                     float* lse, int B, int H, int Hkv, int Lq, int Lk, int D, int causal,
+                     int window, float scale, const uint64_t* mask_bits, int group_tiles,
+                     int mode, float tau, uint8_t* route_out, void* stream);
+
+/* Bytes of workspace lamp_attn_fwd needs for these sizes (q8, k8 and the scales, each
+ * 256-byte aligned).  0 on invalid arguments. */
+size_t lamp_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int D, int mode);
+
+/* Give the library a caller-owned device workspace (ptr may be NULL to drop it and return
+ * to the cached allocation).  The library uses it for every later lamp_attn_fwd on any
+ * stream until replaced; the caller keeps ownership and must keep it alive. */
+int lamp_set_workspace(void* ptr, size_t bytes);
+
+/* Synchronises `stream`, then reports and clears the device-side error word: LAMP_OK, or
+ * LAMP_ERR_TIMEOUT when a kernel's bounded wait gave up since the last check (the kernel
+ * then stopped early and its outputs are undefined), or LAMP_ERR_CUDA. */
+int lamp_check(void* stream);
+
+/* Launches a one-block kernel that waits, with a limit of `wait_ns` nanoseconds, on a
+ * barrier nothing will ever complete, so that the bounded-wait error path can be tested
+ * without faulting or hanging the GPU.  A later lamp_check() returns LAMP_ERR_TIMEOUT. */
+int lamp_selftest_timeout(uint64_t wait_ns, void* stream);
+
+/* Thread-local description of the last error returned by a lamp_* call on this thread. */
+const char* lamp_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LAMP_H */

@@ -1,0 +1,226 @@
+"""Tile-routed mixed-precision prefill attention for B200 (sm_100a).
+
+A thin ctypes binding over the C ABI in ``include/lamp.h`` (library
+``mixed_precision_tiled_b200/_build/liblamp.so``).  Every function below only marshals
+arguments (torch tensors or integer device pointers -> raw pointers, the current CUDA stream)
+and raises ``LampError`` on a non-zero status; all computation runs in the library's CUDA
+kernels.  There is no CPU path: if the library is missing, importing the first entry point
+fails loudly.
+
+The method (TileMix page, section 2; LampAttention abstract): Q and K are quantised per block
+to 8 bits; QK^T score tiles are computed in 8 bits, except tiles routed to 16 bits by a packed
+per-query-tile bitmask (one bit per group of key tiles, 0 = FP16) or flagged by the look-ahead
+rule (8-bit tile max within tau of the running row max); both feed one online softmax and a
+16-bit P.V.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "_build", "liblamp.so")
+
+LAMP_OK, LAMP_ERR_INVALID, LAMP_ERR_UNSUPPORTED, LAMP_ERR_CUDA, LAMP_ERR_TIMEOUT = range(5)
+ROUTE_BITMASK, ROUTE_ADAPTIVE = 0x0, 0x1
+FMT_INT8, FMT_E4M3 = 0x0, 0x2
+IN_FP16, IN_BF16 = 0x0, 0x4
+OUT_F32, OUT_INDTYPE = 0x0, 0x8
+
+EXPORTS = ("lamp_tile_shape", "lamp_mask_words", "lamp_quant_qk", "lamp_build_mask",
+           "lamp_attn_fwd", "lamp_attn_fwd_q8", "lamp_workspace_size", "lamp_set_workspace",
+           "lamp_check", "lamp_selftest_timeout", "lamp_last_error")
+
+
+class LampError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"lamp error {code}: {msg}")
+        self.code = code
+
+
+_lib = None
+_lock = threading.Lock()
+_vp, _i, _f, _u64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_uint64, ctypes.c_size_t
+
+
+def lib():
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(f"{LIB_PATH} is missing: run `python -m mixed_precision_tiled_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            sig = {
+                "lamp_tile_shape": (_i, [_i, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
+                "lamp_mask_words": (_i, [_i, _i, _i]),
+                "lamp_quant_qk": (_i, [_vp, _vp, _vp, _vp, _vp, _vp] + [_i] * 7 + [_vp]),
+                "lamp_build_mask": (_i, [_vp] + [_i] * 6 + [_f, _u64, _vp]),
+                "lamp_attn_fwd": (_i, [_vp] * 5 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp]),
+                "lamp_attn_fwd_q8": (_i, [_vp] * 9 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp, _vp]),
+                "lamp_workspace_size": (_sz, [_i] * 7),
+                "lamp_set_workspace": (_i, [_vp, _sz]),
+                "lamp_check": (_i, [_vp]),
+                "lamp_selftest_timeout": (_i, [_u64, _vp]),
+                "lamp_last_error": (ctypes.c_char_p, []),
+            }
+            for name, (res, args) in sig.items():
+                fn = getattr(L, name)
+                fn.restype, fn.argtypes = res, args
+            _lib = L
+    return _lib
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(code: int):
+    if code != LAMP_OK:
+        raise LampError(code, lib().lamp_last_error().decode())
+
+
+def mode_bits(route="bitmask", fmt="int8", dtype="bf16", out="f32") -> int:
+    return ((ROUTE_ADAPTIVE if route == "adaptive" else ROUTE_BITMASK)
+            | (FMT_E4M3 if fmt == "e4m3" else FMT_INT8)
+            | (IN_BF16 if dtype == "bf16" else IN_FP16)
+            | (OUT_INDTYPE if out == "in" else OUT_F32))
+
+
+# ------------------------------------------------------------ C-ABI wrappers ----------
+
+def lamp_tile_shape(D: int):
+    bm, bn = _i(), _i()
+    _check(lib().lamp_tile_shape(D, ctypes.byref(bm), ctypes.byref(bn)))
+    return bm.value, bn.value
+
+
+def lamp_mask_words(Lk: int, D: int, group_tiles: int) -> int:
+    w = lib().lamp_mask_words(Lk, D, group_tiles)
+    if w < 0:
+        raise LampError(LAMP_ERR_INVALID, "invalid arguments to lamp_mask_words")
+    return w
+
+
+def lamp_quant_qk(q, k, q8, k8, q_scale, k_scale, B, H, Hkv, Lq, Lk, D, mode, stream=None):
+    _check(lib().lamp_quant_qk(_ptr(q), _ptr(k), _ptr(q8), _ptr(k8), _ptr(q_scale), _ptr(k_scale),
+                               B, H, Hkv, Lq, Lk, D, mode, _stream(stream)))
+
+
+def lamp_build_mask(mask_bits, B, H, Lq, Lk, D, group_tiles, fp16_fraction, seed, stream=None):
+    _check(lib().lamp_build_mask(_ptr(mask_bits), B, H, Lq, Lk, D, group_tiles,
+                                 float(fp16_fraction), int(seed) & (2**64 - 1), _stream(stream)))
+
+
+def lamp_attn_fwd(q, k, v, o, lse, B, H, Hkv, Lq, Lk, D, causal, window, scale, mask_bits,
+                  group_tiles, mode, tau, stream=None):
+    _check(lib().lamp_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Lq, Lk,
+                               D, int(causal), int(window), float(scale), _ptr(mask_bits),
+                               int(group_tiles), int(mode), float(tau), _stream(stream)))
+
+
+def lamp_attn_fwd_q8(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D, causal,
+                     window, scale, mask_bits, group_tiles, mode, tau, route_out=None,
+                     stream=None):
+    _check(lib().lamp_attn_fwd_q8(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(q_scale),
+                                  _ptr(k_scale), _ptr(o), _ptr(lse), B, H, Hkv, Lq, Lk, D,
+                                  int(causal), int(window), float(scale), _ptr(mask_bits),
+                                  int(group_tiles), int(mode), float(tau), _ptr(route_out),
+                                  _stream(stream)))
+
+
+def lamp_workspace_size(B, H, Hkv, Lq, Lk, D, mode=0) -> int:
+    return int(lib().lamp_workspace_size(B, H, Hkv, Lq, Lk, D, mode))
+
+
+def lamp_set_workspace(ptr, nbytes: int):
+    _check(lib().lamp_set_workspace(_ptr(ptr), int(nbytes)))
+
+
+def lamp_check(stream=None):
+    _check(lib().lamp_check(_stream(stream)))
+
+
+def lamp_selftest_timeout(wait_ns: int, stream=None):
+    _check(lib().lamp_selftest_timeout(int(wait_ns), _stream(stream)))
+
+
+def lamp_last_error() -> str:
+    return lib().lamp_last_error().decode()
+
+
+# ------------------------------------------------------------ torch conveniences ------
+# Allocation of outputs with torch (device memory is PyTorch's job here); the arithmetic
+# stays in the library.
+
+def attention(q, k, v, *, causal=False, window=0, scale=0.0, mask_bits=None, group_tiles=1,
+              route="bitmask", fmt="int8", tau=0.0, out="f32", stream=None):
+    """O, lse for q [B,H,Lq,D], k/v [B,Hkv,Lk,D] (fp16/bf16 CUDA tensors)."""
+    import torch
+    B, H, Lq, D = q.shape
+    _, Hkv, Lk, _ = k.shape
+    dtype = "bf16" if q.dtype == torch.bfloat16 else "fp16"
+    o = torch.empty((B, H, Lq, D), device=q.device,
+                    dtype=torch.float32 if out == "f32" else q.dtype)
+    lse = torch.empty((B, H, Lq), device=q.device, dtype=torch.float32)
+    lamp_attn_fwd(q, k, v, o, lse, B, H, Hkv, Lq, Lk, D, causal, window, scale, mask_bits,
+                  group_tiles, mode_bits(route, fmt, dtype, out), tau, stream)
+    return o, lse
+
+
+def quantize(q, k, *, fmt="int8", stream=None):
+    """(q8, k8, q_scale, k_scale) for q [B,H,Lq,D], k [B,Hkv,Lk,D]."""
+    import torch
+    B, H, Lq, D = q.shape
+    _, Hkv, Lk, _ = k.shape
+    bm, bn = lamp_tile_shape(D)
+    q8 = torch.empty(q.shape, device=q.device, dtype=torch.uint8)
+    k8 = torch.empty(k.shape, device=k.device, dtype=torch.uint8)
+    qs = torch.empty((B, H, -(-Lq // bm)), device=q.device, dtype=torch.float32)
+    ks = torch.empty((B, Hkv, -(-Lk // bn)), device=q.device, dtype=torch.float32)
+    dtype = "bf16" if q.dtype == torch.bfloat16 else "fp16"
+    lamp_quant_qk(q, k, q8, k8, qs, ks, B, H, Hkv, Lq, Lk, D, mode_bits(fmt=fmt, dtype=dtype),
+                  stream)
+    return q8, k8, qs, ks
+
+
+def build_mask(B, H, Lq, Lk, D, group_tiles, fp16_fraction, seed, device="cuda", stream=None):
+    import torch
+    bm, _ = lamp_tile_shape(D)
+    W = lamp_mask_words(Lk, D, group_tiles)
+    m = torch.empty((B, H, -(-Lq // bm), W), device=device, dtype=torch.int64)
+    lamp_build_mask(m, B, H, Lq, Lk, D, group_tiles, fp16_fraction, seed, stream)
+    return m
+
+
+def attention_q8(q, k, v, q8, k8, q_scale, k_scale, *, causal=False, window=0, scale=0.0,
+                 mask_bits=None, group_tiles=1, route="bitmask", fmt="int8", tau=0.0,
+                 out="f32", want_route=False, stream=None):
+    import torch
+    B, H, Lq, D = q.shape
+    _, Hkv, Lk, _ = k.shape
+    bm, bn = lamp_tile_shape(D)
+    dtype = "bf16" if q.dtype == torch.bfloat16 else "fp16"
+    o = torch.empty((B, H, Lq, D), device=q.device,
+                    dtype=torch.float32 if out == "f32" else q.dtype)
+    lse = torch.empty((B, H, Lq), device=q.device, dtype=torch.float32)
+    rmap = (torch.empty((B, H, -(-Lq // bm), -(-Lk // bn)), device=q.device, dtype=torch.uint8)
+            if want_route else None)
+    lamp_attn_fwd_q8(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D, causal,
+                     window, scale, mask_bits, group_tiles, mode_bits(route, fmt, dtype, out),
+                     tau, rmap, stream)
+    return (o, lse, rmap) if want_route else (o, lse)

@@ -1,0 +1,700 @@
+// Routed mixed-precision attention forward for sm_100a.
+//
+// What it computes (TileMix page, section 2 "How It Works"; LampAttention abstract):
+// softmax(scale * Q K^T) V over the visible (causal / sliding-window) pairs, where each score
+// tile (routing tile BM x BN) is either the 8-bit product of per-block quantised Q and K,
+// rescaled by the two block scales, or the 16-bit product of the inputs.  The choice comes from
+// a packed bitmask (one bit per group of key tiles, 0 = 16-bit) or from the look-ahead rule
+// (recompute in 16 bits when some row's 8-bit tile max reaches the running row max minus tau).
+// Both paths update one online-softmax state (m, l) per row; P.V is 16-bit.
+//
+// B200 design:
+//   * one CTA per (batch, head, 128-row query tile); grid ordered longest-first (causal);
+//   * warp 4 (one thread) streams Q16/Q8 once and then K8 / K16 / V tiles with TMA into a
+//     ring of shared-memory slots (128-byte or 64-byte swizzled, the layouts the tensor core
+//     reads), each slot guarded by full/empty mbarriers;
+//   * warp 5 (one thread) issues tcgen05 MMAs: S = Q8 K8^T (kind::i8 into int32 TMEM or
+//     kind::f8f6f4 into fp32 TMEM), S = Q16 K16^T (kind::f16), O += P V with P read from TMEM;
+//     the S buffer is double-buffered so S(t+1) runs on the tensor core while rows of S(t)
+//     are in the softmax;
+//   * warps 0-3 own one query row per thread (TMEM lane = row): they read S from TMEM,
+//     dequantise, mask, vote on the look-ahead rule, run the online softmax (MUFU ex2), store
+//     P as packed 16-bit pairs into the S columns, rescale O in TMEM when the row max grows,
+//     and write O / lse at the end;
+//   * routing tiles of 64 query rows (D = 64, 256) are stacked two per 128-row MMA; a key
+//     tile whose two halves need different precisions runs the 8-bit MMA first, then the
+//     16-bit MMA into the same TMEM columns after every row has read its 8-bit scores.
+// Every mbarrier wait is bounded; on a timeout the CTA records the failure, stops, drains its
+// in-flight copies and MMAs, frees its TMEM and exits.
+#pragma once
+
+#include <cuda.h>
+
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace lamp {
+
+__device__ uint32_t g_lamp_error;  // device-side error word, read and cleared by lamp_check
+
+// where-codes recorded with a timeout (bits 8..15 of the error word)
+enum : uint32_t {
+  W_QFULL = 1, W_EMPTY = 2, W_FULL = 3, W_SFULL = 4, W_S16 = 5, W_VOTE = 6, W_PFULL = 7,
+  W_ODONE = 8, W_DRAIN = 9, W_SELFTEST = 10
+};
+
+struct AttnParams {
+  CUtensorMap tm_q16;  // [B*H][Lq][D] 16-bit, box 64 x 128 x 1, 128B swizzle
+  CUtensorMap tm_k16;  // [B*Hkv][Lk][D] 16-bit, box 64 x BN x 1, 128B swizzle
+  CUtensorMap tm_v;    // [B*Hkv][Lk][D] 16-bit, box 64 x BN x 1, 128B swizzle
+  CUtensorMap tm_q8;   // [B*H][Lq][D] 8-bit, box min(D,128) x 128 x 1
+  CUtensorMap tm_k8;   // [B*Hkv][Lk][D] 8-bit, box min(D,128) x BN x 1
+  const float* q_scale;  // [B][H][nQT]
+  const float* k_scale;  // [B][Hkv][nKT]
+  const uint64_t* mask;  // [B][H][nQT][W] or null
+  void* o;
+  float* lse;
+  uint8_t* route;
+  int B, H, Hkv, Lq, Lk;
+  int n_ct, nqt, nkt, mask_words, group_tiles;
+  int causal, window;
+  float scale_log2, tau_log2;
+  int adaptive, e4m3, bf16, out_f32;
+  uint64_t wait_ns;
+};
+
+template <int D_, int BN_, bool STACK_>
+struct AttnCfg {
+  static constexpr int D = D_;
+  static constexpr int BN = BN_;
+  static constexpr bool STACK = STACK_;        // routing tiles of 64 rows, two per MMA tile
+  static constexpr int BM = STACK ? 64 : 128;  // routing tile rows
+  static constexpr int MT = 128;               // MMA tile rows
+  static constexpr int Q16_BYTES = MT * D * 2;
+  static constexpr int Q8_BYTES = MT * D;
+  static constexpr int SLOT_BYTES = BN * D * 2;
+  static constexpr int NS = (D == 64) ? 8 : (D == 128 ? 5 : 2);
+  static constexpr bool Q8_SW64 = (D == 64);  // 64-byte rows of 8-bit codes
+  static constexpr int C16 = D / 64;           // 128-byte chunks of a 16-bit row
+  static constexpr int C8 = (D == 64) ? 1 : D / 128;
+  static constexpr int TMEM_O = 2 * BN;
+  static constexpr int TMEM_COLS = (2 * BN + D) <= 256 ? 256 : 512;
+  static constexpr int OFF_Q16 = 0;
+  static constexpr int OFF_Q8 = Q16_BYTES;
+  static constexpr int OFF_SLOTS = Q16_BYTES + Q8_BYTES;
+  static constexpr int OFF_BAR = OFF_SLOTS + NS * SLOT_BYTES;
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
+  static_assert(OFF_Q8 % 1024 == 0 && OFF_SLOTS % 1024 == 0 && SLOT_BYTES % 1024 == 0, "align");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static_assert(2 * BN + D <= 512, "tmem");
+};
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t full[8];
+  uint64_t empty[8];
+  uint64_t s_full[2];
+  uint64_t s16_full[2];
+  uint64_t vote[2];
+  uint64_t p_full[2];
+  uint64_t o_done;
+  uint64_t drain;
+  uint32_t tmem_base;
+  uint32_t abort;
+  uint32_t votes[2][4];
+};
+
+// Per-key-tile routing plan, computed identically by the three roles.
+struct Plan {
+  bool first16;    // first (or only) S MMA is 16-bit
+  bool two_phase;  // an 8-bit S is followed by a possible 16-bit S in the same columns
+  bool live[2];    // routing half h has a visible pair in this key tile
+  bool b16[2];     // bitmask: routing half h is 16-bit
+};
+
+struct Geo {
+  int b, h, kvh, ct, q0, kt_lo, n;
+  int half_lo[2], half_hi[2];  // visible key range (union) of each routing half; lo > hi = none
+};
+
+__device__ __forceinline__ void visible_range(const AttnParams& p, int i, int& lo, int& hi) {
+  if (!p.causal) {
+    lo = 0;
+    hi = p.Lk - 1;
+    return;
+  }
+  const int off = p.Lk - p.Lq;
+  hi = min(i + off, p.Lk - 1);
+  lo = (p.window > 0) ? max(0, i + off - p.window + 1) : 0;
+}
+
+template <class C>
+__device__ __forceinline__ Geo make_geo(const AttnParams& p) {
+  Geo g;
+  const int BH = p.B * p.H;
+  const int idx = blockIdx.x;
+  g.ct = p.n_ct - 1 - idx / BH;  // longest-first for causal workloads
+  const int bh = idx - (idx / BH) * BH;
+  g.b = bh / p.H;
+  g.h = bh - g.b * p.H;
+  g.kvh = g.h / (p.H / p.Hkv);
+  g.q0 = g.ct * C::MT;
+  const int nh = C::STACK ? 2 : 1;
+  int lo_all = 1 << 30, hi_all = -1;
+  for (int hh = 0; hh < 2; ++hh) {
+    g.half_lo[hh] = 1;
+    g.half_hi[hh] = 0;
+    if (hh >= nh) continue;
+    const int r0 = g.q0 + hh * C::BM;
+    const int r1 = min(p.Lq, r0 + (C::STACK ? C::BM : C::MT)) - 1;
+    if (r0 > r1) continue;
+    int lo0, hi0, lo1, hi1;
+    visible_range(p, r0, lo0, hi0);
+    visible_range(p, r1, lo1, hi1);
+    const int lo = lo0, hi = hi1;
+    if (hi < 0 || lo > hi) continue;
+    g.half_lo[hh] = lo;
+    g.half_hi[hh] = hi;
+    lo_all = min(lo_all, lo);
+    hi_all = max(hi_all, hi);
+  }
+  if (hi_all < lo_all) {
+    g.kt_lo = 0;
+    g.n = 0;
+  } else {
+    g.kt_lo = lo_all / C::BN;
+    g.n = hi_all / C::BN - g.kt_lo + 1;
+  }
+  return g;
+}
+
+template <class C>
+__device__ __forceinline__ Plan make_plan(const AttnParams& p, const Geo& g, int kt) {
+  Plan pl;
+  const int c0 = kt * C::BN, c1 = min(p.Lk, c0 + C::BN) - 1;
+  bool need8 = false, need16 = false;
+  const int g_idx = kt / p.group_tiles;
+  for (int hh = 0; hh < 2; ++hh) {
+    pl.live[hh] = g.half_lo[hh] <= g.half_hi[hh] && g.half_lo[hh] <= c1 && g.half_hi[hh] >= c0;
+    pl.b16[hh] = false;
+    if (!pl.live[hh] || p.adaptive) continue;
+    int bit = 1;
+    if (p.mask) {
+      const int qt = C::STACK ? 2 * g.ct + hh : g.ct;
+      const uint64_t w =
+          p.mask[(static_cast<size_t>(g.b * p.H + g.h) * p.nqt + qt) * p.mask_words + (g_idx >> 6)];
+      bit = static_cast<int>((w >> (g_idx & 63)) & 1ull);
+    }
+    pl.b16[hh] = (bit == 0);
+    if (bit) need8 = true; else need16 = true;
+  }
+  if (p.adaptive) {
+    pl.first16 = false;
+    pl.two_phase = true;
+  } else {
+    pl.two_phase = need8 && need16;
+    pl.first16 = !need8;
+  }
+  return pl;
+}
+
+// ------------------------------------------------------------------ producer ----------
+
+template <class C>
+__device__ void producer_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars& bars,
+                              const WaitCtx& wc) {
+  uint8_t* sQ16 = smem + C::OFF_Q16;
+  uint8_t* sQ8 = smem + C::OFF_Q8;
+  uint8_t* slots = smem + C::OFF_SLOTS;
+  const int bh_q = g.b * p.H + g.h;
+  const int bh_kv = g.b * p.Hkv + g.kvh;
+
+  prefetch_tmap(&p.tm_q16);
+  prefetch_tmap(&p.tm_k16);
+  prefetch_tmap(&p.tm_v);
+  prefetch_tmap(&p.tm_q8);
+  prefetch_tmap(&p.tm_k8);
+
+  mbar_arrive_expect_tx(&bars.q_full, C::Q16_BYTES + C::Q8_BYTES);
+  for (int c = 0; c < C::C16; ++c)
+    tma_load_3d(sQ16 + c * C::MT * 128, &p.tm_q16, &bars.q_full, c * 64, g.q0, bh_q);
+  for (int c = 0; c < C::C8; ++c)
+    tma_load_3d(sQ8 + c * C::MT * 128, &p.tm_q8, &bars.q_full, c * 128, g.q0, bh_q);
+
+  uint32_t item = 0;
+  bool ok = true;
+  // kind: 0 = K8, 1 = K16, 2 = V
+  auto load = [&](int kind, int kt) -> bool {
+    const int slot = static_cast<int>(item % C::NS);
+    const uint32_t use = item / C::NS;
+    if (use > 0 && !mbar_wait(&bars.empty[slot], (use - 1) & 1u, wc, W_EMPTY)) return false;
+    uint8_t* dst = slots + slot * C::SLOT_BYTES;
+    const int row = kt * C::BN;
+    if (kind == 0) {
+      mbar_arrive_expect_tx(&bars.full[slot], C::BN * C::D);
+      for (int c = 0; c < C::C8; ++c)
+        tma_load_3d(dst + c * C::BN * 128, &p.tm_k8, &bars.full[slot], c * 128, row, bh_kv);
+    } else {
+      const CUtensorMap* tm = (kind == 1) ? &p.tm_k16 : &p.tm_v;
+      mbar_arrive_expect_tx(&bars.full[slot], C::BN * C::D * 2);
+      for (int c = 0; c < C::C16; ++c)
+        tma_load_3d(dst + c * C::BN * 128, tm, &bars.full[slot], c * 64, row, bh_kv);
+    }
+    ++item;
+    return true;
+  };
+
+  Plan cur = make_plan<C>(p, g, g.kt_lo);
+  ok = load(cur.first16 ? 1 : 0, g.kt_lo);
+  for (int t = 0; ok && t < g.n; ++t) {
+    const int kt = g.kt_lo + t;
+    Plan nxt;
+    if (t + 1 < g.n) {
+      nxt = make_plan<C>(p, g, kt + 1);
+      if (!(ok = load(nxt.first16 ? 1 : 0, kt + 1))) break;
+    }
+    if (cur.two_phase && !(ok = load(1, kt))) break;
+    if (!(ok = load(2, kt))) break;
+    cur = nxt;
+  }
+  // Drain: every slot's most recent load must have landed before the CTA may exit.
+  WaitCtx drain = wc;
+  volatile uint32_t never = 0;
+  drain.abort = &never;
+  drain.limit_ns = 50000000ull;
+  const uint32_t first = item > static_cast<uint32_t>(C::NS) ? item - C::NS : 0;
+  for (uint32_t it = first; it < item; ++it)
+    mbar_wait(&bars.full[it % C::NS], (it / C::NS) & 1u, drain, W_DRAIN);
+  mbar_wait(&bars.q_full, 0, drain, W_DRAIN);
+}
+
+// ------------------------------------------------------------------ MMA issuer --------
+
+template <class C>
+__device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars& bars,
+                         uint32_t tbase, const WaitCtx& wc) {
+  const uint32_t sQ16 = smem_u32(smem + C::OFF_Q16);
+  const uint32_t sQ8 = smem_u32(smem + C::OFF_Q8);
+  const uint32_t slots = smem_u32(smem + C::OFF_SLOTS);
+  const uint32_t f16 = p.bf16 ? 1u : 0u;
+  const uint32_t id_s16 = idesc(1, f16, f16, 0, 0, C::BN, 128);
+  const uint32_t id_s8 = p.e4m3 ? idesc(1, 0, 0, 0, 0, C::BN, 128) : idesc(2, 1, 1, 0, 0, C::BN, 128);
+  const uint32_t id_pv = idesc(1, f16, f16, 0, 1, C::D, 128);
+
+  uint32_t item = 0;
+  uint32_t cv[2] = {0, 0}, cp[2] = {0, 0};
+  bool ok = mbar_wait(&bars.q_full, 0, wc, W_QFULL);
+  tc_fence_after();
+
+  auto take = [&](int& slot) -> bool {
+    slot = static_cast<int>(item % C::NS);
+    const uint32_t use = item / C::NS;
+    ++item;
+    if (!mbar_wait(&bars.full[slot], use & 1u, wc, W_FULL)) return false;
+    tc_fence_after();
+    return true;
+  };
+  auto issue_s = [&](int t, bool sixteen, int slot) {
+    const uint32_t dS = tbase + static_cast<uint32_t>((t & 1) * C::BN);
+    const uint32_t ks = slots + slot * C::SLOT_BYTES;
+    if (sixteen) {
+#pragma unroll
+      for (int s = 0; s < C::D / 16; ++s) {
+        const int c = s >> 2, off = (s & 3) * 32;
+        const uint64_t a = sdesc(sQ16 + c * C::MT * 128 + off, 16, 1024, SWZ_128B);
+        const uint64_t b = sdesc(ks + c * C::BN * 128 + off, 16, 1024, SWZ_128B);
+        mma_f16_ss(dS, a, b, id_s16, s > 0 ? 1u : 0u);
+      }
+    } else {
+#pragma unroll
+      for (int s = 0; s < C::D / 32; ++s) {
+        uint64_t a, b;
+        if (C::Q8_SW64) {
+          a = sdesc(sQ8 + s * 32, 16, 512, SWZ_64B);
+          b = sdesc(ks + s * 32, 16, 512, SWZ_64B);
+        } else {
+          const int c = s >> 2, off = (s & 3) * 32;
+          a = sdesc(sQ8 + c * C::MT * 128 + off, 16, 1024, SWZ_128B);
+          b = sdesc(ks + c * C::BN * 128 + off, 16, 1024, SWZ_128B);
+        }
+        if (p.e4m3)
+          mma_f8_ss(dS, a, b, id_s8, s > 0 ? 1u : 0u);
+        else
+          mma_i8_ss(dS, a, b, id_s8, s > 0 ? 1u : 0u);
+      }
+    }
+  };
+
+  Plan cur = make_plan<C>(p, g, g.kt_lo);
+  int slot = 0;
+  if (ok && (ok = take(slot))) {
+    issue_s(0, cur.first16, slot);
+    tc_commit(&bars.s_full[0]);
+    tc_commit(&bars.empty[slot]);
+  }
+  for (int t = 0; ok && t < g.n; ++t) {
+    const int bsel = t & 1;
+    Plan nxt;
+    if (t + 1 < g.n) {
+      nxt = make_plan<C>(p, g, g.kt_lo + t + 1);
+      if (!(ok = take(slot))) break;
+      issue_s(t + 1, nxt.first16, slot);
+      tc_commit(&bars.s_full[(t + 1) & 1]);
+      tc_commit(&bars.empty[slot]);
+    }
+    if (cur.two_phase) {
+      int slot16;
+      if (!(ok = take(slot16))) break;
+      if (!(ok = mbar_wait(&bars.vote[bsel], cv[bsel] & 1u, wc, W_VOTE))) break;
+      ++cv[bsel];
+      tc_fence_after();
+      bool s16;
+      if (p.adaptive) {
+        const volatile uint32_t* vv = bars.votes[bsel];
+        s16 = (vv[0] | vv[1] | vv[2] | vv[3]) != 0;
+      } else {
+        s16 = true;
+      }
+      if (s16) {
+        issue_s(t, true, slot16);
+        tc_commit(&bars.s16_full[bsel]);
+        tc_commit(&bars.empty[slot16]);
+      } else {
+        mbar_arrive(&bars.empty[slot16]);
+      }
+    }
+    if (!(ok = mbar_wait(&bars.p_full[bsel], cp[bsel] & 1u, wc, W_PFULL))) break;
+    ++cp[bsel];
+    tc_fence_after();
+    int slotv;
+    if (!(ok = take(slotv))) break;
+    const uint32_t vs = slots + slotv * C::SLOT_BYTES;
+    const uint32_t pt = tbase + static_cast<uint32_t>(bsel * C::BN);
+#pragma unroll
+    for (int s = 0; s < C::BN / 16; ++s) {
+      const uint64_t b = sdesc(vs + s * 16 * 128, C::BN * 128, 1024, SWZ_128B);
+      mma_f16_ts(tbase + C::TMEM_O, pt + s * 8, b, id_pv, (t > 0 || s > 0) ? 1u : 0u);
+    }
+    tc_commit(&bars.o_done);
+    tc_commit(&bars.empty[slotv]);
+    cur = nxt;
+  }
+  // Every MMA issued by this thread must complete before the TMEM is released.
+  tc_commit(&bars.drain);
+  WaitCtx drain = wc;
+  volatile uint32_t never = 0;
+  drain.abort = &never;
+  drain.limit_ns = 50000000ull;
+  mbar_wait(&bars.drain, 0, drain, W_DRAIN);
+}
+
+// ------------------------------------------------------------------ softmax -----------
+
+// All 32 lanes poll the barrier; the result is made warp-uniform (and the warp reconverged)
+// before any warp-collective tcgen05 instruction follows.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtx& wc,
+                                          uint32_t where) {
+  const bool ok = mbar_wait(bar, parity, wc, where);
+  return __all_sync(0xFFFFFFFFu, ok);
+}
+
+template <class C>
+__device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint32_t tbase,
+                             const WaitCtx& wc) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = warp * 32 + lane;
+  const int i = g.q0 + r;
+  const bool row_valid = i < p.Lq;
+  const int hh = C::STACK ? (r >> 6) : 0;
+  const int qt_r = C::STACK ? 2 * g.ct + hh : g.ct;
+  const int bh_q = g.b * p.H + g.h;
+  const uint32_t lane_base = tbase + (static_cast<uint32_t>(warp * 32) << 16);
+  int lo_r = 1, hi_r = 0;
+  if (row_valid) visible_range(p, i, lo_r, hi_r);
+  const float sq = (row_valid && qt_r < p.nqt) ? __ldg(p.q_scale + static_cast<size_t>(bh_q) * p.nqt + qt_r) : 0.0f;
+  const float* ks_row = p.k_scale + static_cast<size_t>(g.b * p.Hkv + g.kvh) * p.nkt;
+  const float NEG_INF = -__int_as_float(0x7f800000);
+
+  float m = NEG_INF, l_ex = 0.0f, l_rd = 0.0f;
+  uint32_t cs[2] = {0, 0}, c16[2] = {0, 0}, cv[2] = {0, 0};
+  bool ok = true;
+  uint32_t sraw[C::BN];
+
+  auto load_s = [&](int bsel) {
+#pragma unroll
+    for (int c = 0; c < C::BN / 32; ++c) {
+      uint32_t (&dst)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sraw[c * 32]);
+      tmem_ld32(lane_base + static_cast<uint32_t>(bsel * C::BN + c * 32), dst);
+    }
+    tmem_wait_ld();
+  };
+  auto mask_s = [&](int kt) {
+    const int j0 = kt * C::BN;
+    const bool full = row_valid && j0 >= lo_r && j0 + C::BN - 1 <= hi_r;
+    if (!full) {
+#pragma unroll
+      for (int c = 0; c < C::BN; ++c) {
+        const int j = j0 + c;
+        if (!row_valid || j < lo_r || j > hi_r) sraw[c] = __float_as_uint(NEG_INF);
+      }
+    }
+  };
+  auto sf = [&](int c) -> float { return __uint_as_float(sraw[c]); };
+
+  for (int t = 0; ok && t < g.n; ++t) {
+    const int kt = g.kt_lo + t;
+    const int bsel = t & 1;
+    const Plan pl = make_plan<C>(p, g, kt);
+    if (!(ok = warp_wait(&bars.s_full[bsel], cs[bsel] & 1u, wc, W_SFULL))) break;
+    ++cs[bsel];
+    tc_fence_after();
+    load_s(bsel);
+    if (!pl.first16) {
+      const float c8 = sq * __ldg(ks_row + kt) * p.scale_log2;
+      if (p.e4m3) {
+#pragma unroll
+        for (int c = 0; c < C::BN; ++c) sraw[c] = __float_as_uint(sf(c) * c8);
+      } else {
+#pragma unroll
+        for (int c = 0; c < C::BN; ++c)
+          sraw[c] = __float_as_uint(static_cast<float>(static_cast<int>(sraw[c])) * c8);
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < C::BN; ++c) sraw[c] = __float_as_uint(sf(c) * p.scale_log2);
+    }
+    mask_s(kt);
+
+    bool my16 = pl.first16;
+    if (pl.two_phase) {
+      if (p.adaptive) {
+        float t8 = NEG_INF;
+#pragma unroll
+        for (int c = 0; c < C::BN; ++c) t8 = fmaxf(t8, sf(c));
+        const bool vote = (t8 != NEG_INF) && (t8 >= m - p.tau_log2);
+        const uint32_t wv = __any_sync(0xFFFFFFFFu, vote) ? 1u : 0u;
+        if (lane == 0) bars.votes[bsel][warp] = wv;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.vote[bsel]);
+      if (!(ok = warp_wait(&bars.vote[bsel], cv[bsel] & 1u, wc, W_VOTE))) break;
+      ++cv[bsel];
+      bool f[2];
+      if (p.adaptive) {
+        const volatile uint32_t* vv = bars.votes[bsel];
+        if (C::STACK) {
+          f[0] = (vv[0] | vv[1]) != 0;
+          f[1] = (vv[2] | vv[3]) != 0;
+        } else {
+          f[0] = f[1] = (vv[0] | vv[1] | vv[2] | vv[3]) != 0;
+        }
+      } else {
+        f[0] = pl.live[0] && pl.b16[0];
+        f[1] = pl.live[1] && pl.b16[1];
+      }
+      const bool s16 = p.adaptive ? (f[0] || f[1]) : true;
+      my16 = f[hh];
+      if (s16) {
+        if (!(ok = warp_wait(&bars.s16_full[bsel], c16[bsel] & 1u, wc, W_S16))) break;
+        ++c16[bsel];
+        tc_fence_after();
+        if (my16) {
+          load_s(bsel);
+#pragma unroll
+          for (int c = 0; c < C::BN; ++c) sraw[c] = __float_as_uint(sf(c) * p.scale_log2);
+          mask_s(kt);
+        }
+      }
+    }
+    if (p.route && lane == 0 && (warp == 0 || (C::STACK && warp == 2))) {
+      if (pl.live[hh]) {
+        const uint8_t v = my16 ? (pl.two_phase && p.adaptive ? 3 : 2) : 1;
+        p.route[(static_cast<size_t>(bh_q) * p.nqt + qt_r) * p.nkt + kt] = v;
+      }
+    }
+
+    // online softmax on the routed scores (log2 units)
+    float mt = NEG_INF;
+#pragma unroll
+    for (int c = 0; c < C::BN; ++c) mt = fmaxf(mt, sf(c));
+    const float m_new = fmaxf(m, mt);
+    const float m_use = (m_new == NEG_INF) ? 0.0f : m_new;
+    const float alpha = (m == m_new) ? 1.0f : ((m == NEG_INF) ? 0.0f : ex2(m - m_use));
+    float sum_ex = 0.0f, sum_rd = 0.0f;
+#pragma unroll
+    for (int c = 0; c < C::BN; c += 2) {
+      const float p0 = ex2(sf(c) - m_use);
+      const float p1 = ex2(sf(c + 1) - m_use);
+      sum_ex += p0 + p1;
+      uint32_t pk;
+      if (p.bf16) {
+        __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
+        sum_rd += __low2float(v2) + __high2float(v2);
+        pk = *reinterpret_cast<uint32_t*>(&v2);
+      } else {
+        __half2 v2 = __floats2half2_rn(p0, p1);
+        sum_rd += __low2float(v2) + __high2float(v2);
+        pk = *reinterpret_cast<uint32_t*>(&v2);
+      }
+      sraw[c >> 1] = pk;
+    }
+    l_ex = l_ex * alpha + sum_ex;
+    l_rd = l_rd * alpha + sum_rd;
+
+    if (t > 0) {
+      if (!(ok = warp_wait(&bars.o_done, (t - 1) & 1u, wc, W_ODONE))) break;
+      tc_fence_after();
+      if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+#pragma unroll 1
+        for (int c = 0; c < C::D / 32; ++c) {
+          uint32_t ov[32];
+          const uint32_t ta = lane_base + static_cast<uint32_t>(C::TMEM_O + c * 32);
+          tmem_ld32(ta, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tmem_st16(ta, ov);
+          tmem_st16(ta + 16, ov + 16);
+        }
+        tmem_wait_st();
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < C::BN / 32; ++c)
+      tmem_st16(lane_base + static_cast<uint32_t>(bsel * C::BN + c * 16), &sraw[c * 16]);
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars.p_full[bsel]);
+    m = m_new;
+  }
+  if (!ok) return;
+
+  // epilogue: O / l and lse
+  if (g.n > 0) {
+    if (!warp_wait(&bars.o_done, (g.n - 1) & 1u, wc, W_ODONE)) return;
+    tc_fence_after();
+  }
+  const float inv = (l_rd > 0.0f) ? 1.0f / l_rd : 0.0f;
+  const size_t orow = (static_cast<size_t>(bh_q) * p.Lq + (row_valid ? i : 0)) * C::D;
+#pragma unroll 1
+  for (int c = 0; c < C::D / 32; ++c) {
+    uint32_t ov[32];
+    if (g.n > 0) {
+      tmem_ld32(lane_base + static_cast<uint32_t>(C::TMEM_O + c * 32), ov);
+      tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) ov[e] = 0u;
+    }
+    if (!row_valid) continue;
+    if (p.out_f32) {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow + c * 32);
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
+                             __uint_as_float(ov[4 * e + 2]) * inv, __uint_as_float(ov[4 * e + 3]) * inv);
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow + c * 32);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float a = __uint_as_float(ov[8 * e + 2 * q]) * inv;
+          const float b2 = __uint_as_float(ov[8 * e + 2 * q + 1]) * inv;
+          if (p.bf16) {
+            __nv_bfloat162 v2 = __floats2bfloat162_rn(a, b2);
+            w[q] = *reinterpret_cast<uint32_t*>(&v2);
+          } else {
+            __half2 v2 = __floats2half2_rn(a, b2);
+            w[q] = *reinterpret_cast<uint32_t*>(&v2);
+          }
+        }
+        dst[e] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  }
+  if (row_valid && p.lse) {
+    p.lse[static_cast<size_t>(bh_q) * p.Lq + i] =
+        (l_ex > 0.0f) ? m * 0.69314718055994530942f + logf(l_ex) : NEG_INF;
+  }
+}
+
+// ------------------------------------------------------------------ kernel ------------
+
+template <class C>
+__global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  Bars& bars = *reinterpret_cast<Bars*>(smem + C::OFF_BAR);
+  const int warp = threadIdx.x >> 5;
+  const Geo g = make_geo<C>(p);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars.q_full, 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(&bars.full[s], 1);
+      mbar_init(&bars.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars.s_full[b], 1);
+      mbar_init(&bars.s16_full[b], 1);
+      mbar_init(&bars.vote[b], 4);
+      mbar_init(&bars.p_full[b], 4);
+    }
+    mbar_init(&bars.o_done, 1);
+    mbar_init(&bars.drain, 1);
+    bars.abort = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&bars.tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = bars.tmem_base;
+  WaitCtx wc{&bars.abort, &g_lamp_error, p.wait_ns};
+
+  if (warp == 4) {
+    if ((threadIdx.x & 31) == 0 && g.n > 0) producer_role<C>(p, g, smem, bars, wc);
+  } else if (warp == 5) {
+    if ((threadIdx.x & 31) == 0 && g.n > 0) mma_role<C>(p, g, smem, bars, tbase, wc);
+  } else {
+    softmax_role<C>(p, g, bars, tbase, wc);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) {
+    __syncwarp();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
+}
+
+// A one-block kernel whose single wait can never complete: exercises the bounded-wait error
+// path (records a timeout in the error word and returns) without faulting the GPU.
+__global__ void selftest_timeout_kernel(uint64_t wait_ns) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    WaitCtx w{&abort_flag, &g_lamp_error, wait_ns};
+    mbar_wait(&bar, 0, w, W_SELFTEST);
+  }
+  __syncthreads();
+}
+
+}  // namespace lamp

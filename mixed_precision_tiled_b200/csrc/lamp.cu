@@ -1,0 +1,411 @@
+// Host side of the C ABI declared in include/lamp.h: argument checks, TMA tensor maps,
+// workspace management and kernel launches.  All device code is included into this one
+// translation unit so that the device error word is a single file-scope symbol.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/lamp.h"
+#include "attn_fwd.cuh"
+#include "quant.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(LAMP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define LAMP_CUDA(call, what)                  \
+  do {                                         \
+    cudaError_t e_ = (call);                   \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int tile_shape(int D, int* bm, int* bn) {
+  if (D == 64) { *bm = 64; *bn = 64; return LAMP_OK; }
+  if (D == 128) { *bm = 128; *bn = 128; return LAMP_OK; }
+  if (D == 256) { *bm = 64; *bn = 128; return LAMP_OK; }
+  return LAMP_ERR_UNSUPPORTED;
+}
+
+int check_sizes(int B, int H, int Hkv, int Lq, int Lk, int D) {
+  if (B < 1 || H < 1 || Hkv < 1 || Lq < 1 || Lk < 1)
+    return fail(LAMP_ERR_INVALID, "sizes must be positive (B=%d H=%d Hkv=%d Lq=%d Lk=%d)", B, H,
+                Hkv, Lq, Lk);
+  if (H % Hkv != 0) return fail(LAMP_ERR_INVALID, "H (%d) must be a multiple of Hkv (%d)", H, Hkv);
+  int bm, bn;
+  if (tile_shape(D, &bm, &bn) != LAMP_OK)
+    return fail(LAMP_ERR_UNSUPPORTED, "head dimension D=%d not supported (64, 128, 256)", D);
+  if (static_cast<long long>(B) * H * Lq * D >= (1ll << 40) ||
+      static_cast<long long>(B) * H > (1 << 24) || Lq > (1 << 30) || Lk > (1 << 30))
+    return fail(LAMP_ERR_INVALID, "problem too large");
+  return LAMP_OK;
+}
+
+// ---------------------------------------------------------------- tensor maps ---------
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::mutex g_mu;
+
+int get_encode() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode) return LAMP_OK;
+  cudaDriverEntryPointQueryResult q;
+  void* fn = nullptr;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+    return fail(LAMP_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return LAMP_OK;
+}
+
+// 3-D map over [outer][L][D] elements of `ebytes` bytes; box (inner, rows, 1).
+int make_map(CUtensorMap* m, const void* base, int ebytes, int D, int L, int outer, int inner,
+             int rows, CUtensorMapSwizzle swz) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
+                        static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * ebytes,
+                           static_cast<cuuint64_t>(D) * L * ebytes};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(inner), static_cast<cuuint32_t>(rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, ebytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                        3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LAMP_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return LAMP_OK;
+}
+
+// ---------------------------------------------------------------- workspace -----------
+
+struct Workspace {
+  void* user = nullptr;
+  size_t user_bytes = 0;
+  void* cached[64] = {};
+  size_t cached_bytes[64] = {};
+};
+Workspace g_ws;
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct WsLayout {
+  size_t q8, k8, qs, ks, total;
+};
+
+WsLayout ws_layout(int B, int H, int Hkv, int Lq, int Lk, int D) {
+  int bm, bn;
+  tile_shape(D, &bm, &bn);
+  const size_t nqt = (Lq + bm - 1) / bm, nkt = (Lk + bn - 1) / bn;
+  WsLayout w;
+  w.q8 = 0;
+  w.k8 = align256(static_cast<size_t>(B) * H * Lq * D);
+  w.qs = w.k8 + align256(static_cast<size_t>(B) * Hkv * Lk * D);
+  w.ks = w.qs + align256(static_cast<size_t>(B) * H * nqt * sizeof(float));
+  w.total = w.ks + align256(static_cast<size_t>(B) * Hkv * nkt * sizeof(float));
+  return w;
+}
+
+int get_workspace(size_t need, void** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_ws.user) {
+    if (g_ws.user_bytes < need)
+      return fail(LAMP_ERR_INVALID, "workspace too small: %zu bytes set, %zu needed", g_ws.user_bytes, need);
+    *out = g_ws.user;
+    return LAMP_OK;
+  }
+  int dev = 0;
+  LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(LAMP_ERR_INVALID, "device index out of range");
+  if (g_ws.cached_bytes[dev] < need) {
+    if (g_ws.cached[dev]) {
+      LAMP_CUDA(cudaDeviceSynchronize(), "cudaDeviceSynchronize");
+      cudaFree(g_ws.cached[dev]);
+      g_ws.cached[dev] = nullptr;
+      g_ws.cached_bytes[dev] = 0;
+    }
+    void* p = nullptr;
+    LAMP_CUDA(cudaMalloc(&p, need), "cudaMalloc(workspace)");
+    g_ws.cached[dev] = p;
+    g_ws.cached_bytes[dev] = need;
+  }
+  *out = g_ws.cached[dev];
+  return LAMP_OK;
+}
+
+// ---------------------------------------------------------------- launches ------------
+
+int launch_quant(const void* x, void* codes, float* scales, int outer, int L, int D, int blk,
+                 bool bf16, bool e4m3, cudaStream_t st) {
+  const int nb = (L + blk - 1) / blk;
+  const long long grid = static_cast<long long>(outer) * nb;
+  if (grid > 0x7FFFFFFF) return fail(LAMP_ERR_INVALID, "too many quantisation blocks");
+  auto* xs = static_cast<const uint16_t*>(x);
+  auto* cs = static_cast<uint8_t*>(codes);
+  dim3 g(static_cast<unsigned>(grid)), b(lamp::QUANT_THREADS);
+  if (bf16 && e4m3)
+    lamp::quant_kernel<true, true><<<g, b, 0, st>>>(xs, cs, scales, L, D, blk, nb);
+  else if (bf16)
+    lamp::quant_kernel<true, false><<<g, b, 0, st>>>(xs, cs, scales, L, D, blk, nb);
+  else if (e4m3)
+    lamp::quant_kernel<false, true><<<g, b, 0, st>>>(xs, cs, scales, L, D, blk, nb);
+  else
+    lamp::quant_kernel<false, false><<<g, b, 0, st>>>(xs, cs, scales, L, D, blk, nb);
+  LAMP_CUDA(cudaGetLastError(), "quant_kernel launch");
+  return LAMP_OK;
+}
+
+int quant_qk(const void* q, const void* k, void* q8, void* k8, float* q_scale, float* k_scale,
+             int B, int H, int Hkv, int Lq, int Lk, int D, int mode, cudaStream_t st) {
+  int bm, bn;
+  tile_shape(D, &bm, &bn);
+  const bool bf16 = (mode & LAMP_IN_BF16) != 0, e4m3 = (mode & LAMP_FMT_E4M3) != 0;
+  if (q) {
+    int r = launch_quant(q, q8, q_scale, B * H, Lq, D, bm, bf16, e4m3, st);
+    if (r) return r;
+  }
+  if (k) {
+    int r = launch_quant(k, k8, k_scale, B * Hkv, Lk, D, bn, bf16, e4m3, st);
+    if (r) return r;
+  }
+  return LAMP_OK;
+}
+
+template <class C>
+int launch_attn_cfg(const lamp::AttnParams& p, int grid, cudaStream_t st) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    LAMP_CUDA(cudaFuncSetAttribute(lamp::attn_fwd_kernel<C>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES),
+              "cudaFuncSetAttribute");
+    attr_set[dev] = true;
+  }
+  lamp::attn_fwd_kernel<C><<<grid, 192, C::SMEM_BYTES, st>>>(p);
+  LAMP_CUDA(cudaGetLastError(), "attn_fwd_kernel launch");
+  return LAMP_OK;
+}
+
+using Cfg64 = lamp::AttnCfg<64, 64, true>;
+using Cfg128 = lamp::AttnCfg<128, 128, false>;
+using Cfg256 = lamp::AttnCfg<256, 128, true>;
+
+int attn_q8(const void* q, const void* k, const void* v, const void* q8, const void* k8,
+            const float* q_scale, const float* k_scale, void* o, float* lse, int B, int H,
+            int Hkv, int Lq, int Lk, int D, int causal, int window, float scale,
+            const uint64_t* mask_bits, int group_tiles, int mode, float tau, uint8_t* route_out,
+            cudaStream_t st) {
+  int r = check_sizes(B, H, Hkv, Lq, Lk, D);
+  if (r) return r;
+  if (!q || !k || !v || !q8 || !k8 || !q_scale || !k_scale || !o)
+    return fail(LAMP_ERR_INVALID, "null operand pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q8) || !aligned16(k8) ||
+      !aligned16(o))
+    return fail(LAMP_ERR_INVALID, "q, k, v, q8, k8 and o must be 16-byte aligned");
+  if (causal != 0 && causal != 1) return fail(LAMP_ERR_INVALID, "causal must be 0 or 1");
+  if (window < 0) return fail(LAMP_ERR_INVALID, "window must be >= 0");
+  if (window > 0 && !causal)
+    return fail(LAMP_ERR_UNSUPPORTED, "a sliding window needs causal = 1");
+  if ((mode & ~0xFu) != 0) return fail(LAMP_ERR_INVALID, "unknown mode bits 0x%x", mode);
+  const bool adaptive = (mode & LAMP_ROUTE_ADAPTIVE) != 0;
+  if (!adaptive && group_tiles < 1) return fail(LAMP_ERR_INVALID, "group_tiles must be >= 1");
+  if (adaptive && !(tau == tau)) return fail(LAMP_ERR_INVALID, "tau is NaN");
+  if (!(scale == scale)) return fail(LAMP_ERR_INVALID, "scale is NaN");
+  if ((r = get_encode())) return r;
+
+  int bm, bn;
+  tile_shape(D, &bm, &bn);
+  lamp::AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int BHq = B * H, BHk = B * Hkv;
+  if ((r = make_map(&p.tm_q16, q, 2, D, Lq, BHq, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))) return r;
+  if ((r = make_map(&p.tm_k16, k, 2, D, Lk, BHk, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B))) return r;
+  if ((r = make_map(&p.tm_v, v, 2, D, Lk, BHk, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B))) return r;
+  const CUtensorMapSwizzle sw8 = (D == 64) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  const int in8 = (D == 64) ? 64 : 128;
+  if ((r = make_map(&p.tm_q8, q8, 1, D, Lq, BHq, in8, 128, sw8))) return r;
+  if ((r = make_map(&p.tm_k8, k8, 1, D, Lk, BHk, in8, bn, sw8))) return r;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  const int nqt = (Lq + bm - 1) / bm, nkt = (Lk + bn - 1) / bn;
+  const int gt = adaptive ? 1 : group_tiles;
+  const int ng = (nkt + gt - 1) / gt;
+  p.mask = adaptive ? nullptr : mask_bits;
+  p.mask_words = (ng + 63) / 64;
+  p.group_tiles = gt;
+  p.o = o;
+  p.lse = lse;
+  p.route = route_out;
+  p.B = B; p.H = H; p.Hkv = Hkv; p.Lq = Lq; p.Lk = Lk;
+  p.n_ct = (Lq + 127) / 128;
+  p.nqt = nqt;
+  p.nkt = nkt;
+  p.causal = causal;
+  p.window = window;
+  const float sc = (scale > 0.0f) ? scale : 1.0f / std::sqrt(static_cast<float>(D));
+  const float log2e = 1.4426950408889634f;
+  p.scale_log2 = sc * log2e;
+  p.tau_log2 = adaptive ? tau * log2e : 0.0f;
+  p.adaptive = adaptive ? 1 : 0;
+  p.e4m3 = (mode & LAMP_FMT_E4M3) ? 1 : 0;
+  p.bf16 = (mode & LAMP_IN_BF16) ? 1 : 0;
+  p.out_f32 = (mode & LAMP_OUT_INDTYPE) ? 0 : 1;
+  p.wait_ns = 2000000000ull;  // 2 s per wait: far beyond any legitimate stall
+  const long long grid = static_cast<long long>(BHq) * p.n_ct;
+  if (grid > 0x7FFFFFFF) return fail(LAMP_ERR_INVALID, "grid too large");
+  if (route_out)
+    LAMP_CUDA(cudaMemsetAsync(route_out, 0, static_cast<size_t>(BHq) * nqt * nkt, st), "memset route");
+  if (D == 64) return launch_attn_cfg<Cfg64>(p, static_cast<int>(grid), st);
+  if (D == 128) return launch_attn_cfg<Cfg128>(p, static_cast<int>(grid), st);
+  return launch_attn_cfg<Cfg256>(p, static_cast<int>(grid), st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int lamp_tile_shape(int D, int* bm, int* bn) {
+  if (!bm || !bn) return fail(LAMP_ERR_INVALID, "null output pointer");
+  int r = tile_shape(D, bm, bn);
+  if (r) return fail(r, "head dimension D=%d not supported (64, 128, 256)", D);
+  return LAMP_OK;
+}
+
+int lamp_mask_words(int Lk, int D, int group_tiles) {
+  int bm, bn;
+  if (Lk < 1 || group_tiles < 1 || tile_shape(D, &bm, &bn) != LAMP_OK) return -1;
+  const int nkt = (Lk + bn - 1) / bn;
+  const int ng = (nkt + group_tiles - 1) / group_tiles;
+  return (ng + 63) / 64;
+}
+
+int lamp_quant_qk(const void* q, const void* k, void* q8, void* k8, float* q_scale,
+                  float* k_scale, int B, int H, int Hkv, int Lq, int Lk, int D, int mode,
+                  void* stream) {
+  int r = check_sizes(B, H, Hkv, Lq, Lk, D);
+  if (r) return r;
+  if ((q == nullptr) != (q8 == nullptr) || (q == nullptr) != (q_scale == nullptr))
+    return fail(LAMP_ERR_INVALID, "q, q8 and q_scale must be all set or all null");
+  if ((k == nullptr) != (k8 == nullptr) || (k == nullptr) != (k_scale == nullptr))
+    return fail(LAMP_ERR_INVALID, "k, k8 and k_scale must be all set or all null");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q8) || !aligned16(k8))
+    return fail(LAMP_ERR_INVALID, "q, k, q8, k8 must be 16-byte aligned");
+  return quant_qk(q, k, q8, k8, q_scale, k_scale, B, H, Hkv, Lq, Lk, D, mode,
+                  static_cast<cudaStream_t>(stream));
+}
+
+int lamp_build_mask(uint64_t* mask_bits, int B, int H, int Lq, int Lk, int D, int group_tiles,
+                    float fp16_fraction, uint64_t seed, void* stream) {
+  if (!mask_bits) return fail(LAMP_ERR_INVALID, "null mask pointer");
+  int r = check_sizes(B, H, 1, Lq, Lk, D);
+  if (r) return r;
+  if (group_tiles < 1) return fail(LAMP_ERR_INVALID, "group_tiles must be >= 1");
+  if (!(fp16_fraction >= 0.0f && fp16_fraction <= 1.0f))
+    return fail(LAMP_ERR_INVALID, "fp16_fraction must be in [0, 1]");
+  int bm, bn;
+  tile_shape(D, &bm, &bn);
+  const int nqt = (Lq + bm - 1) / bm, nkt = (Lk + bn - 1) / bn;
+  const int ng = (nkt + group_tiles - 1) / group_tiles;
+  const int W = (ng + 63) / 64;
+  const long long rows = static_cast<long long>(B) * H * nqt;
+  const long long total = rows * W;
+  const int threads = 256;
+  const long long blocks = std::min<long long>((total + threads - 1) / threads, 148 * 16);
+  lamp::mask_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      mask_bits, rows, ng, W, static_cast<double>(fp16_fraction), seed);
+  LAMP_CUDA(cudaGetLastError(), "mask_kernel launch");
+  return LAMP_OK;
+}
+
+int lamp_attn_fwd_q8(const void* q, const void* k, const void* v, const void* q8,
+                     const void* k8, const float* q_scale, const float* k_scale, void* o,
+                     float* lse, int B, int H, int Hkv, int Lq, int Lk, int D, int causal,
+                     int window, float scale, const uint64_t* mask_bits, int group_tiles,
+                     int mode, float tau, uint8_t* route_out, void* stream) {
+  return attn_q8(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D, causal,
+                 window, scale, mask_bits, group_tiles, mode, tau, route_out,
+                 static_cast<cudaStream_t>(stream));
+}
+
+size_t lamp_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int D, int mode) {
+  (void)mode;
+  int bm, bn;
+  if (B < 1 || H < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || tile_shape(D, &bm, &bn) != LAMP_OK)
+    return 0;
+  return ws_layout(B, H, Hkv, Lq, Lk, D).total;
+}
+
+int lamp_set_workspace(void* ptr, size_t bytes) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (ptr && (reinterpret_cast<uintptr_t>(ptr) & 255u))
+    return fail(LAMP_ERR_INVALID, "workspace must be 256-byte aligned");
+  g_ws.user = ptr;
+  g_ws.user_bytes = ptr ? bytes : 0;
+  return LAMP_OK;
+}
+
+int lamp_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                  int H, int Hkv, int Lq, int Lk, int D, int causal, int window, float scale,
+                  const uint64_t* mask_bits, int group_tiles, int mode, float tau, void* stream) {
+  int r = check_sizes(B, H, Hkv, Lq, Lk, D);
+  if (r) return r;
+  if (!q || !k || !v || !o) return fail(LAMP_ERR_INVALID, "null operand pointer");
+  const WsLayout w = ws_layout(B, H, Hkv, Lq, Lk, D);
+  void* ws = nullptr;
+  if ((r = get_workspace(w.total, &ws))) return r;
+  auto* base = static_cast<uint8_t*>(ws);
+  uint8_t* q8 = base + w.q8;
+  uint8_t* k8 = base + w.k8;
+  float* qs = reinterpret_cast<float*>(base + w.qs);
+  float* ks = reinterpret_cast<float*>(base + w.ks);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(LAMP_ERR_INVALID, "q, k, v and o must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((r = quant_qk(q, k, q8, k8, qs, ks, B, H, Hkv, Lq, Lk, D, mode, st))) return r;
+  return attn_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D, causal, window, scale,
+                 mask_bits, group_tiles, mode, tau, nullptr, st);
+}
+
+int lamp_check(void* stream) {
+  LAMP_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)), "cudaStreamSynchronize");
+  uint32_t v = 0;
+  LAMP_CUDA(cudaMemcpyFromSymbol(&v, lamp::g_lamp_error, sizeof(v)), "read error word");
+  if (v) {
+    const uint32_t zero = 0;
+    LAMP_CUDA(cudaMemcpyToSymbol(lamp::g_lamp_error, &zero, sizeof(zero)), "clear error word");
+    return fail(LAMP_ERR_TIMEOUT, "a device wait gave up (error word 0x%x, site %u)", v, (v >> 8) & 0xFFu);
+  }
+  return LAMP_OK;
+}
+
+int lamp_selftest_timeout(uint64_t wait_ns, void* stream) {
+  if (wait_ns == 0 || wait_ns > 10000000000ull)
+    return fail(LAMP_ERR_INVALID, "wait_ns must be in (0, 1e10]");
+  lamp::selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(wait_ns);
+  LAMP_CUDA(cudaGetLastError(), "selftest launch");
+  return LAMP_OK;
+}
+
+const char* lamp_last_error(void) { return g_err; }
+
+}  // extern "C"

@@ -1,0 +1,116 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the header
+declares, and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import mixed_precision_tiled_b200 as mpt
+from mixed_precision_tiled_b200 import build as mbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    mbuild.build()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "lamp.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(lamp_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = header_functions()
+    assert len(names) >= 11
+    out = subprocess.check_output(["nm", "-D", "--defined-only", mbuild.LIB]).decode()
+    exported = set(re.findall(r" T (lamp_\w+)", out))
+    assert set(names) <= exported, set(names) - exported
+    assert set(names) == set(mpt.EXPORTS)
+    L = ctypes.CDLL(mbuild.LIB)
+    for n in names:
+        getattr(L, n)
+
+
+def test_tile_shapes_and_mask_words():
+    assert mpt.lamp_tile_shape(64) == (64, 64)
+    assert mpt.lamp_tile_shape(128) == (128, 128)
+    assert mpt.lamp_tile_shape(256) == (64, 128)
+    with pytest.raises(mpt.LampError) as e:
+        mpt.lamp_tile_shape(96)
+    assert e.value.code == mpt.LAMP_ERR_UNSUPPORTED
+    # config geometry: W = ceil(ceil(nKT / g) / 64)
+    assert mpt.lamp_mask_words(4096, 128, 4) == 1
+    assert mpt.lamp_mask_words(131072, 128, 8) == 2
+    assert mpt.lamp_mask_words(65536, 128, 8) == 1
+    assert mpt.lamp_mask_words(16384, 256, 2) == 1
+    assert mpt.lamp_mask_words(8193, 128, 1) == 2   # 65 key tiles
+    with pytest.raises(mpt.LampError):
+        mpt.lamp_mask_words(0, 128, 1)
+
+
+def _attn_args(**kw):
+    a = dict(q=0x1000, k=0x2000, v=0x3000, o=0x4000, lse=0x5000, B=1, H=4, Hkv=2, Lq=128,
+             Lk=128, D=128, causal=1, window=0, scale=0.0, mask_bits=None, group_tiles=1,
+             mode=0, tau=0.0)
+    a.update(kw)
+    return a
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(H=3, Hkv=2), mpt.LAMP_ERR_INVALID),
+    (dict(B=0), mpt.LAMP_ERR_INVALID),
+    (dict(Lq=0), mpt.LAMP_ERR_INVALID),
+    (dict(D=80), mpt.LAMP_ERR_UNSUPPORTED),
+    (dict(q=None), mpt.LAMP_ERR_INVALID),
+])
+def test_attn_fwd_rejects_bad_arguments_on_host(bad, code):
+    with pytest.raises(mpt.LampError) as e:
+        mpt.lamp_attn_fwd(**_attn_args(**bad), stream=0)
+    assert e.value.code == code
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(q=0x1001), mpt.LAMP_ERR_INVALID),            # misaligned
+    (dict(causal=0, window=16), mpt.LAMP_ERR_UNSUPPORTED),
+    (dict(window=-1), mpt.LAMP_ERR_INVALID),
+    (dict(group_tiles=0), mpt.LAMP_ERR_INVALID),
+    (dict(mode=0x30), mpt.LAMP_ERR_INVALID),
+    (dict(mode=1, tau=float("nan")), mpt.LAMP_ERR_INVALID),
+])
+def test_attn_fwd_q8_rejects_bad_arguments_on_host(bad, code):
+    a = _attn_args(**bad)
+    with pytest.raises(mpt.LampError) as e:
+        mpt.lamp_attn_fwd_q8(a["q"], a["k"], a["v"], 0x6000, 0x7000, 0x8000, 0x9000, a["o"],
+                             a["lse"], a["B"], a["H"], a["Hkv"], a["Lq"], a["Lk"], a["D"],
+                             a["causal"], a["window"], a["scale"], a["mask_bits"],
+                             a["group_tiles"], a["mode"], a["tau"], None, stream=0)
+    assert e.value.code == code
+
+
+def test_quant_and_mask_reject_bad_arguments_on_host():
+    with pytest.raises(mpt.LampError):
+        mpt.lamp_quant_qk(0x1000, None, 0x2000, None, None, None, 1, 1, 1, 64, 64, 64, 0, stream=0)
+    with pytest.raises(mpt.LampError):
+        mpt.lamp_quant_qk(0x1008, None, 0x2000, None, 0x3000, None, 1, 1, 1, 64, 64, 64, 0,
+                          stream=0)
+    with pytest.raises(mpt.LampError):
+        mpt.lamp_build_mask(None, 1, 1, 64, 64, 64, 1, 0.5, 1, stream=0)
+    with pytest.raises(mpt.LampError):
+        mpt.lamp_build_mask(0x1000, 1, 1, 64, 64, 64, 1, 1.5, 1, stream=0)
+    with pytest.raises(mpt.LampError):
+        mpt.lamp_selftest_timeout(0, stream=0)
+
+
+def test_workspace_size_and_alignment():
+    n = mpt.lamp_workspace_size(1, 32, 8, 4096, 4096, 128)
+    # q8 + k8 bytes plus the two scale arrays, each 256-byte aligned
+    assert n == 32 * 4096 * 128 + 8 * 4096 * 128 + 32 * 32 * 4 + 8 * 32 * 4
+    assert mpt.lamp_workspace_size(1, 1, 1, 1, 1, 96) == 0
+    with pytest.raises(mpt.LampError):
+        mpt.lamp_set_workspace(0x1010, 1024)
+    mpt.lamp_set_workspace(None, 0)

@@ -1,0 +1,193 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on seeded inputs.
+
+Small cases span several tiles and a ragged tail and are compared element by element; the
+full-size workloads are compared on seeded samples of query rows (bitmask routing: rows are
+independent) or whole query tiles (adaptive routing: a tile's decisions depend on all its
+rows), in the launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mixed_precision_tiled_b200 as mpt
+import oracle
+from workloads import CONFIGS, make_workload, sample_rows, sample_tiles
+
+from _parity import EXACT_MAX_ABS, mask_to_numpy, parity_case, to_dev
+
+pytestmark = pytest.mark.gpu
+
+TINY = CONFIGS["tiny"]
+GQA = CONFIGS["gqa4k"]
+
+
+def small(base, **kw):
+    return base.replace(**kw)
+
+
+# ----------------------------------------------------------------- quantiser / mask ----
+
+@pytest.mark.parametrize("D,L,dtype,fmt", [(64, 256, "fp16", "int8"), (128, 600, "bf16", "int8"),
+                                           (128, 600, "bf16", "e4m3"), (256, 200, "bf16", "int8"),
+                                           (256, 130, "fp16", "e4m3")])
+def test_quantiser_bit_exact(D, L, dtype, fmt):
+    bm, bn = mpt.lamp_tile_shape(D)
+    w = small(GQA, D=D, Lq=L, Lk=L, B=2, H=4, Hkv=2, bm=bm, bn=bn, dtype=dtype)
+    t = make_workload(w)
+    q, k = to_dev(t.q_bits, dtype), to_dev(t.k_bits, dtype)
+    q8, k8, qs, ks = mpt.quantize(q, k, fmt=fmt)
+    torch.cuda.synchronize()
+    rq, rqs = oracle.quantize(t.q, bm, fmt)
+    rk, rks = oracle.quantize(t.k, bn, fmt)
+    assert np.array_equal(q8.cpu().numpy(), rq) and np.array_equal(qs.cpu().numpy(), rqs)
+    assert np.array_equal(k8.cpu().numpy(), rk) and np.array_equal(ks.cpu().numpy(), rks)
+
+
+@pytest.mark.parametrize("name", ["gqa4k", "gemma_local16k", "long32k"])
+def test_quantiser_bit_exact_full_size(name):
+    w = CONFIGS[name]
+    t = make_workload(w)
+    q, k = to_dev(t.q_bits, w.dtype), to_dev(t.k_bits, w.dtype)
+    q8, k8, qs, ks = mpt.quantize(q, k, fmt=w.fmt)
+    torch.cuda.synchronize()
+    rq, rqs = oracle.quantize(t.q, w.bm, w.fmt)
+    rk, rks = oracle.quantize(t.k, w.bn, w.fmt)
+    assert np.array_equal(qs.cpu().numpy(), rqs) and np.array_equal(ks.cpu().numpy(), rks)
+    assert np.array_equal(q8.cpu().numpy(), rq) and np.array_equal(k8.cpu().numpy(), rk)
+
+
+def test_quantiser_e4m3_full_size_adaptive_workload():
+    w = CONFIGS["adaptive8k"]
+    t = make_workload(w)
+    q, k = to_dev(t.q_bits, w.dtype), to_dev(t.k_bits, w.dtype)
+    q8, k8, qs, ks = mpt.quantize(q, k, fmt="e4m3")
+    torch.cuda.synchronize()
+    rk, rks = oracle.quantize(t.k, w.bn, "e4m3")
+    assert np.array_equal(ks.cpu().numpy(), rks) and np.array_equal(k8.cpu().numpy(), rk)
+    rq, rqs = oracle.quantize(t.q, w.bm, "e4m3")
+    assert np.array_equal(qs.cpu().numpy(), rqs) and np.array_equal(q8.cpu().numpy(), rq)
+
+
+@pytest.mark.parametrize("B,H,L,D,g,p", [(1, 1, 256, 64, 1, 0.25), (2, 32, 4096, 128, 4, 0.2),
+                                         (1, 32, 131072, 128, 8, 0.1), (1, 8, 16384, 256, 2, 0.3),
+                                         (1, 2, 8193, 128, 1, 0.5)])
+def test_mask_builder_bit_exact(B, H, L, D, g, p):
+    bm, bn = mpt.lamp_tile_shape(D)
+    m = mpt.build_mask(B, H, L, L, D, g, p, 1234)
+    torch.cuda.synchronize()
+    nqt, nkt = -(-L // bm), -(-L // bn)
+    ref = oracle.build_mask(B, H, nqt, nkt, g, p, 1234)
+    assert np.array_equal(mask_to_numpy(m), ref)
+
+
+# ----------------------------------------------------------------- attention, small ----
+
+def test_tiny_workload():
+    parity_case(TINY)
+
+
+@pytest.mark.parametrize("p", [0.0, 0.3, 1.0])
+def test_d128_causal_gqa_ragged(p):
+    w = small(GQA, B=2, H=4, Hkv=2, Lq=600, Lk=600, group_tiles=2)
+    parity_case(w, p_fp16=p)
+
+
+def test_d128_noncausal_ragged_both():
+    w = small(GQA, B=1, H=2, Hkv=1, Lq=300, Lk=520, causal=False, group_tiles=1)
+    parity_case(w, p_fp16=0.4)
+
+
+@pytest.mark.parametrize("Lq,Lk", [(200, 700), (700, 200)])
+def test_d128_causal_bottom_right(Lq, Lk):
+    w = small(GQA, B=1, H=2, Hkv=2, Lq=Lq, Lk=Lk, group_tiles=1, plant_frac=0.0)
+    parity_case(w, p_fp16=0.5)
+
+
+@pytest.mark.parametrize("dtype,p", [("fp16", 0.5), ("bf16", 0.5), ("bf16", 0.0)])
+def test_d64_stacked_tiles(dtype, p):
+    w = small(TINY, B=1, H=2, Hkv=1, Lq=320, Lk=320, causal=True, dtype=dtype, values="structured",
+              plant_frac=0.02)
+    parity_case(w, p_fp16=p)
+
+
+@pytest.mark.parametrize("window", [0, 200])
+def test_d256_stacked_window(window):
+    w = small(CONFIGS["gemma_local16k"], B=1, H=4, Hkv=2, Lq=700, Lk=700, window=window)
+    parity_case(w)
+
+
+@pytest.mark.parametrize("fmt", ["int8", "e4m3"])
+def test_all_8bit_and_e4m3_bitmask(fmt):
+    w = small(GQA, B=1, H=2, Hkv=1, Lq=512, Lk=512)
+    parity_case(w, none8=True, fmt=fmt)
+    parity_case(w, p_fp16=0.3, fmt=fmt)
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_all_16bit_routing_is_exact_attention(dtype):
+    w = small(GQA, B=1, H=2, Hkv=1, Lq=384, Lk=384, dtype=dtype, values="iid", plant_frac=0.0)
+    g, r = parity_case(w, all16=True)
+    err = np.abs(g["o"] - r["o"]).max()
+    assert err <= EXACT_MAX_ABS, err
+
+
+def test_v_ones_gives_ones():
+    for w, kw in [(small(GQA, B=1, H=2, Hkv=1, Lq=400, Lk=400), dict(p_fp16=0.3)),
+                  (small(CONFIGS["adaptive8k"], B=1, H=2, Hkv=1, Lq=400, Lk=400), {}),
+                  (small(TINY, Lq=200, Lk=200, causal=True), dict(p_fp16=0.5))]:
+        g, _ = parity_case(w, v_ones=True, **kw)
+        assert np.abs(g["o"][np.isfinite(g["lse"])] - 1.0).max() < 1e-5
+
+
+def test_output_in_input_dtype():
+    w = small(GQA, B=1, H=2, Hkv=1, Lq=256, Lk=256)
+    g, r = parity_case(w, p_fp16=0.3, out="in")
+    assert np.abs(g["o"] - r["o"]).max() < 2e-2
+
+
+@pytest.mark.parametrize("fmt", ["int8", "e4m3"])
+@pytest.mark.parametrize("tau", [-1e30, 2.0, 4.0, 8.0])
+def test_adaptive_small(fmt, tau):
+    w = small(CONFIGS["adaptive8k"], B=1, H=4, Hkv=2, Lq=768, Lk=768)
+    g, r = parity_case(w, fmt=fmt, tau=tau)
+    live = g["route"] != 0
+    assert set(np.unique(g["route"][live]).tolist()) <= {1, 3}
+    if tau < 0:  # only tiles holding a row's first visible key can be flagged
+        assert np.all(g["route"][..., 0] == 3)
+        assert np.all(g["route"][..., 1:][live[..., 1:]] == 1)
+
+
+@pytest.mark.parametrize("base", ["tiny", "gemma_local16k"])
+def test_adaptive_stacked(base):
+    b = CONFIGS[base]
+    w = small(b, B=1, H=2, Hkv=1, Lq=330, Lk=330, causal=True, route="adaptive", tau=3.0,
+              values="structured", plant_frac=0.02, window=0)
+    parity_case(w, fmt="int8", tau=3.0)
+
+
+# ----------------------------------------------------------------- full size, sampled --
+
+@pytest.mark.parametrize("name", ["gqa4k", "gemma_local16k", "long32k"])
+def test_full_size_bitmask_sampled_rows(name):
+    w = CONFIGS[name]
+    rows = sample_rows(w, 64)
+    parity_case(w, rows=rows, check_codes=False)
+
+
+def test_full_size_adaptive_sampled_tiles():
+    w = CONFIGS["adaptive8k"]
+    tiles = sample_tiles(w, 1)
+    rows = (tiles[..., None] * w.bm + np.arange(w.bm)[None, None, None, :]).reshape(w.B, w.H, -1)
+    parity_case(w, rows=rows, check_codes=False)
+
+
+# ----------------------------------------------------------------- failure path -------
+
+def test_bounded_wait_reports_timeout():
+    mpt.lamp_selftest_timeout(1_000_000)  # 1 ms on a barrier nothing completes
+    with pytest.raises(mpt.LampError) as e:
+        mpt.lamp_check()
+    assert e.value.code == mpt.LAMP_ERR_TIMEOUT
+    mpt.lamp_check()  # the error word was cleared; the context is still usable
+    x = torch.ones(4, device="cuda")
+    assert float(x.sum()) == 4.0
