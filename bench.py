@@ -38,6 +38,7 @@ from workloads import CONFIGS, make_workload, sample_rows  # noqa: E402
 
 METRIC = "prefill attention TFLOP/s vs FP16-routed fraction; % of blended tensor roofline"
 KERNEL_SOURCES = ["mixed_precision_tiled_b200/csrc/attn_fwd.cuh",
+                  "mixed_precision_tiled_b200/csrc/attn_fwd_pp.cuh",
                   "mixed_precision_tiled_b200/csrc/ptx.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
 
@@ -125,29 +126,46 @@ class ClockSampler:
         self.uuid, self.proc = uuid, None
 
     def __enter__(self):
+        import threading
         cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                "-lms", "100"]
         if self.uuid:
             cmd += ["-i", self.uuid]
+        self.lines, self.t0 = [], None
+        first = threading.Event()
         try:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
                                          text=True)
         except OSError:
             self.proc = None
-        time.sleep(0.3)
+            return self
+
+        def reader():
+            for l in self.proc.stdout:
+                if l.strip():
+                    self.lines.append((time.monotonic(), l))
+                    first.set()
+            first.set()
+
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
+        first.wait(timeout=10.0)  # sampling is running before the timed region starts
+        self.t0 = time.monotonic()
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
+        t1 = time.monotonic()
         if self.proc:
-            time.sleep(0.25)
+            time.sleep(0.15)
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+            self.thread.join(timeout=5)
+        # keep the samples taken during the timed region (plus one either side)
+        inside = [l for (ts, l) in self.lines if self.t0 - 0.15 <= ts <= t1 + 0.15]
+        self.lines = inside or [l for (_, l) in self.lines]
 
     def summary(self):
         sm, mx, reasons = [], None, set()
@@ -453,7 +471,8 @@ def main():
                          "frac": round(achieved / peak_blend, 4), "traffic": traffic,
                          "peak_basis": f"blended: F8/P8 + F16/P16, P16 = {peaks['bf16']} TFLOP/s "
                                        f"bf16 burst ({peaks['source']}), P8 = 2 x P16 (nominal ratio)",
-                         "kernel": "attn_fwd_kernel", "attn_ms": round(att_ms, 4)},
+                         "kernel": "attn_fwd_pp_kernel" if w.D == 128 else "attn_fwd_kernel",
+                         "attn_ms": round(att_ms, 4)},
             "e2e": {"value": round(F * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 4)},

@@ -15,6 +15,7 @@
 
 #include "../../include/lamp.h"
 #include "attn_fwd.cuh"
+#include "attn_fwd_pp.cuh"
 #include "quant.cuh"
 
 namespace {
@@ -206,6 +207,29 @@ int launch_attn_cfg(const lamp::AttnParams& p, int grid, cudaStream_t st) {
   return LAMP_OK;
 }
 
+int launch_attn_pp(const lamp::AttnParams& p, int grid, cudaStream_t st) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    LAMP_CUDA(cudaFuncSetAttribute(lamp::attn_fwd_pp_kernel<true>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   lamp::PPCfg::SMEM_BYTES),
+              "cudaFuncSetAttribute");
+    LAMP_CUDA(cudaFuncSetAttribute(lamp::attn_fwd_pp_kernel<false>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   lamp::PPCfg::SMEM_BYTES),
+              "cudaFuncSetAttribute");
+    attr_set[dev] = true;
+  }
+  if (p.bf16)
+    lamp::attn_fwd_pp_kernel<true><<<grid, 384, lamp::PPCfg::SMEM_BYTES, st>>>(p);
+  else
+    lamp::attn_fwd_pp_kernel<false><<<grid, 384, lamp::PPCfg::SMEM_BYTES, st>>>(p);
+  LAMP_CUDA(cudaGetLastError(), "attn_fwd_pp_kernel launch");
+  return LAMP_OK;
+}
+
 using Cfg64 = lamp::AttnCfg<64, 64, true>;
 using Cfg128 = lamp::AttnCfg<128, 128, false>;
 using Cfg256 = lamp::AttnCfg<256, 128, true>;
@@ -276,6 +300,10 @@ int attn_q8(const void* q, const void* k, const void* v, const void* q8, const v
   if (route_out)
     LAMP_CUDA(cudaMemsetAsync(route_out, 0, static_cast<size_t>(BHq) * nqt * nkt, st), "memset route");
   if (D == 64) return launch_attn_cfg<Cfg64>(p, static_cast<int>(grid), st);
+  if (D == 128 && !p.e4m3) {
+    const long long pgrid = static_cast<long long>(BHq) * ((nqt + 1) / 2);
+    return launch_attn_pp(p, static_cast<int>(pgrid), st);
+  }
   if (D == 128) return launch_attn_cfg<Cfg128>(p, static_cast<int>(grid), st);
   return launch_attn_cfg<Cfg256>(p, static_cast<int>(grid), st);
 }
