@@ -36,7 +36,6 @@
 
 namespace lamp {
 
-__device__ uint32_t g_lamp_error;  // device-side error word, read and cleared by lamp_check
 
 // where-codes recorded with a timeout (bits 8..15 of the error word)
 enum : uint32_t {
@@ -204,7 +203,7 @@ __device__ __forceinline__ Plan make_plan(const AttnParams& p, const Geo& g, int
 
 template <class C>
 __device__ void producer_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars& bars,
-                              const WaitCtx& wc) {
+                              const WaitCtx wc) {
   uint8_t* sQ16 = smem + C::OFF_Q16;
   uint8_t* sQ8 = smem + C::OFF_Q8;
   uint8_t* slots = smem + C::OFF_SLOTS;
@@ -260,10 +259,7 @@ __device__ void producer_role(const AttnParams& p, const Geo& g, uint8_t* smem, 
     cur = nxt;
   }
   // Drain: every slot's most recent load must have landed before the CTA may exit.
-  WaitCtx drain = wc;
-  volatile uint32_t never = 0;
-  drain.abort = &never;
-  drain.limit_ns = 50000000ull;
+  const WaitCtx drain{0u, 50000u};  // no abort word: in-flight work always completes
   const uint32_t first = item > static_cast<uint32_t>(C::NS) ? item - C::NS : 0;
   for (uint32_t it = first; it < item; ++it)
     mbar_wait(&bars.full[it % C::NS], (it / C::NS) & 1u, drain, W_DRAIN);
@@ -274,7 +270,7 @@ __device__ void producer_role(const AttnParams& p, const Geo& g, uint8_t* smem, 
 
 template <class C>
 __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars& bars,
-                         uint32_t tbase, const WaitCtx& wc) {
+                         uint32_t tbase, const WaitCtx wc) {
   const uint32_t sQ16 = smem_u32(smem + C::OFF_Q16);
   const uint32_t sQ8 = smem_u32(smem + C::OFF_Q8);
   const uint32_t slots = smem_u32(smem + C::OFF_SLOTS);
@@ -383,10 +379,7 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
   }
   // Every MMA issued by this thread must complete before the TMEM is released.
   tc_commit(&bars.drain);
-  WaitCtx drain = wc;
-  volatile uint32_t never = 0;
-  drain.abort = &never;
-  drain.limit_ns = 50000000ull;
+  const WaitCtx drain{0u, 50000u};  // no abort word: in-flight work always completes
   mbar_wait(&bars.drain, 0, drain, W_DRAIN);
 }
 
@@ -394,7 +387,7 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
 
 // All 32 lanes poll the barrier; the result is made warp-uniform (and the warp reconverged)
 // before any warp-collective tcgen05 instruction follows.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtx& wc,
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtx wc,
                                           uint32_t where) {
   const bool ok = mbar_wait(bar, parity, wc, where);
   return __all_sync(0xFFFFFFFFu, ok);
@@ -402,7 +395,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
 
 template <class C>
 __device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint32_t tbase,
-                             const WaitCtx& wc) {
+                             const WaitCtx wc) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = warp * 32 + lane;
   const int i = g.q0 + r;
@@ -660,7 +653,7 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = bars.tmem_base;
-  WaitCtx wc{&bars.abort, &g_lamp_error, p.wait_ns};
+  const WaitCtx wc{smem_u32(&bars.abort), static_cast<uint32_t>(p.wait_ns / 1000)};
 
   if (warp == 4) {
     if ((threadIdx.x & 31) == 0 && g.n > 0) producer_role<C>(p, g, smem, bars, wc);
@@ -691,7 +684,7 @@ __global__ void selftest_timeout_kernel(uint64_t wait_ns) {
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    WaitCtx w{&abort_flag, &g_lamp_error, wait_ns};
+    const WaitCtx w{smem_u32(&abort_flag), static_cast<uint32_t>(wait_ns / 1000)};
     mbar_wait(&bar, 0, w, W_SELFTEST);
   }
   __syncthreads();

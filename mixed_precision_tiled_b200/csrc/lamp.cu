@@ -207,27 +207,29 @@ int launch_attn_cfg(const lamp::AttnParams& p, int grid, cudaStream_t st) {
   return LAMP_OK;
 }
 
-int launch_attn_pp(const lamp::AttnParams& p, int grid, cudaStream_t st) {
+template <bool BF16, bool ADAPTIVE>
+int launch_attn_pp_t(const lamp::AttnParams& p, int grid, cudaStream_t st) {
   static bool attr_set[64] = {};
   int dev = 0;
   LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    LAMP_CUDA(cudaFuncSetAttribute(lamp::attn_fwd_pp_kernel<true>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   lamp::PPCfg::SMEM_BYTES),
-              "cudaFuncSetAttribute");
-    LAMP_CUDA(cudaFuncSetAttribute(lamp::attn_fwd_pp_kernel<false>,
+    LAMP_CUDA(cudaFuncSetAttribute(lamp::attn_fwd_pp_kernel<BF16, ADAPTIVE>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    lamp::PPCfg::SMEM_BYTES),
               "cudaFuncSetAttribute");
     attr_set[dev] = true;
   }
-  if (p.bf16)
-    lamp::attn_fwd_pp_kernel<true><<<grid, 384, lamp::PPCfg::SMEM_BYTES, st>>>(p);
-  else
-    lamp::attn_fwd_pp_kernel<false><<<grid, 384, lamp::PPCfg::SMEM_BYTES, st>>>(p);
+  lamp::attn_fwd_pp_kernel<BF16, ADAPTIVE>
+      <<<grid, lamp::PPCfg::THREADS, lamp::PPCfg::SMEM_BYTES, st>>>(p);
   LAMP_CUDA(cudaGetLastError(), "attn_fwd_pp_kernel launch");
   return LAMP_OK;
+}
+
+int launch_attn_pp(const lamp::AttnParams& p, int grid, cudaStream_t st) {
+  if (p.bf16) return p.adaptive ? launch_attn_pp_t<true, true>(p, grid, st)
+                                : launch_attn_pp_t<true, false>(p, grid, st);
+  return p.adaptive ? launch_attn_pp_t<false, true>(p, grid, st)
+                    : launch_attn_pp_t<false, false>(p, grid, st);
 }
 
 using Cfg64 = lamp::AttnCfg<64, 64, true>;

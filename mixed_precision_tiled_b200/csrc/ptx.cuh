@@ -55,27 +55,53 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As above, but the thread may sleep (up to `hint_ns`) until the phase completes instead of
+// returning at once: waiting warps then take no issue slots from working ones.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ uint32_t g_lamp_error;  // device-side error word, read and cleared by lamp_check
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t saddr) {
+  uint32_t v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(saddr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void sts_u32(uint32_t saddr, uint32_t v) {
+  asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(saddr), "r"(v) : "memory");
+}
+
 // Shared abort word of a CTA: set by the first wait that times out, read by every other wait
-// so that all roles stop waiting once one has given up.
+// so that all roles stop waiting once one has given up.  Kept to two 32-bit values so that
+// waiting costs the softmax threads no registers.
 struct WaitCtx {
-  volatile uint32_t* abort;   // shared memory
-  uint32_t* dev_error;        // global error word (bit field of reasons)
-  uint64_t limit_ns;
+  uint32_t abort;     // shared-memory address of the abort word (0: no abort word)
+  uint32_t limit_us;  // time limit of one wait
 };
 
 // Wait for completion of the phase with the given parity.  Returns false when the time limit
 // passed or another role of the CTA gave up; the first timing-out thread records the failure.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w,
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx w,
                                           uint32_t where) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 63u) {
-      if (*w.abort) return false;
-      if (globaltimer_ns() - t0 > w.limit_ns) {
-        *w.abort = 1u;
-        atomicOr(w.dev_error, 1u | (where << 8));
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+    if ((it & 7u) == 7u) {
+      if (w.abort && lds_u32(w.abort)) return false;
+      if (globaltimer_ns() - t0 > static_cast<uint64_t>(w.limit_us) * 1000ull) {
+        if (w.abort) sts_u32(w.abort, 1u);
+        atomicOr(&g_lamp_error, 1u | (where << 8));
         return false;
       }
     }
