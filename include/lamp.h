@@ -116,6 +116,27 @@ int lamp_attn_fwd_q8(const void* q, const void* k, const void* v, const void* q8
                      int window, float scale, const uint64_t* mask_bits, int group_tiles,
                      int mode, float tau, uint8_t* route_out, void* stream);
 
+/* Same operation and arguments as lamp_attn_fwd, for callers that cannot allocate device
+ * memory: code whose device memory is all owned by another allocator (a framework's caching
+ * allocator that has already reserved it), or latency-bound serving loops that must not call
+ * cudaMalloc / cudaFree, which may synchronise the whole device and take unbounded time.
+ * This entry point allocates nothing.  (The pages have no counterpart to it.)
+ *   - Scratch for the 8-bit Q, K and their block scales lives in one file-scope device array
+ *     of LAMP_NOALLOC_MAX_BYTES, which every GPU that loads this library holds until the
+ *     process exits.  Problems needing more (lamp_workspace_size(...) > the maximum) are
+ *     rejected with LAMP_ERR_INVALID before anything is launched.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents; every byte a call
+ *     reads is written earlier in the same call, so nothing needs clearing.  Calls whose work
+ *     overlaps on the GPU (different streams, no ordering between them) race on the array.
+ *   - The caller still passes (and owns) q, k, v, o, lse and mask_bits. */
+#define LAMP_NOALLOC_MAX_BYTES (32u << 20)
+int lamp_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int H, int Hkv, int Lq, int Lk, int D, int causal, int window,
+                          float scale, const uint64_t* mask_bits, int group_tiles, int mode,
+                          float tau, void* stream);
+
 /* Bytes of workspace lamp_attn_fwd needs for these sizes (q8, k8 and the scales, each
  * 256-byte aligned).  0 on invalid arguments. */
 size_t lamp_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int D, int mode);

@@ -29,8 +29,9 @@ IN_FP16, IN_BF16 = 0x0, 0x4
 OUT_F32, OUT_INDTYPE = 0x0, 0x8
 
 EXPORTS = ("lamp_tile_shape", "lamp_mask_words", "lamp_quant_qk", "lamp_build_mask",
-           "lamp_attn_fwd", "lamp_attn_fwd_q8", "lamp_workspace_size", "lamp_set_workspace",
-           "lamp_check", "lamp_selftest_timeout", "lamp_last_error")
+           "lamp_attn_fwd", "lamp_attn_fwd_q8", "lamp_attn_fwd_noalloc", "lamp_workspace_size",
+           "lamp_set_workspace", "lamp_check", "lamp_selftest_timeout", "lamp_last_error")
+NOALLOC_MAX_BYTES = 32 << 20  # LAMP_NOALLOC_MAX_BYTES
 
 
 class LampError(RuntimeError):
@@ -59,6 +60,7 @@ def lib():
                 "lamp_build_mask": (_i, [_vp] + [_i] * 6 + [_f, _u64, _vp]),
                 "lamp_attn_fwd": (_i, [_vp] * 5 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp]),
                 "lamp_attn_fwd_q8": (_i, [_vp] * 9 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp, _vp]),
+                "lamp_attn_fwd_noalloc": (_i, [_vp] * 5 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp]),
                 "lamp_workspace_size": (_sz, [_i] * 7),
                 "lamp_set_workspace": (_i, [_vp, _sz]),
                 "lamp_check": (_i, [_vp]),
@@ -131,6 +133,15 @@ def lamp_attn_fwd(q, k, v, o, lse, B, H, Hkv, Lq, Lk, D, causal, window, scale, 
     _check(lib().lamp_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Lq, Lk,
                                D, int(causal), int(window), float(scale), _ptr(mask_bits),
                                int(group_tiles), int(mode), float(tau), _stream(stream)))
+
+
+def lamp_attn_fwd_noalloc(q, k, v, o, lse, B, H, Hkv, Lq, Lk, D, causal, window, scale,
+                          mask_bits, group_tiles, mode, tau, stream=None):
+    """lamp_attn_fwd without any device allocation (scratch in a fixed device array)."""
+    _check(lib().lamp_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv,
+                                       Lq, Lk, D, int(causal), int(window), float(scale),
+                                       _ptr(mask_bits), int(group_tiles), int(mode), float(tau),
+                                       _stream(stream)))
 
 
 def lamp_attn_fwd_q8(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D, causal,

@@ -18,6 +18,11 @@
 #include "attn_fwd_pp.cuh"
 #include "quant.cuh"
 
+// Scratch of lamp_attn_fwd_noalloc: a file-scope device array that every GPU loading this
+// library holds until the process exits.  In host code the symbol is only a stand-in; its
+// device address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[LAMP_NOALLOC_MAX_BYTES];
+
 namespace {
 
 thread_local char g_err[512] = "";
@@ -411,6 +416,57 @@ int lamp_attn_fwd(const void* q, const void* k, const void* v, void* o, float* l
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return fail(LAMP_ERR_INVALID, "q, k, v and o must be 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((r = quant_qk(q, k, q8, k8, qs, ks, B, H, Hkv, Lq, Lk, D, mode, st))) return r;
+  return attn_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D, causal, window, scale,
+                 mask_bits, group_tiles, mode, tau, nullptr, st);
+}
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_base[64] = {};
+
+// Device address of the scratch array on the current device (looked up once per device).
+int noalloc_base(void** out) {
+  int dev = 0;
+  LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(LAMP_ERR_INVALID, "device index out of range");
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_base[dev]) {
+    void* p = nullptr;
+    LAMP_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
+    if (!p) return fail(LAMP_ERR_CUDA, "scratch array has no device address");
+    g_noalloc_base[dev] = p;
+  }
+  *out = g_noalloc_base[dev];
+  return LAMP_OK;
+}
+}  // namespace
+
+int lamp_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int H, int Hkv, int Lq, int Lk, int D, int causal, int window,
+                          float scale, const uint64_t* mask_bits, int group_tiles, int mode,
+                          float tau, void* stream) {
+  int r = check_sizes(B, H, Hkv, Lq, Lk, D);
+  if (r) return r;
+  if (!q || !k || !v || !o) return fail(LAMP_ERR_INVALID, "null operand pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(LAMP_ERR_INVALID, "q, k, v and o must be 16-byte aligned");
+  const WsLayout w = ws_layout(B, H, Hkv, Lq, Lk, D);
+  if (w.total > static_cast<size_t>(LAMP_NOALLOC_MAX_BYTES))
+    return fail(LAMP_ERR_INVALID,
+                "problem needs %zu bytes of scratch; lamp_attn_fwd_noalloc holds at most %zu "
+                "(use lamp_attn_fwd with a workspace)",
+                w.total, static_cast<size_t>(LAMP_NOALLOC_MAX_BYTES));
+  void* ws = nullptr;
+  if ((r = noalloc_base(&ws))) return r;
+  auto* base = static_cast<uint8_t*>(ws);
+  uint8_t* q8 = base + w.q8;
+  uint8_t* k8 = base + w.k8;
+  float* qs = reinterpret_cast<float*>(base + w.qs);
+  float* ks = reinterpret_cast<float*>(base + w.ks);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Every byte of the scratch that the attention reads is written first by the quantiser of
+  // the same call, so nothing needs clearing between calls.
   if ((r = quant_qk(q, k, q8, k8, qs, ks, B, H, Hkv, Lq, Lk, D, mode, st))) return r;
   return attn_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D, causal, window, scale,
                  mask_bits, group_tiles, mode, tau, nullptr, st);
