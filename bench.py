@@ -186,6 +186,40 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def reduce_max(values, device, dist_mod=None):
+    """Element-wise max of per-rank timings (the slowest rank sets the job's time)."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist_mod is not None and dist_mod.is_available() and dist_mod.is_initialized() \
+            and dist_mod.get_world_size() > 1:
+        dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def quantiser_bandwidth(mpt, torch, dev, stream, peaks, n=20):
+    """Quantiser alone on a 16-bit tensor larger than L2 (32 x 32768 x 128 bf16 = 268 MB):
+    algorithmic bytes = 2 read + 1 written per element + 4 per block scale."""
+    B, H, L, D = 1, 32, 32768, 128
+    x = torch.randn((B, H, L, D), device=dev, dtype=torch.bfloat16)
+    codes = torch.empty(x.shape, device=dev, dtype=torch.uint8)
+    scales = torch.empty((B, H, L // 128), device=dev, dtype=torch.float32)
+    mode = mpt.mode_bits(fmt="int8", dtype="bf16")
+    for _ in range(3):
+        mpt.lamp_quant_qk(x, None, codes, None, scales, None, B, H, H, L, L, D, mode, stream)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n)]
+    for i in range(n):
+        ev[2 * i].record(stream)
+        mpt.lamp_quant_qk(x, None, codes, None, scales, None, B, H, H, L, L, D, mode, stream)
+        ev[2 * i + 1].record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.fmean(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(n))
+    nbytes = x.numel() * 3 + scales.numel() * 4
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"kernel": "quant_kernel", "tensor": "bf16 [1,32,32768,128] (268 MB > L2), INT8, 128-row blocks",
+            "algorithmic_bytes": nbytes, "ms": round(ms, 4), "achieved_gbs": round(gbs, 1),
+            "peak_gbs": peaks["hbm_gbs"], "frac": round(gbs / peaks["hbm_gbs"], 4)}
+
+
 def cpu_baseline(w, mask_np, t, seconds_target=10.0):
     """The oracle as it stands on a bounded row sample of the workload (host cores)."""
     import oracle
@@ -372,12 +406,7 @@ def main():
         if world > 1:
             dist.barrier()
     mpt.lamp_check(stream)
-    tot_ms = float(sum(step_ms))
-    att_ms = float(statistics.fmean(attn_ms))
-    if world > 1:
-        tt = torch.tensor([tot_ms, att_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        tot_ms, att_ms = float(tt[0]), float(tt[1])
+    tot_ms, att_ms = reduce_max([sum(step_ms), statistics.fmean(attn_ms)], dev, dist)
     ms_per_step = tot_ms / args.steps
     value = world * F / (ms_per_step * 1e-3) / 1e12
 
@@ -413,11 +442,7 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / n_e2e
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt[0])
+    e2e_ms, = reduce_max([e0.elapsed_time(e1) / n_e2e], dev, dist)
     mpt.lamp_check(stream)
     h2d = (q.numel() + k.numel() + v.numel()) * q.element_size()
     d2h = o.numel() * 4 + lse.numel() * 4
@@ -443,6 +468,8 @@ def main():
                                 "roofline_frac": round((f8 / P8 + f16 / P16) / (a * 1e-3), 3)}
         step()  # restore the configured mask
         torch.cuda.synchronize()
+
+    quant = quantiser_bandwidth(mpt, torch, dev, stream, peaks) if not args.no_sweep else None
 
     T_roof = F8 / P8 + F16 / P16
     achieved = F / (att_ms * 1e-3) / 1e12
@@ -481,6 +508,8 @@ def main():
         }
         if sweep:
             line["sweep_fp16_fraction"] = sweep
+        if quant:
+            line["quantiser"] = quant
         if world == 1 and not args.no_cpu_baseline:
             import oracle  # noqa: F401  (CPU baseline leg only)
             mask_np = mask.cpu().numpy().view(np.uint64) if bitmask else None
