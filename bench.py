@@ -34,7 +34,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import CONFIGS, make_workload, sample_rows  # noqa: E402
+from workloads import CONFIGS, make_workload, sample_rows, sample_tiles  # noqa: E402
 
 METRIC = "prefill attention TFLOP/s vs FP16-routed fraction; % of blended tensor roofline"
 KERNEL_SOURCES = ["mixed_precision_tiled_b200/csrc/attn_fwd.cuh",
@@ -220,38 +220,70 @@ def quantiser_bandwidth(mpt, torch, dev, stream, peaks, n=20):
             "peak_gbs": peaks["hbm_gbs"], "frac": round(gbs / peaks["hbm_gbs"], 4)}
 
 
-def cpu_baseline(w, mask_np, t, seconds_target=10.0):
-    """The oracle as it stands on a bounded row sample of the workload (host cores)."""
+def oracle_rows(w, n_per_head, seed):
+    """Seeded query rows per (batch, head) for an oracle sample.  In adaptive mode a row's routing
+    depends on every row of its query tile, so the sample is made of whole query tiles."""
+    if w.route != "adaptive":
+        return sample_rows(w, n_per_head, seed=seed)
+    tiles = sample_tiles(w, max(1, n_per_head // w.bm), seed=seed)
+    rows = (tiles[..., None] * w.bm + np.arange(w.bm)).reshape(w.B, w.H, -1)
+    return np.unique(np.minimum(rows, w.Lq - 1), axis=-1) if w.Lq % w.bm else rows
+
+
+def row_flops(w, rows):
+    """4 * D * (visible keys) summed over the sampled rows."""
+    off = w.Lk - w.Lq
+    i = rows.reshape(-1).astype(np.int64)
+    if not w.causal:
+        return int(4 * w.D * w.Lk * i.size)
+    hi = np.minimum(i + off, w.Lk - 1)
+    lo = np.maximum(0, i + off - w.window + 1) if w.window > 0 else np.zeros_like(i)
+    return int(4 * w.D * np.maximum(0, hi - lo + 1).sum())
+
+
+def cpu_baseline(w, mask_np, t, seconds_target=15.0):
+    """The oracle as it stands on a bounded sample of the workload's query rows (host cores).
+
+    The sample grows from 4 rows per (batch, head) until one oracle call takes about
+    `seconds_target` or covers every row; the last call is the one reported."""
     import oracle
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
-    pairs_row = lambda rows: sum(
-        max(0, min(i + w.Lk - w.Lq, w.Lk - 1) - (max(0, i + w.Lk - w.Lq - w.window + 1)
-                                                 if w.window > 0 else 0) + 1)
-        if w.causal else w.Lk for i in rows.reshape(-1).tolist())
     kw = dict(bm=w.bm, bn=w.bn, causal=w.causal, window=w.window, mask=mask_np,
               group_tiles=w.group_tiles, route=w.route, fmt=w.fmt, tau=w.tau, threads=cores)
-    probe = sample_rows(w, 4, seed=w.seed + 99)
-    t0 = time.perf_counter()
-    oracle.attention(t.q, t.k, t.v, rows=probe, **kw)
-    dt = time.perf_counter() - t0
-    rate = pairs_row(probe) / max(dt, 1e-6)  # pairs per second
-    per_head_rows = max(4, min(w.Lq, int(4 * seconds_target / max(dt, 1e-6))))
-    if w.route == "adaptive":  # whole query tiles (decisions depend on every row of a tile)
-        per_head_rows = max(w.bm, (per_head_rows // w.bm) * w.bm)
-    rows = sample_rows(w, per_head_rows, seed=w.seed + 98)
-    t0 = time.perf_counter()
-    oracle.attention(t.q, t.k, t.v, rows=rows, **kw)
-    dt = time.perf_counter() - t0
-    flops = 4 * w.D * pairs_row(rows)
+    n = 4 if w.route != "adaptive" else w.bm
+    while True:
+        rows = oracle_rows(w, n, seed=w.seed + 98)
+        t0 = time.perf_counter()
+        oracle.attention(t.q, t.k, t.v, rows=rows, **kw)
+        dt = time.perf_counter() - t0
+        if dt >= 0.5 * seconds_target or rows.shape[-1] >= w.Lq:
+            break
+        n = min(w.Lq, max(2 * n, int(n * seconds_target / max(dt, 1e-3))))
+    flops = row_flops(w, rows)
+    whole = rows.shape[-1] >= w.Lq
+    what = (f"the whole workload {w.name}" if whole else
+            f"{rows.shape[-1]} seeded query rows per (batch, head) of {w.name}")
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"{per_head_rows} seeded query rows per (batch, head) of {w.name} "
-                      f"({rows.size} rows, {flops / 1e9:.1f} GFLOP, {dt:.1f} s)",
-            "seconds": dt, "probe_rate_pairs_per_s": rate}
+            "sample": f"{what} ({rows.size} rows, {flops / 1e9:.1f} GFLOP, {dt:.1f} s)",
+            "seconds": dt}
 
 
 # ------------------------------------------------------------------ reference arm -------
 
-def run_reference(args):
+def head_problem(w, t, mask, b, h):
+    """The single-(batch, head) problem of query head h of batch b: the same data, B=H=Hkv=1."""
+    kv = h // (w.H // w.Hkv)
+    sub = w.replace(B=1, H=1, Hkv=1)
+    m = mask[b:b + 1, h:h + 1] if mask is not None else None
+    return sub, t.q[b:b + 1, h:h + 1], t.k[b:b + 1, kv:kv + 1], t.v[b:b + 1, kv:kv + 1], m
+
+
+def run_reference(args, budget_s=150.0):
+    """The oracle as it stands, timed on the host cores, on the CUDA arm's workload and metric.
+
+    Each step runs the oracle on one seeded (batch, head) and a seeded sample of its query rows
+    (whole query tiles in adaptive mode); the sample size is set during warm-up so that the whole
+    run takes about `budget_s` seconds."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
@@ -265,31 +297,30 @@ def run_reference(args):
     mask = (oracle.build_mask(w.B, w.H, w.nqt, w.nkt, w.group_tiles, w.p_fp16, w.mask_seed)
             if w.route == "bitmask" else None)
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
-    kw = dict(bm=w.bm, bn=w.bn, causal=w.causal, window=w.window, mask=mask,
-              group_tiles=w.group_tiles, route=w.route, fmt=w.fmt, tau=w.tau, threads=cores)
-    # Each step: the oracle on a fresh seeded sample of query rows (1 per head; whole query tiles
-    # in adaptive mode), so that warm-up + steps stay within a few minutes.
-    per = w.bm if w.route == "adaptive" else 1
-    flops_total, secs = 0, 0.0
+    per_step = max(0.01, budget_s / max(1, args.steps + args.warmup))
+    n_min = w.bm if w.route == "adaptive" else 1
+    n = n_min
+    rng = np.random.Generator(np.random.PCG64(w.seed + 1000))
+    flops_total, secs, rows_total = 0, 0.0, 0
     for s in range(args.warmup + args.steps):
-        rows = sample_rows(w, per, seed=w.seed + 1000 + s)
-        if w.route == "adaptive":
-            qt = rows[..., :1] // w.bm
-            rows = qt * w.bm + np.arange(w.bm)[None, None, :]
-            rows = np.minimum(rows, w.Lq - 1)
+        b, h = int(rng.integers(w.B)), int(rng.integers(w.H))
+        sub, q, k, v, m = head_problem(w, t, mask, b, h)
+        rows = oracle_rows(sub, n, seed=w.seed + 1000 + s)
+        kw = dict(bm=w.bm, bn=w.bn, causal=w.causal, window=w.window, mask=m,
+                  group_tiles=w.group_tiles, route=w.route, fmt=w.fmt, tau=w.tau, threads=cores)
         t0 = time.perf_counter()
-        oracle.attention(t.q, t.k, t.v, rows=rows, **kw)
+        oracle.attention(q, k, v, rows=rows, **kw)
         dt = time.perf_counter() - t0
-        if s >= args.warmup:
-            secs += dt
-            off = w.Lk - w.Lq
-            for i in rows.reshape(-1).tolist():
-                hi = min(i + off, w.Lk - 1) if w.causal else w.Lk - 1
-                lo = (max(0, i + off - w.window + 1) if w.window > 0 else 0) if w.causal else 0
-                flops_total += 4 * w.D * max(0, hi - lo + 1)
+        if s < args.warmup:  # size the per-step sample from the warm-up calls
+            n = int(min(w.Lq, max(n_min, n * per_step / max(dt, 1e-4))))
+            continue
+        secs += dt
+        rows_total += rows.size
+        flops_total += row_flops(sub, rows)
     value = flops_total / secs / 1e12 if secs > 0 else 0.0
-    sample = (f"{per} seeded query row(s) per (batch, head) per step of {w.name}; "
-              f"{args.steps} timed steps, {secs:.2f} s")
+    sample = (f"per step one seeded (batch, head) of {w.name} and {n} seeded query rows of it"
+              f"{' (whole query tiles)' if w.route == 'adaptive' else ''}; {args.steps} timed "
+              f"steps, {rows_total} rows, {flops_total / 1e9:.2f} GFLOP, {secs:.2f} s")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": secs / max(args.steps, 1) * 1e3, "higher_is_better": True,
