@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -160,23 +161,58 @@ int get_workspace(size_t need, void** out) {
 
 // ---------------------------------------------------------------- launches ------------
 
-int launch_quant(const void* x, void* codes, float* scales, int outer, int L, int D, int blk,
-                 bool bf16, bool e4m3, cudaStream_t st) {
-  const int nb = (L + blk - 1) / blk;
-  const long long grid = static_cast<long long>(outer) * nb;
-  if (grid > 0x7FFFFFFF) return fail(LAMP_ERR_INVALID, "too many quantisation blocks");
-  auto* xs = static_cast<const uint16_t*>(x);
-  auto* cs = static_cast<uint8_t*>(codes);
-  dim3 g(static_cast<unsigned>(grid)), b(lamp::QUANT_THREADS);
-  if (bf16 && e4m3)
-    lamp::quant_kernel<true, true><<<g, b, 0, st>>>(xs, cs, scales, L, D, blk, nb);
-  else if (bf16)
-    lamp::quant_kernel<true, false><<<g, b, 0, st>>>(xs, cs, scales, L, D, blk, nb);
-  else if (e4m3)
-    lamp::quant_kernel<false, true><<<g, b, 0, st>>>(xs, cs, scales, L, D, blk, nb);
-  else
-    lamp::quant_kernel<false, false><<<g, b, 0, st>>>(xs, cs, scales, L, D, blk, nb);
+constexpr uint32_t kWaitUs = 2000000u;  // 2 s per wait: far beyond any legitimate stall
+
+int sm_count(int* n) {
+  static int cached[64] = {};
+  int dev = 0;
+  LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(LAMP_ERR_CUDA, "device index out of range");
+  if (!cached[dev])
+    LAMP_CUDA(cudaDeviceGetAttribute(&cached[dev], cudaDevAttrMultiProcessorCount, dev),
+              "cudaDeviceGetAttribute(multiProcessorCount)");
+  *n = cached[dev];
+  return LAMP_OK;
+}
+
+template <bool BF16, bool E4M3, int VEC>
+int launch_quant_v(const lamp::QuantJob& j0, const lamp::QuantJob& j1, int D, cudaStream_t st) {
+  using P = lamp::QuantPipe<VEC>;
+  static bool attr_set[64] = {};
+  int dev = 0, nsm = 0;
+  LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (int r = sm_count(&nsm)) return r;
+  if (!attr_set[dev]) {
+    LAMP_CUDA(cudaFuncSetAttribute(lamp::quant_kernel<BF16, E4M3, VEC>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM_BYTES),
+              "cudaFuncSetAttribute");
+    attr_set[dev] = true;
+  }
+  const int total = j0.blocks + j1.blocks;
+  const int grid = std::min(total, nsm * P::CTAS_PER_SM);
+  lamp::quant_kernel<BF16, E4M3, VEC>
+      <<<grid, lamp::QUANT_THREADS, P::SMEM_BYTES, st>>>(j0, j1, D, kWaitUs);
   LAMP_CUDA(cudaGetLastError(), "quant_kernel launch");
+  return LAMP_OK;
+}
+
+template <bool BF16, bool E4M3>
+int launch_quant_t(const lamp::QuantJob& j0, const lamp::QuantJob& j1, int D, int vec,
+                   cudaStream_t st) {
+  if (vec <= 1) return launch_quant_v<BF16, E4M3, 1>(j0, j1, D, st);
+  if (vec <= 4) return launch_quant_v<BF16, E4M3, 4>(j0, j1, D, st);
+  return launch_quant_v<BF16, E4M3, 8>(j0, j1, D, st);
+}
+
+// Job for `outer` runs of L rows in blocks of blk rows; an empty job when x is NULL.
+int quant_job(const void* x, void* codes, float* scales, int outer, int L, int blk,
+              lamp::QuantJob* j) {
+  *j = lamp::QuantJob{static_cast<const uint16_t*>(x), static_cast<uint8_t*>(codes), scales, L,
+                      blk, (L + blk - 1) / blk, 0};
+  if (!x) return LAMP_OK;
+  const long long blocks = static_cast<long long>(outer) * j->nb;
+  if (blocks > 0x3FFFFFFF) return fail(LAMP_ERR_INVALID, "too many quantisation blocks");
+  j->blocks = static_cast<int>(blocks);
   return LAMP_OK;
 }
 
@@ -185,15 +221,17 @@ int quant_qk(const void* q, const void* k, void* q8, void* k8, float* q_scale, f
   int bm, bn;
   tile_shape(D, &bm, &bn);
   const bool bf16 = (mode & LAMP_IN_BF16) != 0, e4m3 = (mode & LAMP_FMT_E4M3) != 0;
-  if (q) {
-    int r = launch_quant(q, q8, q_scale, B * H, Lq, D, bm, bf16, e4m3, st);
-    if (r) return r;
-  }
-  if (k) {
-    int r = launch_quant(k, k8, k_scale, B * Hkv, Lk, D, bn, bf16, e4m3, st);
-    if (r) return r;
-  }
-  return LAMP_OK;
+  lamp::QuantJob jq, jk;
+  if (int r = quant_job(q, q8, q_scale, B * H, Lq, bm, &jq)) return r;
+  if (int r = quant_job(k, k8, k_scale, B * Hkv, Lk, bn, &jk)) return r;
+  if (jq.blocks + jk.blocks == 0) return LAMP_OK;
+  // 16-byte vectors per thread for the larger block
+  const int vec = (std::max(q ? bm : 0, k ? bn : 0) * D / 8 + lamp::QUANT_THREADS - 1) /
+                  lamp::QUANT_THREADS;
+  if (bf16 && e4m3) return launch_quant_t<true, true>(jq, jk, D, vec, st);
+  if (bf16) return launch_quant_t<true, false>(jq, jk, D, vec, st);
+  if (e4m3) return launch_quant_t<false, true>(jq, jk, D, vec, st);
+  return launch_quant_t<false, false>(jq, jk, D, vec, st);
 }
 
 template <class C>
@@ -301,7 +339,7 @@ int attn_q8(const void* q, const void* k, const void* v, const void* q8, const v
   p.e4m3 = (mode & LAMP_FMT_E4M3) ? 1 : 0;
   p.bf16 = (mode & LAMP_IN_BF16) ? 1 : 0;
   p.out_f32 = (mode & LAMP_OUT_INDTYPE) ? 0 : 1;
-  p.wait_ns = 2000000000ull;  // 2 s per wait: far beyond any legitimate stall
+  p.wait_ns = kWaitUs * 1000ull;
   const long long grid = static_cast<long long>(BHq) * p.n_ct;
   if (grid > 0x7FFFFFFF) return fail(LAMP_ERR_INVALID, "grid too large");
   if (route_out)

@@ -11,7 +11,7 @@ import torch
 
 import mixed_precision_tiled_b200 as mpt
 import oracle
-from workloads import CONFIGS, make_workload, sample_rows, sample_tiles
+from workloads import CONFIGS, make_workload, sample_rows, sample_tiles, to_16bit
 
 from _parity import EXACT_MAX_ABS, mask_to_numpy, parity_case, to_dev
 
@@ -66,6 +66,63 @@ def test_quantiser_e4m3_full_size_adaptive_workload():
     assert np.array_equal(ks.cpu().numpy(), rks) and np.array_equal(k8.cpu().numpy(), rk)
     rq, rqs = oracle.quantize(t.q, w.bm, "e4m3")
     assert np.array_equal(qs.cpu().numpy(), rqs) and np.array_equal(q8.cpu().numpy(), rq)
+
+
+def _edge_blocks(fmt, dtype, D=128, L=600, seed=5):
+    """Blocks of 128 rows that stress the quantiser's rounding: exact ties of the 8-bit format
+    (absmax chosen so that the scale is 1), an all-zero block, a block of subnormal values (a
+    subnormal scale), a normal random block and a ragged last block."""
+    rng = np.random.default_rng(seed)
+    top = 127.0 if fmt == "int8" else 448.0
+    x = np.zeros((1, 1, L, D), np.float32)
+    if fmt == "int8":
+        ties = rng.integers(-127, 127, size=(128, D)) + 0.5   # half-integers: round to even
+    else:
+        grid = np.array([1.0625, 17.0, 1.5 * 2.0 ** -9, 0.3125 * 2 ** -4, 208.0, 3.75])
+        ties = rng.choice(grid, size=(128, D)) * rng.choice([-1.0, 1.0], size=(128, D))
+    ties[0, 0] = top                                          # absmax -> scale exactly 1
+    x[0, 0, 0:128] = ties
+    # rows 128..255 stay zero
+    x[0, 0, 256:384] = rng.standard_normal((128, D)) * 2.0 ** -130   # subnormal in fp32 / bf16
+    x[0, 0, 384:512] = rng.standard_normal((128, D)) * np.exp(rng.standard_normal((128, D)))
+    x[0, 0, 512:] = rng.standard_normal((L - 512, D)) * 3.0
+    if dtype == "fp16":
+        x[0, 0, 256:384] = rng.standard_normal((128, D)) * 2.0 ** -20  # fp16 subnormals
+    bits, vals = to_16bit(x, dtype)
+    return bits, vals
+
+
+@pytest.mark.parametrize("fmt", ["int8", "e4m3"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_quantiser_rounding_edge_blocks(fmt, dtype):
+    bits, vals = _edge_blocks(fmt, dtype)
+    q = to_dev(bits, dtype)
+    q8, k8, qs, ks = mpt.quantize(q, q, fmt=fmt)
+    torch.cuda.synchronize()
+    rq, rqs = oracle.quantize(vals, 128, fmt)
+    assert np.array_equal(qs.cpu().numpy(), rqs) and np.array_equal(ks.cpu().numpy(), rqs)
+    assert np.array_equal(q8.cpu().numpy(), rq) and np.array_equal(k8.cpu().numpy(), rq)
+    assert rqs[0, 0, 1] == 0 and 0 < rqs[0, 0, 2] < 2.0 ** -126 or dtype == "fp16"
+
+
+def test_quantiser_q_only_and_k_only_calls():
+    w = small(GQA, D=128, Lq=300, Lk=520, B=1, H=4, Hkv=2)
+    t = make_workload(w)
+    q, k = to_dev(t.q_bits, w.dtype), to_dev(t.k_bits, w.dtype)
+    q8 = torch.zeros(q.shape, device="cuda", dtype=torch.uint8)
+    k8 = torch.zeros(k.shape, device="cuda", dtype=torch.uint8)
+    qs = torch.zeros((1, 4, 3), device="cuda", dtype=torch.float32)
+    ks = torch.zeros((1, 2, 5), device="cuda", dtype=torch.float32)
+    mode = mpt.mode_bits(fmt="int8", dtype=w.dtype)
+    mpt.lamp_quant_qk(q, None, q8, None, qs, None, 1, 4, 2, 300, 520, 128, mode)
+    torch.cuda.synchronize()
+    assert int(k8.count_nonzero()) == 0 and int(ks.count_nonzero()) == 0
+    mpt.lamp_quant_qk(None, k, None, k8, None, ks, 1, 4, 2, 300, 520, 128, mode)
+    torch.cuda.synchronize()
+    rq, rqs = oracle.quantize(t.q, 128, "int8")
+    rk, rks = oracle.quantize(t.k, 128, "int8")
+    assert np.array_equal(q8.cpu().numpy(), rq) and np.array_equal(qs.cpu().numpy(), rqs)
+    assert np.array_equal(k8.cpu().numpy(), rk) and np.array_equal(ks.cpu().numpy(), rks)
 
 
 @pytest.mark.parametrize("B,H,L,D,g,p", [(1, 1, 256, 64, 1, 0.25), (2, 32, 4096, 128, 4, 0.2),
