@@ -221,6 +221,27 @@ def quantiser_bandwidth(mpt, torch, dev, stream, peaks, n=20):
             "peak_gbs": peaks["hbm_gbs"], "frac": round(gbs / peaks["hbm_gbs"], 4)}
 
 
+def tensor_probe(mpt, torch, stream, iters=4096):
+    """Measured rate of the tcgen05 MMA shapes the attention kernel issues (one CTA per SM,
+    back-to-back MMAs of M = 128 into one TMEM accumulator), in TFLOP/s (TOP/s for INT8)."""
+    shapes = {"bf16_ss": (0, 16), "i8_ss": (1, 32), "bf16_ts": (2, 16)}
+    nsm = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    out = {}
+    for name, (kind, K) in shapes.items():
+        for n in (64, 128, 256):
+            mpt.lamp_mma_probe(kind, n, 64, stream)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            mpt.lamp_mma_probe(kind, n, iters, stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            ops = 2 * 128 * n * K * 8 * iters * nsm
+            out[f"{name}_n{n}"] = round(ops / (ms * 1e-3) / 1e12, 1)
+    mpt.lamp_check(stream)
+    return out
+
+
 def attn_kernel_name(w):
     """The attention kernel the library dispatches for this workload."""
     return "attn_fwd_pp_kernel" if (w.D == 128 and w.fmt == "int8") else "attn_fwd_kernel"
@@ -513,6 +534,7 @@ def main():
         torch.cuda.synchronize()
 
     quant = quantiser_bandwidth(mpt, torch, dev, stream, peaks) if not args.no_sweep else None
+    probe = tensor_probe(mpt, torch, stream) if not args.no_sweep else None
 
     T_roof = F8 / P8 + F16 / P16
     achieved = F / (att_ms * 1e-3) / 1e12
@@ -553,6 +575,8 @@ def main():
             line["sweep_fp16_fraction"] = sweep
         if quant:
             line["quantiser"] = quant
+        if probe:
+            line["tensor_probe_tflops"] = probe
         if world == 1 and not args.no_cpu_baseline:
             import oracle  # noqa: F401  (CPU baseline leg only)
             mask_np = mask.cpu().numpy().view(np.uint64) if bitmask else None

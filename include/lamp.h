@@ -156,6 +156,16 @@ int lamp_check(void* stream);
  * without faulting or hanging the GPU.  A later lamp_check() returns LAMP_ERR_TIMEOUT. */
 int lamp_selftest_timeout(uint64_t wait_ns, void* stream);
 
+/* Tensor-core throughput probe (measurement only; the pages have no counterpart): launches one
+ * CTA per SM on `stream`; the CTA's elected thread issues iters x 8 back-to-back tcgen05 MMAs of
+ * M = 128, N = n into one TMEM accumulator, with descriptors built once, and waits for them.
+ * kind: 0 = kind::f16 bf16 with A and B in shared memory (K = 16 per MMA), 1 = kind::i8 with A
+ * and B in shared memory (K = 32), 2 = kind::f16 bf16 with A in tensor memory and B in shared
+ * memory (K = 16).  Operands are zero.  Work = 2 * 128 * n * K * 8 * iters operations per SM;
+ * the caller times the launch (CUDA events on `stream`).  n: 64, 128 or 256; iters in
+ * [1, 2^20].  Returns LAMP_OK or LAMP_ERR_INVALID / LAMP_ERR_CUDA. */
+int lamp_mma_probe(int kind, int n, int iters, void* stream);
+
 /* Thread-local description of the last error returned by a lamp_* call on this thread. */
 const char* lamp_last_error(void);
 

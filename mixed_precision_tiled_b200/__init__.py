@@ -30,7 +30,8 @@ OUT_F32, OUT_INDTYPE = 0x0, 0x8
 
 EXPORTS = ("lamp_tile_shape", "lamp_mask_words", "lamp_quant_qk", "lamp_build_mask",
            "lamp_attn_fwd", "lamp_attn_fwd_q8", "lamp_attn_fwd_noalloc", "lamp_workspace_size",
-           "lamp_set_workspace", "lamp_check", "lamp_selftest_timeout", "lamp_last_error")
+           "lamp_set_workspace", "lamp_check", "lamp_selftest_timeout", "lamp_mma_probe",
+           "lamp_last_error")
 NOALLOC_MAX_BYTES = 32 << 20  # LAMP_NOALLOC_MAX_BYTES
 
 
@@ -65,6 +66,7 @@ def lib():
                 "lamp_set_workspace": (_i, [_vp, _sz]),
                 "lamp_check": (_i, [_vp]),
                 "lamp_selftest_timeout": (_i, [_u64, _vp]),
+                "lamp_mma_probe": (_i, [_i, _i, _i, _vp]),
                 "lamp_last_error": (ctypes.c_char_p, []),
             }
             for name, (res, args) in sig.items():
@@ -164,6 +166,10 @@ def lamp_set_workspace(ptr, nbytes: int):
 
 def lamp_check(stream=None):
     _check(lib().lamp_check(_stream(stream)))
+
+
+def lamp_mma_probe(kind: int, n: int, iters: int, stream=None):
+    _check(lib().lamp_mma_probe(int(kind), int(n), int(iters), _stream(stream)))
 
 
 def lamp_selftest_timeout(wait_ns: int, stream=None):

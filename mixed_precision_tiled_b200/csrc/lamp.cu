@@ -17,6 +17,7 @@
 #include "../../include/lamp.h"
 #include "attn_fwd.cuh"
 #include "attn_fwd_pp.cuh"
+#include "mma_probe.cuh"
 #include "quant.cuh"
 
 // Scratch of lamp_attn_fwd_noalloc: a file-scope device array that every GPU loading this
@@ -355,6 +356,32 @@ int attn_q8(const void* q, const void* k, const void* v, const void* q8, const v
 
 }  // namespace
 
+namespace {
+template <int KIND, int N>
+int probe_launch(int nsm, int iters, cudaStream_t st) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(LAMP_ERR_UNSUPPORTED, "device index %d", dev);
+  if (!attr_set[dev]) {
+    LAMP_CUDA(cudaFuncSetAttribute(lamp::mma_probe_kernel<KIND, N>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, lamp::PROBE_SMEM),
+              "cudaFuncSetAttribute");
+    attr_set[dev] = true;
+  }
+  lamp::mma_probe_kernel<KIND, N><<<nsm, lamp::PROBE_THREADS, lamp::PROBE_SMEM, st>>>(iters, kWaitUs);
+  LAMP_CUDA(cudaGetLastError(), "mma_probe_kernel launch");
+  return LAMP_OK;
+}
+
+template <int KIND>
+int probe_n(int n, int nsm, int iters, cudaStream_t st) {
+  if (n == 64) return probe_launch<KIND, 64>(nsm, iters, st);
+  if (n == 128) return probe_launch<KIND, 128>(nsm, iters, st);
+  return probe_launch<KIND, 256>(nsm, iters, st);
+}
+}  // namespace
+
 extern "C" {
 
 int lamp_tile_shape(int D, int* bm, int* bn) {
@@ -528,6 +555,19 @@ int lamp_selftest_timeout(uint64_t wait_ns, void* stream) {
   lamp::selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(wait_ns);
   LAMP_CUDA(cudaGetLastError(), "selftest launch");
   return LAMP_OK;
+}
+
+int lamp_mma_probe(int kind, int n, int iters, void* stream) {
+  if (kind < lamp::PROBE_F16_SS || kind > lamp::PROBE_F16_TS)
+    return fail(LAMP_ERR_INVALID, "probe kind must be 0, 1 or 2");
+  if (n != 64 && n != 128 && n != 256) return fail(LAMP_ERR_INVALID, "probe N must be 64, 128 or 256");
+  if (iters < 1 || iters > (1 << 20)) return fail(LAMP_ERR_INVALID, "probe iters out of range");
+  int nsm = 0;
+  if (int r = sm_count(&nsm)) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (kind == lamp::PROBE_F16_SS) return probe_n<lamp::PROBE_F16_SS>(n, nsm, iters, st);
+  if (kind == lamp::PROBE_I8_SS) return probe_n<lamp::PROBE_I8_SS>(n, nsm, iters, st);
+  return probe_n<lamp::PROBE_F16_TS>(n, nsm, iters, st);
 }
 
 const char* lamp_last_error(void) { return g_err; }

@@ -114,3 +114,12 @@ def test_workspace_size_and_alignment():
     with pytest.raises(mpt.LampError):
         mpt.lamp_set_workspace(0x1010, 1024)
     mpt.lamp_set_workspace(None, 0)
+
+
+@pytest.mark.parametrize("kind,n,iters", [(3, 128, 8), (-1, 128, 8), (0, 120, 8), (0, 272, 8),
+                                          (1, 0, 8), (1, 192, 8), (2, 128, 0),
+                                          (2, 128, (1 << 20) + 1)])
+def test_mma_probe_rejects_bad_shapes_on_host(kind, n, iters):
+    with pytest.raises(mpt.LampError) as e:
+        mpt.lamp_mma_probe(kind, n, iters, stream=0)
+    assert e.value.code == mpt.LAMP_ERR_INVALID

@@ -248,3 +248,11 @@ def test_bounded_wait_reports_timeout():
     mpt.lamp_check()  # the error word was cleared; the context is still usable
     x = torch.ones(4, device="cuda")
     assert float(x.sum()) == 4.0
+
+
+def test_mma_probe_runs():
+    for kind in (0, 1, 2):
+        for n in (64, 128, 256):
+            mpt.lamp_mma_probe(kind, n, 8)
+    torch.cuda.synchronize()
+    mpt.lamp_check()
