@@ -150,18 +150,46 @@ __device__ __forceinline__ bool tile_b16(const AttnParams& p, const MaskRow& m, 
   return ((w >> (gi & 63)) & 1ull) == 0;
 }
 
-// Routing of key tile kt for both query tiles.
+// Key-tile cursor of the producer and MMA warps: the tile's group index advances with the
+// tile, so that no integer division sits on the issue path.
+struct KtCursor {
+  int kt, gi, rem;
+};
+
+__device__ __forceinline__ KtCursor kt_first(const AttnParams& p, int kt0) {
+  KtCursor c;
+  c.kt = kt0;
+  c.gi = kt0 / p.group_tiles;
+  c.rem = kt0 - c.gi * p.group_tiles;
+  return c;
+}
+
+__device__ __forceinline__ void kt_next(const AttnParams& p, KtCursor& c) {
+  ++c.kt;
+  if (++c.rem == p.group_tiles) {
+    c.rem = 0;
+    ++c.gi;
+  }
+}
+
+__device__ __forceinline__ bool group_b16(const AttnParams& p, const MaskRow& m, int gi) {
+  if (p.adaptive) return false;
+  const uint64_t w = (gi >> 6) ? m.w1 : m.w0;
+  return ((w >> (gi & 63)) & 1ull) == 0;
+}
+
+// Routing of key tile c.kt for both query tiles.
 struct PPPlan {
   bool live0, live1, b16_0, b16_1, need8, need16;
 };
 
 __device__ __forceinline__ PPPlan pp_plan(const AttnParams& p, const PPGeo& g, const MaskRow& m0,
-                                          const MaskRow& m1, int kt) {
+                                          const MaskRow& m1, const KtCursor& c) {
   PPPlan pl;
-  pl.live0 = tile_live(g, p, 0, kt);
-  pl.live1 = tile_live(g, p, 1, kt);
-  pl.b16_0 = pl.live0 && tile_b16(p, m0, kt);
-  pl.b16_1 = pl.live1 && tile_b16(p, m1, kt);
+  pl.live0 = tile_live(g, p, 0, c.kt);
+  pl.live1 = tile_live(g, p, 1, c.kt);
+  pl.b16_0 = pl.live0 && group_b16(p, m0, c.gi);
+  pl.b16_1 = pl.live1 && group_b16(p, m1, c.gi);
   if (p.adaptive) {
     pl.need8 = pl.need16 = pl.live0 || pl.live1;
   } else {
@@ -217,12 +245,12 @@ __device__ void pp_producer(const AttnParams& p, const PPGeo& g, uint8_t* smem, 
   };
   // Per key tile, in the MMA warp's order of first use within each ring: K8, K16, V.
   bool ok = true;
-  for (int t = 0; ok && t < g.n; ++t) {
-    const int kt = g.kt_lo + t;
-    const PPPlan pl = pp_plan(p, g, m0, m1, kt);
-    if (pl.need8 && !(ok = load8(kt))) break;
-    if (pl.need16 && !(ok = load16(&p.tm_k16, kt))) break;
-    if (!(ok = load16(&p.tm_v, kt))) break;
+  KtCursor cur = kt_first(p, g.kt_lo);
+  for (int t = 0; ok && t < g.n; ++t, kt_next(p, cur)) {
+    const PPPlan pl = pp_plan(p, g, m0, m1, cur);
+    if (pl.need8 && !(ok = load8(cur.kt))) break;
+    if (pl.need16 && !(ok = load16(&p.tm_k16, cur.kt))) break;
+    if (!(ok = load16(&p.tm_v, cur.kt))) break;
   }
   // Drain: every slot's most recent load must have landed before the CTA may exit.
   const WaitCtx drain{0u, 50000u};  // no abort word: in-flight work always completes
@@ -235,15 +263,26 @@ __device__ void pp_producer(const AttnParams& p, const PPGeo& g, uint8_t* smem, 
 
 // ------------------------------------------------------------------ MMA issuer --------
 
+// Run by the whole MMA warp: every lane takes the same waits and computes the same (uniform)
+// descriptors; the elected lane issues the MMAs and commits.  Shared-memory descriptors are
+// built once per operand region and advanced by constant offsets (16-byte units) per K step.
 __device__ void pp_mma(const AttnParams& p, const PPGeo& g, uint8_t* smem, PPBars& bars,
                        uint32_t tbase, const WaitCtx wc) {
   using C = PPCfg;
+  const bool leader = elect_one();
   const uint32_t sbase = smem_u32(smem);
   const MaskRow m0 = load_mask_row(p, g, 0), m1 = load_mask_row(p, g, 1);
   const uint32_t f16 = p.bf16 ? 1u : 0u;
   const uint32_t id_s16 = idesc(1, f16, f16, 0, 0, C::BN, 128);
   const uint32_t id_s8 = idesc(2, 1, 1, 0, 0, C::BN, 128);  // INT8 only
   const uint32_t id_pv = idesc(1, f16, f16, 0, 1, C::D, 128);
+  // K-major operands: 128-byte rows, 8-row groups 1024 bytes apart; one K step = 32 bytes.
+  const uint64_t d_q16 = sdesc(sbase + C::OFF_Q16, 16, 1024, SWZ_128B);
+  const uint64_t d_q8 = sdesc(sbase + C::OFF_Q8, 16, 1024, SWZ_128B);
+  const uint64_t d_k8 = sdesc(sbase + C::OFF_R8, 16, 1024, SWZ_128B);
+  const uint64_t d_k16 = sdesc(sbase + C::OFF_R16, 16, 1024, SWZ_128B);
+  // V (MN-major): 64-column atoms BN * 128 bytes apart; one K step = 16 keys = 2048 bytes.
+  const uint64_t d_v = sdesc(sbase + C::OFF_R16, C::BN * 128, 1024, SWZ_128B);
 
   uint32_t n8 = 0, n16 = 0;
   uint32_t cv0 = 0, cv1 = 0, cp0 = 0, cp1 = 0;
@@ -277,52 +316,61 @@ __device__ void pp_mma(const AttnParams& p, const PPGeo& g, uint8_t* smem, PPBar
   auto issue_s = [&](int x, bool sixteen, int slot) {
     const uint32_t dS = tbase + static_cast<uint32_t>(x * C::BN);
     if (sixteen) {
-      const uint32_t ks = sbase + C::OFF_R16 + slot * C::KV_BYTES;
-      const uint32_t qa = sbase + C::OFF_Q16 + x * C::Q16_BYTES;
       if (!lamp_chk(slot >= 0 && slot < C::NS16, 5)) return;
+      const uint64_t qa = d_q16 + static_cast<uint64_t>(x * (C::Q16_BYTES >> 4));
+      const uint64_t kb = d_k16 + static_cast<uint64_t>(slot * (C::KV_BYTES >> 4));
+      if (leader) {
 #pragma unroll
-      for (int s = 0; s < C::D / 16; ++s) {
-        const int c = s >> 2, off = (s & 3) * 32;
-        mma_f16_ss(dS, sdesc(qa + c * C::MT * 128 + off, 16, 1024, SWZ_128B),
-                   sdesc(ks + c * C::BN * 128 + off, 16, 1024, SWZ_128B), id_s16, s > 0 ? 1u : 0u);
+        for (int s = 0; s < C::D / 16; ++s) {
+          const uint64_t off = static_cast<uint64_t>((s >> 2) * ((C::MT * 128) >> 4) + (s & 3) * 2);
+          mma_f16_ss(dS, qa + off, kb + off, id_s16, s > 0 ? 1u : 0u);
+        }
       }
     } else {
-      const uint32_t ks = sbase + C::OFF_R8 + slot * C::K8_BYTES;
-      const uint32_t qa = sbase + C::OFF_Q8 + x * C::Q8_BYTES;
       if (!lamp_chk(slot >= 0 && slot < C::NS8, 5)) return;
+      const uint64_t qa = d_q8 + static_cast<uint64_t>(x * (C::Q8_BYTES >> 4));
+      const uint64_t kb = d_k8 + static_cast<uint64_t>(slot * (C::K8_BYTES >> 4));
+      if (leader) {
 #pragma unroll
-      for (int s = 0; s < C::D / 32; ++s)
-        mma_i8_ss(dS, sdesc(qa + s * 32, 16, 1024, SWZ_128B), sdesc(ks + s * 32, 16, 1024, SWZ_128B),
-                  id_s8, s > 0 ? 1u : 0u);
+        for (int s = 0; s < C::D / 32; ++s)
+          mma_i8_ss(dS, qa + static_cast<uint64_t>(s * 2), kb + static_cast<uint64_t>(s * 2), id_s8,
+                    s > 0 ? 1u : 0u);
+      }
     }
+  };
+  auto commit = [&](uint64_t* bar) {
+    if (leader) tc_commit(bar);
   };
   auto first_s = [&](int x, bool b16, const Items& it) {
     const bool sixteen = !p.adaptive && b16;
     issue_s(x, sixteen, sixteen ? it.k16 : it.k8);
-    tc_commit(&bars.s_full[x]);
+    commit(&bars.s_full[x]);
   };
   auto pv = [&](int x, int vslot, bool acc) {
-    const uint32_t vs = sbase + C::OFF_R16 + vslot * C::KV_BYTES;
+    const uint64_t vb = d_v + static_cast<uint64_t>(vslot * (C::KV_BYTES >> 4));
     const uint32_t pt = tbase + static_cast<uint32_t>(x * C::BN);
     const uint32_t ot = tbase + static_cast<uint32_t>(2 * C::BN + x * C::D);
     // P (16-bit pairs) sits in columns 0-63 of S_X
+    if (leader) {
 #pragma unroll
-    for (int s = 0; s < C::BN / 16; ++s) {
-      const uint64_t b = sdesc(vs + s * 16 * 128, C::BN * 128, 1024, SWZ_128B);
-      mma_f16_ts(ot, pt + s * 8, b, id_pv, (acc || s > 0) ? 1u : 0u);
+      for (int s = 0; s < C::BN / 16; ++s)
+        mma_f16_ts(ot, pt + s * 8, vb + static_cast<uint64_t>(s * ((16 * 128) >> 4)), id_pv,
+                   (acc || s > 0) ? 1u : 0u);
     }
   };
 
   Items cur{-1, -1, -1}, nxt{-1, -1, -1};
-  PPPlan pl = pp_plan(p, g, m0, m1, g.kt_lo);
+  KtCursor kc = kt_first(p, g.kt_lo);
+  PPPlan pl = pp_plan(p, g, m0, m1, kc);
   if (ok && g.n > 0 && (ok = take_k(pl, cur))) {
     if (pl.live0) first_s(0, pl.b16_0, cur);
     if (pl.live1) first_s(1, pl.b16_1, cur);
   }
   for (int t = 0; ok && t < g.n; ++t) {
-    const int kt = g.kt_lo + t;
     const bool has_next = t + 1 < g.n;
-    const PPPlan pn = has_next ? pp_plan(p, g, m0, m1, kt + 1) : PPPlan{};
+    KtCursor kn = kc;
+    kt_next(p, kn);
+    const PPPlan pn = has_next ? pp_plan(p, g, m0, m1, kn) : PPPlan{};
     if (p.adaptive) {
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
@@ -337,14 +385,14 @@ __device__ void pp_mma(const AttnParams& p, const PPGeo& g, uint8_t* smem, PPBar
         for (int w = 0; w < 4; ++w) any |= vv[w];
         if (any) {
           issue_s(x, true, cur.k16);
-          tc_commit(&bars.s16_full[x]);
+          commit(&bars.s16_full[x]);
         }
       }
       if (!ok) break;
     }
     // every QK^T MMA of this key tile has been issued: release its K slots when they finish
-    if (cur.k8 >= 0) tc_commit(&bars.empty8[cur.k8]);
-    if (cur.k16 >= 0) tc_commit(&bars.empty16[cur.k16]);
+    if (cur.k8 >= 0) commit(&bars.empty8[cur.k8]);
+    if (cur.k16 >= 0) commit(&bars.empty16[cur.k16]);
     if (!(ok = take16(cur.v))) break;
     bool taken_next = false;
 #pragma unroll
@@ -368,13 +416,14 @@ __device__ void pp_mma(const AttnParams& p, const PPGeo& g, uint8_t* smem, PPBar
       }
     }
     if (!ok) break;
-    tc_commit(&bars.empty16[cur.v]);
+    commit(&bars.empty16[cur.v]);
     cur = nxt;
     pl = pn;
+    kc = kn;
   }
-  tc_commit(&bars.o_done[0]);
-  tc_commit(&bars.o_done[1]);
-  tc_commit(&bars.drain);
+  commit(&bars.o_done[0]);
+  commit(&bars.o_done[1]);
+  commit(&bars.drain);
   const WaitCtx drain{0u, 50000u};  // no abort word: in-flight work always completes
   mbar_wait(&bars.drain, 0, drain, W_DRAIN);
 }
@@ -725,7 +774,7 @@ __global__ void __launch_bounds__(PPCfg::THREADS, 1)
     if (warp == 8) {
       if ((threadIdx.x & 31) == 0 && g.n > 0) pp_producer(p, g, smem, bars, wc);
     } else if (warp == 9) {
-      if ((threadIdx.x & 31) == 0 && g.n > 0) pp_mma(p, g, smem, bars, tbase, wc);
+      if (g.n > 0) pp_mma(p, g, smem, bars, tbase, wc);
     }
   }
   tc_fence_before();

@@ -227,6 +227,19 @@ __device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a, uint64_t 
       : "memory");
 }
 
+// One lane of a converged warp (the same lane for every lane): the warp runs the MMA issue
+// loop together, so that descriptors and slot indices stay warp-uniform, and the elected lane
+// issues the single-thread tcgen05 instructions.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // Arrive (once) on `bar` when every tcgen05 async operation issued so far by this thread
 // has completed.
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
