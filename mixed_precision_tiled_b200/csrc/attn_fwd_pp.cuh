@@ -142,14 +142,6 @@ __device__ __forceinline__ bool tile_live(const PPGeo& g, const AttnParams& p, i
   return lo <= hi && lo <= c1 && hi >= c0;
 }
 
-// bitmask routing: true = the tile of this query tile at key tile kt is 16-bit
-__device__ __forceinline__ bool tile_b16(const AttnParams& p, const MaskRow& m, int kt) {
-  if (p.adaptive) return false;
-  const int gi = kt / p.group_tiles;
-  const uint64_t w = (gi >> 6) ? m.w1 : m.w0;
-  return ((w >> (gi & 63)) & 1ull) == 0;
-}
-
 // Key-tile cursor of the producer and MMA warps: the tile's group index advances with the
 // tile, so that no integer division sits on the issue path.
 struct KtCursor {
@@ -172,6 +164,7 @@ __device__ __forceinline__ void kt_next(const AttnParams& p, KtCursor& c) {
   }
 }
 
+// bitmask routing: true = tiles of routing group gi of this query tile are 16-bit
 __device__ __forceinline__ bool group_b16(const AttnParams& p, const MaskRow& m, int gi) {
   if (p.adaptive) return false;
   const uint64_t w = (gi >> 6) ? m.w1 : m.w0;
@@ -454,6 +447,23 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return r;
 }
 
+
+// acc + the low / high 16-bit half of a packed pair (bf16 or fp16), one rounding: sums the
+// rounded P values as the P.V MMA sees them, without unpacking them.
+template <bool BF16>
+__device__ __forceinline__ float add_lo16(float acc, uint32_t pk) {
+  float r;
+  if (BF16) asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.bf16 %0, lo, %2;\n\t}" : "=f"(r) : "r"(pk), "f"(acc));
+  else asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.f16 %0, lo, %2;\n\t}" : "=f"(r) : "r"(pk), "f"(acc));
+  return r;
+}
+template <bool BF16>
+__device__ __forceinline__ float add_hi16(float acc, uint32_t pk) {
+  float r;
+  if (BF16) asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.bf16 %0, hi, %2;\n\t}" : "=f"(r) : "r"(pk), "f"(acc));
+  else asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.f16 %0, hi, %2;\n\t}" : "=f"(r) : "r"(pk), "f"(acc));
+  return r;
+}
 // A thread owns row r of query tile X.  Per key tile: read the row of S from TMEM, turn it
 // into fp32 values of the raw product (exact int32 -> fp32 for 8-bit tiles), mask, take the
 // row max, vote (look-ahead rule), exponentiate against the lazy reference max, pack P as
@@ -499,18 +509,10 @@ __device__ void pp_softmax(const AttnParams& p, const PPGeo& g, uint8_t* smem, P
       tmem_ld32(lane_base + s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&raw[c * 32]));
     tmem_wait_ld();
   };
-  // int32 accumulators -> exact fp32 (|acc| < 2^22): (acc + 1.5*2^23 as bits) - 1.5*2^23
+  // int32 accumulators -> fp32, exact (|acc| < 2^22)
   auto int_to_float = [&]() {
 #pragma unroll
-    for (int c = 0; c < N; c += 2) {
-      const uint64_t v = f2_add(f2_pack(__uint_as_float(raw[c] + 0x4B400000u),
-                                        __uint_as_float(raw[c + 1] + 0x4B400000u)),
-                                f2_pack(-12582912.0f, -12582912.0f));
-      float a, b;
-      f2_unpack(v, a, b);
-      raw[c] = __float_as_uint(a);
-      raw[c + 1] = __float_as_uint(b);
-    }
+    for (int c = 0; c < N; ++c) raw[c] = __float_as_uint(static_cast<float>(static_cast<int>(raw[c])));
   };
   // keep columns [a, b] of the tile (the row's visible keys), -inf elsewhere; branch-free
   auto apply_mask = [&](int j0) {
@@ -531,18 +533,22 @@ __device__ void pp_softmax(const AttnParams& p, const PPGeo& g, uint8_t* smem, P
     return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
   };
 
-  // next live tile and its K scale, fetched one tile ahead (off the critical path)
-  int t_next = 0;
-  while (t_next < g.n && !tile_live(g, p, x, g.kt_lo + t_next)) ++t_next;
-  float ks_n = (t_next < g.n) ? __ldg(ks_row + g.kt_lo + t_next) : 0.0f;
+  // The live key tiles of query tile X form one range [kt_first, kt_last] (causal and window
+  // limits are monotone in the row); the K scale of the next tile is fetched one tile ahead
+  // and the tile's routing group advances with it.
+  const int lo_x = x ? g.lo[1] : g.lo[0], hi_x = x ? g.hi[1] : g.hi[0];
+  const int kt_first = (lo_x <= hi_x) ? lo_x / N : 1, kt_last = (lo_x <= hi_x) ? hi_x / N : 0;
+  float ks_n = (kt_first <= kt_last) ? __ldg(ks_row + kt_first) : 0.0f;
+  int gi = kt_first / p.group_tiles, grem = kt_first - gi * p.group_tiles;
 
-  while (ok && t_next < g.n) {
-    const int t = t_next;
-    const int kt = g.kt_lo + t;
+  for (int kt = kt_first; ok && kt <= kt_last; ++kt) {
     const float ks = ks_n;
-    ++t_next;
-    while (t_next < g.n && !tile_live(g, p, x, g.kt_lo + t_next)) ++t_next;
-    if (t_next < g.n) ks_n = __ldg(ks_row + g.kt_lo + t_next);
+    if (kt < kt_last) ks_n = __ldg(ks_row + kt + 1);
+    const int gcur = gi;
+    if (++grem == p.group_tiles) {
+      grem = 0;
+      ++gi;
+    }
 
     if (!(ok = warp_wait(&bars.s_full[x], cs & 1u, wc, W_SFULL))) break;
     ++cs;
@@ -550,7 +556,7 @@ __device__ void pp_softmax(const AttnParams& p, const PPGeo& g, uint8_t* smem, P
     load_s();
     const int j0 = kt * N;
     const bool full = row_valid && j0 >= lo_r && j0 + N - 1 <= hi_r;
-    bool sixteen = !ADAPTIVE && tile_b16(p, mrow, kt);
+    bool sixteen = !ADAPTIVE && group_b16(p, mrow, gcur);
     // (a zero block scale would turn masked -inf entries into NaN: keep it positive; the
     // scores of an all-zero block are 0 either way)
     float cscale = sixteen ? p.scale_log2 : fmaxf(sq_scale * ks, 1e-30f);
@@ -623,42 +629,40 @@ __device__ void pp_softmax(const AttnParams& p, const PPGeo& g, uint8_t* smem, P
     const float mu = (m_ref == NEG_INF) ? 0.0f : m_ref;
     const uint64_t c2 = f2_pack(cscale, cscale);
     const uint64_t nb2 = f2_pack(-mu, -mu);
-    uint64_t se0 = 0, se1 = 0, sr0 = 0, sr1 = 0;
+    uint64_t se0 = 0, se1 = 0;
+    float sr0 = 0.f, sr1 = 0.f, sr2 = 0.f, sr3 = 0.f;
 #pragma unroll
     for (int c = 0; c < N; c += 2) {
       float x0, x1;
       f2_unpack(f2_fma(f2_pack(__uint_as_float(raw[c]), __uint_as_float(raw[c + 1])), c2, nb2),
                 x0, x1);
-      const float p0 = ex2(x0), p1 = ex2(x1);
+      float p0, p1;
+      p0 = ex2(x0); p1 = ex2(x1);
       uint32_t pk;
-      float r0, r1;
       if (BF16) {
         __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
         pk = *reinterpret_cast<uint32_t*>(&h2);
-        r0 = __uint_as_float(pk << 16);
-        r1 = __uint_as_float(pk & 0xFFFF0000u);
       } else {
         __half2 h2 = __floats2half2_rn(p0, p1);
         pk = *reinterpret_cast<uint32_t*>(&h2);
-        r0 = __low2float(h2);
-        r1 = __high2float(h2);
       }
       if (c & 2) {
         se1 = f2_add(se1, f2_pack(p0, p1));
-        sr1 = f2_add(sr1, f2_pack(r0, r1));
+        sr2 = add_lo16<BF16>(sr2, pk);
+        sr3 = add_hi16<BF16>(sr3, pk);
       } else {
         se0 = f2_add(se0, f2_pack(p0, p1));
-        sr0 = f2_add(sr0, f2_pack(r0, r1));
+        sr0 = add_lo16<BF16>(sr0, pk);
+        sr1 = add_hi16<BF16>(sr1, pk);
       }
       raw[c >> 1] = pk;
       if ((c & 31) == 30) tmem_st16(lane_base + s_col + (c >> 5) * 16, &raw[(c >> 5) * 16]);
     }
     {
-      float a0, a1, b0, b1;
+      float a0, a1;
       f2_unpack(f2_add(se0, se1), a0, a1);
-      f2_unpack(f2_add(sr0, sr1), b0, b1);
       l_ex += a0 + a1;
-      l_rd += b0 + b1;
+      l_rd += (sr0 + sr1) + (sr2 + sr3);
     }
     tmem_wait_st();
     tc_fence_before();
