@@ -67,12 +67,14 @@ struct PPBars {
   uint64_t s_full[2];
   uint64_t s16_full[2];
   uint64_t vote[2];
-  uint64_t p_full[2];
+  uint64_t p_half[2];  // P of keys 0-63 of query tile X is in TMEM
+  uint64_t p_full[2];  // all of P of query tile X is in TMEM
   uint64_t o_done[2];
   uint64_t drain;
   uint32_t tmem_base;
   uint32_t abort;
   uint32_t votes[2][4];
+  uint64_t mask[2][2];  // routing mask words of query tiles 0 and 1 (all ones: no mask)
 };
 static_assert(sizeof(PPBars) <= 512, "barrier block");
 
@@ -170,19 +172,26 @@ __device__ __forceinline__ bool group_b16(const AttnParams& p, const MaskRow& m,
   const uint64_t w = (gi >> 6) ? m.w1 : m.w0;
   return ((w >> (gi & 63)) & 1ull) == 0;
 }
+// As above, with the mask row of query tile x read from shared memory (it costs the issuing
+// warps no registers).
+__device__ __forceinline__ bool group_b16(const AttnParams& p, const PPBars& bars, int x, int gi) {
+  if (p.adaptive) return false;
+  const uint64_t w = bars.mask[x][(gi >> 6) & 1];
+  return ((w >> (gi & 63)) & 1ull) == 0;
+}
 
 // Routing of key tile c.kt for both query tiles.
 struct PPPlan {
   bool live0, live1, b16_0, b16_1, need8, need16;
 };
 
-__device__ __forceinline__ PPPlan pp_plan(const AttnParams& p, const PPGeo& g, const MaskRow& m0,
-                                          const MaskRow& m1, const KtCursor& c) {
+__device__ __forceinline__ PPPlan pp_plan(const AttnParams& p, const PPGeo& g, const PPBars& bars,
+                                          const KtCursor& c) {
   PPPlan pl;
   pl.live0 = tile_live(g, p, 0, c.kt);
   pl.live1 = tile_live(g, p, 1, c.kt);
-  pl.b16_0 = pl.live0 && group_b16(p, m0, c.gi);
-  pl.b16_1 = pl.live1 && group_b16(p, m1, c.gi);
+  pl.b16_0 = pl.live0 && group_b16(p, bars, 0, c.gi);
+  pl.b16_1 = pl.live1 && group_b16(p, bars, 1, c.gi);
   if (p.adaptive) {
     pl.need8 = pl.need16 = pl.live0 || pl.live1;
   } else {
@@ -199,7 +208,6 @@ __device__ void pp_producer(const AttnParams& p, const PPGeo& g, uint8_t* smem, 
   using C = PPCfg;
   const int bh_q = g.b * p.H + g.h;
   const int bh_kv = g.b * p.Hkv + g.kvh;
-  const MaskRow m0 = load_mask_row(p, g, 0), m1 = load_mask_row(p, g, 1);
   prefetch_tmap(&p.tm_q16);
   prefetch_tmap(&p.tm_k16);
   prefetch_tmap(&p.tm_v);
@@ -240,7 +248,7 @@ __device__ void pp_producer(const AttnParams& p, const PPGeo& g, uint8_t* smem, 
   bool ok = true;
   KtCursor cur = kt_first(p, g.kt_lo);
   for (int t = 0; ok && t < g.n; ++t, kt_next(p, cur)) {
-    const PPPlan pl = pp_plan(p, g, m0, m1, cur);
+    const PPPlan pl = pp_plan(p, g, bars, cur);
     if (pl.need8 && !(ok = load8(cur.kt))) break;
     if (pl.need16 && !(ok = load16(&p.tm_k16, cur.kt))) break;
     if (!(ok = load16(&p.tm_v, cur.kt))) break;
@@ -259,12 +267,15 @@ __device__ void pp_producer(const AttnParams& p, const PPGeo& g, uint8_t* smem, 
 // Run by the whole MMA warp: every lane takes the same waits and computes the same (uniform)
 // descriptors; the elected lane issues the MMAs and commits.  Shared-memory descriptors are
 // built once per operand region and advanced by constant offsets (16-byte units) per K step.
+// Ring cursors (slot, phase) advance in the producer's load order; the plan of a key tile is
+// two range tests and two mask bits, with the routing group advanced per tile.  Operands of
+// the next key tile are taken before the wait for P, so that only MMAs lie between a P tile's
+// arrival and the next QK^T.
 __device__ void pp_mma(const AttnParams& p, const PPGeo& g, uint8_t* smem, PPBars& bars,
                        uint32_t tbase, const WaitCtx wc) {
   using C = PPCfg;
   const bool leader = elect_one();
   const uint32_t sbase = smem_u32(smem);
-  const MaskRow m0 = load_mask_row(p, g, 0), m1 = load_mask_row(p, g, 1);
   const uint32_t f16 = p.bf16 ? 1u : 0u;
   const uint32_t id_s16 = idesc(1, f16, f16, 0, 0, C::BN, 128);
   const uint32_t id_s8 = idesc(2, 1, 1, 0, 0, C::BN, 128);  // INT8 only
@@ -277,34 +288,46 @@ __device__ void pp_mma(const AttnParams& p, const PPGeo& g, uint8_t* smem, PPBar
   // V (MN-major): 64-column atoms BN * 128 bytes apart; one K step = 16 keys = 2048 bytes.
   const uint64_t d_v = sdesc(sbase + C::OFF_R16, C::BN * 128, 1024, SWZ_128B);
 
-  uint32_t n8 = 0, n16 = 0;
-  uint32_t cv0 = 0, cv1 = 0, cp0 = 0, cp1 = 0;
-  bool started0 = false, started1 = false;
+  // packed cursors (few registers: this warp's budget is small): bit 0 K8 slot, bit 1 K8 phase,
+  // bits 2-3 16-bit slot, bit 4 16-bit phase; bits 8+x vote phase, 10+x P phase, 12+x started
+  uint32_t st = 0;
+  const int ra0 = (g.lo[0] <= g.hi[0]) ? g.lo[0] / C::BN : (1 << 30);
+  const int rb0 = (g.lo[0] <= g.hi[0]) ? g.hi[0] / C::BN : -1;
+  const int ra1 = (g.lo[1] <= g.hi[1]) ? g.lo[1] / C::BN : (1 << 30);
+  const int rb1 = (g.lo[1] <= g.hi[1]) ? g.hi[1] / C::BN : -1;
+  const bool adaptive = p.adaptive != 0;
   bool ok = mbar_wait(&bars.q_full, 0, wc, W_QFULL);
   tc_fence_after();
 
-  struct Items { int k8, k16, v; };
-  auto take8 = [&](int& slot) -> bool {
-    slot = static_cast<int>(n8 % C::NS8);
-    const uint32_t use = n8 / C::NS8;
-    ++n8;
-    if (!mbar_wait(&bars.full8[slot], use & 1u, wc, W_FULL)) return false;
-    tc_fence_after();
-    return true;
+  struct Items { int k8, k16; };
+  static_assert(C::NS8 == 2 && C::NS16 <= 4, "cursor packing");
+  auto take8 = [&]() -> int {
+    const int slot = static_cast<int>(st & 1u);
+    ok = ok && mbar_wait(&bars.full8[slot], (st >> 1) & 1u, wc, W_FULL);
+    st = (slot == C::NS8 - 1) ? ((st & ~1u) ^ 2u) : (st + 1u);
+    return slot;
   };
-  auto take16 = [&](int& slot) -> bool {
-    slot = static_cast<int>(n16 % C::NS16);
-    const uint32_t use = n16 / C::NS16;
-    ++n16;
-    if (!mbar_wait(&bars.full16[slot], use & 1u, wc, W_FULL)) return false;
-    tc_fence_after();
-    return true;
+  auto take16 = [&]() -> int {
+    const int slot = static_cast<int>((st >> 2) & 3u);
+    ok = ok && mbar_wait(&bars.full16[slot], (st >> 4) & 1u, wc, W_FULL);
+    st = (slot == C::NS16 - 1) ? ((st & ~12u) ^ 16u) : (st + 4u);
+    return slot;
   };
-  auto take_k = [&](const PPPlan& pl, Items& it) -> bool {
-    it.k8 = it.k16 = it.v = -1;
-    if (pl.need8 && !take8(it.k8)) return false;
-    if (pl.need16 && !take16(it.k16)) return false;
-    return true;
+  // plan bits: 1 live0, 2 live1, 4 b16_0, 8 b16_1, 16 need8, 32 need16
+  auto plan = [&](int kt, int gi) -> uint32_t {
+    const bool l0 = kt >= ra0 && kt <= rb0, l1 = kt >= ra1 && kt <= rb1;
+    const bool h0 = l0 && group_b16(p, bars, 0, gi), h1 = l1 && group_b16(p, bars, 1, gi);
+    const bool n8 = adaptive ? (l0 || l1) : ((l0 && !h0) || (l1 && !h1));
+    const bool n16 = adaptive ? (l0 || l1) : (h0 || h1);
+    return (l0 ? 1u : 0u) | (l1 ? 2u : 0u) | (h0 ? 4u : 0u) | (h1 ? 8u : 0u) | (n8 ? 16u : 0u) |
+           (n16 ? 32u : 0u);
+  };
+  auto live = [](uint32_t pl, int x) { return (pl >> x) & 1u; };
+  auto b16 = [](uint32_t pl, int x) { return ((pl >> (2 + x)) & 1u) != 0; };
+  auto take_k = [&](uint32_t pl, Items& it) {
+    it.k8 = (pl & 16u) ? take8() : -1;
+    it.k16 = (pl & 32u) ? take16() : -1;
+    tc_fence_after();
   };
   auto issue_s = [&](int x, bool sixteen, int slot) {
     const uint32_t dS = tbase + static_cast<uint32_t>(x * C::BN);
@@ -334,43 +357,48 @@ __device__ void pp_mma(const AttnParams& p, const PPGeo& g, uint8_t* smem, PPBar
   auto commit = [&](uint64_t* bar) {
     if (leader) tc_commit(bar);
   };
-  auto first_s = [&](int x, bool b16, const Items& it) {
-    const bool sixteen = !p.adaptive && b16;
+  auto first_s = [&](int x, bool b16x, const Items& it) {
+    const bool sixteen = !adaptive && b16x;
     issue_s(x, sixteen, sixteen ? it.k16 : it.k8);
     commit(&bars.s_full[x]);
   };
-  auto pv = [&](int x, int vslot, bool acc) {
+  // P.V over keys [64 * half, 64 * half + 64) of the tile; P (16-bit pairs) sits in columns
+  // 0-63 of S_X, keys 0-63 in columns 0-31
+  auto pv = [&](int x, int vslot, int half, bool acc) {
     const uint64_t vb = d_v + static_cast<uint64_t>(vslot * (C::KV_BYTES >> 4));
     const uint32_t pt = tbase + static_cast<uint32_t>(x * C::BN);
     const uint32_t ot = tbase + static_cast<uint32_t>(2 * C::BN + x * C::D);
-    // P (16-bit pairs) sits in columns 0-63 of S_X
     if (leader) {
 #pragma unroll
-      for (int s = 0; s < C::BN / 16; ++s)
+      for (int s = 4 * half; s < 4 * half + 4; ++s)
         mma_f16_ts(ot, pt + s * 8, vb + static_cast<uint64_t>(s * ((16 * 128) >> 4)), id_pv,
                    (acc || s > 0) ? 1u : 0u);
     }
   };
 
-  Items cur{-1, -1, -1}, nxt{-1, -1, -1};
-  KtCursor kc = kt_first(p, g.kt_lo);
-  PPPlan pl = pp_plan(p, g, m0, m1, kc);
-  if (ok && g.n > 0 && (ok = take_k(pl, cur))) {
-    if (pl.live0) first_s(0, pl.b16_0, cur);
-    if (pl.live1) first_s(1, pl.b16_1, cur);
+  Items cur{-1, -1}, nxt{-1, -1};
+  int kt = g.kt_lo;
+  int gi = kt / p.group_tiles, grem = kt - gi * p.group_tiles;
+  uint32_t pl = plan(kt, gi);
+  if (ok && g.n > 0) {
+    take_k(pl, cur);
+    if (ok && live(pl, 0)) first_s(0, b16(pl, 0), cur);
+    if (ok && live(pl, 1)) first_s(1, b16(pl, 1), cur);
   }
-  for (int t = 0; ok && t < g.n; ++t) {
-    const bool has_next = t + 1 < g.n;
-    KtCursor kn = kc;
-    kt_next(p, kn);
-    const PPPlan pn = has_next ? pp_plan(p, g, m0, m1, kn) : PPPlan{};
-    if (p.adaptive) {
+  const int kt_end = g.kt_lo + g.n;
+  for (; ok && kt < kt_end; ++kt) {
+    const bool has_next = kt + 1 < kt_end;
+    if (++grem == p.group_tiles) {
+      grem = 0;
+      ++gi;
+    }
+    const uint32_t pn = has_next ? plan(kt + 1, gi) : 0u;
+    if (adaptive) {
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
-        if (!ok || !(x ? pl.live1 : pl.live0)) continue;
-        uint32_t& cv = x ? cv1 : cv0;
-        if (!(ok = mbar_wait(&bars.vote[x], cv & 1u, wc, W_VOTE))) break;
-        ++cv;
+        if (!ok || !live(pl, x)) continue;
+        if (!(ok = mbar_wait(&bars.vote[x], (st >> (8 + x)) & 1u, wc, W_VOTE))) break;
+        st ^= 1u << (8 + x);
         tc_fence_after();
         const volatile uint32_t* vv = bars.votes[x];
         uint32_t any = 0;
@@ -386,33 +414,31 @@ __device__ void pp_mma(const AttnParams& p, const PPGeo& g, uint8_t* smem, PPBar
     // every QK^T MMA of this key tile has been issued: release its K slots when they finish
     if (cur.k8 >= 0) commit(&bars.empty8[cur.k8]);
     if (cur.k16 >= 0) commit(&bars.empty16[cur.k16]);
-    if (!(ok = take16(cur.v))) break;
-    bool taken_next = false;
+    // V of this tile and K of the next were loaded long ago: take them before waiting for P
+    const int vslot = take16();
+    if (has_next) take_k(pn, nxt);
+    tc_fence_after();
+    if (!ok) break;
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
       if (!ok) break;
-      if (x ? pl.live1 : pl.live0) {
-        uint32_t& cp = x ? cp1 : cp0;
-        bool& started = x ? started1 : started0;
-        if (!(ok = mbar_wait(&bars.p_full[x], cp & 1u, wc, W_PFULL))) break;
-        ++cp;
+      if (live(pl, x)) {
+        const uint32_t cp = (st >> (10 + x)) & 1u;
+        // the first half of P is published while the softmax exponentiates the second
+        if (!(ok = mbar_wait(&bars.p_half[x], cp, wc, W_PFULL))) break;
         tc_fence_after();
-        pv(x, cur.v, started);
-        started = true;
+        pv(x, vslot, 0, ((st >> (12 + x)) & 1u) != 0);
+        if (!(ok = mbar_wait(&bars.p_full[x], cp, wc, W_PFULL))) break;
+        tc_fence_after();
+        pv(x, vslot, 1, true);
+        st = (st ^ (1u << (10 + x))) | (1u << (12 + x));
       }
-      if (has_next && (x ? pn.live1 : pn.live0)) {
-        if (!taken_next) {
-          if (!(ok = take_k(pn, nxt))) break;
-          taken_next = true;
-        }
-        first_s(x, x ? pn.b16_1 : pn.b16_0, nxt);
-      }
+      if (has_next && live(pn, x)) first_s(x, b16(pn, x), nxt);
     }
     if (!ok) break;
-    commit(&bars.empty16[cur.v]);
+    commit(&bars.empty16[vslot]);
     cur = nxt;
     pl = pn;
-    kc = kn;
   }
   commit(&bars.o_done[0]);
   commit(&bars.o_done[1]);
@@ -470,6 +496,13 @@ __device__ __forceinline__ float add_hi16(float acc, uint32_t pk) {
 // 16-bit pairs into the row's S columns 0-63 (each 32-column chunk stored as soon as it is
 // ready), and keep two row sums: of the exact p (for lse) and of the rounded p that the P.V
 // MMA multiplies (for O).
+//
+// The warpgroup's first warp also issues its query tile's MMAs (the elected lane issues; all
+// lanes keep the same, warp-uniform ring state): as soon as the whole P tile is in TMEM it
+// issues P.V and the next key tile's QK^T, so that no other warp stands between a finished P
+// and the tensor core.  Both warpgroups take every key tile's ring slots in the producer's
+// order (passing the tiles their query tile does not see) and release each slot with a
+// commit: a slot is free once both have released it.
 template <bool BF16, bool ADAPTIVE>
 __device__ void pp_softmax(const AttnParams& p, const PPGeo& g, uint8_t* smem, PPBars& bars,
                            uint32_t tbase, const WaitCtx wc) {
@@ -493,7 +526,6 @@ __device__ void pp_softmax(const AttnParams& p, const PPGeo& g, uint8_t* smem, P
   const float* ks_row = p.k_scale + static_cast<size_t>(g.b * p.Hkv + g.kvh) * p.nkt;
   const float NEG_INF = -__int_as_float(0x7f800000);
   const float sq_scale = sq * p.scale_log2;
-  const MaskRow mrow = load_mask_row(p, g, x);
   (void)smem;
 
   float m_ref = NEG_INF;   // max used for the exponentials (lazy)
@@ -556,7 +588,7 @@ __device__ void pp_softmax(const AttnParams& p, const PPGeo& g, uint8_t* smem, P
     load_s();
     const int j0 = kt * N;
     const bool full = row_valid && j0 >= lo_r && j0 + N - 1 <= hi_r;
-    bool sixteen = !ADAPTIVE && group_b16(p, mrow, gcur);
+    bool sixteen = !ADAPTIVE && group_b16(p, bars, x, gcur);
     // (a zero block scale would turn masked -inf entries into NaN: keep it positive; the
     // scores of an all-zero block are 0 either way)
     float cscale = sixteen ? p.scale_log2 : fmaxf(sq_scale * ks, 1e-30f);
@@ -656,6 +688,14 @@ __device__ void pp_softmax(const AttnParams& p, const PPGeo& g, uint8_t* smem, P
         sr1 = add_hi16<BF16>(sr1, pk);
       }
       raw[c >> 1] = pk;
+      if (c == 94) {
+        // P of keys 0-63 (stored with the chunks of columns 0-63) is in TMEM: publish it, so
+        // that the first half of P.V overlaps the exponentials of the second half
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.p_half[x]);
+      }
       if ((c & 31) == 30) tmem_st16(lane_base + s_col + (c >> 5) * 16, &raw[(c >> 5) * 16]);
     }
     {
@@ -736,7 +776,6 @@ __global__ void __launch_bounds__(PPCfg::THREADS, 1)
   }
   PPBars& bars = *reinterpret_cast<PPBars*>(smem + C::OFF_BAR);
   const int warp = threadIdx.x >> 5;
-  const PPGeo g = pp_geo(p);
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
     for (int s = 0; s < C::NS8; ++s) {
@@ -751,10 +790,17 @@ __global__ void __launch_bounds__(PPCfg::THREADS, 1)
       mbar_init(&bars.s_full[x], 1);
       mbar_init(&bars.s16_full[x], 1);
       mbar_init(&bars.vote[x], 4);
+      mbar_init(&bars.p_half[x], 4);
       mbar_init(&bars.p_full[x], 4);
       mbar_init(&bars.o_done[x], 1);
     }
     mbar_init(&bars.drain, 1);
+    const PPGeo g0 = pp_geo(p);
+    for (int x = 0; x < 2; ++x) {
+      const MaskRow m = load_mask_row(p, g0, x);
+      bars.mask[x][0] = m.w0;
+      bars.mask[x][1] = m.w1;
+    }
     bars.abort = 0;
     fence_mbarrier_init();
   }
@@ -772,12 +818,17 @@ __global__ void __launch_bounds__(PPCfg::THREADS, 1)
   // (128 * 104 + 256 * 200 = 64512 = 384 * 168).
   if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory");
+    // each role derives the tile geometry itself: nothing computed before the role split stays
+    // live in the smaller register budget of the other roles
+    const PPGeo g = pp_geo(p);
     pp_softmax<BF16, ADAPTIVE>(p, g, smem, bars, tbase, wc);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 104;\n" ::: "memory");
     if (warp == 8) {
+      const PPGeo g = pp_geo(p);
       if ((threadIdx.x & 31) == 0 && g.n > 0) pp_producer(p, g, smem, bars, wc);
     } else if (warp == 9) {
+      const PPGeo g = pp_geo(p);
       if (g.n > 0) pp_mma(p, g, smem, bars, tbase, wc);
     }
   }
