@@ -62,6 +62,7 @@ struct PPCfg {
 
 struct PPBars {
   uint64_t q_full;
+  uint64_t q_empty;  // every QK^T MMA of the current work item has completed: Q may be reloaded
   uint64_t full8[PPCfg::NS8], empty8[PPCfg::NS8];
   uint64_t full16[PPCfg::NS16], empty16[PPCfg::NS16];
   uint64_t s_full[2];
@@ -70,11 +71,12 @@ struct PPBars {
   uint64_t p_half[2];  // P of keys 0-63 of query tile X is in TMEM
   uint64_t p_full[2];  // all of P of query tile X is in TMEM
   uint64_t o_done[2];
+  uint64_t o_free[2];  // the epilogue has read O of query tile X: the next item may overwrite it
   uint64_t drain;
   uint32_t tmem_base;
   uint32_t abort;
   uint32_t votes[2][4];
-  uint64_t mask[2][2];  // routing mask words of query tiles 0 and 1 (all ones: no mask)
+  uint64_t mask[2][2][2];  // [item parity][query tile][word] routing mask (all ones: no mask)
 };
 static_assert(sizeof(PPBars) <= 512, "barrier block");
 
@@ -83,10 +85,19 @@ struct PPGeo {
   int lo[2], hi[2];  // visible key range (union) of query tile X; lo > hi = none
 };
 
-__device__ __forceinline__ PPGeo pp_geo(const AttnParams& p) {
+// Persistent CTAs: work item j = (batch, head, pair of query tiles), numbered longest-first;
+// round r gives CTA c the item r * G + c (r even) or r * G + G - 1 - c (r odd), a snake that
+// keeps the CTAs' total work close.  -1: no item left.
+__device__ __forceinline__ int pp_item(const AttnParams& p, int r) {
+  const long long n_items = static_cast<long long>(p.B) * p.H * ((p.nqt + 1) / 2);
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  const long long j = static_cast<long long>(r) * G + ((r & 1) ? G - 1 - c : c);
+  return j < n_items ? static_cast<int>(j) : -1;
+}
+
+__device__ __forceinline__ PPGeo pp_geo(const AttnParams& p, int idx) {
   PPGeo g;
   const int BH = p.B * p.H;
-  const int idx = blockIdx.x;
   const int n_pairs = (p.nqt + 1) / 2;
   g.pair = n_pairs - 1 - idx / BH;  // longest-first
   const int bh = idx - (idx / BH) * BH;
@@ -174,9 +185,10 @@ __device__ __forceinline__ bool group_b16(const AttnParams& p, const MaskRow& m,
 }
 // As above, with the mask row of query tile x read from shared memory (it costs the issuing
 // warps no registers).
-__device__ __forceinline__ bool group_b16(const AttnParams& p, const PPBars& bars, int x, int gi) {
+__device__ __forceinline__ bool group_b16(const AttnParams& p, const PPBars& bars, int slot, int x,
+                                          int gi) {
   if (p.adaptive) return false;
-  const uint64_t w = bars.mask[x][(gi >> 6) & 1];
+  const uint64_t w = bars.mask[slot][x][(gi >> 6) & 1];
   return ((w >> (gi & 63)) & 1ull) == 0;
 }
 
@@ -186,12 +198,12 @@ struct PPPlan {
 };
 
 __device__ __forceinline__ PPPlan pp_plan(const AttnParams& p, const PPGeo& g, const PPBars& bars,
-                                          const KtCursor& c) {
+                                          int slot, const KtCursor& c) {
   PPPlan pl;
   pl.live0 = tile_live(g, p, 0, c.kt);
   pl.live1 = tile_live(g, p, 1, c.kt);
-  pl.b16_0 = pl.live0 && group_b16(p, bars, 0, c.gi);
-  pl.b16_1 = pl.live1 && group_b16(p, bars, 1, c.gi);
+  pl.b16_0 = pl.live0 && group_b16(p, bars, slot, 0, c.gi);
+  pl.b16_1 = pl.live1 && group_b16(p, bars, slot, 1, c.gi);
   if (p.adaptive) {
     pl.need8 = pl.need16 = pl.live0 || pl.live1;
   } else {
@@ -203,26 +215,19 @@ __device__ __forceinline__ PPPlan pp_plan(const AttnParams& p, const PPGeo& g, c
 
 // ------------------------------------------------------------------ producer ----------
 
-__device__ void pp_producer(const AttnParams& p, const PPGeo& g, uint8_t* smem, PPBars& bars,
-                            const WaitCtx wc) {
+// One lane: for each work item of this CTA, Q16 and Q8 of both query tiles (once the previous
+// item's QK^T MMAs have completed) and the item's routing mask rows, then every key tile's K8,
+// K16 and V in the MMA warp's order of first use within each ring.  The rings run on across
+// items.
+__device__ void pp_producer(const AttnParams& p, uint8_t* smem, PPBars& bars, const WaitCtx wc) {
   using C = PPCfg;
-  const int bh_q = g.b * p.H + g.h;
-  const int bh_kv = g.b * p.Hkv + g.kvh;
   prefetch_tmap(&p.tm_q16);
   prefetch_tmap(&p.tm_k16);
   prefetch_tmap(&p.tm_v);
   prefetch_tmap(&p.tm_q8);
   prefetch_tmap(&p.tm_k8);
-  if (!lamp_chk(bh_q < p.B * p.H && bh_kv < p.B * p.Hkv, 3)) return;
-  mbar_arrive_expect_tx(&bars.q_full, 2 * (C::Q16_BYTES + C::Q8_BYTES));
-  for (int x = 0; x < 2; ++x) {
-    const int row = g.q0 + x * C::MT;
-    for (int c = 0; c < 2; ++c)
-      tma_load_3d(smem + C::OFF_Q16 + x * C::Q16_BYTES + c * C::MT * 128, &p.tm_q16, &bars.q_full,
-                  c * 64, row, bh_q);
-    tma_load_3d(smem + C::OFF_Q8 + x * C::Q8_BYTES, &p.tm_q8, &bars.q_full, 0, row, bh_q);
-  }
   uint32_t n8 = 0, n16 = 0;
+  int bh_kv = 0;
   auto load8 = [&](int kt) -> bool {
     const int slot = static_cast<int>(n8 % C::NS8);
     const uint32_t use = n8 / C::NS8;
@@ -244,14 +249,37 @@ __device__ void pp_producer(const AttnParams& p, const PPGeo& g, uint8_t* smem, 
     ++n16;
     return true;
   };
-  // Per key tile, in the MMA warp's order of first use within each ring: K8, K16, V.
   bool ok = true;
-  KtCursor cur = kt_first(p, g.kt_lo);
-  for (int t = 0; ok && t < g.n; ++t, kt_next(p, cur)) {
-    const PPPlan pl = pp_plan(p, g, bars, cur);
-    if (pl.need8 && !(ok = load8(cur.kt))) break;
-    if (pl.need16 && !(ok = load16(&p.tm_k16, cur.kt))) break;
-    if (!(ok = load16(&p.tm_v, cur.kt))) break;
+  int r = 0;
+  for (; ok; ++r) {
+    const int item = pp_item(p, r);
+    if (item < 0) break;
+    const PPGeo g = pp_geo(p, item);
+    const int bh_q = g.b * p.H + g.h;
+    bh_kv = g.b * p.Hkv + g.kvh;
+    if (!lamp_chk(bh_q < p.B * p.H && bh_kv < p.B * p.Hkv, 3)) { ok = false; break; }
+    if (r > 0 && !(ok = mbar_wait(&bars.q_empty, (r - 1) & 1u, wc, W_EMPTY))) break;
+    // the item's mask rows, read by the MMA warp after it has seen this item's Q arrive
+    for (int x = 0; x < 2; ++x) {
+      const MaskRow m = load_mask_row(p, g, x);
+      bars.mask[r & 1][x][0] = m.w0;
+      bars.mask[r & 1][x][1] = m.w1;
+    }
+    mbar_arrive_expect_tx(&bars.q_full, 2 * (C::Q16_BYTES + C::Q8_BYTES));
+    for (int x = 0; x < 2; ++x) {
+      const int row = g.q0 + x * C::MT;
+      for (int c = 0; c < 2; ++c)
+        tma_load_3d(smem + C::OFF_Q16 + x * C::Q16_BYTES + c * C::MT * 128, &p.tm_q16,
+                    &bars.q_full, c * 64, row, bh_q);
+      tma_load_3d(smem + C::OFF_Q8 + x * C::Q8_BYTES, &p.tm_q8, &bars.q_full, 0, row, bh_q);
+    }
+    KtCursor cur = kt_first(p, g.kt_lo);
+    for (int t = 0; ok && t < g.n; ++t, kt_next(p, cur)) {
+      const PPPlan pl = pp_plan(p, g, bars, r & 1, cur);
+      if (pl.need8 && !(ok = load8(cur.kt))) break;
+      if (pl.need16 && !(ok = load16(&p.tm_k16, cur.kt))) break;
+      if (!(ok = load16(&p.tm_v, cur.kt))) break;
+    }
   }
   // Drain: every slot's most recent load must have landed before the CTA may exit.
   const WaitCtx drain{0u, 50000u};  // no abort word: in-flight work always completes
@@ -259,7 +287,7 @@ __device__ void pp_producer(const AttnParams& p, const PPGeo& g, uint8_t* smem, 
     mbar_wait(&bars.full8[it % C::NS8], (it / C::NS8) & 1u, drain, W_DRAIN);
   for (uint32_t it = n16 > static_cast<uint32_t>(C::NS16) ? n16 - C::NS16 : 0; it < n16; ++it)
     mbar_wait(&bars.full16[it % C::NS16], (it / C::NS16) & 1u, drain, W_DRAIN);
-  mbar_wait(&bars.q_full, 0, drain, W_DRAIN);
+  if (r > 0) mbar_wait(&bars.q_full, (r - 1) & 1u, drain, W_DRAIN);
 }
 
 // ------------------------------------------------------------------ MMA issuer --------
@@ -267,19 +295,23 @@ __device__ void pp_producer(const AttnParams& p, const PPGeo& g, uint8_t* smem, 
 // Run by the whole MMA warp: every lane takes the same waits and computes the same (uniform)
 // descriptors; the elected lane issues the MMAs and commits.  Shared-memory descriptors are
 // built once per operand region and advanced by constant offsets (16-byte units) per K step.
-// Ring cursors (slot, phase) advance in the producer's load order; the plan of a key tile is
-// two range tests and two mask bits, with the routing group advanced per tile.  Operands of
-// the next key tile are taken before the wait for P, so that only MMAs lie between a P tile's
-// arrival and the next QK^T.
-__device__ void pp_mma(const AttnParams& p, const PPGeo& g, uint8_t* smem, PPBars& bars,
-                       uint32_t tbase, const WaitCtx wc) {
+// Ring cursors (slot, phase) advance in the producer's load order and run on across work
+// items; the plan of a key tile is two range tests and two mask bits, with the routing group
+// advanced per tile.  Operands of the next key tile are taken before the wait for P, so that
+// only MMAs lie between a P tile's arrival and the next QK^T.  Per work item: wait for its Q,
+// and before the first QK^T of a query tile for the previous item's epilogue to have read O;
+// at the end release Q and publish O.
+template <bool BF16, bool ADAPTIVE>
+__device__ void pp_mma(const AttnParams& p, uint8_t* smem, PPBars& bars, uint32_t tbase,
+                       const WaitCtx wc) {
   using C = PPCfg;
   const bool leader = elect_one();
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t f16 = p.bf16 ? 1u : 0u;
-  const uint32_t id_s16 = idesc(1, f16, f16, 0, 0, C::BN, 128);
-  const uint32_t id_s8 = idesc(2, 1, 1, 0, 0, C::BN, 128);  // INT8 only
-  const uint32_t id_pv = idesc(1, f16, f16, 0, 1, C::D, 128);
+  constexpr uint32_t f16 = BF16 ? 1u : 0u;
+  constexpr uint32_t id_s16 = idesc(1, f16, f16, 0, 0, C::BN, 128);
+  constexpr uint32_t id_s8 = idesc(2, 1, 1, 0, 0, C::BN, 128);  // INT8 only
+  constexpr uint32_t id_pv = idesc(1, f16, f16, 0, 1, C::D, 128);
+  constexpr bool adaptive = ADAPTIVE;
   // K-major operands: 128-byte rows, 8-row groups 1024 bytes apart; one K step = 32 bytes.
   const uint64_t d_q16 = sdesc(sbase + C::OFF_Q16, 16, 1024, SWZ_128B);
   const uint64_t d_q8 = sdesc(sbase + C::OFF_Q8, 16, 1024, SWZ_128B);
@@ -289,16 +321,11 @@ __device__ void pp_mma(const AttnParams& p, const PPGeo& g, uint8_t* smem, PPBar
   const uint64_t d_v = sdesc(sbase + C::OFF_R16, C::BN * 128, 1024, SWZ_128B);
 
   // packed cursors (few registers: this warp's budget is small): bit 0 K8 slot, bit 1 K8 phase,
-  // bits 2-3 16-bit slot, bit 4 16-bit phase; bits 8+x vote phase, 10+x P phase, 12+x started
+  // bits 2-3 16-bit slot, bit 4 16-bit phase; bits 8+x vote phase, 10+x P phase, 12+x started,
+  // 14+x O of query tile x not yet released by the previous item's epilogue, 16+x O of this
+  // item published
   uint32_t st = 0;
-  const int ra0 = (g.lo[0] <= g.hi[0]) ? g.lo[0] / C::BN : (1 << 30);
-  const int rb0 = (g.lo[0] <= g.hi[0]) ? g.hi[0] / C::BN : -1;
-  const int ra1 = (g.lo[1] <= g.hi[1]) ? g.lo[1] / C::BN : (1 << 30);
-  const int rb1 = (g.lo[1] <= g.hi[1]) ? g.hi[1] / C::BN : -1;
-  const bool adaptive = p.adaptive != 0;
-  bool ok = mbar_wait(&bars.q_full, 0, wc, W_QFULL);
-  tc_fence_after();
-
+  bool ok = true;
   struct Items { int k8, k16; };
   static_assert(C::NS8 == 2 && C::NS16 <= 4, "cursor packing");
   auto take8 = [&]() -> int {
@@ -312,15 +339,6 @@ __device__ void pp_mma(const AttnParams& p, const PPGeo& g, uint8_t* smem, PPBar
     ok = ok && mbar_wait(&bars.full16[slot], (st >> 4) & 1u, wc, W_FULL);
     st = (slot == C::NS16 - 1) ? ((st & ~12u) ^ 16u) : (st + 4u);
     return slot;
-  };
-  // plan bits: 1 live0, 2 live1, 4 b16_0, 8 b16_1, 16 need8, 32 need16
-  auto plan = [&](int kt, int gi) -> uint32_t {
-    const bool l0 = kt >= ra0 && kt <= rb0, l1 = kt >= ra1 && kt <= rb1;
-    const bool h0 = l0 && group_b16(p, bars, 0, gi), h1 = l1 && group_b16(p, bars, 1, gi);
-    const bool n8 = adaptive ? (l0 || l1) : ((l0 && !h0) || (l1 && !h1));
-    const bool n16 = adaptive ? (l0 || l1) : (h0 || h1);
-    return (l0 ? 1u : 0u) | (l1 ? 2u : 0u) | (h0 ? 4u : 0u) | (h1 ? 8u : 0u) | (n8 ? 16u : 0u) |
-           (n16 ? 32u : 0u);
   };
   auto live = [](uint32_t pl, int x) { return (pl >> x) & 1u; };
   auto b16 = [](uint32_t pl, int x) { return ((pl >> (2 + x)) & 1u) != 0; };
@@ -357,6 +375,14 @@ __device__ void pp_mma(const AttnParams& p, const PPGeo& g, uint8_t* smem, PPBar
   auto commit = [&](uint64_t* bar) {
     if (leader) tc_commit(bar);
   };
+  // the previous item's epilogue must have read O of query tile x (phase r - 1 of o_free) before
+  // this item's first P.V overwrites it
+  auto o_released = [&](int x, int r) {
+    if ((st >> (14 + x)) & 1u) {
+      ok = ok && mbar_wait(&bars.o_free[x], (r - 1) & 1u, wc, W_ODONE);
+      st &= ~(1u << (14 + x));
+    }
+  };
   auto first_s = [&](int x, bool b16x, const Items& it) {
     const bool sixteen = !adaptive && b16x;
     issue_s(x, sixteen, sixteen ? it.k16 : it.k8);
@@ -376,72 +402,110 @@ __device__ void pp_mma(const AttnParams& p, const PPGeo& g, uint8_t* smem, PPBar
     }
   };
 
-  Items cur{-1, -1}, nxt{-1, -1};
-  int kt = g.kt_lo;
-  int gi = kt / p.group_tiles, grem = kt - gi * p.group_tiles;
-  uint32_t pl = plan(kt, gi);
-  if (ok && g.n > 0) {
-    take_k(pl, cur);
-    if (ok && live(pl, 0)) first_s(0, b16(pl, 0), cur);
-    if (ok && live(pl, 1)) first_s(1, b16(pl, 1), cur);
-  }
-  const int kt_end = g.kt_lo + g.n;
-  for (; ok && kt < kt_end; ++kt) {
-    const bool has_next = kt + 1 < kt_end;
-    if (++grem == p.group_tiles) {
-      grem = 0;
-      ++gi;
+  for (int r = 0; ok; ++r) {
+    const int item = pp_item(p, r);
+    if (item < 0) break;
+    const PPGeo g = pp_geo(p, item);
+    const int ms = r & 1;  // mask slot of this item
+    const int ra0 = (g.lo[0] <= g.hi[0]) ? g.lo[0] / C::BN : (1 << 30);
+    const int rb0 = (g.lo[0] <= g.hi[0]) ? g.hi[0] / C::BN : -1;
+    const int ra1 = (g.lo[1] <= g.hi[1]) ? g.lo[1] / C::BN : (1 << 30);
+    const int rb1 = (g.lo[1] <= g.hi[1]) ? g.hi[1] / C::BN : -1;
+    // plan bits: 1 live0, 2 live1, 4 b16_0, 8 b16_1, 16 need8, 32 need16
+    auto plan = [&](int kt, int gi) -> uint32_t {
+      const bool l0 = kt >= ra0 && kt <= rb0, l1 = kt >= ra1 && kt <= rb1;
+      const bool h0 = l0 && group_b16(p, bars, ms, 0, gi), h1 = l1 && group_b16(p, bars, ms, 1, gi);
+      const bool n8 = adaptive ? (l0 || l1) : ((l0 && !h0) || (l1 && !h1));
+      const bool n16 = adaptive ? (l0 || l1) : (h0 || h1);
+      return (l0 ? 1u : 0u) | (l1 ? 2u : 0u) | (h0 ? 4u : 0u) | (h1 ? 8u : 0u) | (n8 ? 16u : 0u) |
+             (n16 ? 32u : 0u);
+    };
+    if (!(ok = mbar_wait(&bars.q_full, ms, wc, W_QFULL))) break;
+    tc_fence_after();
+    st &= ~((3u << 12) | (3u << 16));  // no P.V of this item yet, O not published
+    if (r > 0) st |= 3u << 14;         // O of both tiles held by the previous item's epilogue
+
+    Items cur{-1, -1}, nxt{-1, -1};
+    int kt = g.kt_lo;
+    int gi = kt / p.group_tiles, grem = kt - gi * p.group_tiles;
+    uint32_t pl = plan(kt, gi);
+    if (g.n > 0) {
+      take_k(pl, cur);
+      if (ok && live(pl, 0)) first_s(0, b16(pl, 0), cur);
+      if (ok && live(pl, 1)) first_s(1, b16(pl, 1), cur);
     }
-    const uint32_t pn = has_next ? plan(kt + 1, gi) : 0u;
-    if (adaptive) {
+    const int kt_end = g.kt_lo + g.n;
+    for (; ok && kt < kt_end; ++kt) {
+      const bool has_next = kt + 1 < kt_end;
+      if (++grem == p.group_tiles) {
+        grem = 0;
+        ++gi;
+      }
+      const uint32_t pn = has_next ? plan(kt + 1, gi) : 0u;
+      if (adaptive) {
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if (!ok || !live(pl, x)) continue;
+          if (!(ok = mbar_wait(&bars.vote[x], (st >> (8 + x)) & 1u, wc, W_VOTE))) break;
+          st ^= 1u << (8 + x);
+          tc_fence_after();
+          const volatile uint32_t* vv = bars.votes[x];
+          uint32_t any = 0;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) any |= vv[w];
+          if (any) {
+            issue_s(x, true, cur.k16);
+            commit(&bars.s16_full[x]);
+          }
+        }
+        if (!ok) break;
+      }
+      // every QK^T MMA of this key tile has been issued: release its K slots when they finish,
+      // and Q once the item's last key tile is reached
+      if (cur.k8 >= 0) commit(&bars.empty8[cur.k8]);
+      if (cur.k16 >= 0) commit(&bars.empty16[cur.k16]);
+      if (!has_next) commit(&bars.q_empty);
+      // V of this tile and K of the next were loaded long ago: take them before waiting for P
+      const int vslot = take16();
+      if (has_next) take_k(pn, nxt);
+      tc_fence_after();
+      if (!ok) break;
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
-        if (!ok || !live(pl, x)) continue;
-        if (!(ok = mbar_wait(&bars.vote[x], (st >> (8 + x)) & 1u, wc, W_VOTE))) break;
-        st ^= 1u << (8 + x);
-        tc_fence_after();
-        const volatile uint32_t* vv = bars.votes[x];
-        uint32_t any = 0;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) any |= vv[w];
-        if (any) {
-          issue_s(x, true, cur.k16);
-          commit(&bars.s16_full[x]);
+        if (!ok) break;
+        if (live(pl, x)) {
+          const uint32_t cp = (st >> (10 + x)) & 1u;
+          // the first half of P is published while the softmax exponentiates the second
+          const bool started = ((st >> (12 + x)) & 1u) != 0;
+          if (!started) o_released(x, r);
+          if (!(ok = ok && mbar_wait(&bars.p_half[x], cp, wc, W_PFULL))) break;
+          tc_fence_after();
+          pv(x, vslot, 0, started);
+          if (!(ok = mbar_wait(&bars.p_full[x], cp, wc, W_PFULL))) break;
+          tc_fence_after();
+          pv(x, vslot, 1, true);
+          st = (st ^ (1u << (10 + x))) | (1u << (12 + x));
+          if (!(has_next && live(pn, x))) {  // the query tile's last key tile: publish O
+            commit(&bars.o_done[x]);
+            st |= 1u << (16 + x);
+          }
         }
+        if (has_next && live(pn, x)) first_s(x, b16(pn, x), nxt);
       }
       if (!ok) break;
+      commit(&bars.empty16[vslot]);
+      cur = nxt;
+      pl = pn;
     }
-    // every QK^T MMA of this key tile has been issued: release its K slots when they finish
-    if (cur.k8 >= 0) commit(&bars.empty8[cur.k8]);
-    if (cur.k16 >= 0) commit(&bars.empty16[cur.k16]);
-    // V of this tile and K of the next were loaded long ago: take them before waiting for P
-    const int vslot = take16();
-    if (has_next) take_k(pn, nxt);
-    tc_fence_after();
     if (!ok) break;
-#pragma unroll
-    for (int x = 0; x < 2; ++x) {
-      if (!ok) break;
-      if (live(pl, x)) {
-        const uint32_t cp = (st >> (10 + x)) & 1u;
-        // the first half of P is published while the softmax exponentiates the second
-        if (!(ok = mbar_wait(&bars.p_half[x], cp, wc, W_PFULL))) break;
-        tc_fence_after();
-        pv(x, vslot, 0, ((st >> (12 + x)) & 1u) != 0);
-        if (!(ok = mbar_wait(&bars.p_full[x], cp, wc, W_PFULL))) break;
-        tc_fence_after();
-        pv(x, vslot, 1, true);
-        st = (st ^ (1u << (10 + x))) | (1u << (12 + x));
+    if (g.n == 0) commit(&bars.q_empty);
+    for (int x = 0; x < 2; ++x) {  // a query tile without a visible key tile: O is zero
+      if (!((st >> (16 + x)) & 1u)) {
+        o_released(x, r);
+        commit(&bars.o_done[x]);
       }
-      if (has_next && live(pn, x)) first_s(x, b16(pn, x), nxt);
     }
-    if (!ok) break;
-    commit(&bars.empty16[vslot]);
-    cur = nxt;
-    pl = pn;
   }
-  commit(&bars.o_done[0]);
-  commit(&bars.o_done[1]);
   commit(&bars.drain);
   const WaitCtx drain{0u, 50000u};  // no abort word: in-flight work always completes
   mbar_wait(&bars.drain, 0, drain, W_DRAIN);
@@ -503,9 +567,14 @@ __device__ __forceinline__ float add_hi16(float acc, uint32_t pk) {
 // and the tensor core.  Both warpgroups take every key tile's ring slots in the producer's
 // order (passing the tiles their query tile does not see) and release each slot with a
 // commit: a slot is free once both have released it.
+// One work item of the softmax role (it = the CTA's item count, the parity of its per-item
+// barrier phases).  The phase counters of the per-tile barriers run on across items.  Returns
+// false when a wait gave up.
 template <bool BF16, bool ADAPTIVE>
-__device__ void pp_softmax(const AttnParams& p, const PPGeo& g, uint8_t* smem, PPBars& bars,
-                           uint32_t tbase, const WaitCtx wc) {
+__device__ __forceinline__ bool pp_softmax_item(const AttnParams& p, const PPGeo& g, PPBars& bars,
+                                                uint32_t tbase, const WaitCtx wc, int it,
+                                                uint32_t& cs, uint32_t& c16, uint32_t& cvv,
+                                                uint32_t (&raw)[PPCfg::BN]) {
   using C = PPCfg;
   constexpr int N = C::BN;
   const int warp = threadIdx.x >> 5;
@@ -526,14 +595,12 @@ __device__ void pp_softmax(const AttnParams& p, const PPGeo& g, uint8_t* smem, P
   const float* ks_row = p.k_scale + static_cast<size_t>(g.b * p.Hkv + g.kvh) * p.nkt;
   const float NEG_INF = -__int_as_float(0x7f800000);
   const float sq_scale = sq * p.scale_log2;
-  (void)smem;
+  const MaskRow mrow = load_mask_row(p, g, x);
 
   float m_ref = NEG_INF;   // max used for the exponentials (lazy)
   float m_true = NEG_INF;  // true running max of the used scores (look-ahead rule)
   float l_ex = 0.0f, l_rd = 0.0f;
-  uint32_t cs = 0, c16 = 0, cvv = 0;
   bool ok = true, any_pv = false;
-  uint32_t raw[N];
 
   auto load_s = [&]() {
 #pragma unroll
@@ -588,7 +655,7 @@ __device__ void pp_softmax(const AttnParams& p, const PPGeo& g, uint8_t* smem, P
     load_s();
     const int j0 = kt * N;
     const bool full = row_valid && j0 >= lo_r && j0 + N - 1 <= hi_r;
-    bool sixteen = !ADAPTIVE && group_b16(p, bars, x, gcur);
+    bool sixteen = !ADAPTIVE && group_b16(p, mrow, gcur);
     // (a zero block scale would turn masked -inf entries into NaN: keep it positive; the
     // scores of an all-zero block are 0 either way)
     float cscale = sixteen ? p.scale_log2 : fmaxf(sq_scale * ks, 1e-30f);
@@ -710,42 +777,43 @@ __device__ void pp_softmax(const AttnParams& p, const PPGeo& g, uint8_t* smem, P
     if (lane == 0) mbar_arrive(&bars.p_full[x]);
     any_pv = true;
   }
-  if (!ok) return;
+  if (!ok) return false;
 
-  // epilogue: O / l and lse
+  // epilogue: O / l and lse.  O is read from TMEM in one go and released at once, so that the
+  // next item's P.V may start while this one is normalised and stored.
+  if (!warp_wait(&bars.o_done[x], it & 1, wc, W_ODONE)) return false;
+  tc_fence_after();
   if (any_pv) {
-    if (!warp_wait(&bars.o_done[x], 0, wc, W_ODONE)) return;
-    tc_fence_after();
+#pragma unroll
+    for (int c = 0; c < C::D / 32; ++c)
+      tmem_ld32(lane_base + o_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&raw[c * 32]));
+    tmem_wait_ld();
+  } else {
+#pragma unroll
+    for (int e = 0; e < C::D; ++e) raw[e] = 0u;
   }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&bars.o_free[x]);
   const float inv = (l_rd > 0.0f) ? 1.0f / l_rd : 0.0f;
   const size_t orow = (static_cast<size_t>(bh_q) * p.Lq + (row_valid ? i : 0)) * C::D;
-#pragma unroll 1
-  for (int c = 0; c < C::D / 32; ++c) {
-    uint32_t ov[32];
-    if (any_pv) {
-      tmem_ld32(lane_base + o_col + c * 32, ov);
-      tmem_wait_ld();
-    } else {
-#pragma unroll
-      for (int e = 0; e < 32; ++e) ov[e] = 0u;
-    }
-    if (!row_valid) continue;
-    if (!lamp_chk(orow + c * 32 + 32 <= static_cast<size_t>(p.B) * p.H * p.Lq * C::D, 12)) continue;
+  if (row_valid &&
+      lamp_chk(orow + C::D <= static_cast<size_t>(p.B) * p.H * p.Lq * C::D, 12)) {
     if (p.out_f32) {
-      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow + c * 32);
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow);
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
-        dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
-                             __uint_as_float(ov[4 * e + 2]) * inv, __uint_as_float(ov[4 * e + 3]) * inv);
+      for (int e = 0; e < C::D / 4; ++e)
+        dst[e] = make_float4(__uint_as_float(raw[4 * e]) * inv, __uint_as_float(raw[4 * e + 1]) * inv,
+                             __uint_as_float(raw[4 * e + 2]) * inv, __uint_as_float(raw[4 * e + 3]) * inv);
     } else {
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow + c * 32);
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
+      for (int e = 0; e < C::D / 8; ++e) {
         uint32_t w[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const float a = __uint_as_float(ov[8 * e + 2 * q]) * inv;
-          const float b2 = __uint_as_float(ov[8 * e + 2 * q + 1]) * inv;
+          const float a = __uint_as_float(raw[8 * e + 2 * q]) * inv;
+          const float b2 = __uint_as_float(raw[8 * e + 2 * q + 1]) * inv;
           if (BF16) {
             __nv_bfloat162 v2 = __floats2bfloat162_rn(a, b2);
             w[q] = *reinterpret_cast<uint32_t*>(&v2);
@@ -761,6 +829,20 @@ __device__ void pp_softmax(const AttnParams& p, const PPGeo& g, uint8_t* smem, P
   if (row_valid && p.lse)
     p.lse[static_cast<size_t>(bh_q) * p.Lq + i] =
         (l_ex > 0.0f) ? m_ref * 0.69314718055994530942f + logf(l_ex) : NEG_INF;
+  return true;
+}
+
+// The softmax role: the CTA's work items in turn.
+template <bool BF16, bool ADAPTIVE>
+__device__ void pp_softmax(const AttnParams& p, PPBars& bars, uint32_t tbase, const WaitCtx wc) {
+  uint32_t cs = 0, c16 = 0, cvv = 0;
+  uint32_t raw[PPCfg::BN];
+  for (int it = 0;; ++it) {
+    const int item = pp_item(p, it);
+    if (item < 0) break;
+    const PPGeo g = pp_geo(p, item);
+    if (!pp_softmax_item<BF16, ADAPTIVE>(p, g, bars, tbase, wc, it, cs, c16, cvv, raw)) break;
+  }
 }
 
 // ------------------------------------------------------------------ kernel ------------
@@ -778,6 +860,7 @@ __global__ void __launch_bounds__(PPCfg::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
+    mbar_init(&bars.q_empty, 1);
     for (int s = 0; s < C::NS8; ++s) {
       mbar_init(&bars.full8[s], 1);
       mbar_init(&bars.empty8[s], 1);
@@ -793,14 +876,9 @@ __global__ void __launch_bounds__(PPCfg::THREADS, 1)
       mbar_init(&bars.p_half[x], 4);
       mbar_init(&bars.p_full[x], 4);
       mbar_init(&bars.o_done[x], 1);
+      mbar_init(&bars.o_free[x], 4);
     }
     mbar_init(&bars.drain, 1);
-    const PPGeo g0 = pp_geo(p);
-    for (int x = 0; x < 2; ++x) {
-      const MaskRow m = load_mask_row(p, g0, x);
-      bars.mask[x][0] = m.w0;
-      bars.mask[x][1] = m.w1;
-    }
     bars.abort = 0;
     fence_mbarrier_init();
   }
@@ -816,20 +894,17 @@ __global__ void __launch_bounds__(PPCfg::THREADS, 1)
   // Register split within the launch allotment of 384 x 168: the control warpgroup gives
   // back to 104 per thread, the two softmax warpgroups grow to 200
   // (128 * 104 + 256 * 200 = 64512 = 384 * 168).
+  // Every role walks the same sequence of work items (pp_item) and derives each item's geometry
+  // itself.
   if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory");
-    // each role derives the tile geometry itself: nothing computed before the role split stays
-    // live in the smaller register budget of the other roles
-    const PPGeo g = pp_geo(p);
-    pp_softmax<BF16, ADAPTIVE>(p, g, smem, bars, tbase, wc);
+    pp_softmax<BF16, ADAPTIVE>(p, bars, tbase, wc);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 104;\n" ::: "memory");
     if (warp == 8) {
-      const PPGeo g = pp_geo(p);
-      if ((threadIdx.x & 31) == 0 && g.n > 0) pp_producer(p, g, smem, bars, wc);
+      if ((threadIdx.x & 31) == 0) pp_producer(p, smem, bars, wc);
     } else if (warp == 9) {
-      const PPGeo g = pp_geo(p);
-      if (g.n > 0) pp_mma(p, g, smem, bars, tbase, wc);
+      pp_mma<BF16, ADAPTIVE>(p, smem, bars, tbase, wc);
     }
   }
   tc_fence_before();

@@ -347,7 +347,12 @@ int attn_q8(const void* q, const void* k, const void* v, const void* q8, const v
     LAMP_CUDA(cudaMemsetAsync(route_out, 0, static_cast<size_t>(BHq) * nqt * nkt, st), "memset route");
   if (D == 64) return launch_attn_cfg<Cfg64>(p, static_cast<int>(grid), st);
   if (D == 128 && !p.e4m3) {
-    const long long pgrid = static_cast<long long>(BHq) * ((nqt + 1) / 2);
+    // persistent CTAs: one per SM (the kernel fills the SM's shared and tensor memory), each
+    // walking its share of the (batch, head, query-tile pair) work items
+    const long long items = static_cast<long long>(BHq) * ((nqt + 1) / 2);
+    int nsm = 0;
+    if (int r = sm_count(&nsm)) return r;
+    const long long pgrid = std::min<long long>(items, nsm);
     return launch_attn_pp(p, static_cast<int>(pgrid), st);
   }
   if (D == 128) return launch_attn_cfg<Cfg128>(p, static_cast<int>(grid), st);
