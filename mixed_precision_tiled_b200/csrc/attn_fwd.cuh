@@ -268,16 +268,28 @@ __device__ void producer_role(const AttnParams& p, const Geo& g, uint8_t* smem, 
 
 // ------------------------------------------------------------------ MMA issuer --------
 
-template <class C>
+template <class C, bool BF16, bool E4M3>
 __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars& bars,
                          uint32_t tbase, const WaitCtx wc) {
+  // The whole warp runs this loop (warp-uniform state and descriptors); the elected lane issues
+  // the MMAs, commits and the one plain arrival.  Shared-memory descriptors are built once per
+  // operand region and advanced by constant offsets (16-byte units).
+  const bool leader = elect_one();
   const uint32_t sQ16 = smem_u32(smem + C::OFF_Q16);
   const uint32_t sQ8 = smem_u32(smem + C::OFF_Q8);
   const uint32_t slots = smem_u32(smem + C::OFF_SLOTS);
-  const uint32_t f16 = p.bf16 ? 1u : 0u;
-  const uint32_t id_s16 = idesc(1, f16, f16, 0, 0, C::BN, 128);
-  const uint32_t id_s8 = p.e4m3 ? idesc(1, 0, 0, 0, 0, C::BN, 128) : idesc(2, 1, 1, 0, 0, C::BN, 128);
-  const uint32_t id_pv = idesc(1, f16, f16, 0, 1, C::D, 128);
+  constexpr uint32_t f16 = BF16 ? 1u : 0u;
+  constexpr uint32_t id_s16 = idesc(1, f16, f16, 0, 0, C::BN, 128);
+  constexpr uint32_t id_s8 = E4M3 ? idesc(1, 0, 0, 0, 0, C::BN, 128) : idesc(2, 1, 1, 0, 0, C::BN, 128);
+  constexpr uint32_t id_pv = idesc(1, f16, f16, 0, 1, C::D, 128);
+  // 16-bit K-major operands: 128-byte rows (64 elements), row chunks of 64 elements MT * 128 or
+  // BN * 128 bytes apart; 8-bit operands likewise (64-byte rows with 64-byte swizzle at D = 64)
+  const uint64_t d_q16 = sdesc(sQ16, 16, 1024, SWZ_128B);
+  const uint64_t d_k16 = sdesc(slots, 16, 1024, SWZ_128B);
+  const uint64_t d_q8 = C::Q8_SW64 ? sdesc(sQ8, 16, 512, SWZ_64B) : sdesc(sQ8, 16, 1024, SWZ_128B);
+  const uint64_t d_k8 = C::Q8_SW64 ? sdesc(slots, 16, 512, SWZ_64B) : sdesc(slots, 16, 1024, SWZ_128B);
+  const uint64_t d_v = sdesc(slots, C::BN * 128, 1024, SWZ_128B);
+  constexpr uint64_t SLOT_D = C::SLOT_BYTES >> 4;
 
   uint32_t item = 0;
   uint32_t cv[2] = {0, 0}, cp[2] = {0, 0};
@@ -294,41 +306,46 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
   };
   auto issue_s = [&](int t, bool sixteen, int slot) {
     const uint32_t dS = tbase + static_cast<uint32_t>((t & 1) * C::BN);
-    const uint32_t ks = slots + slot * C::SLOT_BYTES;
     if (sixteen) {
+      const uint64_t kb = d_k16 + slot * SLOT_D;
+      if (leader) {
 #pragma unroll
-      for (int s = 0; s < C::D / 16; ++s) {
-        const int c = s >> 2, off = (s & 3) * 32;
-        const uint64_t a = sdesc(sQ16 + c * C::MT * 128 + off, 16, 1024, SWZ_128B);
-        const uint64_t b = sdesc(ks + c * C::BN * 128 + off, 16, 1024, SWZ_128B);
-        mma_f16_ss(dS, a, b, id_s16, s > 0 ? 1u : 0u);
+        for (int s = 0; s < C::D / 16; ++s) {
+          const uint64_t qo = static_cast<uint64_t>((s >> 2) * ((C::MT * 128) >> 4) + (s & 3) * 2);
+          const uint64_t ko = static_cast<uint64_t>((s >> 2) * ((C::BN * 128) >> 4) + (s & 3) * 2);
+          mma_f16_ss(dS, d_q16 + qo, kb + ko, id_s16, s > 0 ? 1u : 0u);
+        }
       }
     } else {
+      const uint64_t kb = d_k8 + slot * SLOT_D;
+      if (leader) {
 #pragma unroll
-      for (int s = 0; s < C::D / 32; ++s) {
-        uint64_t a, b;
-        if (C::Q8_SW64) {
-          a = sdesc(sQ8 + s * 32, 16, 512, SWZ_64B);
-          b = sdesc(ks + s * 32, 16, 512, SWZ_64B);
-        } else {
-          const int c = s >> 2, off = (s & 3) * 32;
-          a = sdesc(sQ8 + c * C::MT * 128 + off, 16, 1024, SWZ_128B);
-          b = sdesc(ks + c * C::BN * 128 + off, 16, 1024, SWZ_128B);
+        for (int s = 0; s < C::D / 32; ++s) {
+          uint64_t qo, ko;
+          if (C::Q8_SW64) {
+            qo = ko = static_cast<uint64_t>(s * 2);
+          } else {
+            qo = static_cast<uint64_t>((s >> 2) * ((C::MT * 128) >> 4) + (s & 3) * 2);
+            ko = static_cast<uint64_t>((s >> 2) * ((C::BN * 128) >> 4) + (s & 3) * 2);
+          }
+          if (E4M3)
+            mma_f8_ss(dS, d_q8 + qo, kb + ko, id_s8, s > 0 ? 1u : 0u);
+          else
+            mma_i8_ss(dS, d_q8 + qo, kb + ko, id_s8, s > 0 ? 1u : 0u);
         }
-        if (p.e4m3)
-          mma_f8_ss(dS, a, b, id_s8, s > 0 ? 1u : 0u);
-        else
-          mma_i8_ss(dS, a, b, id_s8, s > 0 ? 1u : 0u);
       }
     }
+  };
+  auto commit = [&](uint64_t* bar) {
+    if (leader) tc_commit(bar);
   };
 
   Plan cur = make_plan<C>(p, g, g.kt_lo);
   int slot = 0;
   if (ok && (ok = take(slot))) {
     issue_s(0, cur.first16, slot);
-    tc_commit(&bars.s_full[0]);
-    tc_commit(&bars.empty[slot]);
+    commit(&bars.s_full[0]);
+    commit(&bars.empty[slot]);
   }
   for (int t = 0; ok && t < g.n; ++t) {
     const int bsel = t & 1;
@@ -337,8 +354,8 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
       nxt = make_plan<C>(p, g, g.kt_lo + t + 1);
       if (!(ok = take(slot))) break;
       issue_s(t + 1, nxt.first16, slot);
-      tc_commit(&bars.s_full[(t + 1) & 1]);
-      tc_commit(&bars.empty[slot]);
+      commit(&bars.s_full[(t + 1) & 1]);
+      commit(&bars.empty[slot]);
     }
     if (cur.two_phase) {
       int slot16;
@@ -355,9 +372,9 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
       }
       if (s16) {
         issue_s(t, true, slot16);
-        tc_commit(&bars.s16_full[bsel]);
-        tc_commit(&bars.empty[slot16]);
-      } else {
+        commit(&bars.s16_full[bsel]);
+        commit(&bars.empty[slot16]);
+      } else if (leader) {
         mbar_arrive(&bars.empty[slot16]);
       }
     }
@@ -366,36 +383,84 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
     tc_fence_after();
     int slotv;
     if (!(ok = take(slotv))) break;
-    const uint32_t vs = slots + slotv * C::SLOT_BYTES;
+    const uint64_t vb = d_v + slotv * SLOT_D;
     const uint32_t pt = tbase + static_cast<uint32_t>(bsel * C::BN);
+    if (leader) {
 #pragma unroll
-    for (int s = 0; s < C::BN / 16; ++s) {
-      const uint64_t b = sdesc(vs + s * 16 * 128, C::BN * 128, 1024, SWZ_128B);
-      mma_f16_ts(tbase + C::TMEM_O, pt + s * 8, b, id_pv, (t > 0 || s > 0) ? 1u : 0u);
+      for (int s = 0; s < C::BN / 16; ++s)
+        mma_f16_ts(tbase + C::TMEM_O, pt + s * 8, vb + static_cast<uint64_t>(s * ((16 * 128) >> 4)),
+                   id_pv, (t > 0 || s > 0) ? 1u : 0u);
     }
-    tc_commit(&bars.o_done);
-    tc_commit(&bars.empty[slotv]);
+    commit(&bars.o_done);
+    commit(&bars.empty[slotv]);
     cur = nxt;
   }
   // Every MMA issued by this thread must complete before the TMEM is released.
-  tc_commit(&bars.drain);
+  commit(&bars.drain);
   const WaitCtx drain{0u, 50000u};  // no abort word: in-flight work always completes
   mbar_wait(&bars.drain, 0, drain, W_DRAIN);
 }
 
-// ------------------------------------------------------------------ softmax -----------
-
-// All 32 lanes poll the barrier; the result is made warp-uniform (and the warp reconverged)
-// before any warp-collective tcgen05 instruction follows.
+// Bounded wait by a whole warp: true only if every lane saw the phase complete.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtx wc,
                                           uint32_t where) {
   const bool ok = mbar_wait(bar, parity, wc, where);
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
-template <class C>
+// Packed f32x2 helpers and the mixed-precision adds of the softmax.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// acc + the low / high 16-bit half of a packed pair (bf16 or fp16), one rounding: sums the
+// rounded P values as the P.V MMA sees them, without unpacking them.
+template <bool BF16>
+__device__ __forceinline__ float add_lo16(float acc, uint32_t pk) {
+  float r;
+  if (BF16) asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.bf16 %0, lo, %2;\n\t}" : "=f"(r) : "r"(pk), "f"(acc));
+  else asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.f16 %0, lo, %2;\n\t}" : "=f"(r) : "r"(pk), "f"(acc));
+  return r;
+}
+template <bool BF16>
+__device__ __forceinline__ float add_hi16(float acc, uint32_t pk) {
+  float r;
+  if (BF16) asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.bf16 %0, hi, %2;\n\t}" : "=f"(r) : "r"(pk), "f"(acc));
+  else asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.f16 %0, hi, %2;\n\t}" : "=f"(r) : "r"(pk), "f"(acc));
+  return r;
+}
+
+// One thread per row of the 128-row MMA tile (the TMEM lane).  Per key tile: read S, turn it
+// into fp32 values of the raw product (exact int32 -> fp32 for INT8 tiles; E4M3 and 16-bit
+// tiles accumulate in fp32), mask, take the row max, vote (look-ahead rule), exponentiate
+// against a lazy reference max (it moves only when the row max exceeds it by more than 8 in
+// log2 units, so O is rarely rescaled), pack P as 16-bit pairs into the tile's S columns
+// (each 32-column chunk stored when ready), and keep two row sums: of the exact p (for lse)
+// and of the rounded p that the P.V MMA multiplies (for O).
+template <class C, bool BF16, bool E4M3>
 __device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint32_t tbase,
                              const WaitCtx wc) {
+  constexpr int N = C::BN;
+  constexpr float RESCALE_THRESH = 8.0f;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = warp * 32 + lane;
   const int i = g.q0 + r;
@@ -409,32 +474,41 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint
   const float sq = (row_valid && qt_r < p.nqt) ? __ldg(p.q_scale + static_cast<size_t>(bh_q) * p.nqt + qt_r) : 0.0f;
   const float* ks_row = p.k_scale + static_cast<size_t>(g.b * p.Hkv + g.kvh) * p.nkt;
   const float NEG_INF = -__int_as_float(0x7f800000);
+  const float sq_scale = sq * p.scale_log2;
 
-  float m = NEG_INF, l_ex = 0.0f, l_rd = 0.0f;
+  float m_ref = NEG_INF;   // max used for the exponentials (lazy)
+  float m_true = NEG_INF;  // true running max of the used scores (look-ahead rule)
+  float l_ex = 0.0f, l_rd = 0.0f;
   uint32_t cs[2] = {0, 0}, c16[2] = {0, 0}, cv[2] = {0, 0};
   bool ok = true;
-  uint32_t sraw[C::BN];
+  uint32_t raw[N];
 
   auto load_s = [&](int bsel) {
 #pragma unroll
-    for (int c = 0; c < C::BN / 32; ++c) {
-      uint32_t (&dst)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sraw[c * 32]);
-      tmem_ld32(lane_base + static_cast<uint32_t>(bsel * C::BN + c * 32), dst);
-    }
+    for (int c = 0; c < N / 32; ++c)
+      tmem_ld32(lane_base + static_cast<uint32_t>(bsel * N + c * 32),
+                *reinterpret_cast<uint32_t(*)[32]>(&raw[c * 32]));
     tmem_wait_ld();
   };
-  auto mask_s = [&](int kt) {
-    const int j0 = kt * C::BN;
-    const bool full = row_valid && j0 >= lo_r && j0 + C::BN - 1 <= hi_r;
-    if (!full) {
+  auto int_to_float = [&]() {  // exact: |int32 product| < 2^22
 #pragma unroll
-      for (int c = 0; c < C::BN; ++c) {
-        const int j = j0 + c;
-        if (!row_valid || j < lo_r || j > hi_r) sraw[c] = __float_as_uint(NEG_INF);
-      }
-    }
+    for (int c = 0; c < N; ++c) raw[c] = __float_as_uint(static_cast<float>(static_cast<int>(raw[c])));
   };
-  auto sf = [&](int c) -> float { return __uint_as_float(sraw[c]); };
+  auto apply_mask = [&](int j0) {  // keep the row's visible columns, -inf elsewhere
+    const int a = row_valid ? lo_r - j0 : N;
+    const int b = row_valid ? hi_r - j0 : -1;
+#pragma unroll
+    for (int c = 0; c < N; ++c) raw[c] = (c < a || c > b) ? 0xff800000u : raw[c];
+  };
+  auto raw_max = [&]() -> float {
+    float m0 = NEG_INF, m1 = NEG_INF;
+#pragma unroll
+    for (int c = 0; c < N; c += 4) {
+      m0 = max3(m0, __uint_as_float(raw[c]), __uint_as_float(raw[c + 1]));
+      m1 = max3(m1, __uint_as_float(raw[c + 2]), __uint_as_float(raw[c + 3]));
+    }
+    return fmaxf(m0, m1);
+  };
 
   for (int t = 0; ok && t < g.n; ++t) {
     const int kt = g.kt_lo + t;
@@ -444,29 +518,20 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint
     ++cs[bsel];
     tc_fence_after();
     load_s(bsel);
-    if (!pl.first16) {
-      const float c8 = sq * __ldg(ks_row + kt) * p.scale_log2;
-      if (p.e4m3) {
-#pragma unroll
-        for (int c = 0; c < C::BN; ++c) sraw[c] = __float_as_uint(sf(c) * c8);
-      } else {
-#pragma unroll
-        for (int c = 0; c < C::BN; ++c)
-          sraw[c] = __float_as_uint(static_cast<float>(static_cast<int>(sraw[c])) * c8);
-      }
-    } else {
-#pragma unroll
-      for (int c = 0; c < C::BN; ++c) sraw[c] = __float_as_uint(sf(c) * p.scale_log2);
-    }
-    mask_s(kt);
+    const int j0 = kt * N;
+    const bool full = row_valid && j0 >= lo_r && j0 + N - 1 <= hi_r;
+    bool sixteen = pl.first16;
+    // (a zero block scale would turn masked -inf entries into NaN: keep it positive)
+    float cscale = sixteen ? p.scale_log2 : fmaxf(sq_scale * __ldg(ks_row + kt), 1e-30f);
+    if (!sixteen && !E4M3) int_to_float();
+    if (!full) apply_mask(j0);
+    float tmax = raw_max();
 
     bool my16 = pl.first16;
     if (pl.two_phase) {
       if (p.adaptive) {
-        float t8 = NEG_INF;
-#pragma unroll
-        for (int c = 0; c < C::BN; ++c) t8 = fmaxf(t8, sf(c));
-        const bool vote = (t8 != NEG_INF) && (t8 >= m - p.tau_log2);
+        const float t8 = (tmax == NEG_INF) ? NEG_INF : tmax * cscale;
+        const bool vote = (t8 != NEG_INF) && (t8 >= m_true - p.tau_log2);
         const uint32_t wv = __any_sync(0xFFFFFFFFu, vote) ? 1u : 0u;
         if (lane == 0) bars.votes[bsel][warp] = wv;
       }
@@ -496,9 +561,10 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint
         tc_fence_after();
         if (my16) {
           load_s(bsel);
-#pragma unroll
-          for (int c = 0; c < C::BN; ++c) sraw[c] = __float_as_uint(sf(c) * p.scale_log2);
-          mask_s(kt);
+          sixteen = true;
+          cscale = p.scale_log2;
+          if (!full) apply_mask(j0);
+          tmax = raw_max();
         }
       }
     }
@@ -509,60 +575,84 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint
       }
     }
 
-    // online softmax on the routed scores (log2 units)
-    float mt = NEG_INF;
-#pragma unroll
-    for (int c = 0; c < C::BN; ++c) mt = fmaxf(mt, sf(c));
-    const float m_new = fmaxf(m, mt);
-    const float m_use = (m_new == NEG_INF) ? 0.0f : m_new;
-    const float alpha = (m == m_new) ? 1.0f : ((m == NEG_INF) ? 0.0f : ex2(m - m_use));
-    float sum_ex = 0.0f, sum_rd = 0.0f;
-#pragma unroll
-    for (int c = 0; c < C::BN; c += 2) {
-      const float p0 = ex2(sf(c) - m_use);
-      const float p1 = ex2(sf(c + 1) - m_use);
-      sum_ex += p0 + p1;
-      uint32_t pk;
-      if (p.bf16) {
-        __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
-        sum_rd += __low2float(v2) + __high2float(v2);
-        pk = *reinterpret_cast<uint32_t*>(&v2);
-      } else {
-        __half2 v2 = __floats2half2_rn(p0, p1);
-        sum_rd += __low2float(v2) + __high2float(v2);
-        pk = *reinterpret_cast<uint32_t*>(&v2);
-      }
-      sraw[c >> 1] = pk;
-    }
-    l_ex = l_ex * alpha + sum_ex;
-    l_rd = l_rd * alpha + sum_rd;
+    const float tl = (tmax == NEG_INF) ? NEG_INF : tmax * cscale;  // log2 units
+    m_true = fmaxf(m_true, tl);
+    const bool move = (tl != NEG_INF) && (m_ref == NEG_INF || tl > m_ref + RESCALE_THRESH);
+    const float new_ref = move ? tl : m_ref;
+    const float alpha = move ? ((m_ref == NEG_INF) ? 0.0f : ex2(m_ref - new_ref)) : 1.0f;
+    l_ex *= alpha;
+    l_rd *= alpha;
+    m_ref = new_ref;
 
-    if (t > 0) {
+    // p = 2^(value * cscale - m_ref); masked entries hold -inf and give 0.  Each 32-column
+    // chunk of P (16 packed columns) is stored into this tile's S buffer as soon as it is ready:
+    // P.V of the tile two steps back, which read that buffer, completed before S was written.
+    const float mu = (m_ref == NEG_INF) ? 0.0f : m_ref;
+    const uint64_t c2 = f2_pack(cscale, cscale);
+    const uint64_t nb2 = f2_pack(-mu, -mu);
+    uint64_t se0 = 0, se1 = 0;
+    float sr0 = 0.f, sr1 = 0.f, sr2 = 0.f, sr3 = 0.f;
+#pragma unroll
+    for (int c = 0; c < N; c += 2) {
+      float x0, x1;
+      f2_unpack(f2_fma(f2_pack(__uint_as_float(raw[c]), __uint_as_float(raw[c + 1])), c2, nb2),
+                x0, x1);
+      const float p0 = ex2(x0), p1 = ex2(x1);
+      uint32_t pk;
+      if (BF16) {
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+        pk = *reinterpret_cast<uint32_t*>(&h2);
+      } else {
+        __half2 h2 = __floats2half2_rn(p0, p1);
+        pk = *reinterpret_cast<uint32_t*>(&h2);
+      }
+      if (c & 2) {
+        se1 = f2_add(se1, f2_pack(p0, p1));
+        sr2 = add_lo16<BF16>(sr2, pk);
+        sr3 = add_hi16<BF16>(sr3, pk);
+      } else {
+        se0 = f2_add(se0, f2_pack(p0, p1));
+        sr0 = add_lo16<BF16>(sr0, pk);
+        sr1 = add_hi16<BF16>(sr1, pk);
+      }
+      raw[c >> 1] = pk;
+      if ((c & 31) == 30)
+        tmem_st16(lane_base + static_cast<uint32_t>(bsel * N + (c >> 5) * 16), &raw[(c >> 5) * 16]);
+    }
+    {
+      float a0, a1;
+      f2_unpack(f2_add(se0, se1), a0, a1);
+      l_ex += a0 + a1;
+      l_rd += (sr0 + sr1) + (sr2 + sr3);
+    }
+
+    if (t > 0) {  // P.V of the previous tile has completed: O may be rescaled
       if (!(ok = warp_wait(&bars.o_done, (t - 1) & 1u, wc, W_ODONE))) break;
       tc_fence_after();
       if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+        const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll 1
-        for (int c = 0; c < C::D / 32; ++c) {
-          uint32_t ov[32];
-          const uint32_t ta = lane_base + static_cast<uint32_t>(C::TMEM_O + c * 32);
-          tmem_ld32(ta, ov);
+        for (int c = 0; c < C::D / 16; ++c) {
+          uint32_t ov[16];
+          const uint32_t ta = lane_base + static_cast<uint32_t>(C::TMEM_O + c * 16);
+          tmem_ld16(ta, ov);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          for (int e = 0; e < 16; e += 2) {
+            float lo, hi;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1])), a2, 0ull),
+                      lo, hi);
+            ov[e] = __float_as_uint(lo);
+            ov[e + 1] = __float_as_uint(hi);
+          }
           tmem_st16(ta, ov);
-          tmem_st16(ta + 16, ov + 16);
         }
-        tmem_wait_st();
       }
     }
-#pragma unroll
-    for (int c = 0; c < C::BN / 32; ++c)
-      tmem_st16(lane_base + static_cast<uint32_t>(bsel * C::BN + c * 16), &sraw[c * 16]);
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars.p_full[bsel]);
-    m = m_new;
   }
   if (!ok) return;
 
@@ -599,7 +689,7 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint
         for (int q = 0; q < 4; ++q) {
           const float a = __uint_as_float(ov[8 * e + 2 * q]) * inv;
           const float b2 = __uint_as_float(ov[8 * e + 2 * q + 1]) * inv;
-          if (p.bf16) {
+          if (BF16) {
             __nv_bfloat162 v2 = __floats2bfloat162_rn(a, b2);
             w[q] = *reinterpret_cast<uint32_t*>(&v2);
           } else {
@@ -613,13 +703,13 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint
   }
   if (row_valid && p.lse) {
     p.lse[static_cast<size_t>(bh_q) * p.Lq + i] =
-        (l_ex > 0.0f) ? m * 0.69314718055994530942f + logf(l_ex) : NEG_INF;
+        (l_ex > 0.0f) ? m_ref * 0.69314718055994530942f + logf(l_ex) : NEG_INF;
   }
 }
 
 // ------------------------------------------------------------------ kernel ------------
 
-template <class C>
+template <class C, bool BF16, bool E4M3>
 __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -658,9 +748,9 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const __grid_constant_
   if (warp == 4) {
     if ((threadIdx.x & 31) == 0 && g.n > 0) producer_role<C>(p, g, smem, bars, wc);
   } else if (warp == 5) {
-    if ((threadIdx.x & 31) == 0 && g.n > 0) mma_role<C>(p, g, smem, bars, tbase, wc);
+    if (g.n > 0) mma_role<C, BF16, E4M3>(p, g, smem, bars, tbase, wc);
   } else {
-    softmax_role<C>(p, g, bars, tbase, wc);
+    softmax_role<C, BF16, E4M3>(p, g, bars, tbase, wc);
   }
 
   tc_fence_before();

@@ -513,47 +513,8 @@ __device__ void pp_mma(const AttnParams& p, uint8_t* smem, PPBars& bars, uint32_
 
 // ------------------------------------------------------------------ softmax -----------
 
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ float max3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
+// (f32x2 helpers, max3 and the mixed-precision adds come from attn_fwd.cuh)
 
-
-// acc + the low / high 16-bit half of a packed pair (bf16 or fp16), one rounding: sums the
-// rounded P values as the P.V MMA sees them, without unpacking them.
-template <bool BF16>
-__device__ __forceinline__ float add_lo16(float acc, uint32_t pk) {
-  float r;
-  if (BF16) asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.bf16 %0, lo, %2;\n\t}" : "=f"(r) : "r"(pk), "f"(acc));
-  else asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.f16 %0, lo, %2;\n\t}" : "=f"(r) : "r"(pk), "f"(acc));
-  return r;
-}
-template <bool BF16>
-__device__ __forceinline__ float add_hi16(float acc, uint32_t pk) {
-  float r;
-  if (BF16) asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.bf16 %0, hi, %2;\n\t}" : "=f"(r) : "r"(pk), "f"(acc));
-  else asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.f16 %0, hi, %2;\n\t}" : "=f"(r) : "r"(pk), "f"(acc));
-  return r;
-}
 // A thread owns row r of query tile X.  Per key tile: read the row of S from TMEM, turn it
 // into fp32 values of the raw product (exact int32 -> fp32 for 8-bit tiles), mask, take the
 // row max, vote (look-ahead rule), exponentiate against the lazy reference max, pack P as
