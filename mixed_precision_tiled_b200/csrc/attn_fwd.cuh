@@ -10,17 +10,18 @@
 //
 // B200 design:
 //   * one CTA per (batch, head, 128-row query tile); grid ordered longest-first (causal);
-//   * warp 4 (one thread) streams Q16/Q8 once and then K8 / K16 / V tiles with TMA into a
+//   * warp 8 (one thread) streams Q16/Q8 once and then K8 / K16 / V tiles with TMA into a
 //     ring of shared-memory slots (128-byte or 64-byte swizzled, the layouts the tensor core
 //     reads), each slot guarded by full/empty mbarriers;
-//   * warp 5 (one thread) issues tcgen05 MMAs: S = Q8 K8^T (kind::i8 into int32 TMEM or
-//     kind::f8f6f4 into fp32 TMEM), S = Q16 K16^T (kind::f16), O += P V with P read from TMEM;
-//     the S buffer is double-buffered so S(t+1) runs on the tensor core while rows of S(t)
-//     are in the softmax;
-//   * warps 0-3 own one query row per thread (TMEM lane = row): they read S from TMEM,
-//     dequantise, mask, vote on the look-ahead rule, run the online softmax (MUFU ex2), store
-//     P as packed 16-bit pairs into the S columns, rescale O in TMEM when the row max grows,
-//     and write O / lse at the end;
+//   * warp 9 issues tcgen05 MMAs (the whole warp runs the loop, one elected lane issues):
+//     S = Q8 K8^T (kind::i8 into int32 TMEM or kind::f8f6f4 into fp32 TMEM), S = Q16 K16^T
+//     (kind::f16), O += P V with P read from TMEM; the S buffer is double-buffered so S(t+1)
+//     runs on the tensor core while rows of S(t) are in the softmax;
+//   * warps 0-7 own one query row per two threads (TMEM lane = row; warps 0-3 columns 0..BN/2,
+//     warps 4-7 the rest): they read S from TMEM, dequantise, mask, exchange the half-row
+//     maxima, vote on the look-ahead rule, run the online softmax (MUFU ex2, lazy reference
+//     max), store P as packed 16-bit pairs into the S columns, rescale O in TMEM when the
+//     reference moves, and write O / lse at the end;
 //   * routing tiles of 64 query rows (D = 64, 256) are stacked two per 128-row MMA; a key
 //     tile whose two halves need different precisions runs the 8-bit MMA first, then the
 //     16-bit MMA into the same TMEM columns after every row has read its 8-bit scores.
@@ -40,7 +41,7 @@ namespace lamp {
 // where-codes recorded with a timeout (bits 8..15 of the error word)
 enum : uint32_t {
   W_QFULL = 1, W_EMPTY = 2, W_FULL = 3, W_SFULL = 4, W_S16 = 5, W_VOTE = 6, W_PFULL = 7,
-  W_ODONE = 8, W_DRAIN = 9, W_SELFTEST = 10
+  W_ODONE = 8, W_DRAIN = 9, W_SELFTEST = 10, W_XCH = 11
 };
 
 struct AttnParams {
@@ -84,7 +85,9 @@ struct AttnCfg {
   static constexpr int OFF_SLOTS = Q16_BYTES + Q8_BYTES;
   static constexpr int OFF_BAR = OFF_SLOTS + NS * SLOT_BYTES;
   static constexpr int BAR_BYTES = 512;
-  static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
+  static constexpr int OFF_XCH = OFF_BAR + BAR_BYTES;  // row-pair exchange: float [2][2][MT]
+  static constexpr int SMEM_BYTES = OFF_XCH + 2 * 2 * MT * 4;  // dynamic base is 1024-aligned
+  static constexpr int THREADS = 320;  // 8 softmax warps (two per row), producer, MMA
   static_assert(OFF_Q8 % 1024 == 0 && OFF_SLOTS % 1024 == 0 && SLOT_BYTES % 1024 == 0, "align");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   static_assert(2 * BN + D <= 512, "tmem");
@@ -102,8 +105,10 @@ struct Bars {
   uint64_t drain;
   uint32_t tmem_base;
   uint32_t abort;
-  uint32_t votes[2][4];
+  uint32_t votes[2][8];
+  uint64_t xbar[4];  // row-pair exchange of lane quadrant q (64 arrivals)
 };
+static_assert(sizeof(Bars) <= 512, "barrier block");
 
 // Per-key-tile routing plan, computed identically by the three roles.
 struct Plan {
@@ -366,7 +371,10 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
       bool s16;
       if (p.adaptive) {
         const volatile uint32_t* vv = bars.votes[bsel];
-        s16 = (vv[0] | vv[1] | vv[2] | vv[3]) != 0;
+        uint32_t any = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) any |= vv[w];
+        s16 = any != 0;
       } else {
         s16 = true;
       }
@@ -385,11 +393,14 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
     if (!(ok = take(slotv))) break;
     const uint64_t vb = d_v + slotv * SLOT_D;
     const uint32_t pt = tbase + static_cast<uint32_t>(bsel * C::BN);
+    // P (16-bit pairs): each softmax column half packs its keys into the first half of its own
+    // S columns, so keys [BN/2 * h, BN/2 * (h + 1)) sit at columns BN/2 * h + [0, BN/4)
+    constexpr int SPH = C::BN / 32;  // K steps of 16 keys per column half
     if (leader) {
 #pragma unroll
       for (int s = 0; s < C::BN / 16; ++s)
-        mma_f16_ts(tbase + C::TMEM_O, pt + s * 8, vb + static_cast<uint64_t>(s * ((16 * 128) >> 4)),
-                   id_pv, (t > 0 || s > 0) ? 1u : 0u);
+        mma_f16_ts(tbase + C::TMEM_O, pt + (s / SPH) * (C::BN / 2) + (s % SPH) * 8,
+                   vb + static_cast<uint64_t>(s * ((16 * 128) >> 4)), id_pv, (t > 0 || s > 0) ? 1u : 0u);
     }
     commit(&bars.o_done);
     commit(&bars.empty[slotv]);
@@ -449,61 +460,80 @@ __device__ __forceinline__ float add_hi16(float acc, uint32_t pk) {
   return r;
 }
 
-// One thread per row of the 128-row MMA tile (the TMEM lane).  Per key tile: read S, turn it
-// into fp32 values of the raw product (exact int32 -> fp32 for INT8 tiles; E4M3 and 16-bit
-// tiles accumulate in fp32), mask, take the row max, vote (look-ahead rule), exponentiate
-// against a lazy reference max (it moves only when the row max exceeds it by more than 8 in
-// log2 units, so O is rarely rescaled), pack P as 16-bit pairs into the tile's S columns
-// (each 32-column chunk stored when ready), and keep two row sums: of the exact p (for lse)
-// and of the rounded p that the P.V MMA multiplies (for O).
+// Two threads per row of the 128-row MMA tile (the TMEM lane): the thread of column half h
+// (warps 4h .. 4h + 3) handles key columns [BN/2 * h, BN/2 * (h + 1)) of each key tile.  Per
+// key tile: read its half row of S, turn it into fp32 values of the raw product (exact int32 ->
+// fp32 for INT8 tiles; E4M3 and 16-bit tiles accumulate in fp32), mask, take the half-row max
+// and combine it with the partner's through shared memory (an mbarrier per lane quadrant, so
+// that every wait is bounded; the exchange slots alternate with the S buffer), vote (look-ahead
+// rule), exponentiate against a lazy reference max (it moves only when the row max exceeds it
+// by more than 8 in log2 units, so O is rarely rescaled), pack P as 16-bit pairs into the first
+// half of the thread's own S columns (each 32-column chunk stored when ready), and keep two
+// partial row sums: of the exact p (for lse) and of the rounded p that the P.V MMA multiplies
+// (for O).  Both threads of a row take identical decisions from identical inputs.
 template <class C, bool BF16, bool E4M3>
-__device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint32_t tbase,
-                             const WaitCtx wc) {
-  constexpr int N = C::BN;
+__device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars& bars,
+                             uint32_t tbase, const WaitCtx wc) {
+  constexpr int N = C::BN, NH = C::BN / 2;
   constexpr float RESCALE_THRESH = 8.0f;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = warp * 32 + lane;
+  const int h = warp >> 2;   // column half
+  const int q4 = warp & 3;   // TMEM lane quadrant
+  const int r = q4 * 32 + lane;
   const int i = g.q0 + r;
   const bool row_valid = i < p.Lq;
   const int hh = C::STACK ? (r >> 6) : 0;
   const int qt_r = C::STACK ? 2 * g.ct + hh : g.ct;
   const int bh_q = g.b * p.H + g.h;
-  const uint32_t lane_base = tbase + (static_cast<uint32_t>(warp * 32) << 16);
+  const uint32_t lane_base = tbase + (static_cast<uint32_t>(q4 * 32) << 16);
   int lo_r = 1, hi_r = 0;
   if (row_valid) visible_range(p, i, lo_r, hi_r);
   const float sq = (row_valid && qt_r < p.nqt) ? __ldg(p.q_scale + static_cast<size_t>(bh_q) * p.nqt + qt_r) : 0.0f;
   const float* ks_row = p.k_scale + static_cast<size_t>(g.b * p.Hkv + g.kvh) * p.nkt;
   const float NEG_INF = -__int_as_float(0x7f800000);
   const float sq_scale = sq * p.scale_log2;
+  const uint32_t xch = smem_u32(smem + C::OFF_XCH) + static_cast<uint32_t>(r * 4);
+  uint64_t* xbar = &bars.xbar[q4];
 
   float m_ref = NEG_INF;   // max used for the exponentials (lazy)
   float m_true = NEG_INF;  // true running max of the used scores (look-ahead rule)
   float l_ex = 0.0f, l_rd = 0.0f;
-  uint32_t cs[2] = {0, 0}, c16[2] = {0, 0}, cv[2] = {0, 0};
+  uint32_t cs[2] = {0, 0}, c16[2] = {0, 0}, cv[2] = {0, 0}, nx = 0;
   bool ok = true;
-  uint32_t raw[N];
+  uint32_t raw[NH];
 
+  // Publish v in this thread's exchange slot of parity `par` and return the partner's value.
+  // The slot's previous value (two key tiles back) has been read: the partner read it before
+  // it published that tile's P, which the MMA warp waited for before issuing this tile's S.
+  auto exchange = [&](int par, float v, float& other) -> bool {
+    sts_u32(xch + static_cast<uint32_t>((par * 2 + h) * C::MT * 4), __float_as_uint(v));
+    mbar_arrive(xbar);
+    if (!mbar_wait(xbar, nx & 1u, wc, W_XCH)) return false;
+    ++nx;
+    other = __uint_as_float(lds_u32(xch + static_cast<uint32_t>((par * 2 + (h ^ 1)) * C::MT * 4)));
+    return true;
+  };
   auto load_s = [&](int bsel) {
 #pragma unroll
-    for (int c = 0; c < N / 32; ++c)
-      tmem_ld32(lane_base + static_cast<uint32_t>(bsel * N + c * 32),
+    for (int c = 0; c < NH / 32; ++c)
+      tmem_ld32(lane_base + static_cast<uint32_t>(bsel * N + h * NH + c * 32),
                 *reinterpret_cast<uint32_t(*)[32]>(&raw[c * 32]));
     tmem_wait_ld();
   };
   auto int_to_float = [&]() {  // exact: |int32 product| < 2^22
 #pragma unroll
-    for (int c = 0; c < N; ++c) raw[c] = __float_as_uint(static_cast<float>(static_cast<int>(raw[c])));
+    for (int c = 0; c < NH; ++c) raw[c] = __float_as_uint(static_cast<float>(static_cast<int>(raw[c])));
   };
-  auto apply_mask = [&](int j0) {  // keep the row's visible columns, -inf elsewhere
-    const int a = row_valid ? lo_r - j0 : N;
+  auto apply_mask = [&](int j0) {  // keep the row's visible columns of this half, -inf elsewhere
+    const int a = row_valid ? lo_r - j0 : NH;
     const int b = row_valid ? hi_r - j0 : -1;
 #pragma unroll
-    for (int c = 0; c < N; ++c) raw[c] = (c < a || c > b) ? 0xff800000u : raw[c];
+    for (int c = 0; c < NH; ++c) raw[c] = (c < a || c > b) ? 0xff800000u : raw[c];
   };
   auto raw_max = [&]() -> float {
     float m0 = NEG_INF, m1 = NEG_INF;
 #pragma unroll
-    for (int c = 0; c < N; c += 4) {
+    for (int c = 0; c < NH; c += 4) {
       m0 = max3(m0, __uint_as_float(raw[c]), __uint_as_float(raw[c + 1]));
       m1 = max3(m1, __uint_as_float(raw[c + 2]), __uint_as_float(raw[c + 3]));
     }
@@ -518,14 +548,16 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint
     ++cs[bsel];
     tc_fence_after();
     load_s(bsel);
-    const int j0 = kt * N;
-    const bool full = row_valid && j0 >= lo_r && j0 + N - 1 <= hi_r;
+    const int j0 = kt * N + h * NH;
+    const bool full = row_valid && j0 >= lo_r && j0 + NH - 1 <= hi_r;
     bool sixteen = pl.first16;
     // (a zero block scale would turn masked -inf entries into NaN: keep it positive)
     float cscale = sixteen ? p.scale_log2 : fmaxf(sq_scale * __ldg(ks_row + kt), 1e-30f);
     if (!sixteen && !E4M3) int_to_float();
     if (!full) apply_mask(j0);
-    float tmax = raw_max();
+    float tmax = raw_max(), other;
+    if (!(ok = exchange(bsel, tmax, other))) break;
+    tmax = fmaxf(tmax, other);
 
     bool my16 = pl.first16;
     if (pl.two_phase) {
@@ -543,11 +575,11 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint
       bool f[2];
       if (p.adaptive) {
         const volatile uint32_t* vv = bars.votes[bsel];
-        if (C::STACK) {
-          f[0] = (vv[0] | vv[1]) != 0;
-          f[1] = (vv[2] | vv[3]) != 0;
+        if (C::STACK) {  // rows 0-63: quadrants 0, 1; rows 64-127: quadrants 2, 3
+          f[0] = (vv[0] | vv[1] | vv[4] | vv[5]) != 0;
+          f[1] = (vv[2] | vv[3] | vv[6] | vv[7]) != 0;
         } else {
-          f[0] = f[1] = (vv[0] | vv[1] | vv[2] | vv[3]) != 0;
+          f[0] = f[1] = (vv[0] | vv[1] | vv[2] | vv[3] | vv[4] | vv[5] | vv[6] | vv[7]) != 0;
         }
       } else {
         f[0] = pl.live[0] && pl.b16[0];
@@ -559,16 +591,18 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint
         if (!(ok = warp_wait(&bars.s16_full[bsel], c16[bsel] & 1u, wc, W_S16))) break;
         ++c16[bsel];
         tc_fence_after();
-        if (my16) {
+        if (my16) {  // (both threads of a row take this branch or neither)
           load_s(bsel);
           sixteen = true;
           cscale = p.scale_log2;
           if (!full) apply_mask(j0);
           tmax = raw_max();
+          if (!(ok = exchange(bsel, tmax, other))) break;
+          tmax = fmaxf(tmax, other);
         }
       }
     }
-    if (p.route && lane == 0 && (warp == 0 || (C::STACK && warp == 2))) {
+    if (p.route && h == 0 && lane == 0 && (q4 == 0 || (C::STACK && q4 == 2))) {
       if (pl.live[hh]) {
         const uint8_t v = my16 ? (pl.two_phase && p.adaptive ? 3 : 2) : 1;
         p.route[(static_cast<size_t>(bh_q) * p.nqt + qt_r) * p.nkt + kt] = v;
@@ -585,15 +619,15 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint
     m_ref = new_ref;
 
     // p = 2^(value * cscale - m_ref); masked entries hold -inf and give 0.  Each 32-column
-    // chunk of P (16 packed columns) is stored into this tile's S buffer as soon as it is ready:
-    // P.V of the tile two steps back, which read that buffer, completed before S was written.
+    // chunk of P (16 packed columns) goes into this tile's S buffer as soon as it is ready: P.V
+    // of the tile two steps back, which read that buffer, completed before S was written.
     const float mu = (m_ref == NEG_INF) ? 0.0f : m_ref;
     const uint64_t c2 = f2_pack(cscale, cscale);
     const uint64_t nb2 = f2_pack(-mu, -mu);
     uint64_t se0 = 0, se1 = 0;
     float sr0 = 0.f, sr1 = 0.f, sr2 = 0.f, sr3 = 0.f;
 #pragma unroll
-    for (int c = 0; c < N; c += 2) {
+    for (int c = 0; c < NH; c += 2) {
       float x0, x1;
       f2_unpack(f2_fma(f2_pack(__uint_as_float(raw[c]), __uint_as_float(raw[c + 1])), c2, nb2),
                 x0, x1);
@@ -617,7 +651,8 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint
       }
       raw[c >> 1] = pk;
       if ((c & 31) == 30)
-        tmem_st16(lane_base + static_cast<uint32_t>(bsel * N + (c >> 5) * 16), &raw[(c >> 5) * 16]);
+        tmem_st16(lane_base + static_cast<uint32_t>(bsel * N + h * NH + (c >> 5) * 16),
+                  &raw[(c >> 5) * 16]);
     }
     {
       float a0, a1;
@@ -629,12 +664,12 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint
     if (t > 0) {  // P.V of the previous tile has completed: O may be rescaled
       if (!(ok = warp_wait(&bars.o_done, (t - 1) & 1u, wc, W_ODONE))) break;
       tc_fence_after();
-      if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+      if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {  // each thread rescales its half of O
         const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll 1
-        for (int c = 0; c < C::D / 16; ++c) {
+        for (int c = 0; c < C::D / 32; ++c) {
           uint32_t ov[16];
-          const uint32_t ta = lane_base + static_cast<uint32_t>(C::TMEM_O + c * 16);
+          const uint32_t ta = lane_base + static_cast<uint32_t>(C::TMEM_O + h * (C::D / 2) + c * 16);
           tmem_ld16(ta, ov);
           tmem_wait_ld();
 #pragma unroll
@@ -656,18 +691,27 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint
   }
   if (!ok) return;
 
-  // epilogue: O / l and lse
+  // epilogue: combine the two halves' row sums, then O / l and lse
   if (g.n > 0) {
     if (!warp_wait(&bars.o_done, (g.n - 1) & 1u, wc, W_ODONE)) return;
     tc_fence_after();
   }
-  const float inv = (l_rd > 0.0f) ? 1.0f / l_rd : 0.0f;
-  const size_t orow = (static_cast<size_t>(bh_q) * p.Lq + (row_valid ? i : 0)) * C::D;
+  const int par = g.n & 1;  // the exchange slots of parity n & 1 were last read two tiles back
+  float other_rd, other_ex;
+  if (!exchange(par, l_rd, other_rd)) return;
+  mbar_arrive(xbar);  // a phase without a write: both partners have read the l_rd slots
+  if (!mbar_wait(xbar, nx & 1u, wc, W_XCH)) return;
+  ++nx;
+  if (!exchange(par, l_ex, other_ex)) return;
+  const float l_rd_t = l_rd + other_rd, l_ex_t = l_ex + other_ex;
+  const float inv = (l_rd_t > 0.0f) ? 1.0f / l_rd_t : 0.0f;
+  constexpr int DH = C::D / 2;
+  const size_t orow = (static_cast<size_t>(bh_q) * p.Lq + (row_valid ? i : 0)) * C::D + h * DH;
 #pragma unroll 1
-  for (int c = 0; c < C::D / 32; ++c) {
+  for (int c = 0; c < DH / 32; ++c) {
     uint32_t ov[32];
     if (g.n > 0) {
-      tmem_ld32(lane_base + static_cast<uint32_t>(C::TMEM_O + c * 32), ov);
+      tmem_ld32(lane_base + static_cast<uint32_t>(C::TMEM_O + h * DH + c * 32), ov);
       tmem_wait_ld();
     } else {
 #pragma unroll
@@ -701,19 +745,21 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, Bars& bars, uint
       }
     }
   }
-  if (row_valid && p.lse) {
+  if (h == 0 && row_valid && p.lse) {
     p.lse[static_cast<size_t>(bh_q) * p.Lq + i] =
-        (l_ex > 0.0f) ? m_ref * 0.69314718055994530942f + logf(l_ex) : NEG_INF;
+        (l_ex_t > 0.0f) ? m_ref * 0.69314718055994530942f + logf(l_ex_t) : NEG_INF;
   }
 }
 
 // ------------------------------------------------------------------ kernel ------------
 
 template <class C, bool BF16, bool E4M3>
-__global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+__global__ void __launch_bounds__(C::THREADS, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0) {  // the layouts need a 1024-aligned base
+    if (threadIdx.x == 0) atomicOr(&g_lamp_error, 0x4u);
+    return;
+  }
   Bars& bars = *reinterpret_cast<Bars*>(smem + C::OFF_BAR);
   const int warp = threadIdx.x >> 5;
   const Geo g = make_geo<C>(p);
@@ -727,15 +773,16 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const __grid_constant_
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars.s_full[b], 1);
       mbar_init(&bars.s16_full[b], 1);
-      mbar_init(&bars.vote[b], 4);
-      mbar_init(&bars.p_full[b], 4);
+      mbar_init(&bars.vote[b], 8);
+      mbar_init(&bars.p_full[b], 8);
     }
     mbar_init(&bars.o_done, 1);
     mbar_init(&bars.drain, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&bars.xbar[q], 64);
     bars.abort = 0;
     fence_mbarrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(&bars.tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -745,18 +792,18 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const __grid_constant_
   const uint32_t tbase = bars.tmem_base;
   const WaitCtx wc{smem_u32(&bars.abort), static_cast<uint32_t>(p.wait_ns / 1000)};
 
-  if (warp == 4) {
+  if (warp == 8) {
     if ((threadIdx.x & 31) == 0 && g.n > 0) producer_role<C>(p, g, smem, bars, wc);
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (g.n > 0) mma_role<C, BF16, E4M3>(p, g, smem, bars, tbase, wc);
   } else {
-    softmax_role<C, BF16, E4M3>(p, g, bars, tbase, wc);
+    softmax_role<C, BF16, E4M3>(p, g, smem, bars, tbase, wc);
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) {
+  if (warp == 9) {
     __syncwarp();
     tmem_dealloc(tbase, C::TMEM_COLS);
   }

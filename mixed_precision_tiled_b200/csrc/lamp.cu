@@ -246,7 +246,7 @@ int launch_attn_cfg_t(const lamp::AttnParams& p, int grid, cudaStream_t st) {
               "cudaFuncSetAttribute");
     attr_set[dev] = true;
   }
-  lamp::attn_fwd_kernel<C, BF16, E4M3><<<grid, 192, C::SMEM_BYTES, st>>>(p);
+  lamp::attn_fwd_kernel<C, BF16, E4M3><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(p);
   LAMP_CUDA(cudaGetLastError(), "attn_fwd_kernel launch");
   return LAMP_OK;
 }
