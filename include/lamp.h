@@ -21,7 +21,8 @@
  *     k_scale [B][Hkv][nKT]; mask_bits [B][H][nQT][W] uint64 words, bit g of a row at word
  *     g>>6, bit g&63 (LSB first).  nQT = ceil(Lq/BM), nKT = ceil(Lk/BN), W = ceil(nG/64),
  *     nG = ceil(nKT/group_tiles), with (BM, BN) from lamp_tile_shape(D).
- *   - q, k, v, q8, k8 must be 16-byte aligned (TMA); D must be 64, 128 or 256.
+ *   - q, k, v, q8, k8 must be 16-byte aligned (TMA) and o 32-byte aligned (32-byte stores);
+ *     D must be 64, 128 or 256.
  *   - Return value: LAMP_OK or an error code.  Arguments are checked synchronously before
  *     anything is launched; on error nothing is enqueued and lamp_last_error() describes the
  *     problem (thread-local string).  Device-side failures (a bounded wait in a kernel that

@@ -760,21 +760,23 @@ __device__ __forceinline__ bool pp_softmax_item(const AttnParams& p, const PPGeo
   const size_t orow = (static_cast<size_t>(bh_q) * p.Lq + (row_valid ? i : 0)) * C::D;
   if (row_valid &&
       lamp_chk(orow + C::D <= static_cast<size_t>(p.B) * p.H * p.Lq * C::D, 12)) {
+    // 32-byte stores: each thread writes whole sectors of its row
+    auto sc = [&](int e) { return __float_as_uint(__uint_as_float(raw[e]) * inv); };
     if (p.out_f32) {
-      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow);
+      float* dst = static_cast<float*>(p.o) + orow;
 #pragma unroll
-      for (int e = 0; e < C::D / 4; ++e)
-        dst[e] = make_float4(__uint_as_float(raw[4 * e]) * inv, __uint_as_float(raw[4 * e + 1]) * inv,
-                             __uint_as_float(raw[4 * e + 2]) * inv, __uint_as_float(raw[4 * e + 3]) * inv);
+      for (int e = 0; e < C::D; e += 8)
+        st_global_v8(dst + e, sc(e), sc(e + 1), sc(e + 2), sc(e + 3), sc(e + 4), sc(e + 5), sc(e + 6),
+                     sc(e + 7));
     } else {
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow);
+      uint16_t* dst = static_cast<uint16_t*>(p.o) + orow;
 #pragma unroll
-      for (int e = 0; e < C::D / 8; ++e) {
-        uint32_t w[4];
+      for (int e = 0; e < C::D; e += 16) {
+        uint32_t w[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float a = __uint_as_float(raw[8 * e + 2 * q]) * inv;
-          const float b2 = __uint_as_float(raw[8 * e + 2 * q + 1]) * inv;
+        for (int q = 0; q < 8; ++q) {
+          const float a = __uint_as_float(raw[e + 2 * q]) * inv;
+          const float b2 = __uint_as_float(raw[e + 2 * q + 1]) * inv;
           if (BF16) {
             __nv_bfloat162 v2 = __floats2bfloat162_rn(a, b2);
             w[q] = *reinterpret_cast<uint32_t*>(&v2);
@@ -783,7 +785,7 @@ __device__ __forceinline__ bool pp_softmax_item(const AttnParams& p, const PPGeo
             w[q] = *reinterpret_cast<uint32_t*>(&v2);
           }
         }
-        dst[e] = make_uint4(w[0], w[1], w[2], w[3]);
+        st_global_v8(dst + e, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
       }
     }
   }

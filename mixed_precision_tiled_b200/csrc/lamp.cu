@@ -48,6 +48,8 @@ int cuda_fail(cudaError_t e, const char* what) {
   } while (0)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// O is written with 32-byte stores
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 int tile_shape(int D, int* bm, int* bn) {
   if (D == 64) { *bm = 64; *bn = 64; return LAMP_OK; }
@@ -298,8 +300,8 @@ int attn_q8(const void* q, const void* k, const void* v, const void* q8, const v
   if (!q || !k || !v || !q8 || !k8 || !q_scale || !k_scale || !o)
     return fail(LAMP_ERR_INVALID, "null operand pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q8) || !aligned16(k8) ||
-      !aligned16(o))
-    return fail(LAMP_ERR_INVALID, "q, k, v, q8, k8 and o must be 16-byte aligned");
+      !aligned32(o))
+    return fail(LAMP_ERR_INVALID, "q, k, v, q8, k8 must be 16-byte and o 32-byte aligned");
   if (causal != 0 && causal != 1) return fail(LAMP_ERR_INVALID, "causal must be 0 or 1");
   if (window < 0) return fail(LAMP_ERR_INVALID, "window must be >= 0");
   if (window > 0 && !causal)
@@ -491,8 +493,8 @@ int lamp_attn_fwd(const void* q, const void* k, const void* v, void* o, float* l
   uint8_t* k8 = base + w.k8;
   float* qs = reinterpret_cast<float*>(base + w.qs);
   float* ks = reinterpret_cast<float*>(base + w.ks);
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
-    return fail(LAMP_ERR_INVALID, "q, k, v and o must be 16-byte aligned");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned32(o))
+    return fail(LAMP_ERR_INVALID, "q, k, v must be 16-byte and o 32-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((r = quant_qk(q, k, q8, k8, qs, ks, B, H, Hkv, Lq, Lk, D, mode, st))) return r;
   return attn_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D, causal, window, scale,
@@ -527,8 +529,8 @@ int lamp_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
   int r = check_sizes(B, H, Hkv, Lq, Lk, D);
   if (r) return r;
   if (!q || !k || !v || !o) return fail(LAMP_ERR_INVALID, "null operand pointer");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
-    return fail(LAMP_ERR_INVALID, "q, k, v and o must be 16-byte aligned");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned32(o))
+    return fail(LAMP_ERR_INVALID, "q, k, v must be 16-byte and o 32-byte aligned");
   const WsLayout w = ws_layout(B, H, Hkv, Lq, Lk, D);
   if (w.total > static_cast<size_t>(LAMP_NOALLOC_MAX_BYTES))
     return fail(LAMP_ERR_INVALID,

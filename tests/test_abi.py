@@ -76,6 +76,7 @@ def test_attn_fwd_rejects_bad_arguments_on_host(bad, code):
 
 @pytest.mark.parametrize("bad,code", [
     (dict(q=0x1001), mpt.LAMP_ERR_INVALID),            # misaligned
+    (dict(o=0x5010), mpt.LAMP_ERR_INVALID),            # O written with 32-byte stores
     (dict(causal=0, window=16), mpt.LAMP_ERR_UNSUPPORTED),
     (dict(window=-1), mpt.LAMP_ERR_INVALID),
     (dict(group_tiles=0), mpt.LAMP_ERR_INVALID),
