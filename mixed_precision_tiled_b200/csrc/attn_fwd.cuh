@@ -297,7 +297,9 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
   constexpr uint64_t SLOT_D = C::SLOT_BYTES >> 4;
 
   uint32_t item = 0;
-  uint32_t cv[2] = {0, 0}, cp[2] = {0, 0};
+  // phase bits per S buffer (bit b: buffer b) of the vote barriers; the P barrier of buffer b
+  // completes at every use, its phase is (t >> 1) & 1 (registers only: no indexed arrays)
+  uint32_t cvb = 0;
   bool ok = mbar_wait(&bars.q_full, 0, wc, W_QFULL);
   tc_fence_after();
 
@@ -365,8 +367,8 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
     if (cur.two_phase) {
       int slot16;
       if (!(ok = take(slot16))) break;
-      if (!(ok = mbar_wait(&bars.vote[bsel], cv[bsel] & 1u, wc, W_VOTE))) break;
-      ++cv[bsel];
+      if (!(ok = mbar_wait(&bars.vote[bsel], (cvb >> bsel) & 1u, wc, W_VOTE))) break;
+      cvb ^= 1u << bsel;
       tc_fence_after();
       bool s16;
       if (p.adaptive) {
@@ -386,8 +388,7 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
         mbar_arrive(&bars.empty[slot16]);
       }
     }
-    if (!(ok = mbar_wait(&bars.p_full[bsel], cp[bsel] & 1u, wc, W_PFULL))) break;
-    ++cp[bsel];
+    if (!(ok = mbar_wait(&bars.p_full[bsel], static_cast<uint32_t>(t >> 1) & 1u, wc, W_PFULL))) break;
     tc_fence_after();
     int slotv;
     if (!(ok = take(slotv))) break;
@@ -498,7 +499,9 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
   float m_ref = NEG_INF;   // max used for the exponentials (lazy)
   float m_true = NEG_INF;  // true running max of the used scores (look-ahead rule)
   float l_ex = 0.0f, l_rd = 0.0f;
-  uint32_t cs[2] = {0, 0}, c16[2] = {0, 0}, cv[2] = {0, 0}, nx = 0;
+  // phase bits per S buffer (bit b: buffer b) of the vote and 16-bit S barriers; the S barrier
+  // of buffer b completes at every use, its phase is (t >> 1) & 1
+  uint32_t cvb = 0, c16b = 0, nx = 0;
   bool ok = true;
   uint32_t raw[NH];
 
@@ -544,8 +547,7 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
     const int kt = g.kt_lo + t;
     const int bsel = t & 1;
     const Plan pl = make_plan<C>(p, g, kt);
-    if (!(ok = warp_wait(&bars.s_full[bsel], cs[bsel] & 1u, wc, W_SFULL))) break;
-    ++cs[bsel];
+    if (!(ok = warp_wait(&bars.s_full[bsel], static_cast<uint32_t>(t >> 1) & 1u, wc, W_SFULL))) break;
     tc_fence_after();
     load_s(bsel);
     const int j0 = kt * N + h * NH;
@@ -570,26 +572,26 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.vote[bsel]);
-      if (!(ok = warp_wait(&bars.vote[bsel], cv[bsel] & 1u, wc, W_VOTE))) break;
-      ++cv[bsel];
-      bool f[2];
+      if (!(ok = warp_wait(&bars.vote[bsel], (cvb >> bsel) & 1u, wc, W_VOTE))) break;
+      cvb ^= 1u << bsel;
+      bool f0, f1;
       if (p.adaptive) {
         const volatile uint32_t* vv = bars.votes[bsel];
         if (C::STACK) {  // rows 0-63: quadrants 0, 1; rows 64-127: quadrants 2, 3
-          f[0] = (vv[0] | vv[1] | vv[4] | vv[5]) != 0;
-          f[1] = (vv[2] | vv[3] | vv[6] | vv[7]) != 0;
+          f0 = (vv[0] | vv[1] | vv[4] | vv[5]) != 0;
+          f1 = (vv[2] | vv[3] | vv[6] | vv[7]) != 0;
         } else {
-          f[0] = f[1] = (vv[0] | vv[1] | vv[2] | vv[3] | vv[4] | vv[5] | vv[6] | vv[7]) != 0;
+          f0 = f1 = (vv[0] | vv[1] | vv[2] | vv[3] | vv[4] | vv[5] | vv[6] | vv[7]) != 0;
         }
       } else {
-        f[0] = pl.live[0] && pl.b16[0];
-        f[1] = pl.live[1] && pl.b16[1];
+        f0 = pl.live[0] && pl.b16[0];
+        f1 = pl.live[1] && pl.b16[1];
       }
-      const bool s16 = p.adaptive ? (f[0] || f[1]) : true;
-      my16 = f[hh];
+      const bool s16 = p.adaptive ? (f0 || f1) : true;
+      my16 = hh ? f1 : f0;
       if (s16) {
-        if (!(ok = warp_wait(&bars.s16_full[bsel], c16[bsel] & 1u, wc, W_S16))) break;
-        ++c16[bsel];
+        if (!(ok = warp_wait(&bars.s16_full[bsel], (c16b >> bsel) & 1u, wc, W_S16))) break;
+        c16b ^= 1u << bsel;
         tc_fence_after();
         if (my16) {  // (both threads of a row take this branch or neither)
           load_s(bsel);
@@ -603,7 +605,7 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
       }
     }
     if (p.route && h == 0 && lane == 0 && (q4 == 0 || (C::STACK && q4 == 2))) {
-      if (pl.live[hh]) {
+      if (hh ? pl.live[1] : pl.live[0]) {
         const uint8_t v = my16 ? (pl.two_phase && p.adaptive ? 3 : 2) : 1;
         p.route[(static_cast<size_t>(bh_q) * p.nqt + qt_r) * p.nkt + kt] = v;
       }
