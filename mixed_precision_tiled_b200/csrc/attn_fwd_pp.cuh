@@ -81,15 +81,28 @@ struct PPBars {
 static_assert(sizeof(PPBars) <= 512, "barrier block");
 
 struct PPGeo {
-  int b, h, kvh, pair, q0, kt_lo, n;
-  int lo[2], hi[2];  // visible key range (union) of query tile X; lo > hi = none
+  int b, kvh, kt_lo, n;
+  int h[2], q0[2], qt[2];  // head, first row and query-tile index of query tile X
+  int lo[2], hi[2];        // visible key range (union) of query tile X; lo > hi = none
 };
 
-// Persistent CTAs: work item j = (batch, head, pair of query tiles), numbered longest-first;
-// round r gives CTA c the item r * G + c (r even) or r * G + G - 1 - c (r odd), a snake that
-// keeps the CTAs' total work close.  -1: no item left.
+// Work items.  With an even number of query heads per KV head (grouped-query attention) an item
+// is one 128-row query tile of two heads of the same KV group: both query tiles see the same
+// key tiles, so the two softmax warpgroups stay in step to the item's end, and every K / V tile
+// is still loaded once for both.  Otherwise an item is two consecutive query tiles of one head.
+// Items are numbered longest-first (causal).
+__device__ __forceinline__ bool pp_head_pairs(const AttnParams& p) {
+  return ((p.H / p.Hkv) & 1) == 0;
+}
+__device__ __forceinline__ long long pp_n_items(const AttnParams& p) {
+  return pp_head_pairs(p) ? static_cast<long long>(p.B) * (p.H / 2) * p.nqt
+                          : static_cast<long long>(p.B) * p.H * ((p.nqt + 1) / 2);
+}
+
+// Persistent CTAs: round r gives CTA c the item r * G + c (r even) or r * G + G - 1 - c (r odd),
+// a snake that keeps the CTAs' total work close.  -1: no item left.
 __device__ __forceinline__ int pp_item(const AttnParams& p, int r) {
-  const long long n_items = static_cast<long long>(p.B) * p.H * ((p.nqt + 1) / 2);
+  const long long n_items = pp_n_items(p);
   const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
   const long long j = static_cast<long long>(r) * G + ((r & 1) ? G - 1 - c : c);
   return j < n_items ? static_cast<int>(j) : -1;
@@ -97,19 +110,35 @@ __device__ __forceinline__ int pp_item(const AttnParams& p, int r) {
 
 __device__ __forceinline__ PPGeo pp_geo(const AttnParams& p, int idx) {
   PPGeo g;
-  const int BH = p.B * p.H;
-  const int n_pairs = (p.nqt + 1) / 2;
-  g.pair = n_pairs - 1 - idx / BH;  // longest-first
-  const int bh = idx - (idx / BH) * BH;
-  g.b = bh / p.H;
-  g.h = bh - g.b * p.H;
-  g.kvh = g.h / (p.H / p.Hkv);
-  g.q0 = g.pair * 2 * PPCfg::MT;
+  if (pp_head_pairs(p)) {
+    const int BH2 = p.B * (p.H / 2);
+    const int qt = p.nqt - 1 - idx / BH2;  // longest-first
+    const int bhp = idx - (idx / BH2) * BH2;
+    g.b = bhp / (p.H / 2);
+    const int hp = bhp - g.b * (p.H / 2);
+    for (int x = 0; x < 2; ++x) {
+      g.h[x] = 2 * hp + x;
+      g.q0[x] = qt * PPCfg::MT;
+      g.qt[x] = qt;
+    }
+  } else {
+    const int BH = p.B * p.H;
+    const int n_pairs = (p.nqt + 1) / 2;
+    const int pair = n_pairs - 1 - idx / BH;  // longest-first
+    const int bh = idx - (idx / BH) * BH;
+    g.b = bh / p.H;
+    for (int x = 0; x < 2; ++x) {
+      g.h[x] = bh - g.b * p.H;
+      g.q0[x] = (2 * pair + x) * PPCfg::MT;
+      g.qt[x] = 2 * pair + x;
+    }
+  }
+  g.kvh = g.h[0] / (p.H / p.Hkv);
   int lo_all = 1 << 30, hi_all = -1;
   for (int x = 0; x < 2; ++x) {
     g.lo[x] = 1;
     g.hi[x] = 0;
-    const int r0 = g.q0 + x * PPCfg::MT;
+    const int r0 = g.q0[x];
     const int r1 = min(p.Lq, r0 + PPCfg::MT) - 1;
     if (r0 > r1) continue;
     int lo0, hi0, lo1, hi1;
@@ -138,9 +167,10 @@ struct MaskRow {
 
 __device__ __forceinline__ MaskRow load_mask_row(const AttnParams& p, const PPGeo& g, int x) {
   MaskRow m{~0ull, ~0ull};
-  const int qt = 2 * g.pair + x;
+  const int qt = x ? g.qt[1] : g.qt[0];
+  const int hx = x ? g.h[1] : g.h[0];
   if (!p.mask || p.adaptive || qt >= p.nqt) return m;
-  const size_t base = (static_cast<size_t>(g.b * p.H + g.h) * p.nqt + qt) * p.mask_words;
+  const size_t base = (static_cast<size_t>(g.b * p.H + hx) * p.nqt + qt) * p.mask_words;
   if (lamp_chk(base + p.mask_words <= static_cast<size_t>(p.B) * p.H * p.nqt * p.mask_words, 1)) {
     const unsigned long long* mp = reinterpret_cast<const unsigned long long*>(p.mask);
     m.w0 = __ldg(mp + base);
@@ -255,9 +285,8 @@ __device__ void pp_producer(const AttnParams& p, uint8_t* smem, PPBars& bars, co
     const int item = pp_item(p, r);
     if (item < 0) break;
     const PPGeo g = pp_geo(p, item);
-    const int bh_q = g.b * p.H + g.h;
     bh_kv = g.b * p.Hkv + g.kvh;
-    if (!lamp_chk(bh_q < p.B * p.H && bh_kv < p.B * p.Hkv, 3)) { ok = false; break; }
+    if (!lamp_chk(g.b * p.H + g.h[1] < p.B * p.H && bh_kv < p.B * p.Hkv, 3)) { ok = false; break; }
     if (r > 0 && !(ok = mbar_wait(&bars.q_empty, (r - 1) & 1u, wc, W_EMPTY))) break;
     // the item's mask rows, read by the MMA warp after it has seen this item's Q arrive
     for (int x = 0; x < 2; ++x) {
@@ -267,7 +296,8 @@ __device__ void pp_producer(const AttnParams& p, uint8_t* smem, PPBars& bars, co
     }
     mbar_arrive_expect_tx(&bars.q_full, 2 * (C::Q16_BYTES + C::Q8_BYTES));
     for (int x = 0; x < 2; ++x) {
-      const int row = g.q0 + x * C::MT;
+      const int row = g.q0[x];
+      const int bh_q = g.b * p.H + g.h[x];
       for (int c = 0; c < 2; ++c)
         tma_load_3d(smem + C::OFF_Q16 + x * C::Q16_BYTES + c * C::MT * 128, &p.tm_q16,
                     &bars.q_full, c * 64, row, bh_q);
@@ -543,10 +573,10 @@ __device__ __forceinline__ bool pp_softmax_item(const AttnParams& p, const PPGeo
   const int q4 = warp & 3;                  // TMEM lane quadrant
   const int lane = threadIdx.x & 31;
   const int r = q4 * 32 + lane;
-  const int i = g.q0 + x * C::MT + r;
+  const int i = (x ? g.q0[1] : g.q0[0]) + r;
   const bool row_valid = i < p.Lq;
-  const int qt = 2 * g.pair + x;
-  const int bh_q = g.b * p.H + g.h;
+  const int qt = x ? g.qt[1] : g.qt[0];
+  const int bh_q = g.b * p.H + (x ? g.h[1] : g.h[0]);
   const uint32_t lane_base = tbase + (static_cast<uint32_t>(q4 * 32) << 16);
   const uint32_t s_col = static_cast<uint32_t>(x * C::BN);
   const uint32_t o_col = static_cast<uint32_t>(2 * C::BN + x * C::D);

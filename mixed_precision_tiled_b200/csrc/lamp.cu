@@ -359,7 +359,10 @@ int attn_q8(const void* q, const void* k, const void* v, const void* q8, const v
   if (D == 128 && !p.e4m3) {
     // persistent CTAs: one per SM (the kernel fills the SM's shared and tensor memory), each
     // walking its share of the (batch, head, query-tile pair) work items
-    const long long items = static_cast<long long>(BHq) * ((nqt + 1) / 2);
+    // (work items as in the kernel: query-tile pairs of two heads of one KV group when the
+    // group size is even, else pairs of consecutive query tiles of one head)
+    const long long items = ((H / Hkv) % 2 == 0) ? static_cast<long long>(B) * (H / 2) * nqt
+                                                 : static_cast<long long>(BHq) * ((nqt + 1) / 2);
     int nsm = 0;
     if (int r = sm_count(&nsm)) return r;
     const long long pgrid = std::min<long long>(items, nsm);
