@@ -86,9 +86,12 @@ def tile_pairs(w) -> np.ndarray:
 
 
 def blended_flops(w, route_map: np.ndarray):
-    """(F8, F16, F_total): FLOPs of 8-bit QK tiles, of 16-bit QK tiles + P.V, and the metric's."""
+    """(F8, F16, F_total, 16-bit fraction): FLOPs of 8-bit QK tiles, of 16-bit QK tiles + P.V,
+    the metric's FLOPs, and the fraction of visible pairs scored in 16 bits.  Route codes: 1
+    8-bit, 2 16-bit by the mask, 3 recomputed by the look-ahead rule; a recomputed tile counts
+    its 8-bit pass too (the rule needs the 8-bit tile max of every tile to decide)."""
     pairs = tile_pairs(w)[None, None]  # broadcast over B, H
-    p8 = int((pairs * (route_map == 1)).sum())
+    p8 = int((pairs * ((route_map == 1) | (route_map == 3))).sum())
     p16 = int((pairs * ((route_map == 2) | (route_map == 3))).sum())
     total = int((pairs * (route_map != 0)).sum())
     F8 = 2 * w.D * p8
@@ -414,8 +417,10 @@ def main():
         flush.view(torch.int64).sum()
     bitmask = w.route == "bitmask"
 
-    def step(ev_a=None, ev_b=None, p_fp16=None):
-        mpt.lamp_quant_qk(q, k, q8, k8, qs, ks, B, H, Hkv, Lq, Lk, D, mode, stream)
+    def step(ev_a=None, ev_b=None, p_fp16=None, mode_=None, tau_=None):
+        md = mode if mode_ is None else mode_
+        tu = w.tau if tau_ is None else tau_
+        mpt.lamp_quant_qk(q, k, q8, k8, qs, ks, B, H, Hkv, Lq, Lk, D, md, stream)
         if bitmask:
             mpt.lamp_build_mask(mask, B, H, Lq, Lk, D, w.group_tiles,
                                 w.p_fp16 if p_fp16 is None else p_fp16, w.mask_seed, stream)
@@ -423,19 +428,19 @@ def main():
             ev_a.record(stream)
         mpt.lamp_attn_fwd_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D,
                              int(w.causal), w.window, 0.0, mask if bitmask else None,
-                             w.group_tiles, mode, w.tau, None, stream)
+                             w.group_tiles, md, tu, None, stream)
         if ev_b is not None:
             ev_b.record(stream)
 
     launches_per_step = 1 + (1 if bitmask else 0) + 1  # quantiser (Q and K), mask, attention
 
-    def timed(n, p_fp16=None):
+    def timed(n, **kw):
         """Per-step and attention-kernel device times (ms) over n steps, L2 flushed between."""
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
         for i in range(n):
             flush_l2()
             ev[i][0].record(stream)
-            step(ev[i][1], ev[i][2], p_fp16)
+            step(ev[i][1], ev[i][2], **kw)
             ev[i][3].record(stream)
         torch.cuda.synchronize()
         st = [ev[i][0].elapsed_time(ev[i][3]) for i in range(n)]
@@ -532,6 +537,26 @@ def main():
                                 "roofline_frac": round((f8 / P8 + f16 / P16) / (a * 1e-3), 3)}
         step()  # restore the configured mask
         torch.cuda.synchronize()
+    # look-ahead workloads: tau x 8-bit format, with the rerouted (recomputed) tile fraction
+    if not bitmask and not args.no_sweep:
+        for fmt in ("int8", "e4m3"):
+            md = mpt.mode_bits(w.route, fmt, w.dtype)
+            for tau in (2.0, 4.0, 8.0):
+                step(mode_=md, tau_=tau)
+                mpt.lamp_attn_fwd_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D,
+                                     int(w.causal), w.window, 0.0, None, w.group_tiles, md, tau,
+                                     rmap, stream)
+                torch.cuda.synchronize()
+                f8, f16, ff, fr = blended_flops(w, rmap.cpu().numpy())
+                n = max(10, args.steps // 10)
+                _, at = timed(n, mode_=md, tau_=tau)
+                a = float(statistics.fmean(at))
+                sweep[f"{fmt} tau={tau:g}"] = {
+                    "rerouted_fraction": round(fr, 4),
+                    "attn_tflops": round(ff / (a * 1e-3) / 1e12, 1),
+                    "roofline_frac": round((f8 / P8 + f16 / P16) / (a * 1e-3), 3)}
+        step()  # restore the configured format and tau
+        torch.cuda.synchronize()
 
     quant = quantiser_bandwidth(mpt, torch, dev, stream, peaks) if not args.no_sweep else None
     probe = tensor_probe(mpt, torch, stream) if not args.no_sweep else None
@@ -572,7 +597,7 @@ def main():
             "gpu_launches": launches_per_step * args.steps,
         }
         if sweep:
-            line["sweep_fp16_fraction"] = sweep
+            line["sweep_fp16_fraction" if bitmask else "sweep_tau_format"] = sweep
         if quant:
             line["quantiser"] = quant
         if probe:

@@ -22,9 +22,13 @@
 //     maxima, vote on the look-ahead rule, run the online softmax (MUFU ex2, lazy reference
 //     max), store P as packed 16-bit pairs into the S columns, rescale O in TMEM when the
 //     reference moves, and write O / lse at the end;
-//   * routing tiles of 64 query rows (D = 64, 256) are stacked two per 128-row MMA; a key
-//     tile whose two halves need different precisions runs the 8-bit MMA first, then the
-//     16-bit MMA into the same TMEM columns after every row has read its 8-bit scores.
+//   * routing tiles of 64 query rows (D = 64, 256) are stacked two per 128-row MMA;
+//   * a two-phase key tile (look-ahead mode, or stacked halves of different precisions) has
+//     an 8-bit and a 16-bit S.  At D = 64 and 128 the 16-bit S has TMEM columns of its own and
+//     is issued right behind the 8-bit one (in look-ahead mode speculatively: the rows read it
+//     only when the vote flags the tile, and the tile's result is the same as if it had been
+//     issued after the vote); at D = 256 it goes into the 8-bit S's columns once every row has
+//     read its 8-bit scores.
 // Every mbarrier wait is bounded; on a timeout the CTA records the failure, stops, drains its
 // in-flight copies and MMAs, frees its TMEM and exits.
 #pragma once
@@ -41,7 +45,7 @@ namespace lamp {
 // where-codes recorded with a timeout (bits 8..15 of the error word)
 enum : uint32_t {
   W_QFULL = 1, W_EMPTY = 2, W_FULL = 3, W_SFULL = 4, W_S16 = 5, W_VOTE = 6, W_PFULL = 7,
-  W_ODONE = 8, W_DRAIN = 9, W_SELFTEST = 10, W_XCH = 11
+  W_ODONE = 8, W_DRAIN = 9, W_SELFTEST = 10, W_XCH = 11, W_ZFREE = 12
 };
 
 struct AttnParams {
@@ -79,7 +83,13 @@ struct AttnCfg {
   static constexpr int C16 = D / 64;           // 128-byte chunks of a 16-bit row
   static constexpr int C8 = (D == 64) ? 1 : D / 128;
   static constexpr int TMEM_O = 2 * BN;
-  static constexpr int TMEM_COLS = (2 * BN + D) <= 256 ? 256 : 512;
+  // A separate TMEM region Z for the 16-bit S of two-phase key tiles, where the columns allow
+  // (D = 64, 128): the 16-bit MMA is then issued right behind the 8-bit one instead of after
+  // every row has read the 8-bit scores.  At D = 256 (S x 2 + O fill all 512 columns) the
+  // 16-bit S goes into the 8-bit S's own columns after the rows have read them.
+  static constexpr bool SEP16 = 3 * BN + D <= 512;
+  static constexpr int TMEM_Z = 2 * BN + D;
+  static constexpr int TMEM_COLS = ((SEP16 ? 3 * BN : 2 * BN) + D) <= 256 ? 256 : 512;
   static constexpr int OFF_Q16 = 0;
   static constexpr int OFF_Q8 = Q16_BYTES;
   static constexpr int OFF_SLOTS = Q16_BYTES + Q8_BYTES;
@@ -103,6 +113,8 @@ struct Bars {
   uint64_t p_full[2];
   uint64_t o_done;
   uint64_t drain;
+  uint64_t z_free;   // the rows have finished with the 16-bit S region Z (8 warp arrivals)
+  uint64_t o_final;  // every P.V of the CTA has completed (one phase)
   uint32_t tmem_base;
   uint32_t abort;
   uint32_t votes[2][8];
@@ -174,12 +186,30 @@ __device__ __forceinline__ Geo make_geo(const AttnParams& p) {
   return g;
 }
 
+// Key tile kt and its mask group g_idx = kt / group_tiles, advanced without a division.
+struct KtPos {
+  int kt, g_idx, rem;
+  __device__ __forceinline__ void init(const AttnParams& p, int kt0) {
+    kt = kt0;
+    g_idx = kt0 / p.group_tiles;
+    rem = kt0 - g_idx * p.group_tiles;
+  }
+  __device__ __forceinline__ void next(const AttnParams& p) {
+    ++kt;
+    if (++rem == p.group_tiles) {
+      rem = 0;
+      ++g_idx;
+    }
+  }
+};
+
 template <class C>
-__device__ __forceinline__ Plan make_plan(const AttnParams& p, const Geo& g, int kt) {
+__device__ __forceinline__ Plan make_plan(const AttnParams& p, const Geo& g, const KtPos& pos) {
   Plan pl;
+  const int kt = pos.kt;
   const int c0 = kt * C::BN, c1 = min(p.Lk, c0 + C::BN) - 1;
   bool need8 = false, need16 = false;
-  const int g_idx = kt / p.group_tiles;
+  const int g_idx = pos.g_idx;
   for (int hh = 0; hh < 2; ++hh) {
     pl.live[hh] = g.half_lo[hh] <= g.half_hi[hh] && g.half_lo[hh] <= c1 && g.half_hi[hh] >= c0;
     pl.b16[hh] = false;
@@ -250,16 +280,24 @@ __device__ void producer_role(const AttnParams& p, const Geo& g, uint8_t* smem, 
     return true;
   };
 
-  Plan cur = make_plan<C>(p, g, g.kt_lo);
+  // Order of the loads = order in which the MMA warp consumes them: the first S operand of
+  // tile t+1 before V of tile t; the 16-bit K of a two-phase tile right behind its 8-bit K
+  // (separate region Z) or after the next tile's first operand (shared columns).
+  KtPos pos;
+  pos.init(p, g.kt_lo);
+  Plan cur = make_plan<C>(p, g, pos);
   ok = load(cur.first16 ? 1 : 0, g.kt_lo);
+  if (ok && C::SEP16 && cur.two_phase) ok = load(1, g.kt_lo);
   for (int t = 0; ok && t < g.n; ++t) {
     const int kt = g.kt_lo + t;
     Plan nxt;
     if (t + 1 < g.n) {
-      nxt = make_plan<C>(p, g, kt + 1);
+      pos.next(p);
+      nxt = make_plan<C>(p, g, pos);
       if (!(ok = load(nxt.first16 ? 1 : 0, kt + 1))) break;
+      if (C::SEP16 && nxt.two_phase && !(ok = load(1, kt + 1))) break;
     }
-    if (cur.two_phase && !(ok = load(1, kt))) break;
+    if (!C::SEP16 && cur.two_phase && !(ok = load(1, kt))) break;
     if (!(ok = load(2, kt))) break;
     cur = nxt;
   }
@@ -311,8 +349,9 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
     tc_fence_after();
     return true;
   };
-  auto issue_s = [&](int t, bool sixteen, int slot) {
-    const uint32_t dS = tbase + static_cast<uint32_t>((t & 1) * C::BN);
+  // S of tile t into TMEM column col (its S buffer, or Z)
+  auto issue_s = [&](uint32_t col, bool sixteen, int slot) {
+    const uint32_t dS = tbase + col;
     if (sixteen) {
       const uint64_t kb = d_k16 + slot * SLOT_D;
       if (leader) {
@@ -346,25 +385,48 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
   auto commit = [&](uint64_t* bar) {
     if (leader) tc_commit(bar);
   };
+  auto buf = [](int t) { return static_cast<uint32_t>((t & 1) * C::BN); };
+  // Separate region Z: the 16-bit S of every two-phase tile goes there right behind the tile's
+  // first S (in adaptive mode speculatively: the rows use it only if the tile is flagged).  Z is
+  // rewritten once every row has finished with its previous contents (z_free).
+  uint32_t zuse = 0;
+  auto issue_z = [&]() -> bool {
+    int slot16;
+    if (zuse > 0) {
+      if (!mbar_wait(&bars.z_free, (zuse - 1) & 1u, wc, W_ZFREE)) return false;
+      tc_fence_after();
+    }
+    if (!take(slot16)) return false;
+    issue_s(C::TMEM_Z, true, slot16);
+    commit(&bars.s16_full[0]);
+    commit(&bars.empty[slot16]);
+    ++zuse;
+    return true;
+  };
 
-  Plan cur = make_plan<C>(p, g, g.kt_lo);
+  KtPos pos;
+  pos.init(p, g.kt_lo);
+  Plan cur = make_plan<C>(p, g, pos);
   int slot = 0;
   if (ok && (ok = take(slot))) {
-    issue_s(0, cur.first16, slot);
+    issue_s(buf(0), cur.first16, slot);
     commit(&bars.s_full[0]);
     commit(&bars.empty[slot]);
+    if (C::SEP16 && cur.two_phase) ok = issue_z();
   }
   for (int t = 0; ok && t < g.n; ++t) {
     const int bsel = t & 1;
     Plan nxt;
     if (t + 1 < g.n) {
-      nxt = make_plan<C>(p, g, g.kt_lo + t + 1);
+      pos.next(p);
+      nxt = make_plan<C>(p, g, pos);
       if (!(ok = take(slot))) break;
-      issue_s(t + 1, nxt.first16, slot);
+      issue_s(buf(t + 1), nxt.first16, slot);
       commit(&bars.s_full[(t + 1) & 1]);
       commit(&bars.empty[slot]);
+      if (C::SEP16 && nxt.two_phase && !(ok = issue_z())) break;
     }
-    if (cur.two_phase) {
+    if (!C::SEP16 && cur.two_phase) {
       int slot16;
       if (!(ok = take(slot16))) break;
       if (!(ok = mbar_wait(&bars.vote[bsel], (cvb >> bsel) & 1u, wc, W_VOTE))) break;
@@ -381,7 +443,7 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
         s16 = true;
       }
       if (s16) {
-        issue_s(t, true, slot16);
+        issue_s(buf(t), true, slot16);
         commit(&bars.s16_full[bsel]);
         commit(&bars.empty[slot16]);
       } else if (leader) {
@@ -407,6 +469,9 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
     commit(&bars.empty[slotv]);
     cur = nxt;
   }
+  // The epilogue waits for every P.V (the softmax skips most per-tile o_done waits, so that
+  // barrier's phase count cannot tell it when the last one is done).
+  commit(&bars.o_final);
   // Every MMA issued by this thread must complete before the TMEM is released.
   commit(&bars.drain);
   const WaitCtx drain{0u, 50000u};  // no abort word: in-flight work always completes
@@ -502,6 +567,7 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
   // phase bits per S buffer (bit b: buffer b) of the vote and 16-bit S barriers; the S barrier
   // of buffer b completes at every use, its phase is (t >> 1) & 1
   uint32_t cvb = 0, c16b = 0, nx = 0;
+  uint32_t zc = 0;  // uses of the separate 16-bit region Z so far
   bool ok = true;
   uint32_t raw[NH];
 
@@ -516,10 +582,10 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
     other = __uint_as_float(lds_u32(xch + static_cast<uint32_t>((par * 2 + (h ^ 1)) * C::MT * 4)));
     return true;
   };
-  auto load_s = [&](int bsel) {
+  auto load_s = [&](int col) {  // this thread's half row of the S at TMEM column col
 #pragma unroll
     for (int c = 0; c < NH / 32; ++c)
-      tmem_ld32(lane_base + static_cast<uint32_t>(bsel * N + h * NH + c * 32),
+      tmem_ld32(lane_base + static_cast<uint32_t>(col + h * NH + c * 32),
                 *reinterpret_cast<uint32_t(*)[32]>(&raw[c * 32]));
     tmem_wait_ld();
   };
@@ -543,26 +609,108 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
     return fmaxf(m0, m1);
   };
 
+  auto load_s_async = [&](int col) {  // as load_s, without the wait for the data
+#pragma unroll
+    for (int c = 0; c < NH / 32; ++c)
+      tmem_ld32(lane_base + static_cast<uint32_t>(col + h * NH + c * 32),
+                *reinterpret_cast<uint32_t(*)[32]>(&raw[c * 32]));
+  };
+  // the key block's scale is read one tile ahead (its L2 latency would otherwise sit on the
+  // path of every tile)
+  float ks_nxt = (g.n > 0) ? __ldg(ks_row + g.kt_lo) : 0.0f;
+  // the routing plan is likewise made one tile ahead (its mask read and arithmetic then overlap
+  // the current tile's work)
+  KtPos pos;
+  pos.init(p, g.kt_lo);
+  Plan pl_nxt = make_plan<C>(p, g, pos);
+
   for (int t = 0; ok && t < g.n; ++t) {
     const int kt = g.kt_lo + t;
     const int bsel = t & 1;
-    const Plan pl = make_plan<C>(p, g, kt);
+    const Plan pl = pl_nxt;
+    const float ks_cur = ks_nxt;
+    if (t + 1 < g.n) {
+      ks_nxt = __ldg(ks_row + kt + 1);
+      pos.next(p);
+      pl_nxt = make_plan<C>(p, g, pos);
+    }
     if (!(ok = warp_wait(&bars.s_full[bsel], static_cast<uint32_t>(t >> 1) & 1u, wc, W_SFULL))) break;
     tc_fence_after();
-    load_s(bsel);
     const int j0 = kt * N + h * NH;
     const bool full = row_valid && j0 >= lo_r && j0 + NH - 1 <= hi_r;
-    bool sixteen = pl.first16;
     // (a zero block scale would turn masked -inf entries into NaN: keep it positive)
-    float cscale = sixteen ? p.scale_log2 : fmaxf(sq_scale * __ldg(ks_row + kt), 1e-30f);
-    if (!sixteen && !E4M3) int_to_float();
-    if (!full) apply_mask(j0);
-    float tmax = raw_max(), other;
-    if (!(ok = exchange(bsel, tmax, other))) break;
-    tmax = fmaxf(tmax, other);
-
-    bool my16 = pl.first16;
-    if (pl.two_phase) {
+    const float cs8 = fmaxf(sq_scale * ks_cur, 1e-30f);
+    bool sixteen = pl.first16, my16 = pl.first16;
+    float cscale, tmax, other;
+    if (C::SEP16 && pl.two_phase) {
+      // The 16-bit S is in Z, issued with the tile.  Look-ahead mode: vote on the 8-bit half-row
+      // maximum (a row reaches m - tau iff one of its halves does, so the tile vote needs no
+      // exchange), read Z while the vote completes, and fall back to the 8-bit S only if the
+      // tile is not flagged.  Mixed stacked halves know their precision from the mask.
+      if (p.adaptive) {
+        load_s(bsel * N);
+        if (!E4M3) int_to_float();
+        if (!full) apply_mask(j0);
+        const float hmax = raw_max();
+        const float t8 = (hmax == NEG_INF) ? NEG_INF : hmax * cs8;
+        const bool vote = (t8 != NEG_INF) && (t8 >= m_true - p.tau_log2);
+        const uint32_t wv = __any_sync(0xFFFFFFFFu, vote) ? 1u : 0u;
+        if (lane == 0) bars.votes[bsel][warp] = wv;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.vote[bsel]);
+        if (!(ok = warp_wait(&bars.s16_full[0], zc & 1u, wc, W_S16))) break;
+        tc_fence_after();
+        load_s_async(C::TMEM_Z);
+        ok = warp_wait(&bars.vote[bsel], (cvb >> bsel) & 1u, wc, W_VOTE);
+        tmem_wait_ld();
+        if (!ok) break;
+        cvb ^= 1u << bsel;
+        const volatile uint32_t* vv = bars.votes[bsel];
+        bool f0, f1;
+        if (C::STACK) {  // rows 0-63: quadrants 0, 1; rows 64-127: quadrants 2, 3
+          f0 = (vv[0] | vv[1] | vv[4] | vv[5]) != 0;
+          f1 = (vv[2] | vv[3] | vv[6] | vv[7]) != 0;
+        } else {
+          f0 = f1 = (vv[0] | vv[1] | vv[2] | vv[3] | vv[4] | vv[5] | vv[6] | vv[7]) != 0;
+        }
+        my16 = hh ? f1 : f0;
+        if (!my16) {  // not flagged: back to the 8-bit scores (still in this tile's S buffer)
+          load_s(bsel * N);
+          if (!E4M3) int_to_float();
+        }
+      } else {
+        my16 = hh ? (pl.live[1] && pl.b16[1]) : (pl.live[0] && pl.b16[0]);
+        if (my16) {
+          if (!(ok = warp_wait(&bars.s16_full[0], zc & 1u, wc, W_S16))) break;
+          tc_fence_after();
+          load_s(C::TMEM_Z);
+        } else {
+          load_s(bsel * N);
+          if (!E4M3) int_to_float();
+        }
+      }
+      // (a warp that skipped the s16_full wait cannot fall two phases behind: the next use of
+      // Z needs its z_free arrival)
+      ++zc;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.z_free);
+      sixteen = my16;
+      cscale = my16 ? p.scale_log2 : cs8;
+      if (!full) apply_mask(j0);
+      tmax = raw_max();
+      if (!(ok = exchange(bsel, tmax, other))) break;
+      tmax = fmaxf(tmax, other);
+    } else {
+      load_s(bsel * N);
+      cscale = sixteen ? p.scale_log2 : cs8;
+      if (!sixteen && !E4M3) int_to_float();
+      if (!full) apply_mask(j0);
+      tmax = raw_max();
+      if (!(ok = exchange(bsel, tmax, other))) break;
+      tmax = fmaxf(tmax, other);
+    }
+    if (!C::SEP16 && pl.two_phase) {
       if (p.adaptive) {
         const float t8 = (tmax == NEG_INF) ? NEG_INF : tmax * cscale;
         const bool vote = (t8 != NEG_INF) && (t8 >= m_true - p.tau_log2);
@@ -594,7 +742,7 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
         c16b ^= 1u << bsel;
         tc_fence_after();
         if (my16) {  // (both threads of a row take this branch or neither)
-          load_s(bsel);
+          load_s(bsel * N);
           sixteen = true;
           cscale = p.scale_log2;
           if (!full) apply_mask(j0);
@@ -663,10 +811,14 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
       l_rd += (sr0 + sr1) + (sr2 + sr3);
     }
 
-    if (t > 0) {  // P.V of the previous tile has completed: O may be rescaled
+    // O is rescaled (rarely: lazy reference max) once P.V of the previous tile has completed.
+    // The wait is exact although most tiles skip it: S(t), seen complete above, was issued
+    // after P.V(t-2) and the tensor core completes in issue order, and P.V(t) is issued only
+    // after this warp's P arrival below, so o_done stands at phase t-1 or t.
+    if (t > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
       if (!(ok = warp_wait(&bars.o_done, (t - 1) & 1u, wc, W_ODONE))) break;
       tc_fence_after();
-      if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {  // each thread rescales its half of O
+      {  // each thread rescales its half of O
         const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll 1
         for (int c = 0; c < C::D / 32; ++c) {
@@ -695,7 +847,7 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
 
   // epilogue: combine the two halves' row sums, then O / l and lse
   if (g.n > 0) {
-    if (!warp_wait(&bars.o_done, (g.n - 1) & 1u, wc, W_ODONE)) return;
+    if (!warp_wait(&bars.o_final, 0, wc, W_ODONE)) return;
     tc_fence_after();
   }
   const int par = g.n & 1;  // the exchange slots of parity n & 1 were last read two tiles back
@@ -782,6 +934,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) attn_fwd_kernel(const __grid_co
     }
     mbar_init(&bars.o_done, 1);
     mbar_init(&bars.drain, 1);
+    mbar_init(&bars.z_free, 8);
+    mbar_init(&bars.o_final, 1);
     for (int q = 0; q < 4; ++q) mbar_init(&bars.xbar[q], 64);
     bars.abort = 0;
     fence_mbarrier_init();

@@ -66,3 +66,15 @@ def test_blended_flops_split():
     rmap[rmap == 1] = 2  # all 16-bit
     F8, F16, F, frac = bench.blended_flops(w, rmap)
     assert F8 == 0 and F16 == F and frac == 1.0
+
+
+def test_blended_flops_recomputed_tiles_count_both_passes():
+    # a tile recomputed by the look-ahead rule (route 3) was scored in 8 bits first: its QK^T
+    # counts at both precisions, P.V once
+    w = CONFIGS["adaptive8k"].replace(B=1, H=2, Hkv=1, Lq=1024, Lk=1024)
+    pairs = bench.tile_pairs(w)
+    live = (pairs > 0).astype(np.uint8)
+    rmap = np.broadcast_to(live * 3, (w.B, w.H) + live.shape).copy()
+    F8, F16, F, frac = bench.blended_flops(w, rmap)
+    assert F == 4 * w.D * w.pairs() * w.B * w.H
+    assert F8 == F // 2 and F16 == F and frac == 1.0
