@@ -568,8 +568,9 @@ def main():
     try:
         with open(TRAFFIC_FILE) as f:
             tr = json.load(f)
-        if tr.get("kernel_hash") == kernel_hash() and tr.get("workload") == w.name:
-            traffic = tr.get("traffic_bytes_per_launch")
+        rec = tr.get("records", {}).get(w.name)
+        if rec and tr.get("kernel_hash") == kernel_hash():
+            traffic = rec.get("traffic_bytes_per_launch")
     except (OSError, ValueError):
         pass
 

@@ -1,25 +1,30 @@
 // Routed mixed-precision attention forward, head dimension 128, INT8 8-bit format: two query
-// tiles per CTA, one softmax warpgroup each.  (FP8 E4M3 runs in the single-tile kernel of
-// attn_fwd.cuh.)
+// tiles in flight per CTA, one softmax warpgroup each.  (FP8 E4M3 runs in the single-tile
+// kernel of attn_fwd.cuh.)
 //
 // Same computation as attn_fwd.cuh (TileMix page, section 2 "How It Works": 8-bit or 16-bit
 // score tiles chosen per tile, one shared online softmax; LampAttention abstract: 8-bit
 // products, look-ahead recomputation of sensitive tiles in 16 bits), organised for B200 so
 // that the tensor core works on one query tile while the softmax works on the other:
-//   * a CTA owns two 128-row query tiles A and B of one (batch, head) and streams each key
-//     tile through shared memory once for both: K8 tiles in a ring of 16 KB slots, K16 and V
-//     tiles in a ring of 32 KB slots;
-//   * TMEM holds S_A, S_B (128 columns each) and O_A, O_B (128 each) = all 512 columns;
-//   * warpgroup 0 runs the softmax of A, warpgroup 1 that of B (one row per thread, the row
-//     is the TMEM lane); warp 8 issues TMA loads, warp 9 issues the MMAs in the order
-//       S_A(0) S_B(0) | PV_A(t) S_A(t+1) PV_B(t) S_B(t+1) | ...
+//   * persistent CTAs (one per SM) walk a list of work items, longest first, in a snake order;
+//     an item is two 128-row query tiles X = 0, 1 that read the same K/V: the same query tile
+//     of two heads of one KV group (grouped-query attention with an even group), otherwise two
+//     query tiles of one head.  Each key tile is streamed through shared memory once for both:
+//     K8 tiles in a ring of 16 KB slots, K16 and V tiles in a ring of 32 KB slots;
+//   * TMEM holds S_0, S_1 (128 columns each) and O_0, O_1 (128 each) = all 512 columns;
+//   * warpgroup X runs the softmax of query tile X (one row per thread, the row is the TMEM
+//     lane); warp 8 issues TMA loads, warp 9 issues the MMAs (warp-wide loop, one elected
+//     lane) in the order
+//       S_0(0) S_1(0) | PV_0(t) S_0(t+1) PV_1(t) S_1(t+1) | ...
 //     so that while one warpgroup exponentiates tile t, the tensor core runs the other tile's
-//     P.V and next QK^T;
-//   * softmax arithmetic: exact int32 -> fp32 by the 2^23 magic-number add (ALU + FMA pipes
-//     instead of the MUFU conversion), packed f32x2 FMAs / adds, 3-input max, and a lazy O
-//     rescale: the reference max used for the exponentials only moves when a row max exceeds
-//     it by more than 8 (log2 units), which keeps P <= 256 and makes the TMEM round trip of O
-//     rare; the true running max is tracked separately for the look-ahead rule.
+//     P.V and next QK^T; P.V is issued in two halves as the softmax publishes them, and the
+//     next item's Q loads and first QK^T overlap the current item's last tiles and epilogue;
+//   * softmax arithmetic: exact int32 -> fp32 conversion (exact below 2^24), packed f32x2
+//     FMAs / adds, 3-input max, the rounded row sum by mixed-precision adds of the packed
+//     16-bit P, and a lazy O rescale: the reference max used for the exponentials only moves
+//     when a row max exceeds it by more than 8 (log2 units), which keeps P <= 256 and makes the
+//     TMEM round trip of O rare; the true running max is tracked separately for the look-ahead
+//     rule.
 #pragma once
 
 #include "attn_fwd.cuh"

@@ -78,3 +78,15 @@ def test_blended_flops_recomputed_tiles_count_both_passes():
     F8, F16, F, frac = bench.blended_flops(w, rmap)
     assert F == 4 * w.D * w.pairs() * w.B * w.H
     assert F8 == F // 2 and F16 == F and frac == 1.0
+
+
+def test_traffic_record_format():
+    # per-workload DRAM traffic of the attention launch (ncu), used only while the kernel
+    # sources hash to the recorded value
+    import json
+    with open(bench.TRAFFIC_FILE) as f:
+        tr = json.load(f)
+    assert len(tr["kernel_hash"]) == 16
+    for name, rec in tr["records"].items():
+        assert name in CONFIGS
+        assert rec["traffic_bytes_per_launch"] == rec["dram_bytes_read"] + rec["dram_bytes_write"]
