@@ -69,14 +69,14 @@ __device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
-__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
 __device__ __forceinline__ uint64_t f2sub(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
   return r;
 }
 
@@ -111,9 +111,11 @@ __device__ __forceinline__ bool near_e4m3(float q) {
 }
 
 // Eight 16-bit inputs -> eight 8-bit codes (two 32-bit words), x / s as described above.
-// INT8: t = q + 1.5 * 2^23 holds round-to-nearest-even(q) in its low mantissa bits (exact for
-// |q| < 2^22), so t's low byte is the two's-complement code and t - 1.5 * 2^23 = rint(q); the
-// estimate is near a half-integer when |q - rint(q)| > 0.5 - 2^-12.
+// INT8: t = fma(x, r, 1.5 * 2^23) rounds the exact product e = x * r once, to the integer
+// rint(e) held in t's low mantissa bits (exact for |e| < 2^22), so t's low byte is the two's-
+// complement code; d = fma(x, r, -(t - 1.5 * 2^23)) = e - rint(e), and the estimate is near a
+// half-integer when |d| > 0.5 - 2^-12.  (e is within 2^-23 relative of x / s: one ulp of the
+// reciprocal estimate, the product being exact inside the fma.)
 template <bool BF16, bool E4M3>
 __device__ __forceinline__ uint2 encode8(const uint4 w, float s, float r) {
   constexpr float MAGIC = 12582912.0f;  // 1.5 * 2^23
@@ -144,10 +146,10 @@ __device__ __forceinline__ uint2 encode8(const uint4 w, float s, float r) {
     float dmax = 0.0f;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const uint64_t q2 = f2mul(h2_to_f2<BF16>(ws[e]), r2);
-      const uint64_t t2 = f2add(q2, m2);
+      const uint64_t x2 = h2_to_f2<BF16>(ws[e]);
+      const uint64_t t2 = f2fma(x2, r2, m2);
       float d0, d1;
-      f2unpack(f2sub(q2, f2sub(t2, m2)), d0, d1);
+      f2unpack(f2fma(x2, r2, f2sub(m2, t2)), d0, d1);
       dmax = fmaxf(dmax, fmaxf(fabsf(d0), fabsf(d1)));
       f2unpack(t2, t[2 * e], t[2 * e + 1]);
     }
@@ -196,7 +198,8 @@ template <int VEC>
 struct QuantPipe {
   static constexpr int STAGE_BYTES = VEC * QUANT_THREADS * 16;
   static constexpr int NS = STAGE_BYTES <= 8192 ? 4 : 3;
-  static constexpr int SMEM_BYTES = NS * STAGE_BYTES + NS * 8;
+  // stages, then NS mbarriers, then NS block descriptors (QuantBlock, 32 bytes each)
+  static constexpr int SMEM_BYTES = NS * STAGE_BYTES + NS * 8 + NS * 32;
   static constexpr int CTAS_PER_SM = STAGE_BYTES <= 8192 ? 4 : (STAGE_BYTES <= 32768 ? 2 : 1);
   static constexpr int MIN_CTAS = CTAS_PER_SM > 2 ? 2 : CTAS_PER_SM;  // register bound
 };
@@ -208,6 +211,7 @@ struct QuantBlock {
   float* scale;       // the block's scale
   int nvec;           // 16-byte vectors in it (ragged last block of a run: fewer rows)
 };
+static_assert(sizeof(QuantBlock) == 32, "descriptor slot");
 __device__ __forceinline__ QuantBlock quant_locate(const QuantJob& j0, const QuantJob& j1, int b,
                                                    int D) {
   const bool second = b >= j0.blocks;
@@ -233,6 +237,9 @@ __global__ void __launch_bounds__(QUANT_THREADS, QuantPipe<VEC>::MIN_CTAS)
   using P = QuantPipe<VEC>;
   extern __shared__ __align__(128) uint8_t qsm[];
   uint64_t* full = reinterpret_cast<uint64_t*>(qsm + P::NS * P::STAGE_BYTES);
+  // Block descriptors, written by the issuing thread before the copy's arrival on full[]:
+  // the other threads read them after their wait, so the index arithmetic runs once per block.
+  QuantBlock* desc = reinterpret_cast<QuantBlock*>(qsm + P::NS * P::STAGE_BYTES + P::NS * 8);
   __shared__ uint32_t red[2][QUANT_THREADS / 32];
   __shared__ uint32_t abort_word;
   const int total = j0.blocks + j1.blocks;
@@ -247,6 +254,7 @@ __global__ void __launch_bounds__(QUANT_THREADS, QuantPipe<VEC>::MIN_CTAS)
   __syncthreads();
   auto issue = [&](int i) {  // the CTA's i-th block into stage i % NS
     const QuantBlock qb = quant_locate(j0, j1, first + i * stride, D);
+    desc[i % P::NS] = qb;
     const uint32_t bytes = static_cast<uint32_t>(qb.nvec) * 16u;
     uint64_t* bar = &full[i % P::NS];
     mbar_arrive_expect_tx(bar, bytes);
@@ -260,7 +268,7 @@ __global__ void __launch_bounds__(QUANT_THREADS, QuantPipe<VEC>::MIN_CTAS)
   for (; i < mine; ++i) {
     const int st = i % P::NS;
     const bool ok = mbar_wait(&full[st], (i / P::NS) & 1u, wc, 0x40u);
-    const QuantBlock qb = quant_locate(j0, j1, first + i * stride, D);
+    const QuantBlock qb = desc[st];
     const uint4* src = reinterpret_cast<const uint4*>(qsm + st * P::STAGE_BYTES);
     uint4 buf[VEC];
     uint32_t m2 = 0;
@@ -278,9 +286,8 @@ __global__ void __launch_bounds__(QUANT_THREADS, QuantPipe<VEC>::MIN_CTAS)
     // Every thread has its data in registers and its partial max in red[]: the stage is free.
     if (!__syncthreads_and(ok)) break;
     if (threadIdx.x == 0 && i + P::NS < mine) issue(i + P::NS);
-    mb = red[i & 1][0];
-#pragma unroll
-    for (int k = 1; k < QUANT_THREADS / 32; ++k) mb = max(mb, red[i & 1][k]);
+    // every warp reduces the 16 warp maxima itself (no second barrier)
+    mb = __reduce_max_sync(0xFFFFFFFFu, red[i & 1][threadIdx.x & (QUANT_THREADS / 32 - 1)]);
     const float amax = h16_to_f32(mb, BF16);
     const float s = (amax == 0.0f) ? 0.0f : __fdiv_rn(amax, E4M3 ? 448.0f : 127.0f);
     if (threadIdx.x == 0) *qb.scale = s;
