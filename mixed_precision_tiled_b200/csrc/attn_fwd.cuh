@@ -504,6 +504,31 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// 2^x for a pair on the FMA and ALU pipes instead of the MUFU: 2^x = 2^n * 2^f with n = rint(x)
+// (magic-number rounding) and f = x - n in [-1/2, 1/2], 2^f from a degree-3 polynomial fitted
+// to it for least relative error on that interval (max 7.7e-5, below the 16-bit rounding of
+// P), and n added to the exponent field.  x < -125 gives 0, as the flush-to-zero MUFU ex2 does
+// below -126 (masked scores are -inf).
+__device__ __forceinline__ void ex2_poly2(float x0, float x1, float& p0, float& p1) {
+  auto two = [](float v) { return f2_pack(v, v); };
+  const uint64_t M2 = two(12582912.0f);  // 1.5 * 2^23
+  const uint64_t xx = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t tt = f2_add(xx, M2);
+  const uint64_t fr = f2_sub(xx, f2_sub(tt, M2));
+  uint64_t pp = f2_fma(two(0.05518098175525665f), fr, two(0.2426345944404602f));
+  pp = f2_fma(pp, fr, two(0.6932613253593445f));
+  pp = f2_fma(pp, fr, two(0.9999262094497681f));
+  float r0, r1, t0, t1;
+  f2_unpack(pp, r0, r1);
+  f2_unpack(tt, t0, t1);
+  p0 = (x0 < -125.0f) ? 0.0f : __uint_as_float(__float_as_uint(r0) + (__float_as_uint(t0) << 23));
+  p1 = (x1 < -125.0f) ? 0.0f : __uint_as_float(__float_as_uint(r1) + (__float_as_uint(t1) << 23));
+}
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -542,6 +567,10 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
                              uint32_t tbase, const WaitCtx wc) {
   constexpr int N = C::BN, NH = C::BN / 2;
   constexpr float RESCALE_THRESH = 8.0f;
+  // At D = 128 the two partner warps of a row run their exponentials in lock step on one SM
+  // sub-partition's MUFU; moving one pair in eight to the FMA pipe shortens that phase (at
+  // D = 256 the tensor core sets the pace and the extra instructions cost more than they save).
+  constexpr bool POLY_EX2 = (C::D == 128);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = warp >> 2;   // column half
   const int q4 = warp & 3;   // TMEM lane quadrant
@@ -781,7 +810,13 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
       float x0, x1;
       f2_unpack(f2_fma(f2_pack(__uint_as_float(raw[c]), __uint_as_float(raw[c + 1])), c2, nb2),
                 x0, x1);
-      const float p0 = ex2(x0), p1 = ex2(x1);
+      float p0, p1;
+      if (POLY_EX2 && ((c >> 1) & 7) == 7) {  // one pair in eight on the FMA pipe
+        ex2_poly2(x0, x1, p0, p1);
+      } else {
+        p0 = ex2(x0);
+        p1 = ex2(x1);
+      }
       uint32_t pk;
       if (BF16) {
         __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
