@@ -10,6 +10,8 @@ What it computes, with the pages' passages it follows:
                          Dual-Path Engine", item 2; LampAttention abstract, "8-bit formats").
   * ``build_mask``    -- the packed routing bitmask, one bit per group of key tiles, 0 = FP16,
                          1 = INT8 (TileMix page, section 2, "Packed Bitmasks").
+  * ``build_mask_template`` -- the structured static routing template (TileMix page, section
+                         4, "static, data-free structured templates"; section 3, "SpTrans75").
   * ``attention``     -- routed scores, shared softmax and 16-bit-routed tiles (TileMix page,
                          section 2, "The Dual-Path Engine"; LampAttention abstract for the
                          adaptive 8-bit -> 16-bit recomputation).
@@ -82,6 +84,8 @@ def lib():
             L.orc_build_mask.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                          ctypes.c_uint64]
+            L.orc_build_mask_template.restype = None
+            L.orc_build_mask_template.argtypes = [ctypes.c_void_p] + [ctypes.c_int] * 10
             L.orc_attention.restype = ctypes.c_int
             L.orc_attention.argtypes = [ctypes.POINTER(_Args)]
             _lib = L
@@ -135,6 +139,20 @@ def build_mask(B: int, H: int, nqt: int, nkt: int, group_tiles: int, p_fp16: flo
     W = mask_words(nkt, group_tiles)
     m = np.empty((B, H, nqt, W), dtype=np.uint64)
     lib().orc_build_mask(_ptr(m), B, H, nqt, ng, W, float(p_fp16), int(seed) & (2**64 - 1))
+    return m
+
+
+def build_mask_template(B: int, H: int, Lq: int, Lk: int, bm: int, bn: int, group_tiles: int,
+                        sink: int, band: int, stride: int) -> np.ndarray:
+    """uint64 [B, H, nQT, W] structured static routing template (TileMix page, section 4,
+    "static, data-free structured templates"; section 3, the 75%-INT8 "SpTrans75"
+    configuration): group g of routing row qt is FP16 iff g < sink, |gd - g| < band, or stride
+    divides |gd - g|, gd being the group of the key aligned with the row's last query."""
+    nqt, nkt = -(-Lq // bm), -(-Lk // bn)
+    W = mask_words(nkt, group_tiles)
+    m = np.empty((B, H, nqt, W), dtype=np.uint64)
+    lib().orc_build_mask_template(_ptr(m), B, H, Lq, Lk, bm, bn, group_tiles, int(sink),
+                                  int(band), int(stride))
     return m
 
 

@@ -193,6 +193,37 @@ void orc_build_mask(uint64_t* mask, int B, int H, int nqt, int ng, int W, double
       }
 }
 
+// Structured static routing template (TileMix page, section 4 "Why It Matters": the routing
+// policy is a static, data-free structured template; section 3: the "SpTrans75" configuration
+// routes 75% of the work to INT8).  The pages give no shape; the reading used, after the
+// strided and local layouts of sparse transformers: for the routing row qt, the diagonal key
+// tile kd holds the key aligned with the row's last query, min(Lq, (qt+1) BM) - 1 + Lk - Lq
+// (bottom-right), clamped to [0, nKT - 1]; gd = kd / group_tiles is its group.  Group g is
+// FP16 (bit 0) iff g < sink, or |gd - g| < band, or stride > 0 and |gd - g| is a multiple of
+// stride; every other group is INT8 (bit 1).  Bits at g >= nG are zero.
+void orc_build_mask_template(uint64_t* mask, int B, int H, int Lq, int Lk, int bm, int bn,
+                             int group_tiles, int sink, int band, int stride) {
+  const int nqt = (Lq + bm - 1) / bm, nkt = (Lk + bn - 1) / bn;
+  const int ng = (nkt + group_tiles - 1) / group_tiles;
+  const int W = (ng + 63) / 64 > 0 ? (ng + 63) / 64 : 1;
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h)
+      for (int qt = 0; qt < nqt; ++qt) {
+        uint64_t* row = mask + (((size_t)b * H + h) * nqt + qt) * W;
+        for (int w = 0; w < W; ++w) row[w] = 0;
+        long last_q = std::min<long>(Lq, (long)(qt + 1) * bm) - 1;
+        long kd = (last_q + Lk - Lq) / bn;
+        if (last_q + Lk - Lq < 0) kd = 0;
+        if (kd > nkt - 1) kd = nkt - 1;
+        const long gd = kd / group_tiles;
+        for (int g = 0; g < ng; ++g) {
+          const long d = std::labs(gd - g);
+          const bool fp16 = g < sink || d < band || (stride > 0 && d % stride == 0);
+          if (!fp16) row[g >> 6] |= (1ull << (g & 63));
+        }
+      }
+}
+
 int orc_attention(const orc_args* a) {
   Geometry g{a->B, a->H, a->Hkv, a->Lq, a->Lk, a->D, a->bm, a->bn, a->causal, a->window};
   if (g.H % g.Hkv != 0 || g.D <= 0 || g.bm <= 0 || g.bn <= 0) return 1;

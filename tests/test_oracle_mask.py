@@ -1,9 +1,11 @@
-"""Pins of the oracle's routing-mask template (CPU only).
+"""Pins of the oracle's routing-mask templates (CPU only): the seeded Bernoulli template and
+the structured static template.
 
 Mask layout and polarity follow the TileMix page, section 2 "Packed Bitmasks": one bit per
 group of adjacent key tiles, 0 = FP16, 1 = INT8.  The bits are drawn from SplitMix64, pinned
 here to the generator's published reference outputs.
 """
+import json
 import os
 
 import numpy as np
@@ -66,3 +68,48 @@ def test_mask_draw_matches_threshold_on_generator_output():
             u = oracle.splitmix64_next(seed ^ ((idx * GAMMA) & M64))
             want = 0 if (u >> 11) * 2.0 ** -53 < p else 1
             assert (int(m[0, 0, qt, 0]) >> gi) & 1 == want
+
+
+# ---- structured static routing template (TileMix page, sections 3 and 4) ----------------
+
+def _template_bits(m, ng):
+    return ["".join(str((int(w[g >> 6]) >> (g & 63)) & 1) for g in range(ng)) for w in m]
+
+
+def test_template_matches_hand_derived_tables():
+    with open(os.path.join(GOLDEN, "mask_template_hand.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        m = oracle.build_mask_template(c["B"], c["H"], c["Lq"], c["Lk"], c["bm"], c["bn"],
+                                       c["group_tiles"], c["sink"], c["band"], c["stride"])
+        ng = len(c["bits"][0])
+        assert _template_bits(m[0, 0], ng) == c["bits"], c["name"]
+
+
+def test_template_extremes():
+    # band covering every group -> all FP16; nothing selected -> every group INT8;
+    # stride 1 divides every distance -> all FP16; unused bits stay 0
+    L, bm, gt = 4096, 128, 1
+    ng = L // bm
+    full = oracle.build_mask_template(1, 2, L, L, bm, bm, gt, 0, ng, 0)
+    assert not full.any()
+    none = oracle.build_mask_template(1, 2, L, L, bm, bm, gt, 0, 0, 0)
+    assert np.all(none == np.uint64((1 << ng) - 1))
+    s1 = oracle.build_mask_template(1, 2, L, L, bm, bm, gt, 0, 0, 1)
+    assert not s1.any()
+    # 130 groups need three words; bits 130..191 are zero
+    big = oracle.build_mask_template(1, 1, 130 * 128, 130 * 128, 128, 128, 1, 0, 0, 0)
+    assert big.shape[-1] == 3 and int(big[0, 0, 0, 2]) == 0b11
+
+
+def test_template_is_a_band_around_the_diagonal():
+    # with sink 0 and no stride, row qt's FP16 groups are exactly those within band - 1 of gd;
+    # every (b, h) gets the same data-free template
+    L, bm, gt, band = 8192, 128, 4, 3
+    m = oracle.build_mask_template(2, 3, L, L, bm, bm, gt, 0, band, 0)
+    ng = L // bm // gt
+    for qt in range(L // bm):
+        gd = qt // gt
+        want = "".join("0" if abs(gd - g) < band else "1" for g in range(ng))
+        assert _template_bits(m[1, 2, qt:qt + 1], ng)[0] == want
+    assert np.array_equal(m[0, 0], m[1, 2])
