@@ -52,18 +52,35 @@ def parse():
     ap.add_argument("--workload", default="gqa4k", choices=sorted(CONFIGS))
     ap.add_argument("--p-fp16", type=float, default=None)
     ap.add_argument("--tau", type=float, default=None)
+    ap.add_argument("--template", choices=["bernoulli", "sptrans"], default="bernoulli",
+                    help="bitmask routing template: seeded Bernoulli groups (the workloads' "
+                         "default) or the structured sink/band/stride template whose INT8 share "
+                         "is 1 - FP16 fraction (--p-fp16 0.25 = SpTrans75)")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
 
-def describe(w) -> str:
-    route = (f"bitmask g={w.group_tiles}, {w.p_fp16:.0%} FP16 groups" if w.route == "bitmask"
-             else f"adaptive tau={w.tau}")
+def describe(w, template="bernoulli", params=None) -> str:
+    if w.route != "bitmask":
+        route = f"adaptive tau={w.tau}"
+    elif template == "sptrans":
+        route = (f"bitmask g={w.group_tiles}, structured template sink/band/stride={params} "
+                 f"for {1 - w.p_fp16:.0%} INT8 pairs")
+    else:
+        route = f"bitmask g={w.group_tiles}, {w.p_fp16:.0%} FP16 groups"
     win = f", window {w.window}" if w.window else ""
     return (f"{w.name}: B={w.B} H={w.H} Hkv={w.Hkv} Lq={w.Lq} Lk={w.Lk} D={w.D} {w.dtype}, "
             f"{'causal' if w.causal else 'non-causal'}{win}, {w.bm}x{w.bn} tiles, "
             f"{w.fmt.upper()}, {route}")
+
+
+def template_params(mpt, w, p_fp16):
+    """(sink, band, stride) of the structured template whose INT8 share of the visible pairs is
+    closest to 1 - p_fp16 (the library's host-side search)."""
+    s, b, st, _ = mpt.lamp_template_for_int8_fraction(w.Lq, w.Lk, w.D, w.group_tiles,
+                                                      int(w.causal), w.window, 1.0 - p_fp16)
+    return s, b, st
 
 
 def tile_pairs(w) -> np.ndarray:
@@ -324,8 +341,15 @@ def run_reference(args, budget_s=150.0):
     if args.tau is not None:
         w = w.replace(tau=args.tau)
     t = make_workload(w)
-    mask = (oracle.build_mask(w.B, w.H, w.nqt, w.nkt, w.group_tiles, w.p_fp16, w.mask_seed)
-            if w.route == "bitmask" else None)
+    tp = None
+    if w.route != "bitmask":
+        mask = None
+    elif args.template == "sptrans":
+        import mixed_precision_tiled_b200 as mpt  # host-side parameter search only
+        tp = template_params(mpt, w, w.p_fp16)
+        mask = oracle.build_mask_template(w.B, w.H, w.Lq, w.Lk, w.bm, w.bn, w.group_tiles, *tp)
+    else:
+        mask = oracle.build_mask(w.B, w.H, w.nqt, w.nkt, w.group_tiles, w.p_fp16, w.mask_seed)
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     per_step = max(0.01, budget_s / max(1, args.steps + args.warmup))
     n_min = w.bm if w.route == "adaptive" else 1
@@ -355,7 +379,7 @@ def run_reference(args, budget_s=150.0):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": secs / max(args.steps, 1) * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64+int64", "data": "synthetic",
-            "config": {"workload": describe(w)},
+            "config": {"workload": describe(w, args.template, tp)},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -417,13 +441,23 @@ def main():
         flush.view(torch.int64).sum()
     bitmask = w.route == "bitmask"
 
+    tparams = {}
+
+    def build_mask(pf):
+        if args.template == "sptrans":
+            if pf not in tparams:
+                tparams[pf] = template_params(mpt, w, pf)
+            mpt.lamp_build_mask_template(mask, B, H, Lq, Lk, D, w.group_tiles, *tparams[pf],
+                                         stream)
+        else:
+            mpt.lamp_build_mask(mask, B, H, Lq, Lk, D, w.group_tiles, pf, w.mask_seed, stream)
+
     def step(ev_a=None, ev_b=None, p_fp16=None, mode_=None, tau_=None):
         md = mode if mode_ is None else mode_
         tu = w.tau if tau_ is None else tau_
         mpt.lamp_quant_qk(q, k, q8, k8, qs, ks, B, H, Hkv, Lq, Lk, D, md, stream)
         if bitmask:
-            mpt.lamp_build_mask(mask, B, H, Lq, Lk, D, w.group_tiles,
-                                w.p_fp16 if p_fp16 is None else p_fp16, w.mask_seed, stream)
+            build_mask(w.p_fp16 if p_fp16 is None else p_fp16)
         if ev_a is not None:
             ev_a.record(stream)
         mpt.lamp_attn_fwd_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D,
@@ -492,8 +526,7 @@ def main():
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
         if bitmask:
-            mpt.lamp_build_mask(mask, B, H, Lq, Lk, D, w.group_tiles, w.p_fp16, w.mask_seed,
-                                stream)
+            build_mask(w.p_fp16)
         mpt.lamp_attn_fwd(dq, dk, dv, o, lse, B, H, Hkv, Lq, Lk, D, int(w.causal), w.window,
                           0.0, mask if bitmask else None, w.group_tiles, mode, w.tau, stream)
         ho.copy_(o, non_blocking=True)
@@ -581,7 +614,8 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": f"int8+{w.dtype}" if w.fmt == "int8" else f"e4m3+{w.dtype}",
             "data": "synthetic",
-            "config": {"workload": describe(w), "fp16_fraction_realised": round(frac16, 4),
+            "config": {"workload": describe(w, args.template, tparams.get(w.p_fp16)),
+                       "fp16_fraction_realised": round(frac16, 4),
                        "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
                        "l2": "flushed between steps (256 MiB write, then read back); per-step CUDA events exclude the flush"},
             "roofline": {"bound": "tensor", "achieved": round(achieved, 1),

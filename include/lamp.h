@@ -88,6 +88,38 @@ int lamp_quant_qk(const void* q, const void* k, void* q8, void* k8, float* q_sca
 int lamp_build_mask(uint64_t* mask_bits, int B, int H, int Lq, int Lk, int D, int group_tiles,
                     float fp16_fraction, uint64_t seed, void* stream);
 
+/* Structured static routing template (TileMix page, section 4: the routing policy is a
+ * static, data-free structured template; section 3: the "SpTrans75" configuration routes 75%
+ * of the work to INT8).  The pages give no shape; this one follows the local and strided
+ * layouts of sparse transformers.  For routing row qt (BM query rows) the diagonal key tile
+ *   kd = clamp((min(Lq, (qt+1)*BM) - 1 + Lk - Lq) / BN, 0, nKT - 1),   gd = kd / group_tiles
+ * holds the key aligned with the row's last query (bottom-right), and group g is 16-bit
+ * (bit 0) iff g < sink_groups, or |gd - g| < band_groups, or stride_groups > 0 divides
+ * |gd - g|; every other group is 8-bit (bit 1); bits g >= nG are 0.  Every (batch, head)
+ * gets the same template.  mask_bits: device buffer of B*H*nQT*W uint64 words, fully
+ * written.  Negative template parameters return LAMP_ERR_INVALID. */
+int lamp_build_mask_template(uint64_t* mask_bits, int B, int H, int Lq, int Lk, int D,
+                             int group_tiles, int sink_groups, int band_groups,
+                             int stride_groups, void* stream);
+
+/* Host-side, no GPU work: the fraction of visible (query, key) pairs of one (batch, head)
+ * that the template above routes to 16 bits, with the causal / window limits of
+ * lamp_attn_fwd_q8.  Writes *fp16_fraction (0 when no pair is visible); LAMP_ERR_INVALID for
+ * invalid sizes, parameters or a NULL output. */
+int lamp_template_fraction(int Lq, int Lk, int D, int group_tiles, int causal, int window,
+                           int sink_groups, int band_groups, int stride_groups,
+                           double* fp16_fraction);
+
+/* Host-side, no GPU work: template parameters whose 8-bit share of the visible pairs is
+ * closest to int8_fraction (0.75 for the pages' SpTrans75), searched over sink_groups in
+ * {1, 0}, stride_groups in {0, 2, 3, ..., nG}, band_groups in {1, ..., nG} (the first best in
+ * that order).  Writes the three parameters and the realised 16-bit fraction; NULL outputs
+ * or int8_fraction outside [0, 1] return LAMP_ERR_INVALID. */
+int lamp_template_for_int8_fraction(int Lq, int Lk, int D, int group_tiles, int causal,
+                                    int window, double int8_fraction, int* sink_groups,
+                                    int* band_groups, int* stride_groups,
+                                    double* fp16_fraction);
+
 /* Routed attention forward, end to end: quantises Q and K into the library workspace
  * (lamp_set_workspace, or a cached allocation made on first use with cudaMalloc), then runs
  * the routed attention kernel.  Arguments as lamp_attn_fwd_q8 without the 8-bit operands.

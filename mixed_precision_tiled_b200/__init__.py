@@ -29,7 +29,8 @@ IN_FP16, IN_BF16 = 0x0, 0x4
 OUT_F32, OUT_INDTYPE = 0x0, 0x8
 
 EXPORTS = ("lamp_tile_shape", "lamp_mask_words", "lamp_quant_qk", "lamp_build_mask",
-           "lamp_attn_fwd", "lamp_attn_fwd_q8", "lamp_attn_fwd_noalloc", "lamp_workspace_size",
+           "lamp_build_mask_template", "lamp_template_fraction",
+           "lamp_template_for_int8_fraction", "lamp_attn_fwd", "lamp_attn_fwd_q8", "lamp_attn_fwd_noalloc", "lamp_workspace_size",
            "lamp_set_workspace", "lamp_check", "lamp_selftest_timeout", "lamp_mma_probe",
            "lamp_last_error")
 NOALLOC_MAX_BYTES = 32 << 20  # LAMP_NOALLOC_MAX_BYTES
@@ -59,6 +60,11 @@ def lib():
                 "lamp_mask_words": (_i, [_i, _i, _i]),
                 "lamp_quant_qk": (_i, [_vp, _vp, _vp, _vp, _vp, _vp] + [_i] * 7 + [_vp]),
                 "lamp_build_mask": (_i, [_vp] + [_i] * 6 + [_f, _u64, _vp]),
+                "lamp_build_mask_template": (_i, [_vp] + [_i] * 9 + [_vp]),
+                "lamp_template_fraction": (_i, [_i] * 9 + [ctypes.POINTER(ctypes.c_double)]),
+                "lamp_template_for_int8_fraction": (_i, [_i] * 6 + [ctypes.c_double]
+                                                    + [ctypes.POINTER(_i)] * 3
+                                                    + [ctypes.POINTER(ctypes.c_double)]),
                 "lamp_attn_fwd": (_i, [_vp] * 5 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp]),
                 "lamp_attn_fwd_q8": (_i, [_vp] * 9 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp, _vp]),
                 "lamp_attn_fwd_noalloc": (_i, [_vp] * 5 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp]),
@@ -128,6 +134,31 @@ def lamp_quant_qk(q, k, q8, k8, q_scale, k_scale, B, H, Hkv, Lq, Lk, D, mode, st
 def lamp_build_mask(mask_bits, B, H, Lq, Lk, D, group_tiles, fp16_fraction, seed, stream=None):
     _check(lib().lamp_build_mask(_ptr(mask_bits), B, H, Lq, Lk, D, group_tiles,
                                  float(fp16_fraction), int(seed) & (2**64 - 1), _stream(stream)))
+
+
+def lamp_build_mask_template(mask_bits, B, H, Lq, Lk, D, group_tiles, sink_groups, band_groups,
+                             stride_groups, stream=None):
+    _check(lib().lamp_build_mask_template(_ptr(mask_bits), B, H, Lq, Lk, D, group_tiles,
+                                          sink_groups, band_groups, stride_groups,
+                                          _stream(stream)))
+
+
+def lamp_template_fraction(Lq, Lk, D, group_tiles, causal, window, sink_groups, band_groups,
+                           stride_groups) -> float:
+    out = ctypes.c_double()
+    _check(lib().lamp_template_fraction(Lq, Lk, D, group_tiles, int(causal), window, sink_groups,
+                                        band_groups, stride_groups, ctypes.byref(out)))
+    return out.value
+
+
+def lamp_template_for_int8_fraction(Lq, Lk, D, group_tiles, causal, window, int8_fraction):
+    """(sink_groups, band_groups, stride_groups, realised fp16 fraction)."""
+    s, b, st, fr = _i(), _i(), _i(), ctypes.c_double()
+    _check(lib().lamp_template_for_int8_fraction(Lq, Lk, D, group_tiles, int(causal), window,
+                                                 float(int8_fraction), ctypes.byref(s),
+                                                 ctypes.byref(b), ctypes.byref(st),
+                                                 ctypes.byref(fr)))
+    return s.value, b.value, st.value, fr.value
 
 
 def lamp_attn_fwd(q, k, v, o, lse, B, H, Hkv, Lq, Lk, D, causal, window, scale, mask_bits,
@@ -221,6 +252,17 @@ def build_mask(B, H, Lq, Lk, D, group_tiles, fp16_fraction, seed, device="cuda",
     W = lamp_mask_words(Lk, D, group_tiles)
     m = torch.empty((B, H, -(-Lq // bm), W), device=device, dtype=torch.int64)
     lamp_build_mask(m, B, H, Lq, Lk, D, group_tiles, fp16_fraction, seed, stream)
+    return m
+
+
+def build_mask_template(B, H, Lq, Lk, D, group_tiles, sink_groups, band_groups, stride_groups,
+                        device="cuda", stream=None):
+    import torch
+    bm, _ = lamp_tile_shape(D)
+    W = lamp_mask_words(Lk, D, group_tiles)
+    m = torch.empty((B, H, -(-Lq // bm), W), device=device, dtype=torch.int64)
+    lamp_build_mask_template(m, B, H, Lq, Lk, D, group_tiles, sink_groups, band_groups,
+                             stride_groups, stream)
     return m
 
 

@@ -13,6 +13,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/lamp.h"
 #include "attn_fwd.cuh"
@@ -398,6 +399,58 @@ int probe_n(int n, int nsm, int iters, cudaStream_t st) {
   if (n == 128) return probe_launch<KIND, 128>(nsm, iters, st);
   return probe_launch<KIND, 256>(nsm, iters, st);
 }
+
+// ---- structured static routing template, host side -------------------------------------
+
+// Group of the diagonal key tile of routing row qt: the tile of the key aligned with the
+// row's last query (bottom-right), clamped to the key range.
+long long template_gd(int qt, int bm, int bn, int Lq, int Lk, int nkt, int group_tiles) {
+  const long long aligned = static_cast<long long>(std::min(Lq, (qt + 1) * bm)) - 1 + Lk - Lq;
+  const long long kd = aligned < 0 ? 0 : std::min<long long>(aligned / bn, nkt - 1);
+  return kd / group_tiles;
+}
+
+struct TemplateGeo {
+  int bm, bn, nqt, nkt, ng;
+  std::vector<long long> pairs;  // visible pairs of one (batch, head) per (qt, group)
+  long long total;
+};
+
+// Visible pairs per (routing row, key group) under the causal / window limits of the kernel.
+int template_geo(int Lq, int Lk, int D, int group_tiles, int causal, int window,
+                 TemplateGeo* t) {
+  if (Lq < 1 || Lk < 1 || group_tiles < 1 || window < 0 || Lq > (1 << 30) || Lk > (1 << 30))
+    return fail(LAMP_ERR_INVALID, "invalid template geometry");
+  if (window > 0 && !causal) return fail(LAMP_ERR_UNSUPPORTED, "window needs causal = 1");
+  if (tile_shape(D, &t->bm, &t->bn) != LAMP_OK)
+    return fail(LAMP_ERR_UNSUPPORTED, "head dimension D=%d not supported (64, 128, 256)", D);
+  t->nqt = (Lq + t->bm - 1) / t->bm;
+  t->nkt = (Lk + t->bn - 1) / t->bn;
+  t->ng = (t->nkt + group_tiles - 1) / group_tiles;
+  t->pairs.assign(static_cast<size_t>(t->nqt) * t->ng, 0);
+  t->total = 0;
+  const long long gk = static_cast<long long>(group_tiles) * t->bn;  // keys per group
+  for (int i = 0; i < Lq; ++i) {
+    long long lo = 0, hi = Lk - 1;
+    if (causal) {
+      hi = std::min<long long>(static_cast<long long>(i) + Lk - Lq, Lk - 1);
+      if (window > 0) lo = std::max<long long>(0, static_cast<long long>(i) + Lk - Lq - window + 1);
+    }
+    if (hi < lo) continue;
+    long long* row = t->pairs.data() + static_cast<size_t>(i / t->bm) * t->ng;
+    for (long long g = lo / gk; g <= hi / gk; ++g) {
+      const long long a = std::max(lo, g * gk), b = std::min(hi, (g + 1) * gk - 1);
+      row[g] += b - a + 1;
+      t->total += b - a + 1;
+    }
+  }
+  return LAMP_OK;
+}
+
+bool template_sixteen(long long g, long long gd, int sink, int band, int stride) {
+  const long long d = gd >= g ? gd - g : g - gd;
+  return g < sink || d < band || (stride > 0 && d % stride == 0);
+}
 }  // namespace
 
 extern "C" {
@@ -452,6 +505,107 @@ int lamp_build_mask(uint64_t* mask_bits, int B, int H, int Lq, int Lk, int D, in
   lamp::mask_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
       mask_bits, rows, ng, W, static_cast<double>(fp16_fraction), seed);
   LAMP_CUDA(cudaGetLastError(), "mask_kernel launch");
+  return LAMP_OK;
+}
+
+int lamp_build_mask_template(uint64_t* mask_bits, int B, int H, int Lq, int Lk, int D,
+                             int group_tiles, int sink_groups, int band_groups,
+                             int stride_groups, void* stream) {
+  if (!mask_bits) return fail(LAMP_ERR_INVALID, "null mask pointer");
+  int r = check_sizes(B, H, 1, Lq, Lk, D);
+  if (r) return r;
+  if (group_tiles < 1) return fail(LAMP_ERR_INVALID, "group_tiles must be >= 1");
+  if (sink_groups < 0 || band_groups < 0 || stride_groups < 0)
+    return fail(LAMP_ERR_INVALID, "template parameters must be >= 0");
+  int bm, bn;
+  tile_shape(D, &bm, &bn);
+  const int nqt = (Lq + bm - 1) / bm, nkt = (Lk + bn - 1) / bn;
+  const int ng = (nkt + group_tiles - 1) / group_tiles;
+  const int W = (ng + 63) / 64;
+  const long long rows = static_cast<long long>(B) * H * nqt;
+  const long long total = rows * W;
+  const int threads = 256;
+  const long long blocks = std::min<long long>((total + threads - 1) / threads, 148 * 16);
+  lamp::mask_template_kernel<<<static_cast<unsigned>(blocks), threads, 0,
+                               static_cast<cudaStream_t>(stream)>>>(
+      mask_bits, rows, nqt, ng, W, Lq, Lk, bm, bn, nkt, group_tiles, sink_groups, band_groups,
+      stride_groups);
+  LAMP_CUDA(cudaGetLastError(), "mask_template_kernel launch");
+  return LAMP_OK;
+}
+
+int lamp_template_fraction(int Lq, int Lk, int D, int group_tiles, int causal, int window,
+                           int sink_groups, int band_groups, int stride_groups,
+                           double* fp16_fraction) {
+  if (!fp16_fraction) return fail(LAMP_ERR_INVALID, "null output pointer");
+  if (sink_groups < 0 || band_groups < 0 || stride_groups < 0)
+    return fail(LAMP_ERR_INVALID, "template parameters must be >= 0");
+  TemplateGeo t;
+  int r = template_geo(Lq, Lk, D, group_tiles, causal, window, &t);
+  if (r) return r;
+  long long sixteen = 0;
+  for (int qt = 0; qt < t.nqt; ++qt) {
+    const long long gd = template_gd(qt, t.bm, t.bn, Lq, Lk, t.nkt, group_tiles);
+    for (int g = 0; g < t.ng; ++g)
+      if (template_sixteen(g, gd, sink_groups, band_groups, stride_groups))
+        sixteen += t.pairs[static_cast<size_t>(qt) * t.ng + g];
+  }
+  *fp16_fraction = t.total ? static_cast<double>(sixteen) / static_cast<double>(t.total) : 0.0;
+  return LAMP_OK;
+}
+
+int lamp_template_for_int8_fraction(int Lq, int Lk, int D, int group_tiles, int causal,
+                                    int window, double int8_fraction, int* sink_groups,
+                                    int* band_groups, int* stride_groups,
+                                    double* fp16_fraction) {
+  if (!sink_groups || !band_groups || !stride_groups || !fp16_fraction)
+    return fail(LAMP_ERR_INVALID, "null output pointer");
+  if (!(int8_fraction >= 0.0 && int8_fraction <= 1.0))
+    return fail(LAMP_ERR_INVALID, "int8_fraction must be in [0, 1]");
+  TemplateGeo t;
+  int r = template_geo(Lq, Lk, D, group_tiles, causal, window, &t);
+  if (r) return r;
+  // visible pairs by distance |gd - g| from the diagonal group, split into group 0 (the sink
+  // candidate) and the rest: every candidate is then scored in O(nG)
+  std::vector<long long> h0(t.ng, 0), hr(t.ng, 0);
+  for (int qt = 0; qt < t.nqt; ++qt) {
+    const long long gd = template_gd(qt, t.bm, t.bn, Lq, Lk, t.nkt, group_tiles);
+    for (int g = 0; g < t.ng; ++g) {
+      const long long d = gd >= g ? gd - g : g - gd;
+      (g == 0 ? h0 : hr)[d] += t.pairs[static_cast<size_t>(qt) * t.ng + g];
+    }
+  }
+  long long sink_pairs = 0;
+  for (int d = 0; d < t.ng; ++d) sink_pairs += h0[d];
+  const double target = 1.0 - int8_fraction;
+  double best_err = 2.0, best_frac = 0.0;
+  int best[3] = {0, 0, 0};
+  const int sinks[2] = {1, 0};
+  for (int si = 0; si < 2; ++si) {
+    const int sink = sinks[si];
+    for (int stride = 0; stride <= t.ng; stride = (stride == 0) ? 2 : stride + 1) {
+      for (int band = 1; band <= t.ng; ++band) {
+        long long sixteen = sink ? sink_pairs : 0;
+        for (int d = 0; d < t.ng; ++d) {
+          const bool sel = d < band || (stride > 0 && d % stride == 0);
+          if (sel) sixteen += hr[d] + (sink ? 0 : h0[d]);
+        }
+        const double frac = t.total ? static_cast<double>(sixteen) / t.total : 0.0;
+        const double err = std::fabs(frac - target);
+        if (err < best_err - 1e-12) {
+          best_err = err;
+          best_frac = frac;
+          best[0] = sink;
+          best[1] = band;
+          best[2] = stride;
+        }
+      }
+    }
+  }
+  *sink_groups = best[0];
+  *band_groups = best[1];
+  *stride_groups = best[2];
+  *fp16_fraction = best_frac;
   return LAMP_OK;
 }
 

@@ -10,9 +10,11 @@
 // 8-byte vector stores: 2 bytes in, 1 byte out per element.  Q and K are quantised by one
 // launch.
 //
-// Mask builder: TileMix page, section 2 "Packed Bitmasks" (one bit per group of adjacent key
-// tiles, 0 = FP16, 1 = INT8).  The template is a seeded Bernoulli draw per group bit from a
-// counter-based SplitMix64 hash (Steele, Lea, Flood 2014).
+// Mask builders: TileMix page, section 2 "Packed Bitmasks" (one bit per group of adjacent key
+// tiles, 0 = FP16, 1 = INT8).  Two templates: a seeded Bernoulli draw per group bit from a
+// counter-based SplitMix64 hash (Steele, Lea, Flood 2014), and a structured static template
+// (sink, local band and strided groups in 16 bits; section 4 "static, data-free structured
+// templates").
 #pragma once
 
 #include <cstdint>
@@ -339,6 +341,33 @@ __global__ void mask_kernel(uint64_t* __restrict__ mask, long long rows, int ng,
       const uint64_t u = splitmix64_step(seed ^ (idx * 0x9E3779B97F4A7C15ull));
       const double r = static_cast<double>(u >> 11) * 0x1.0p-53;
       if (!(r < p_fp16)) word |= 1ull << bit;
+    }
+    mask[i] = word;
+  }
+}
+
+// Structured static template: one thread per mask word.  Row qt's diagonal key tile is the
+// tile of the key aligned with its last query row (bottom-right); group g is 16-bit (bit 0)
+// iff g < sink, |gd - g| < band, or stride > 0 divides |gd - g|.
+__global__ void mask_template_kernel(uint64_t* __restrict__ mask, long long rows, int nqt,
+                                     int ng, int W, int Lq, int Lk, int bm, int bn, int nkt,
+                                     int group_tiles, int sink, int band, int stride) {
+  const long long total = rows * W;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long row = i / W;
+    const int w = static_cast<int>(i - row * W);
+    const int qt = static_cast<int>(row % nqt);
+    const long long aligned = static_cast<long long>(min(Lq, (qt + 1) * bm)) - 1 + Lk - Lq;
+    const long long kd = aligned < 0 ? 0 : min(aligned / bn, static_cast<long long>(nkt - 1));
+    const long long gd = kd / group_tiles;
+    uint64_t word = 0;
+    for (int bit = 0; bit < 64; ++bit) {
+      const int g = w * 64 + bit;
+      if (g >= ng) break;
+      const long long d = gd >= g ? gd - g : g - gd;
+      const bool sixteen = g < sink || d < band || (stride > 0 && d % stride == 0);
+      if (!sixteen) word |= 1ull << bit;
     }
     mask[i] = word;
   }

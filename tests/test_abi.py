@@ -124,3 +124,22 @@ def test_mma_probe_rejects_bad_shapes_on_host(kind, n, iters):
     with pytest.raises(mpt.LampError) as e:
         mpt.lamp_mma_probe(kind, n, iters, stream=0)
     assert e.value.code == mpt.LAMP_ERR_INVALID
+
+
+def test_template_calls_reject_bad_arguments_on_host():
+    L = mpt.lib()
+    d = ctypes.c_double()
+    i1, i2, i3 = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    # (a non-null dummy pointer: the call must fail before any launch)
+    assert L.lamp_build_mask_template(None, 1, 1, 256, 256, 64, 1, 0, 1, 0, None) == mpt.LAMP_ERR_INVALID
+    assert L.lamp_build_mask_template(0x1000, 1, 1, 256, 256, 64, 1, -1, 1, 0, None) == mpt.LAMP_ERR_INVALID
+    assert L.lamp_build_mask_template(0x1000, 1, 1, 256, 256, 64, 0, 0, 1, 0, None) == mpt.LAMP_ERR_INVALID
+    assert L.lamp_build_mask_template(0x1000, 1, 1, 256, 256, 96, 1, 0, 1, 0, None) == mpt.LAMP_ERR_UNSUPPORTED
+    assert L.lamp_template_fraction(256, 256, 64, 1, 1, 0, 0, 1, 0, None) == mpt.LAMP_ERR_INVALID
+    assert L.lamp_template_fraction(256, 256, 64, 1, 0, 64, 0, 1, 0, ctypes.byref(d)) == mpt.LAMP_ERR_UNSUPPORTED
+    assert L.lamp_template_fraction(0, 256, 64, 1, 1, 0, 0, 1, 0, ctypes.byref(d)) == mpt.LAMP_ERR_INVALID
+    assert L.lamp_template_for_int8_fraction(256, 256, 64, 1, 1, 0, 1.5, ctypes.byref(i1),
+                                             ctypes.byref(i2), ctypes.byref(i3),
+                                             ctypes.byref(d)) == mpt.LAMP_ERR_INVALID
+    assert L.lamp_template_for_int8_fraction(256, 256, 64, 1, 1, 0, 0.75, None, ctypes.byref(i2),
+                                             ctypes.byref(i3), ctypes.byref(d)) == mpt.LAMP_ERR_INVALID

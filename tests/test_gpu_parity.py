@@ -13,7 +13,8 @@ import mixed_precision_tiled_b200 as mpt
 import oracle
 from workloads import CONFIGS, make_workload, sample_rows, sample_tiles, to_16bit
 
-from _parity import EXACT_MAX_ABS, mask_to_numpy, parity_case, to_dev
+from _parity import (EXACT_MAX_ABS, check_outputs, gpu_run, mask_to_numpy, oracle_run,
+                     parity_case, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -135,6 +136,36 @@ def test_mask_builder_bit_exact(B, H, L, D, g, p):
     nqt, nkt = -(-L // bm), -(-L // bn)
     ref = oracle.build_mask(B, H, nqt, nkt, g, p, 1234)
     assert np.array_equal(mask_to_numpy(m), ref)
+
+
+@pytest.mark.parametrize("B,H,Lq,Lk,D,g,sink,band,stride", [
+    (1, 1, 512, 512, 64, 1, 1, 2, 3), (2, 3, 4096, 4096, 128, 4, 0, 1, 4),
+    (1, 2, 200, 300, 64, 2, 0, 1, 2), (1, 2, 700, 300, 128, 1, 2, 1, 0),
+    (1, 4, 16384, 16384, 256, 2, 1, 1, 4), (1, 1, 130 * 128, 130 * 128, 128, 1, 1, 3, 7)])
+def test_mask_template_bit_exact(B, H, Lq, Lk, D, g, sink, band, stride):
+    bm, bn = mpt.lamp_tile_shape(D)
+    m = mpt.build_mask_template(B, H, Lq, Lk, D, g, sink, band, stride)
+    torch.cuda.synchronize()
+    ref = oracle.build_mask_template(B, H, Lq, Lk, bm, bn, g, sink, band, stride)
+    assert np.array_equal(mask_to_numpy(m), ref)
+
+
+def test_attention_with_sptrans75_template():
+    # the 75%-INT8 structured template chosen by the library's search, end to end against the
+    # oracle on the same mask (GQA, causal, ragged tail)
+    w = CONFIGS["gqa4k"].replace(H=4, Hkv=2, Lq=1000, Lk=1000)
+    sink, band, stride, fr = mpt.lamp_template_for_int8_fraction(w.Lq, w.Lk, w.D, w.group_tiles,
+                                                                  1, 0, 0.75)
+    t = make_workload(w)
+    mask_dev = mpt.build_mask_template(w.B, w.H, w.Lq, w.Lk, w.D, w.group_tiles, sink, band,
+                                       stride)
+    mask = mask_to_numpy(mask_dev)
+    g = gpu_run(w, t, mask_dev=mask_dev)
+    r = oracle_run(w, t, mask=mask)
+    assert np.array_equal(g["route"], r["route"])
+    live = g["route"] > 0
+    assert 0 < (g["route"][live] == 2).mean() < 1
+    check_outputs(g, r, what="sptrans75")
 
 
 # ----------------------------------------------------------------- attention, small ----
