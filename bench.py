@@ -264,7 +264,9 @@ def tensor_probe(mpt, torch, stream, iters=4096):
 
 def attn_kernel_name(w):
     """The attention kernel the library dispatches for this workload."""
-    return "attn_fwd_pp_kernel" if (w.D == 128 and w.fmt == "int8") else "attn_fwd_kernel"
+    wide_mask = w.route == "bitmask" and -(-w.nkt // w.group_tiles) > 128  # more than 2 words
+    return ("attn_fwd_pp_kernel" if (w.D == 128 and w.fmt == "int8" and not wide_mask)
+            else "attn_fwd_kernel")
 
 
 def oracle_rows(w, n_per_head, seed):

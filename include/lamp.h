@@ -170,6 +170,42 @@ int lamp_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
                           float scale, const uint64_t* mask_bits, int group_tiles, int mode,
                           float tau, void* stream);
 
+/* ---- variable-length batches (TileMix page, section 4: GQA and variable-length batches
+ * are supported) --------------------------------------------------------------------------
+ * B sequences of different lengths share one launch.  Sequence b owns query rows
+ * [cu_q[b], cu_q[b+1]) and key rows [cu_k[b], cu_k[b+1]); cu_q / cu_k are device int32 arrays
+ * of B + 1 non-decreasing offsets with cu_q[0] = cu_k[0] = 0, cu_q[B] = total_q, cu_k[B] =
+ * total_k, and no sequence longer than max_q / max_k.  Sequences are independent problems:
+ * causal and window limits, routing tiles and quantisation blocks all start at each
+ * sequence's first row (bottom-right causal alignment within the sequence).
+ * Layouts (head-major, rows packed):
+ *   q, q8, o: [H][total_q][D];  k, v, k8: [Hkv][total_k][D];  lse: [H][total_q];
+ *   q_scale:  [B][H][ceil(max_q/BM)];  k_scale: [B][Hkv][ceil(max_k/BN)] (entries past a
+ *             sequence's own block count are 0);
+ *   mask_bits: [B][H][ceil(max_q/BM)][W], W = lamp_mask_words(max_k, D, group_tiles), the
+ *             layout lamp_build_mask(mask, B, H, max_q, max_k, ...) writes; route_out
+ *             likewise [B][H][ceil(max_q/BM)][ceil(max_k/BN)].
+ * Offsets are read on the device; a sequence whose offsets are decreasing or longer than
+ * max_q / max_k is clipped to [0, max] rows and never written past total_q. */
+int lamp_quant_qk_varlen(const void* q, const void* k, void* q8, void* k8, float* q_scale,
+                         float* k_scale, const int* cu_q, const int* cu_k, int B, int H,
+                         int Hkv, int max_q, int max_k, int total_q, int total_k, int D,
+                         int mode, void* stream);
+int lamp_attn_fwd_q8_varlen(const void* q, const void* k, const void* v, const void* q8,
+                            const void* k8, const float* q_scale, const float* k_scale,
+                            void* o, float* lse, const int* cu_q, const int* cu_k, int B, int H,
+                            int Hkv, int max_q, int max_k, int total_q, int total_k, int D,
+                            int causal, int window, float scale, const uint64_t* mask_bits,
+                            int group_tiles, int mode, float tau, uint8_t* route_out,
+                            void* stream);
+/* Quantise (into the library workspace, as lamp_attn_fwd) and run the routed attention on
+ * a variable-length batch. */
+int lamp_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                         const int* cu_q, const int* cu_k, int B, int H, int Hkv, int max_q,
+                         int max_k, int total_q, int total_k, int D, int causal, int window,
+                         float scale, const uint64_t* mask_bits, int group_tiles, int mode,
+                         float tau, void* stream);
+
 /* Bytes of workspace lamp_attn_fwd needs for these sizes (q8, k8 and the scales, each
  * 256-byte aligned).  0 on invalid arguments. */
 size_t lamp_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int D, int mode);

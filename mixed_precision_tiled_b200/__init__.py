@@ -30,7 +30,8 @@ OUT_F32, OUT_INDTYPE = 0x0, 0x8
 
 EXPORTS = ("lamp_tile_shape", "lamp_mask_words", "lamp_quant_qk", "lamp_build_mask",
            "lamp_build_mask_template", "lamp_template_fraction",
-           "lamp_template_for_int8_fraction", "lamp_attn_fwd", "lamp_attn_fwd_q8", "lamp_attn_fwd_noalloc", "lamp_workspace_size",
+           "lamp_template_for_int8_fraction", "lamp_quant_qk_varlen", "lamp_attn_fwd_q8_varlen",
+           "lamp_attn_fwd_varlen", "lamp_attn_fwd", "lamp_attn_fwd_q8", "lamp_attn_fwd_noalloc", "lamp_workspace_size",
            "lamp_set_workspace", "lamp_check", "lamp_selftest_timeout", "lamp_mma_probe",
            "lamp_last_error")
 NOALLOC_MAX_BYTES = 32 << 20  # LAMP_NOALLOC_MAX_BYTES
@@ -66,6 +67,9 @@ def lib():
                                                     + [ctypes.POINTER(_i)] * 3
                                                     + [ctypes.POINTER(ctypes.c_double)]),
                 "lamp_attn_fwd": (_i, [_vp] * 5 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp]),
+                "lamp_quant_qk_varlen": (_i, [_vp] * 8 + [_i] * 9 + [_vp]),
+                "lamp_attn_fwd_q8_varlen": (_i, [_vp] * 11 + [_i] * 10 + [_f, _vp, _i, _i, _f, _vp, _vp]),
+                "lamp_attn_fwd_varlen": (_i, [_vp] * 7 + [_i] * 10 + [_f, _vp, _i, _i, _f, _vp]),
                 "lamp_attn_fwd_q8": (_i, [_vp] * 9 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp, _vp]),
                 "lamp_attn_fwd_noalloc": (_i, [_vp] * 5 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp]),
                 "lamp_workspace_size": (_sz, [_i] * 7),
@@ -159,6 +163,33 @@ def lamp_template_for_int8_fraction(Lq, Lk, D, group_tiles, causal, window, int8
                                                  ctypes.byref(b), ctypes.byref(st),
                                                  ctypes.byref(fr)))
     return s.value, b.value, st.value, fr.value
+
+
+def lamp_quant_qk_varlen(q, k, q8, k8, q_scale, k_scale, cu_q, cu_k, B, H, Hkv, max_q, max_k,
+                         total_q, total_k, D, mode, stream=None):
+    _check(lib().lamp_quant_qk_varlen(_ptr(q), _ptr(k), _ptr(q8), _ptr(k8), _ptr(q_scale),
+                                      _ptr(k_scale), _ptr(cu_q), _ptr(cu_k), B, H, Hkv, max_q,
+                                      max_k, total_q, total_k, D, mode, _stream(stream)))
+
+
+def lamp_attn_fwd_q8_varlen(q, k, v, q8, k8, q_scale, k_scale, o, lse, cu_q, cu_k, B, H, Hkv,
+                            max_q, max_k, total_q, total_k, D, causal, window, scale, mask_bits,
+                            group_tiles, mode, tau, route_out=None, stream=None):
+    _check(lib().lamp_attn_fwd_q8_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8),
+                                         _ptr(q_scale), _ptr(k_scale), _ptr(o), _ptr(lse),
+                                         _ptr(cu_q), _ptr(cu_k), B, H, Hkv, max_q, max_k, total_q,
+                                         total_k, D, int(causal), window, float(scale),
+                                         _ptr(mask_bits), group_tiles, mode, float(tau),
+                                         _ptr(route_out), _stream(stream)))
+
+
+def lamp_attn_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, B, H, Hkv, max_q, max_k, total_q, total_k,
+                         D, causal, window, scale, mask_bits, group_tiles, mode, tau,
+                         stream=None):
+    _check(lib().lamp_attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_q),
+                                      _ptr(cu_k), B, H, Hkv, max_q, max_k, total_q, total_k, D,
+                                      int(causal), window, float(scale), _ptr(mask_bits),
+                                      group_tiles, mode, float(tau), _stream(stream)))
 
 
 def lamp_attn_fwd(q, k, v, o, lse, B, H, Hkv, Lq, Lk, D, causal, window, scale, mask_bits,

@@ -60,8 +60,13 @@ struct AttnParams {
   void* o;
   float* lse;
   uint8_t* route;
-  int B, H, Hkv, Lq, Lk;
+  int B, H, Hkv, Lq, Lk;  // variable-length batches: Lq, Lk = the longest sequence
   int n_ct, nqt, nkt, mask_words, group_tiles;
+  // variable-length batches: row offsets [B + 1] of the sequences in the packed [heads][rows][D]
+  // tensors (null: dense [B][heads][L][D]); q_rows = rows per head plane of Q, O and lse
+  const int* cu_q;
+  const int* cu_k;
+  int q_rows, k_rows;
   int causal, window;
   float scale_log2, tau_log2;
   int adaptive, e4m3, bf16, out_f32;
@@ -130,19 +135,53 @@ struct Plan {
   bool b16[2];     // bitmask: routing half h is 16-bit
 };
 
+// Rows of one sequence: its lengths and where its rows sit in the Q / K / V / O tensors.
+struct SeqRows {
+  int Lq, Lk;          // this sequence's query and key counts
+  int q_row0, k_row0;  // first row in the head plane (0 for dense batches)
+  int q_plane, kv_plane;  // head plane of Q / O / lse and of K / V (TMA coordinate 2)
+};
+
+// Sequence b, query head h, KV head kvh.  Offsets of a variable-length batch are clipped to
+// the tensors, so a malformed offset array cannot move a load or a store out of bounds.
+__device__ __forceinline__ SeqRows seq_rows(const AttnParams& p, int b, int h, int kvh) {
+  SeqRows s;
+  if (p.cu_q) {
+    const int q0 = min(max(__ldg(p.cu_q + b), 0), p.q_rows);
+    const int k0 = min(max(__ldg(p.cu_k + b), 0), p.k_rows);
+    s.Lq = min(max(__ldg(p.cu_q + b + 1) - q0, 0), min(p.Lq, p.q_rows - q0));
+    s.Lk = min(max(__ldg(p.cu_k + b + 1) - k0, 0), min(p.Lk, p.k_rows - k0));
+    s.q_row0 = q0;
+    s.k_row0 = k0;
+    s.q_plane = h;
+    s.kv_plane = kvh;
+  } else {
+    s.Lq = p.Lq;
+    s.Lk = p.Lk;
+    s.q_row0 = s.k_row0 = 0;
+    s.q_plane = b * p.H + h;
+    s.kv_plane = b * p.Hkv + kvh;
+  }
+  return s;
+}
+
 struct Geo {
   int b, h, kvh, ct, q0, kt_lo, n;
   int half_lo[2], half_hi[2];  // visible key range (union) of each routing half; lo > hi = none
+  SeqRows s;
 };
 
-__device__ __forceinline__ void visible_range(const AttnParams& p, int i, int& lo, int& hi) {
+// Keys visible to query row i of a sequence of Lq queries and Lk keys: bottom-right causal
+// alignment and the sliding window of the kernel arguments.
+__device__ __forceinline__ void visible_range(const AttnParams& p, int Lq, int Lk, int i,
+                                              int& lo, int& hi) {
   if (!p.causal) {
     lo = 0;
-    hi = p.Lk - 1;
+    hi = Lk - 1;
     return;
   }
-  const int off = p.Lk - p.Lq;
-  hi = min(i + off, p.Lk - 1);
+  const int off = Lk - Lq;
+  hi = min(i + off, Lk - 1);
   lo = (p.window > 0) ? max(0, i + off - p.window + 1) : 0;
 }
 
@@ -157,6 +196,7 @@ __device__ __forceinline__ Geo make_geo(const AttnParams& p) {
   g.h = bh - g.b * p.H;
   g.kvh = g.h / (p.H / p.Hkv);
   g.q0 = g.ct * C::MT;
+  g.s = seq_rows(p, g.b, g.h, g.kvh);
   const int nh = C::STACK ? 2 : 1;
   int lo_all = 1 << 30, hi_all = -1;
   for (int hh = 0; hh < 2; ++hh) {
@@ -164,11 +204,11 @@ __device__ __forceinline__ Geo make_geo(const AttnParams& p) {
     g.half_hi[hh] = 0;
     if (hh >= nh) continue;
     const int r0 = g.q0 + hh * C::BM;
-    const int r1 = min(p.Lq, r0 + (C::STACK ? C::BM : C::MT)) - 1;
+    const int r1 = min(g.s.Lq, r0 + (C::STACK ? C::BM : C::MT)) - 1;
     if (r0 > r1) continue;
     int lo0, hi0, lo1, hi1;
-    visible_range(p, r0, lo0, hi0);
-    visible_range(p, r1, lo1, hi1);
+    visible_range(p, g.s.Lq, g.s.Lk, r0, lo0, hi0);
+    visible_range(p, g.s.Lq, g.s.Lk, r1, lo1, hi1);
     const int lo = lo0, hi = hi1;
     if (hi < 0 || lo > hi) continue;
     g.half_lo[hh] = lo;
@@ -207,7 +247,7 @@ template <class C>
 __device__ __forceinline__ Plan make_plan(const AttnParams& p, const Geo& g, const KtPos& pos) {
   Plan pl;
   const int kt = pos.kt;
-  const int c0 = kt * C::BN, c1 = min(p.Lk, c0 + C::BN) - 1;
+  const int c0 = kt * C::BN, c1 = min(g.s.Lk, c0 + C::BN) - 1;
   bool need8 = false, need16 = false;
   const int g_idx = pos.g_idx;
   for (int hh = 0; hh < 2; ++hh) {
@@ -242,8 +282,8 @@ __device__ void producer_role(const AttnParams& p, const Geo& g, uint8_t* smem, 
   uint8_t* sQ16 = smem + C::OFF_Q16;
   uint8_t* sQ8 = smem + C::OFF_Q8;
   uint8_t* slots = smem + C::OFF_SLOTS;
-  const int bh_q = g.b * p.H + g.h;
-  const int bh_kv = g.b * p.Hkv + g.kvh;
+  const int pq = g.s.q_plane, pkv = g.s.kv_plane;
+  const int qrow = g.s.q_row0 + g.q0;
 
   prefetch_tmap(&p.tm_q16);
   prefetch_tmap(&p.tm_k16);
@@ -253,9 +293,9 @@ __device__ void producer_role(const AttnParams& p, const Geo& g, uint8_t* smem, 
 
   mbar_arrive_expect_tx(&bars.q_full, C::Q16_BYTES + C::Q8_BYTES);
   for (int c = 0; c < C::C16; ++c)
-    tma_load_3d(sQ16 + c * C::MT * 128, &p.tm_q16, &bars.q_full, c * 64, g.q0, bh_q);
+    tma_load_3d(sQ16 + c * C::MT * 128, &p.tm_q16, &bars.q_full, c * 64, qrow, pq);
   for (int c = 0; c < C::C8; ++c)
-    tma_load_3d(sQ8 + c * C::MT * 128, &p.tm_q8, &bars.q_full, c * 128, g.q0, bh_q);
+    tma_load_3d(sQ8 + c * C::MT * 128, &p.tm_q8, &bars.q_full, c * 128, qrow, pq);
 
   uint32_t item = 0;
   bool ok = true;
@@ -265,16 +305,16 @@ __device__ void producer_role(const AttnParams& p, const Geo& g, uint8_t* smem, 
     const uint32_t use = item / C::NS;
     if (use > 0 && !mbar_wait(&bars.empty[slot], (use - 1) & 1u, wc, W_EMPTY)) return false;
     uint8_t* dst = slots + slot * C::SLOT_BYTES;
-    const int row = kt * C::BN;
+    const int row = g.s.k_row0 + kt * C::BN;
     if (kind == 0) {
       mbar_arrive_expect_tx(&bars.full[slot], C::BN * C::D);
       for (int c = 0; c < C::C8; ++c)
-        tma_load_3d(dst + c * C::BN * 128, &p.tm_k8, &bars.full[slot], c * 128, row, bh_kv);
+        tma_load_3d(dst + c * C::BN * 128, &p.tm_k8, &bars.full[slot], c * 128, row, pkv);
     } else {
       const CUtensorMap* tm = (kind == 1) ? &p.tm_k16 : &p.tm_v;
       mbar_arrive_expect_tx(&bars.full[slot], C::BN * C::D * 2);
       for (int c = 0; c < C::C16; ++c)
-        tma_load_3d(dst + c * C::BN * 128, tm, &bars.full[slot], c * 64, row, bh_kv);
+        tma_load_3d(dst + c * C::BN * 128, tm, &bars.full[slot], c * 64, row, pkv);
     }
     ++item;
     return true;
@@ -576,13 +616,13 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
   const int q4 = warp & 3;   // TMEM lane quadrant
   const int r = q4 * 32 + lane;
   const int i = g.q0 + r;
-  const bool row_valid = i < p.Lq;
+  const bool row_valid = i < g.s.Lq;
   const int hh = C::STACK ? (r >> 6) : 0;
   const int qt_r = C::STACK ? 2 * g.ct + hh : g.ct;
   const int bh_q = g.b * p.H + g.h;
   const uint32_t lane_base = tbase + (static_cast<uint32_t>(q4 * 32) << 16);
   int lo_r = 1, hi_r = 0;
-  if (row_valid) visible_range(p, i, lo_r, hi_r);
+  if (row_valid) visible_range(p, g.s.Lq, g.s.Lk, i, lo_r, hi_r);
   const float sq = (row_valid && qt_r < p.nqt) ? __ldg(p.q_scale + static_cast<size_t>(bh_q) * p.nqt + qt_r) : 0.0f;
   const float* ks_row = p.k_scale + static_cast<size_t>(g.b * p.Hkv + g.kvh) * p.nkt;
   const float NEG_INF = -__int_as_float(0x7f800000);
@@ -895,7 +935,8 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
   const float l_rd_t = l_rd + other_rd, l_ex_t = l_ex + other_ex;
   const float inv = (l_rd_t > 0.0f) ? 1.0f / l_rd_t : 0.0f;
   constexpr int DH = C::D / 2;
-  const size_t orow = (static_cast<size_t>(bh_q) * p.Lq + (row_valid ? i : 0)) * C::D + h * DH;
+  const size_t orow =
+      (static_cast<size_t>(g.s.q_plane) * p.q_rows + g.s.q_row0 + (row_valid ? i : 0)) * C::D + h * DH;
 #pragma unroll 1
   for (int c = 0; c < DH / 32; ++c) {
     uint32_t ov[32];
@@ -937,7 +978,7 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
     }
   }
   if (h == 0 && row_valid && p.lse) {
-    p.lse[static_cast<size_t>(bh_q) * p.Lq + i] =
+    p.lse[static_cast<size_t>(g.s.q_plane) * p.q_rows + g.s.q_row0 + i] =
         (l_ex_t > 0.0f) ? m_ref * 0.69314718055994530942f + logf(l_ex_t) : NEG_INF;
   }
 }

@@ -89,6 +89,9 @@ struct PPGeo {
   int b, kvh, kt_lo, n;
   int h[2], q0[2], qt[2];  // head, first row and query-tile index of query tile X
   int lo[2], hi[2];        // visible key range (union) of query tile X; lo > hi = none
+  int Lq, Lk;              // the sequence's query and key counts
+  int q_row0, k_row0;      // its first rows in the Q / O / lse and K / V head planes
+  int q_plane[2], kv_plane;  // head planes of query tile X and of the KV head
 };
 
 // Work items.  With an even number of query heads per KV head (grouped-query attention) an item
@@ -139,16 +142,27 @@ __device__ __forceinline__ PPGeo pp_geo(const AttnParams& p, int idx) {
     }
   }
   g.kvh = g.h[0] / (p.H / p.Hkv);
+  for (int x = 0; x < 2; ++x) {
+    const SeqRows sr = seq_rows(p, g.b, g.h[x], g.kvh);
+    g.q_plane[x] = sr.q_plane;
+    if (x == 0) {
+      g.Lq = sr.Lq;
+      g.Lk = sr.Lk;
+      g.q_row0 = sr.q_row0;
+      g.k_row0 = sr.k_row0;
+      g.kv_plane = sr.kv_plane;
+    }
+  }
   int lo_all = 1 << 30, hi_all = -1;
   for (int x = 0; x < 2; ++x) {
     g.lo[x] = 1;
     g.hi[x] = 0;
     const int r0 = g.q0[x];
-    const int r1 = min(p.Lq, r0 + PPCfg::MT) - 1;
+    const int r1 = min(g.Lq, r0 + PPCfg::MT) - 1;
     if (r0 > r1) continue;
     int lo0, hi0, lo1, hi1;
-    visible_range(p, r0, lo0, hi0);
-    visible_range(p, r1, lo1, hi1);
+    visible_range(p, g.Lq, g.Lk, r0, lo0, hi0);
+    visible_range(p, g.Lq, g.Lk, r1, lo1, hi1);
     if (hi1 < 0 || lo0 > hi1) continue;
     g.lo[x] = lo0;
     g.hi[x] = hi1;
@@ -185,7 +199,7 @@ __device__ __forceinline__ MaskRow load_mask_row(const AttnParams& p, const PPGe
 }
 
 __device__ __forceinline__ bool tile_live(const PPGeo& g, const AttnParams& p, int x, int kt) {
-  const int c0 = kt * PPCfg::BN, c1 = min(p.Lk, c0 + PPCfg::BN) - 1;
+  const int c0 = kt * PPCfg::BN, c1 = min(g.Lk, c0 + PPCfg::BN) - 1;
   const int lo = x ? g.lo[1] : g.lo[0], hi = x ? g.hi[1] : g.hi[0];
   return lo <= hi && lo <= c1 && hi >= c0;
 }
@@ -262,14 +276,14 @@ __device__ void pp_producer(const AttnParams& p, uint8_t* smem, PPBars& bars, co
   prefetch_tmap(&p.tm_q8);
   prefetch_tmap(&p.tm_k8);
   uint32_t n8 = 0, n16 = 0;
-  int bh_kv = 0;
+  int pkv = 0, krow0 = 0;  // KV head plane and first key row of the current item's sequence
   auto load8 = [&](int kt) -> bool {
     const int slot = static_cast<int>(n8 % C::NS8);
     const uint32_t use = n8 / C::NS8;
     if (use > 0 && !mbar_wait(&bars.empty8[slot], (use - 1) & 1u, wc, W_EMPTY)) return false;
     mbar_arrive_expect_tx(&bars.full8[slot], C::K8_BYTES);
     tma_load_3d(smem + C::OFF_R8 + slot * C::K8_BYTES, &p.tm_k8, &bars.full8[slot], 0,
-                kt * C::BN, bh_kv);
+                krow0 + kt * C::BN, pkv);
     ++n8;
     return true;
   };
@@ -279,8 +293,8 @@ __device__ void pp_producer(const AttnParams& p, uint8_t* smem, PPBars& bars, co
     if (use > 0 && !mbar_wait(&bars.empty16[slot], (use - 1) & 1u, wc, W_EMPTY)) return false;
     uint8_t* dst = smem + C::OFF_R16 + slot * C::KV_BYTES;
     mbar_arrive_expect_tx(&bars.full16[slot], C::KV_BYTES);
-    tma_load_3d(dst, tm, &bars.full16[slot], 0, kt * C::BN, bh_kv);
-    tma_load_3d(dst + C::BN * 128, tm, &bars.full16[slot], 64, kt * C::BN, bh_kv);
+    tma_load_3d(dst, tm, &bars.full16[slot], 0, krow0 + kt * C::BN, pkv);
+    tma_load_3d(dst + C::BN * 128, tm, &bars.full16[slot], 64, krow0 + kt * C::BN, pkv);
     ++n16;
     return true;
   };
@@ -290,8 +304,12 @@ __device__ void pp_producer(const AttnParams& p, uint8_t* smem, PPBars& bars, co
     const int item = pp_item(p, r);
     if (item < 0) break;
     const PPGeo g = pp_geo(p, item);
-    bh_kv = g.b * p.Hkv + g.kvh;
-    if (!lamp_chk(g.b * p.H + g.h[1] < p.B * p.H && bh_kv < p.B * p.Hkv, 3)) { ok = false; break; }
+    pkv = g.kv_plane;
+    krow0 = g.k_row0;
+    if (!lamp_chk(g.b * p.H + g.h[1] < p.B * p.H && g.b * p.Hkv + g.kvh < p.B * p.Hkv, 3)) {
+      ok = false;
+      break;
+    }
     if (r > 0 && !(ok = mbar_wait(&bars.q_empty, (r - 1) & 1u, wc, W_EMPTY))) break;
     // the item's mask rows, read by the MMA warp after it has seen this item's Q arrive
     for (int x = 0; x < 2; ++x) {
@@ -301,12 +319,12 @@ __device__ void pp_producer(const AttnParams& p, uint8_t* smem, PPBars& bars, co
     }
     mbar_arrive_expect_tx(&bars.q_full, 2 * (C::Q16_BYTES + C::Q8_BYTES));
     for (int x = 0; x < 2; ++x) {
-      const int row = g.q0[x];
-      const int bh_q = g.b * p.H + g.h[x];
+      const int row = g.q_row0 + g.q0[x];
+      const int pq = g.q_plane[x];
       for (int c = 0; c < 2; ++c)
         tma_load_3d(smem + C::OFF_Q16 + x * C::Q16_BYTES + c * C::MT * 128, &p.tm_q16,
-                    &bars.q_full, c * 64, row, bh_q);
-      tma_load_3d(smem + C::OFF_Q8 + x * C::Q8_BYTES, &p.tm_q8, &bars.q_full, 0, row, bh_q);
+                    &bars.q_full, c * 64, row, pq);
+      tma_load_3d(smem + C::OFF_Q8 + x * C::Q8_BYTES, &p.tm_q8, &bars.q_full, 0, row, pq);
     }
     KtCursor cur = kt_first(p, g.kt_lo);
     for (int t = 0; ok && t < g.n; ++t, kt_next(p, cur)) {
@@ -579,14 +597,14 @@ __device__ __forceinline__ bool pp_softmax_item(const AttnParams& p, const PPGeo
   const int lane = threadIdx.x & 31;
   const int r = q4 * 32 + lane;
   const int i = (x ? g.q0[1] : g.q0[0]) + r;
-  const bool row_valid = i < p.Lq;
+  const bool row_valid = i < g.Lq;
   const int qt = x ? g.qt[1] : g.qt[0];
   const int bh_q = g.b * p.H + (x ? g.h[1] : g.h[0]);
   const uint32_t lane_base = tbase + (static_cast<uint32_t>(q4 * 32) << 16);
   const uint32_t s_col = static_cast<uint32_t>(x * C::BN);
   const uint32_t o_col = static_cast<uint32_t>(2 * C::BN + x * C::D);
   int lo_r = 1, hi_r = 0;
-  if (row_valid) visible_range(p, i, lo_r, hi_r);
+  if (row_valid) visible_range(p, g.Lq, g.Lk, i, lo_r, hi_r);
   const float sq = (row_valid && qt < p.nqt) ? __ldg(p.q_scale + static_cast<size_t>(bh_q) * p.nqt + qt) : 0.0f;
   const float* ks_row = p.k_scale + static_cast<size_t>(g.b * p.Hkv + g.kvh) * p.nkt;
   const float NEG_INF = -__int_as_float(0x7f800000);
@@ -792,9 +810,10 @@ __device__ __forceinline__ bool pp_softmax_item(const AttnParams& p, const PPGeo
   __syncwarp();
   if (lane == 0) mbar_arrive(&bars.o_free[x]);
   const float inv = (l_rd > 0.0f) ? 1.0f / l_rd : 0.0f;
-  const size_t orow = (static_cast<size_t>(bh_q) * p.Lq + (row_valid ? i : 0)) * C::D;
+  const int pq = x ? g.q_plane[1] : g.q_plane[0];
+  const size_t orow = (static_cast<size_t>(pq) * p.q_rows + g.q_row0 + (row_valid ? i : 0)) * C::D;
   if (row_valid &&
-      lamp_chk(orow + C::D <= static_cast<size_t>(p.B) * p.H * p.Lq * C::D, 12)) {
+      lamp_chk(orow + C::D <= static_cast<size_t>(p.cu_q ? p.H : p.B * p.H) * p.q_rows * C::D, 12)) {
     // 32-byte stores: each thread writes whole sectors of its row
     auto sc = [&](int e) { return __float_as_uint(__uint_as_float(raw[e]) * inv); };
     if (p.out_f32) {
@@ -825,7 +844,7 @@ __device__ __forceinline__ bool pp_softmax_item(const AttnParams& p, const PPGeo
     }
   }
   if (row_valid && p.lse)
-    p.lse[static_cast<size_t>(bh_q) * p.Lq + i] =
+    p.lse[static_cast<size_t>(pq) * p.q_rows + g.q_row0 + i] =
         (l_ex > 0.0f) ? m_ref * 0.69314718055994530942f + logf(l_ex) : NEG_INF;
   return true;
 }

@@ -123,14 +123,17 @@ struct WsLayout {
   size_t q8, k8, qs, ks, total;
 };
 
-WsLayout ws_layout(int B, int H, int Hkv, int Lq, int Lk, int D) {
+// q_rows / k_rows: rows per head plane of a variable-length batch (0: dense, B * L).
+WsLayout ws_layout(int B, int H, int Hkv, int Lq, int Lk, int D, int q_rows = 0, int k_rows = 0) {
   int bm, bn;
   tile_shape(D, &bm, &bn);
   const size_t nqt = (Lq + bm - 1) / bm, nkt = (Lk + bn - 1) / bn;
+  const size_t qr = q_rows ? static_cast<size_t>(q_rows) : static_cast<size_t>(B) * Lq;
+  const size_t kr = k_rows ? static_cast<size_t>(k_rows) : static_cast<size_t>(B) * Lk;
   WsLayout w;
   w.q8 = 0;
-  w.k8 = align256(static_cast<size_t>(B) * H * Lq * D);
-  w.qs = w.k8 + align256(static_cast<size_t>(B) * Hkv * Lk * D);
+  w.k8 = align256(qr * H * D);
+  w.qs = w.k8 + align256(kr * Hkv * D);
   w.ks = w.qs + align256(static_cast<size_t>(B) * H * nqt * sizeof(float));
   w.total = w.ks + align256(static_cast<size_t>(B) * Hkv * nkt * sizeof(float));
   return w;
@@ -212,7 +215,7 @@ int launch_quant_t(const lamp::QuantJob& j0, const lamp::QuantJob& j1, int D, in
 int quant_job(const void* x, void* codes, float* scales, int outer, int L, int blk,
               lamp::QuantJob* j) {
   *j = lamp::QuantJob{static_cast<const uint16_t*>(x), static_cast<uint8_t*>(codes), scales, L,
-                      blk, (L + blk - 1) / blk, 0};
+                      blk, (L + blk - 1) / blk, 0, nullptr, 0, 0};
   if (!x) return LAMP_OK;
   const long long blocks = static_cast<long long>(outer) * j->nb;
   if (blocks > 0x3FFFFFFF) return fail(LAMP_ERR_INVALID, "too many quantisation blocks");
@@ -220,14 +223,26 @@ int quant_job(const void* x, void* codes, float* scales, int outer, int L, int b
   return LAMP_OK;
 }
 
+// Variable-length batch: run (b, h) is sequence b of head plane h, cu the row offsets.
+void varlen_job(lamp::QuantJob* j, const int* cu, int heads, int total) {
+  if (!j->x) return;
+  j->cu = cu;
+  j->heads = heads;
+  j->total = total;
+}
+
 int quant_qk(const void* q, const void* k, void* q8, void* k8, float* q_scale, float* k_scale,
-             int B, int H, int Hkv, int Lq, int Lk, int D, int mode, cudaStream_t st) {
+             int B, int H, int Hkv, int Lq, int Lk, int D, int mode, cudaStream_t st,
+             const int* cu_q = nullptr, const int* cu_k = nullptr, int total_q = 0,
+             int total_k = 0) {
   int bm, bn;
   tile_shape(D, &bm, &bn);
   const bool bf16 = (mode & LAMP_IN_BF16) != 0, e4m3 = (mode & LAMP_FMT_E4M3) != 0;
   lamp::QuantJob jq, jk;
   if (int r = quant_job(q, q8, q_scale, B * H, Lq, bm, &jq)) return r;
   if (int r = quant_job(k, k8, k_scale, B * Hkv, Lk, bn, &jk)) return r;
+  if (cu_q) varlen_job(&jq, cu_q, H, total_q);
+  if (cu_k) varlen_job(&jk, cu_k, Hkv, total_k);
   if (jq.blocks + jk.blocks == 0) return LAMP_OK;
   // 16-byte vectors per thread for the larger block
   const int vec = (std::max(q ? bm : 0, k ? bn : 0) * D / 8 + lamp::QUANT_THREADS - 1) /
@@ -291,13 +306,19 @@ using Cfg64 = lamp::AttnCfg<64, 64, true>;
 using Cfg128 = lamp::AttnCfg<128, 128, false>;
 using Cfg256 = lamp::AttnCfg<256, 128, true>;
 
+// cu_q / cu_k non-null: variable-length batch of B sequences (at most Lq / Lk rows each) packed
+// into [heads][total][D] tensors.
 int attn_q8(const void* q, const void* k, const void* v, const void* q8, const void* k8,
             const float* q_scale, const float* k_scale, void* o, float* lse, int B, int H,
             int Hkv, int Lq, int Lk, int D, int causal, int window, float scale,
             const uint64_t* mask_bits, int group_tiles, int mode, float tau, uint8_t* route_out,
-            cudaStream_t st) {
+            cudaStream_t st, const int* cu_q = nullptr, const int* cu_k = nullptr,
+            int total_q = 0, int total_k = 0) {
   int r = check_sizes(B, H, Hkv, Lq, Lk, D);
   if (r) return r;
+  const bool varlen = cu_q != nullptr;
+  if (varlen && (!cu_k || total_q < 1 || total_k < 1 || total_q > (1 << 30) || total_k > (1 << 30)))
+    return fail(LAMP_ERR_INVALID, "variable-length batch needs cu_q, cu_k and positive totals");
   if (!q || !k || !v || !q8 || !k8 || !q_scale || !k_scale || !o)
     return fail(LAMP_ERR_INVALID, "null operand pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q8) || !aligned16(k8) ||
@@ -319,13 +340,16 @@ int attn_q8(const void* q, const void* k, const void* v, const void* q8, const v
   lamp::AttnParams p;
   std::memset(&p, 0, sizeof(p));
   const int BHq = B * H, BHk = B * Hkv;
-  if ((r = make_map(&p.tm_q16, q, 2, D, Lq, BHq, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))) return r;
-  if ((r = make_map(&p.tm_k16, k, 2, D, Lk, BHk, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B))) return r;
-  if ((r = make_map(&p.tm_v, v, 2, D, Lk, BHk, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B))) return r;
+  // TMA views [planes][rows][D]: dense (B*H planes of L rows) or packed (H planes of total rows)
+  const int qr = varlen ? total_q : Lq, kr = varlen ? total_k : Lk;
+  const int qpl = varlen ? H : BHq, kpl = varlen ? Hkv : BHk;
+  if ((r = make_map(&p.tm_q16, q, 2, D, qr, qpl, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))) return r;
+  if ((r = make_map(&p.tm_k16, k, 2, D, kr, kpl, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B))) return r;
+  if ((r = make_map(&p.tm_v, v, 2, D, kr, kpl, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B))) return r;
   const CUtensorMapSwizzle sw8 = (D == 64) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   const int in8 = (D == 64) ? 64 : 128;
-  if ((r = make_map(&p.tm_q8, q8, 1, D, Lq, BHq, in8, 128, sw8))) return r;
-  if ((r = make_map(&p.tm_k8, k8, 1, D, Lk, BHk, in8, bn, sw8))) return r;
+  if ((r = make_map(&p.tm_q8, q8, 1, D, qr, qpl, in8, 128, sw8))) return r;
+  if ((r = make_map(&p.tm_k8, k8, 1, D, kr, kpl, in8, bn, sw8))) return r;
   p.q_scale = q_scale;
   p.k_scale = k_scale;
   const int nqt = (Lq + bm - 1) / bm, nkt = (Lk + bn - 1) / bn;
@@ -338,6 +362,10 @@ int attn_q8(const void* q, const void* k, const void* v, const void* q8, const v
   p.lse = lse;
   p.route = route_out;
   p.B = B; p.H = H; p.Hkv = Hkv; p.Lq = Lq; p.Lk = Lk;
+  p.q_rows = qr;
+  p.k_rows = kr;
+  p.cu_q = cu_q;
+  p.cu_k = varlen ? cu_k : nullptr;
   p.n_ct = (Lq + 127) / 128;
   p.nqt = nqt;
   p.nkt = nkt;
@@ -357,7 +385,9 @@ int attn_q8(const void* q, const void* k, const void* v, const void* q8, const v
   if (route_out)
     LAMP_CUDA(cudaMemsetAsync(route_out, 0, static_cast<size_t>(BHq) * nqt * nkt, st), "memset route");
   if (D == 64) return launch_attn_cfg<Cfg64>(p, static_cast<int>(grid), st);
-  if (D == 128 && !p.e4m3) {
+  // The two-tile kernel keeps two mask words per query tile (128 key groups); wider masks go
+  // to the single-tile kernel, which reads any number of words.
+  if (D == 128 && !p.e4m3 && (adaptive || p.mask_words <= 2)) {
     // persistent CTAs: one per SM (the kernel fills the SM's shared and tensor memory), each
     // walking its share of the (batch, head, query-tile pair) work items
     // (work items as in the kernel: query-tile pairs of two heads of one KV group when the
@@ -656,6 +686,66 @@ int lamp_attn_fwd(const void* q, const void* k, const void* v, void* o, float* l
   if ((r = quant_qk(q, k, q8, k8, qs, ks, B, H, Hkv, Lq, Lk, D, mode, st))) return r;
   return attn_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D, causal, window, scale,
                  mask_bits, group_tiles, mode, tau, nullptr, st);
+}
+
+int lamp_quant_qk_varlen(const void* q, const void* k, void* q8, void* k8, float* q_scale,
+                         float* k_scale, const int* cu_q, const int* cu_k, int B, int H,
+                         int Hkv, int max_q, int max_k, int total_q, int total_k, int D,
+                         int mode, void* stream) {
+  int r = check_sizes(B, H, Hkv, max_q, max_k, D);
+  if (r) return r;
+  if ((q == nullptr) != (q8 == nullptr) || (q == nullptr) != (q_scale == nullptr) ||
+      (q != nullptr && (cu_q == nullptr || total_q < 1 || total_q > (1 << 30))))
+    return fail(LAMP_ERR_INVALID, "q, q8, q_scale, cu_q must be all set (total_q > 0) or q null");
+  if ((k == nullptr) != (k8 == nullptr) || (k == nullptr) != (k_scale == nullptr) ||
+      (k != nullptr && (cu_k == nullptr || total_k < 1 || total_k > (1 << 30))))
+    return fail(LAMP_ERR_INVALID, "k, k8, k_scale, cu_k must be all set (total_k > 0) or k null");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q8) || !aligned16(k8))
+    return fail(LAMP_ERR_INVALID, "q, k, q8, k8 must be 16-byte aligned");
+  return quant_qk(q, k, q8, k8, q_scale, k_scale, B, H, Hkv, max_q, max_k, D, mode,
+                  static_cast<cudaStream_t>(stream), cu_q, cu_k, total_q, total_k);
+}
+
+int lamp_attn_fwd_q8_varlen(const void* q, const void* k, const void* v, const void* q8,
+                            const void* k8, const float* q_scale, const float* k_scale,
+                            void* o, float* lse, const int* cu_q, const int* cu_k, int B, int H,
+                            int Hkv, int max_q, int max_k, int total_q, int total_k, int D,
+                            int causal, int window, float scale, const uint64_t* mask_bits,
+                            int group_tiles, int mode, float tau, uint8_t* route_out,
+                            void* stream) {
+  if (!cu_q || !cu_k) return fail(LAMP_ERR_INVALID, "null sequence offsets");
+  return attn_q8(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, max_q, max_k, D, causal,
+                 window, scale, mask_bits, group_tiles, mode, tau, route_out,
+                 static_cast<cudaStream_t>(stream), cu_q, cu_k, total_q, total_k);
+}
+
+int lamp_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                         const int* cu_q, const int* cu_k, int B, int H, int Hkv, int max_q,
+                         int max_k, int total_q, int total_k, int D, int causal, int window,
+                         float scale, const uint64_t* mask_bits, int group_tiles, int mode,
+                         float tau, void* stream) {
+  int r = check_sizes(B, H, Hkv, max_q, max_k, D);
+  if (r) return r;
+  if (!q || !k || !v || !o || !cu_q || !cu_k) return fail(LAMP_ERR_INVALID, "null pointer");
+  if (total_q < 1 || total_k < 1 || total_q > (1 << 30) || total_k > (1 << 30))
+    return fail(LAMP_ERR_INVALID, "totals must be positive");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned32(o))
+    return fail(LAMP_ERR_INVALID, "q, k, v must be 16-byte and o 32-byte aligned");
+  const WsLayout w = ws_layout(B, H, Hkv, max_q, max_k, D, total_q, total_k);
+  void* ws = nullptr;
+  if ((r = get_workspace(w.total, &ws))) return r;
+  auto* base = static_cast<uint8_t*>(ws);
+  uint8_t* q8 = base + w.q8;
+  uint8_t* k8 = base + w.k8;
+  float* qs = reinterpret_cast<float*>(base + w.qs);
+  float* ks = reinterpret_cast<float*>(base + w.ks);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((r = quant_qk(q, k, q8, k8, qs, ks, B, H, Hkv, max_q, max_k, D, mode, st, cu_q, cu_k,
+                    total_q, total_k)))
+    return r;
+  return attn_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, max_q, max_k, D, causal, window,
+                 scale, mask_bits, group_tiles, mode, tau, nullptr, st, cu_q, cu_k, total_q,
+                 total_k);
 }
 
 namespace {

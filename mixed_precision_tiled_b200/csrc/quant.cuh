@@ -26,12 +26,16 @@ namespace lamp {
 constexpr int QUANT_THREADS = 512;
 
 // One quantisation job: `outer` = batch*heads runs of L rows x D channels, blocks of `blk` rows.
+// Variable-length batches (cu != null): run (b, h) is rows [cu[b], cu[b+1]) of head plane h of
+// a [heads][total][D] tensor, at most L rows; scales stay [batch][heads][nb].
 struct QuantJob {
   const uint16_t* x;
   uint8_t* codes;
   float* scales;
-  int L, blk, nb;  // rows per run, rows per block, blocks per run
+  int L, blk, nb;  // rows per run (varlen: the longest sequence), rows per block, blocks per run
   int blocks;      // outer * nb
+  const int* cu;   // varlen: [batch + 1] row offsets, else null
+  int heads, total;
 };
 
 __device__ __forceinline__ float h16_to_f32(uint32_t bits, bool bf16) {
@@ -218,12 +222,19 @@ __device__ __forceinline__ QuantBlock quant_locate(const QuantJob& j0, const Qua
                                                    int D) {
   const bool second = b >= j0.blocks;
   const int id = b - (second ? j0.blocks : 0);
-  const int L = second ? j1.L : j0.L, blk = second ? j1.blk : j0.blk, nb = second ? j1.nb : j0.nb;
-  const int o = id / nb, bi = id - o * nb;
-  const int r0 = bi * blk;
-  const size_t base = (static_cast<size_t>(o) * L + r0) * D;
-  return QuantBlock{(second ? j1.x : j0.x) + base, (second ? j1.codes : j0.codes) + base,
-                    (second ? j1.scales : j0.scales) + id, min(blk, L - r0) * D / 8};
+  const QuantJob& j = second ? j1 : j0;
+  const int o = id / j.nb, bi = id - o * j.nb;
+  const int r0 = bi * j.blk;
+  if (j.cu) {  // rows of sequence o / heads in head plane o % heads, clipped to the tensor
+    const int sb = o / j.heads, h = o - sb * j.heads;
+    const int s0 = min(max(__ldg(j.cu + sb), 0), j.total);
+    const int len = min(max(__ldg(j.cu + sb + 1) - s0, 0), min(j.L, j.total - s0));
+    const int rows = min(max(len - r0, 0), j.blk);
+    const size_t base = (static_cast<size_t>(h) * j.total + s0 + min(r0, len)) * D;
+    return QuantBlock{j.x + base, j.codes + base, j.scales + id, rows * D / 8};
+  }
+  const size_t base = (static_cast<size_t>(o) * j.L + r0) * D;
+  return QuantBlock{j.x + base, j.codes + base, j.scales + id, min(j.blk, j.L - r0) * D / 8};
 }
 
 // Persistent CTAs; CTA c quantises blocks c, c + grid, c + 2 grid, ... of the combined grid
@@ -260,7 +271,8 @@ __global__ void __launch_bounds__(QUANT_THREADS, QuantPipe<VEC>::MIN_CTAS)
     const uint32_t bytes = static_cast<uint32_t>(qb.nvec) * 16u;
     uint64_t* bar = &full[i % P::NS];
     mbar_arrive_expect_tx(bar, bytes);
-    bulk_load(smem_u32(qsm + (i % P::NS) * P::STAGE_BYTES), qb.x, bytes, bar);
+    // (an empty block -- past the end of a short sequence -- completes on the arrival alone)
+    if (bytes) bulk_load(smem_u32(qsm + (i % P::NS) * P::STAGE_BYTES), qb.x, bytes, bar);
   };
   if (threadIdx.x == 0)
     for (int i = 0; i < P::NS && i < mine; ++i) issue(i);

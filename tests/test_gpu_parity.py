@@ -262,6 +262,17 @@ def test_full_size_bitmask_sampled_rows(name):
     parity_case(w, rows=rows, check_codes=False)
 
 
+def test_masks_wider_than_two_words_sampled_rows():
+    # 129 key groups (three mask words) at D = 128: the bits past group 127 must be honoured
+    w = CONFIGS["gqa4k"].replace(B=1, H=2, Hkv=1, Lq=129 * 128, Lk=129 * 128, group_tiles=1,
+                                 p_fp16=0.5)
+    assert mpt.lamp_mask_words(w.Lk, w.D, w.group_tiles) == 3
+    tail = np.array([w.Lq - 128, w.Lq - 64, w.Lq - 1])  # rows of the last query tile see group 128
+    one = np.union1d(np.linspace(0, w.Lq - 1, 45).astype(np.int64), tail)
+    rows = np.broadcast_to(one, (w.B, w.H, one.size)).copy()
+    parity_case(w, rows=rows, check_codes=False)
+
+
 def test_full_size_adaptive_sampled_tiles():
     w = CONFIGS["adaptive8k"]
     tiles = sample_tiles(w, 1)
