@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--workload", default="gqa4k", choices=sorted(CONFIGS))
     ap.add_argument("--p-fp16", type=float, default=None)
     ap.add_argument("--tau", type=float, default=None)
+    ap.add_argument("--varlen", type=int, default=0,
+                    help="run the workload's B*L query rows as a variable-length batch of this "
+                         "many sequences (seeded lengths), through the packed-layout calls")
     ap.add_argument("--template", choices=["bernoulli", "sptrans"], default="bernoulli",
                     help="bitmask routing template: seeded Bernoulli groups (the workloads' "
                          "default) or the structured sink/band/stride template whose INT8 share "
@@ -392,6 +395,163 @@ def run_reference(args, budget_s=150.0):
 
 # ------------------------------------------------------------------ CUDA arm ------------
 
+def varlen_lengths(w, n):
+    """Seeded sequence lengths (uniform in [L/4, L] before scaling) summing to B * L rows."""
+    rng = np.random.Generator(np.random.PCG64(w.seed + 99))
+    x = rng.uniform(0.25, 1.0, size=n)
+    total = w.B * w.Lq
+    lens = np.maximum(1, np.floor(x / x.sum() * total)).astype(np.int64)
+    lens[-1] += total - lens.sum()
+    return [int(v) for v in lens]
+
+
+def run_varlen(args, w, mpt, torch, dist, dev, stream, world, rank):
+    """The workload's B * L query rows as one variable-length batch (self-attention per
+    sequence, causal as the workload), through lamp_quant_qk_varlen + lamp_attn_fwd_q8_varlen
+    (device time) and lamp_attn_fwd_varlen with host buffers (e2e)."""
+    lens = varlen_lengths(w, args.varlen)
+    B, H, Hkv, D = len(lens), w.H, w.Hkv, w.D
+    L = max(lens)
+    total = sum(lens)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
+    gen = torch.Generator(device="cpu").manual_seed(w.seed)
+    q = torch.randn((H, total, D), generator=gen).to(tdt).to(dev)
+    k = torch.randn((Hkv, total, D), generator=gen).to(tdt).to(dev)
+    v = torch.randn((Hkv, total, D), generator=gen).to(tdt).to(dev)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=dev)
+    bm, bn = w.bm, w.bn
+    nqt, nkt = -(-L // bm), -(-L // bn)
+    q8 = torch.empty(q.shape, dtype=torch.uint8, device=dev)
+    k8 = torch.empty(k.shape, dtype=torch.uint8, device=dev)
+    qs = torch.empty((B, H, nqt), dtype=torch.float32, device=dev)
+    ks = torch.empty((B, Hkv, nkt), dtype=torch.float32, device=dev)
+    bitmask = w.route == "bitmask"
+    W = mpt.lamp_mask_words(L, D, w.group_tiles)
+    mask = torch.empty((B, H, nqt, W), dtype=torch.int64, device=dev)
+    o = torch.empty((H, total, D), dtype=torch.float32, device=dev)
+    lse = torch.empty((H, total), dtype=torch.float32, device=dev)
+    mode = mpt.mode_bits(w.route, w.fmt, w.dtype)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step(ev_a=None, ev_b=None):
+        mpt.lamp_quant_qk_varlen(q, k, q8, k8, qs, ks, cu, cu, B, H, Hkv, L, L, total, total, D,
+                                 mode, stream)
+        if bitmask:
+            mpt.lamp_build_mask(mask, B, H, L, L, D, w.group_tiles, w.p_fp16, w.mask_seed, stream)
+        if ev_a is not None:
+            ev_a.record(stream)
+        mpt.lamp_attn_fwd_q8_varlen(q, k, v, q8, k8, qs, ks, o, lse, cu, cu, B, H, Hkv, L, L,
+                                    total, total, D, int(w.causal), w.window, 0.0,
+                                    mask if bitmask else None, w.group_tiles, mode, w.tau, None,
+                                    stream)
+        if ev_b is not None:
+            ev_b.record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    mpt.lamp_check(stream)
+    rmap = torch.empty((B, H, nqt, nkt), dtype=torch.uint8, device=dev)
+    mpt.lamp_attn_fwd_q8_varlen(q, k, v, q8, k8, qs, ks, o, lse, cu, cu, B, H, Hkv, L, L, total,
+                                total, D, int(w.causal), w.window, 0.0, mask if bitmask else None,
+                                w.group_tiles, mode, w.tau, rmap, stream)
+    torch.cuda.synchronize()
+    rm = rmap.cpu().numpy()
+    F8 = F16 = F = 0
+    for b, n in enumerate(lens):
+        wb = w.replace(B=1, Lq=n, Lk=n)
+        f8, f16, f, _ = blended_flops(wb, rm[b:b + 1, :, :wb.nqt, :wb.nkt])
+        F8, F16, F = F8 + f8, F16 + f16, F + f
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    if world > 1:
+        dist.barrier()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    with ClockSampler(uuid if rank == 0 else None) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            flush.view(torch.int64).sum()
+            ev[i][0].record(stream)
+            step(ev[i][1], ev[i][2])
+            ev[i][3].record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    mpt.lamp_check(stream)
+    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    tot_ms, att_ms = reduce_max([sum(step_ms), statistics.fmean(attn_ms)], dev, dist)
+    ms_per_step = tot_ms / args.steps
+    # end to end: pinned host buffers in, O and lse out
+    hq = torch.empty(q.shape, dtype=tdt, pin_memory=True).copy_(q)
+    hk = torch.empty(k.shape, dtype=tdt, pin_memory=True).copy_(k)
+    hv = torch.empty(v.shape, dtype=tdt, pin_memory=True).copy_(v)
+    ho = torch.empty(o.shape, dtype=torch.float32, pin_memory=True)
+    hl = torch.empty(lse.shape, dtype=torch.float32, pin_memory=True)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        if bitmask:
+            mpt.lamp_build_mask(mask, B, H, L, L, D, w.group_tiles, w.p_fp16, w.mask_seed, stream)
+        mpt.lamp_attn_fwd_varlen(dq, dk, dv, o, lse, cu, cu, B, H, Hkv, L, L, total, total, D,
+                                 int(w.causal), w.window, 0.0, mask if bitmask else None,
+                                 w.group_tiles, mode, w.tau, stream)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    n_e2e = max(3, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms, = reduce_max([e0.elapsed_time(e1) / n_e2e], dev, dist)
+    peaks = measured_peaks()
+    P16 = peaks["bf16"] * 1e12
+    T_roof = F8 / (2.0 * P16) + F16 / P16
+    achieved = F / (att_ms * 1e-3) / 1e12
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(world * F / (ms_per_step * 1e-3) / 1e12, 2),
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": f"int8+{w.dtype}" if w.fmt == "int8" else f"e4m3+{w.dtype}",
+            "data": "synthetic",
+            "config": {"workload": describe(w) + f"; as a variable-length batch of {B} sequences",
+                       "lengths": lens, "fp16_fraction_realised": round(2.0 * F16 / F - 1.0, 4) if F else 0.0,
+                       "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "flushed between steps (256 MiB write, then read back); per-step CUDA events exclude the flush"},
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
+                         "peak": round(F / T_roof / 1e12, 1), "unit": "TFLOP/s",
+                         "frac": round(T_roof / (att_ms * 1e-3), 4), "traffic": None,
+                         "peak_basis": f"blended: F8/P8 + F16/P16, P16 = {peaks['bf16']} TFLOP/s "
+                                       f"bf16 burst ({peaks['source']}), P8 = 2 x P16 (nominal ratio)",
+                         "kernel": attn_kernel_name(w), "attn_ms": round(att_ms, 4)},
+            "e2e": {"value": round(F * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": (q.numel() + k.numel() + v.numel()) * q.element_size(),
+                    "d2h_bytes_per_step": o.numel() * 4 + lse.numel() * 4,
+                    "ms_per_step": round(e2e_ms, 4)},
+            "clocks": clk.summary(),
+            "gpu_launches": (3 if bitmask else 2) * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -417,6 +577,8 @@ def main():
         w = w.replace(p_fp16=args.p_fp16)
     if args.tau is not None:
         w = w.replace(tau=args.tau)
+    if args.varlen > 0:
+        return run_varlen(args, w, mpt, torch, dist, dev, stream, world, rank)
     t = make_workload(w)
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
 

@@ -10,6 +10,8 @@
 //
 // B200 design:
 //   * one CTA per (batch, head, 128-row query tile); grid ordered longest-first (causal);
+//     variable-length batches (TileMix page, section 4) take each sequence's lengths and first
+//     rows from offset arrays and address packed [heads][rows][D] tensors;
 //   * warp 8 (one thread) streams Q16/Q8 once and then K8 / K16 / V tiles with TMA into a
 //     ring of shared-memory slots (128-byte or 64-byte swizzled, the layouts the tensor core
 //     reads), each slot guarded by full/empty mbarriers;
