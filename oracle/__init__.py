@@ -61,6 +61,7 @@ class _Args(ctypes.Structure):
         ("hint_margin", ctypes.c_double),
         ("q_codes", ctypes.c_void_p), ("q_scales", ctypes.c_void_p),
         ("k_codes", ctypes.c_void_p), ("k_scales", ctypes.c_void_p),
+        ("skip_tau", ctypes.c_double),
     ]
 
 
@@ -158,13 +159,16 @@ def build_mask_template(B: int, H: int, Lq: int, Lk: int, bm: int, bn: int, grou
 
 def attention(q, k, v, *, bm, bn, causal=False, window=0, scale=None, mask=None, group_tiles=1,
               route="bitmask", fmt="int8", tau=0.0, rows=None, threads=0, want_codes=False,
-              route_hint=None, hint_margin=0.0):
+              route_hint=None, hint_margin=0.0, skip_tau=float("inf")):
     """Routed attention on fp32 values of 16-bit inputs.
 
     q [B,H,Lq,D], k/v [B,Hkv,Lk,D].  ``mask`` uint64 [B,H,nQT,W] or None (all 8-bit) in
     bitmask routing.  ``rows`` int64 [B,H,n] (sorted per head) restricts the output rows.
     Returns a dict with o (fp64 [B,H,R,D]), lse (fp64 [B,H,R]), route (uint8 [B,H,nQT,nKT]:
-    0 dead, 1 8-bit, 2 16-bit by mask, 3 16-bit flagged), margin (fp64, adaptive decisions).
+    0 dead, 1 8-bit, 2 16-bit by mask, 3 16-bit flagged, 4 dropped), margin (fp64, adaptive
+    decisions).  ``skip_tau`` (look-ahead mode; LATTE page, low-precision filtering of the keys
+    far below the row maximum, read per tile): a tile every row of which has t_r < m_r -
+    skip_tau is dropped; +inf never drops.
     """
     q = np.ascontiguousarray(q, dtype=np.float32)
     k = np.ascontiguousarray(k, dtype=np.float32)
@@ -204,6 +208,7 @@ def attention(q, k, v, *, bm, bn, causal=False, window=0, scale=None, mask=None,
     a.o, a.lse, a.route, a.margin = _ptr(o), _ptr(lse), _ptr(rmap), _ptr(margin)
     a.route_hint = _ptr(route_hint)
     a.hint_margin = float(hint_margin)
+    a.skip_tau = float(skip_tau)
     out = {"o": o, "lse": lse, "route": rmap, "margin": margin}
     if want_codes:
         qc = np.empty(q.shape, np.uint8)

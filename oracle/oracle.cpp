@@ -145,7 +145,8 @@ struct orc_args {
   int threads;
   double* o;               // [B,H,R,D]  R = nrows or Lq
   double* lse;             // [B,H,R]
-  uint8_t* route;          // optional [B,H,nQT,nKT]: 0 dead, 1 8-bit, 2 16-bit by mask, 3 16-bit flagged
+  uint8_t* route;          // optional [B,H,nQT,nKT]: 0 dead, 1 8-bit, 2 16-bit by mask, 3 16-bit flagged,
+                           // 4 dropped by the threshold skip
   double* margin;          // optional [B,H,nQT,nKT]: adaptive decision margin (inf elsewhere)
   const uint8_t* route_hint;  // optional [B,H,nQT,nKT]: decisions to follow where margin < hint_margin
   double hint_margin;
@@ -153,6 +154,8 @@ struct orc_args {
   float* q_scales;         // optional [B,H,nQT]
   uint8_t* k_codes;        // optional [B,Hkv,Lk,D]
   float* k_scales;         // optional [B,Hkv,nKT]
+  double skip_tau;         // look-ahead mode: drop a tile every row of which is this far below
+                           // its running max (+inf: never)
 };
 
 double orc_e4m3_decode(uint8_t c) { return e4m3_decode(c); }
@@ -349,6 +352,37 @@ int orc_attention(const orc_args* a) {
         for (int kt = 0; kt < nkt; ++kt) {
           if (!tile_live(kt)) continue;
           long c0 = (long)kt * g.bn, c1 = std::min<long>(g.Lk, c0 + g.bn) - 1;
+          size_t ti = (((size_t)b * g.H + h) * nqt + qt) * nkt + kt;
+          // Threshold skip (LATTE page: low-precision dot products filter the keys far below
+          // the row maximum; here per tile): the tile is dropped iff every row with a visible
+          // key in it has a running max and t_r < m_r - skip_tau.  Its margin: the smallest
+          // (m_r - skip_tau) - t_r when dropped, else the largest t_r - (m_r - skip_tau).
+          if (a->skip_tau != INF) {
+            bool keep = false;
+            double drop_margin = INF, keep_margin = NEG_INF;
+            for (int r = 0; r < rows_in_tile; ++r) {
+              long jl = std::max(lo[r], c0), jh = std::min(hi[r], c1);
+              if (jl > jh) continue;
+              double tr = NEG_INF;
+              for (long j = jl; j <= jh; ++j) tr = std::max(tr, score8(r, j));
+              double thr = m_run[r] - a->skip_tau;
+              if (m_run[r] == NEG_INF || tr >= thr) {
+                keep = true;
+                keep_margin = std::max(keep_margin, m_run[r] == NEG_INF ? INF : tr - thr);
+              } else {
+                drop_margin = std::min(drop_margin, thr - tr);
+              }
+            }
+            double sm = keep ? keep_margin : drop_margin;
+            if (hint && sm < a->hint_margin && (hint[kt] == 1 || hint[kt] == 3 || hint[kt] == 4))
+              keep = (hint[kt] != 4);
+            if (!keep) {
+              tile_route[kt] = 4;
+              if (a->margin) a->margin[ti] = sm;
+              continue;
+            }
+            if (a->margin) a->margin[ti] = sm;
+          }
           // Decision and its margin: the distance the deciding quantity is from the
           // threshold.  Flagged: the largest t_r - (m_r - tau) over voting rows (infinite
           // when some voting row has no running max yet).  Not flagged: the smallest
@@ -374,8 +408,7 @@ int orc_attention(const orc_args* a) {
           if (hint && margin < a->hint_margin && (hint[kt] == 1 || hint[kt] == 3))
             flagged = (hint[kt] == 3);
           tile_route[kt] = flagged ? 3 : 1;
-          size_t ti = (((size_t)b * g.H + h) * nqt + qt) * nkt + kt;
-          if (a->margin) a->margin[ti] = margin;
+          if (a->margin) a->margin[ti] = std::min(a->margin[ti], margin);
           for (int r = 0; r < rows_in_tile; ++r) {
             long jl = std::max(lo[r], c0), jh = std::min(hi[r], c1);
             if (jl > jh) continue;
@@ -406,13 +439,14 @@ int orc_attention(const orc_args* a) {
         double M = NEG_INF;
         for (long j = jl; j <= jh; ++j) {
           int rt = tile_route[j / g.bn];
-          double sc = (rt == 1) ? score8(r, j) : score16(r, j);
+          double sc = (rt == 4) ? NEG_INF : (rt == 1) ? score8(r, j) : score16(r, j);
           srow[j] = sc;
           M = std::max(M, sc);
         }
         double l = 0.0;
         for (int d = 0; d < D; ++d) orow[d] = 0.0;
         for (long j = jl; j <= jh; ++j) {
+          if (srow[j] == NEG_INF) continue;  // a dropped tile's keys
           double p = std::exp(srow[j] - M);
           l += p;
           const float* vj = vh + (size_t)j * D;

@@ -341,3 +341,58 @@ def test_tiny_golden_record_is_reproduced():
     for idx, val in g["o_samples"]:
         assert abs(r["o"][tuple(idx)] - val) < 1e-12
     assert abs(np.abs(r["o"]).sum() - g["o_abs_sum"]) < 1e-9
+
+
+# ---- threshold skip (LATTE page: low-precision filtering of keys far below the row max) ----
+
+def _skip_case():
+    # One query tile of 16 identical rows q = 4*e0; four key tiles with constant scores per tile
+    # 6, 0, -30, 1 (scale 1): the running max after tile 0 is 6.
+    D, bm, bn = 16, 16, 16
+    q = np.zeros((1, 1, 16, D), np.float32)
+    q[..., 0] = 4.0
+    k = np.zeros((1, 1, 64, D), np.float32)
+    for t, sc in enumerate([6.0, 0.0, -30.0, 1.0]):
+        k[0, 0, t * 16:(t + 1) * 16, 0] = sc / 4.0
+        k[0, 0, t * 16:(t + 1) * 16, 1] = 0.25
+    v = np.random.default_rng(1).standard_normal((1, 1, 64, D)).astype(np.float32)
+    return q, k, v, bm, bn
+
+
+def test_skip_drops_exactly_the_tiles_below_the_threshold():
+    q, k, v, bm, bn = _skip_case()
+    for fmt in ("int8", "e4m3"):
+        # tau huge: every kept tile is recomputed in 16 bits, so the output is plain attention
+        # over the kept keys; skip_tau 20 drops tile 2 only (-30 < 6 - 20; 0 and 1 are not)
+        r = oracle.attention(q, k, v, bm=bm, bn=bn, scale=1.0, route="adaptive", fmt=fmt,
+                             tau=1e9, skip_tau=20.0)
+        assert r["route"][0, 0, 0].tolist() == [3, 3, 4, 3]
+        keep = np.ones(64, bool)
+        keep[32:48] = False
+        s = exact_scores(q, k, 1.0)[..., keep]
+        o, lse = softmax_attention(s, v[:, :, keep].astype(np.float64), np.ones((16, 48), bool))
+        assert np.abs(r["o"] - o).max() < 1e-12 and np.abs(r["lse"] - lse).max() < 1e-12
+        # skip_tau 5.5 also drops tile 1 (0 < 6 - 5.5) but keeps tile 3 (1 >= 0.5)
+        r = oracle.attention(q, k, v, bm=bm, bn=bn, scale=1.0, route="adaptive", fmt=fmt,
+                             tau=1e9, skip_tau=5.5)
+        assert r["route"][0, 0, 0].tolist() == [3, 4, 4, 3]
+        # margins: tile 2 dropped by 6 - 5.5 + 30 = 30.5; tile 3 kept by 1 - 0.5 = 0.5
+        assert abs(r["margin"][0, 0, 0, 2] - 30.5) < 0.3
+        assert abs(r["margin"][0, 0, 0, 3] - 0.5) < 0.3
+
+
+def test_skip_infinite_threshold_changes_nothing_and_first_tiles_stay():
+    rng = np.random.default_rng(5)
+    q, k, v = rand_qkv(rng, 1, 2, 1, 200, 200, 64, scale=1.5)
+    kw = dict(bm=64, bn=64, causal=True, route="adaptive", fmt="int8", tau=2.0)
+    a = oracle.attention(q, k, v, **kw)
+    b = oracle.attention(q, k, v, skip_tau=float("inf"), **kw)
+    assert np.array_equal(a["o"], b["o"]) and np.array_equal(a["route"], b["route"])
+    # even skip_tau = 0 never drops a query tile's first live key tile (no running max yet),
+    # so every row keeps some key and its lse stays finite
+    c = oracle.attention(q, k, v, skip_tau=0.0, **kw)
+    assert (c["route"] == 4).any()
+    for qt in range(c["route"].shape[2]):
+        live = np.nonzero(c["route"][0, 0, qt])[0]
+        assert c["route"][0, 0, qt, live[0]] != 4
+    assert np.isfinite(c["lse"]).all()
