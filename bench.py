@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--workload", default="gqa4k", choices=sorted(CONFIGS))
     ap.add_argument("--p-fp16", type=float, default=None)
     ap.add_argument("--tau", type=float, default=None)
+    ap.add_argument("--skip-tau", type=float, default=None,
+                    help="look-ahead workloads: drop tiles this far (natural log) below the "
+                         "running max (threshold skip)")
     ap.add_argument("--varlen", type=int, default=0,
                     help="run the workload's B*L query rows as a variable-length batch of this "
                          "many sequences (seeded lengths), through the packed-layout calls")
@@ -108,14 +111,17 @@ def tile_pairs(w) -> np.ndarray:
 def blended_flops(w, route_map: np.ndarray):
     """(F8, F16, F_total, 16-bit fraction): FLOPs of 8-bit QK tiles, of 16-bit QK tiles + P.V,
     the metric's FLOPs, and the fraction of visible pairs scored in 16 bits.  Route codes: 1
-    8-bit, 2 16-bit by the mask, 3 recomputed by the look-ahead rule; a recomputed tile counts
-    its 8-bit pass too (the rule needs the 8-bit tile max of every tile to decide)."""
+    8-bit, 2 16-bit by the mask, 3 recomputed by the look-ahead rule, 4 dropped by the
+    threshold skip; a recomputed or dropped tile counts its 8-bit pass (the rules need the
+    8-bit tile max of every tile to decide), a dropped tile has no P.V.  The metric's FLOPs
+    count every visible pair."""
     pairs = tile_pairs(w)[None, None]  # broadcast over B, H
-    p8 = int((pairs * ((route_map == 1) | (route_map == 3))).sum())
+    p8 = int((pairs * ((route_map == 1) | (route_map == 3) | (route_map == 4))).sum())
     p16 = int((pairs * ((route_map == 2) | (route_map == 3))).sum())
     total = int((pairs * (route_map != 0)).sum())
+    kept = int((pairs * ((route_map != 0) & (route_map != 4))).sum())  # P.V of kept tiles
     F8 = 2 * w.D * p8
-    F16 = 2 * w.D * p16 + 2 * w.D * total
+    F16 = 2 * w.D * p16 + 2 * w.D * kept
     return F8, F16, 4 * w.D * total, (p16 / total if total else 0.0)
 
 
@@ -265,10 +271,11 @@ def tensor_probe(mpt, torch, stream, iters=4096):
     return out
 
 
-def attn_kernel_name(w):
+def attn_kernel_name(w, skip=False):
     """The attention kernel the library dispatches for this workload."""
     wide_mask = w.route == "bitmask" and -(-w.nkt // w.group_tiles) > 128  # more than 2 words
-    return ("attn_fwd_pp_kernel" if (w.D == 128 and w.fmt == "int8" and not wide_mask)
+    skip = skip and w.route == "adaptive"
+    return ("attn_fwd_pp_kernel" if (w.D == 128 and w.fmt == "int8" and not wide_mask and not skip)
             else "attn_fwd_kernel")
 
 
@@ -624,9 +631,14 @@ def main():
             build_mask(w.p_fp16 if p_fp16 is None else p_fp16)
         if ev_a is not None:
             ev_a.record(stream)
-        mpt.lamp_attn_fwd_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D,
-                             int(w.causal), w.window, 0.0, mask if bitmask else None,
-                             w.group_tiles, md, tu, None, stream)
+        if args.skip_tau is not None and not bitmask:
+            mpt.lamp_attn_fwd_q8_skip(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D,
+                                      int(w.causal), w.window, 0.0, md, tu, args.skip_tau, None,
+                                      stream)
+        else:
+            mpt.lamp_attn_fwd_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D,
+                                 int(w.causal), w.window, 0.0, mask if bitmask else None,
+                                 w.group_tiles, md, tu, None, stream)
         if ev_b is not None:
             ev_b.record(stream)
 
@@ -652,11 +664,17 @@ def main():
 
     # routing map of this configuration (untimed) -> blended-roofline FLOP split
     rmap = torch.empty((B, H, w.nqt, w.nkt), dtype=torch.uint8, device=dev)
-    mpt.lamp_attn_fwd_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D, int(w.causal),
-                         w.window, 0.0, mask if bitmask else None, w.group_tiles, mode, w.tau,
-                         rmap, stream)
+    if args.skip_tau is not None and not bitmask:
+        mpt.lamp_attn_fwd_q8_skip(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D,
+                                  int(w.causal), w.window, 0.0, mode, w.tau, args.skip_tau, rmap,
+                                  stream)
+    else:
+        mpt.lamp_attn_fwd_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D,
+                             int(w.causal), w.window, 0.0, mask if bitmask else None,
+                             w.group_tiles, mode, w.tau, rmap, stream)
     torch.cuda.synchronize()
-    F8, F16, F, frac16 = blended_flops(w, rmap.cpu().numpy())
+    rm = rmap.cpu().numpy()
+    F8, F16, F, frac16 = blended_flops(w, rm)
 
     uuid = None
     try:
@@ -778,8 +796,12 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": f"int8+{w.dtype}" if w.fmt == "int8" else f"e4m3+{w.dtype}",
             "data": "synthetic",
-            "config": {"workload": describe(w, args.template, tparams.get(w.p_fp16)),
+            "config": {"workload": describe(w, args.template, tparams.get(w.p_fp16))
+                                   + (f", threshold skip {args.skip_tau}"
+                                      if args.skip_tau is not None and not bitmask else ""),
                        "fp16_fraction_realised": round(frac16, 4),
+                       "dropped_fraction": round(float((tile_pairs(w)[None, None]
+                                                        * (rm == 4)).sum()) / max(1, F // (4 * w.D)), 4),
                        "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
                        "l2": "flushed between steps (256 MiB write, then read back); per-step CUDA events exclude the flush"},
             "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
@@ -787,7 +809,7 @@ def main():
                          "frac": round(achieved / peak_blend, 4), "traffic": traffic,
                          "peak_basis": f"blended: F8/P8 + F16/P16, P16 = {peaks['bf16']} TFLOP/s "
                                        f"bf16 burst ({peaks['source']}), P8 = 2 x P16 (nominal ratio)",
-                         "kernel": attn_kernel_name(w),
+                         "kernel": attn_kernel_name(w, args.skip_tau is not None),
                          "attn_ms": round(att_ms, 4)},
             "e2e": {"value": round(F * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -141,7 +141,7 @@ int lamp_attn_fwd(const void* q, const void* k, const void* v, void* o, float* l
  *           mode;
  *   route_out: optional device buffer uint8 [B][H][nQT][nKT] receiving the routing decision
  *           of every tile: 0 = no visible pair, 1 = 8-bit, 2 = 16-bit by mask, 3 = 16-bit by
- *           the look-ahead rule.  NULL to skip.
+ *           the look-ahead rule (4 = dropped, lamp_attn_fwd_q8_skip).  NULL to skip.
  * GQA: query head h reads KV head h / (H / Hkv). */
 int lamp_attn_fwd_q8(const void* q, const void* k, const void* v, const void* q8,
                      const void* k8, const float* q_scale, const float* k_scale, void* o,
@@ -169,6 +169,21 @@ int lamp_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
                           int B, int H, int Hkv, int Lq, int Lk, int D, int causal, int window,
                           float scale, const uint64_t* mask_bits, int group_tiles, int mode,
                           float tau, void* stream);
+
+/* Look-ahead routing with a threshold skip (LampAttention abstract: 8-bit products decide which
+ * sub-blocks need 16 bits; LATTE page: low-precision dot products filter out the keys far below
+ * the row maximum).  As lamp_attn_fwd_q8 in look-ahead mode (mode must hold
+ * LAMP_ROUTE_ADAPTIVE; no mask), plus: a live routing tile is dropped -- it contributes
+ * nothing to m, l or O -- iff every row with a visible key in it has a running max m_r and
+ * its 8-bit tile max t_r < m_r - skip_tau; kept tiles follow the look-ahead rule with tau.
+ * skip_tau is in natural-log units, tau <= skip_tau; +inf disables the skip.  A query tile's
+ * first live key tile is never dropped.  route_out marks dropped tiles 4.
+ * LAMP_ERR_INVALID for a NaN skip_tau, skip_tau < tau or a mode without LAMP_ROUTE_ADAPTIVE. */
+int lamp_attn_fwd_q8_skip(const void* q, const void* k, const void* v, const void* q8,
+                          const void* k8, const float* q_scale, const float* k_scale, void* o,
+                          float* lse, int B, int H, int Hkv, int Lq, int Lk, int D, int causal,
+                          int window, float scale, int mode, float tau, float skip_tau,
+                          uint8_t* route_out, void* stream);
 
 /* ---- variable-length batches (TileMix page, section 4: GQA and variable-length batches
  * are supported) --------------------------------------------------------------------------

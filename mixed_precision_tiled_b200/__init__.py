@@ -30,7 +30,7 @@ OUT_F32, OUT_INDTYPE = 0x0, 0x8
 
 EXPORTS = ("lamp_tile_shape", "lamp_mask_words", "lamp_quant_qk", "lamp_build_mask",
            "lamp_build_mask_template", "lamp_template_fraction",
-           "lamp_template_for_int8_fraction", "lamp_quant_qk_varlen", "lamp_attn_fwd_q8_varlen",
+           "lamp_template_for_int8_fraction", "lamp_quant_qk_varlen", "lamp_attn_fwd_q8_varlen", "lamp_attn_fwd_q8_skip",
            "lamp_attn_fwd_varlen", "lamp_attn_fwd", "lamp_attn_fwd_q8", "lamp_attn_fwd_noalloc", "lamp_workspace_size",
            "lamp_set_workspace", "lamp_check", "lamp_selftest_timeout", "lamp_mma_probe",
            "lamp_last_error")
@@ -68,6 +68,7 @@ def lib():
                                                     + [ctypes.POINTER(ctypes.c_double)]),
                 "lamp_attn_fwd": (_i, [_vp] * 5 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp]),
                 "lamp_quant_qk_varlen": (_i, [_vp] * 8 + [_i] * 9 + [_vp]),
+                "lamp_attn_fwd_q8_skip": (_i, [_vp] * 9 + [_i] * 8 + [_f, _i, _f, _f, _vp, _vp]),
                 "lamp_attn_fwd_q8_varlen": (_i, [_vp] * 11 + [_i] * 10 + [_f, _vp, _i, _i, _f, _vp, _vp]),
                 "lamp_attn_fwd_varlen": (_i, [_vp] * 7 + [_i] * 10 + [_f, _vp, _i, _i, _f, _vp]),
                 "lamp_attn_fwd_q8": (_i, [_vp] * 9 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp, _vp]),
@@ -163,6 +164,16 @@ def lamp_template_for_int8_fraction(Lq, Lk, D, group_tiles, causal, window, int8
                                                  ctypes.byref(b), ctypes.byref(st),
                                                  ctypes.byref(fr)))
     return s.value, b.value, st.value, fr.value
+
+
+def lamp_attn_fwd_q8_skip(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D,
+                          causal, window, scale, mode, tau, skip_tau, route_out=None,
+                          stream=None):
+    _check(lib().lamp_attn_fwd_q8_skip(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8),
+                                       _ptr(q_scale), _ptr(k_scale), _ptr(o), _ptr(lse), B, H,
+                                       Hkv, Lq, Lk, D, int(causal), window, float(scale), mode,
+                                       float(tau), float(skip_tau), _ptr(route_out),
+                                       _stream(stream)))
 
 
 def lamp_quant_qk_varlen(q, k, q8, k8, q_scale, k_scale, cu_q, cu_k, B, H, Hkv, max_q, max_k,
@@ -299,7 +310,7 @@ def build_mask_template(B, H, Lq, Lk, D, group_tiles, sink_groups, band_groups, 
 
 def attention_q8(q, k, v, q8, k8, q_scale, k_scale, *, causal=False, window=0, scale=0.0,
                  mask_bits=None, group_tiles=1, route="bitmask", fmt="int8", tau=0.0,
-                 out="f32", want_route=False, stream=None):
+                 out="f32", want_route=False, skip_tau=None, stream=None):
     import torch
     B, H, Lq, D = q.shape
     _, Hkv, Lk, _ = k.shape
@@ -310,7 +321,11 @@ def attention_q8(q, k, v, q8, k8, q_scale, k_scale, *, causal=False, window=0, s
     lse = torch.empty((B, H, Lq), device=q.device, dtype=torch.float32)
     rmap = (torch.empty((B, H, -(-Lq // bm), -(-Lk // bn)), device=q.device, dtype=torch.uint8)
             if want_route else None)
-    lamp_attn_fwd_q8(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D, causal,
-                     window, scale, mask_bits, group_tiles, mode_bits(route, fmt, dtype, out),
-                     tau, rmap, stream)
+    mode = mode_bits(route, fmt, dtype, out)
+    if skip_tau is not None:
+        lamp_attn_fwd_q8_skip(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D,
+                              causal, window, scale, mode, tau, skip_tau, rmap, stream)
+    else:
+        lamp_attn_fwd_q8(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D, causal,
+                         window, scale, mask_bits, group_tiles, mode, tau, rmap, stream)
     return (o, lse, rmap) if want_route else (o, lse)

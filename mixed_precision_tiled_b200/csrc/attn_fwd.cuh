@@ -71,6 +71,8 @@ struct AttnParams {
   int q_rows, k_rows;
   int causal, window;
   float scale_log2, tau_log2;
+  float skip_log2;  // look-ahead mode: drop a tile every row of which is this far below its
+                    // running max (log2 units; +inf: never)
   int adaptive, e4m3, bf16, out_f32;
   uint64_t wait_ns;
 };
@@ -480,7 +482,7 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
         uint32_t any = 0;
 #pragma unroll
         for (int w = 0; w < 8; ++w) any |= vv[w];
-        s16 = any != 0;
+        s16 = (any & 1u) != 0;  // bit 0 of the vote words: recompute
       } else {
         s16 = true;
       }
@@ -712,6 +714,7 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
     // (a zero block scale would turn masked -inf entries into NaN: keep it positive)
     const float cs8 = fmaxf(sq_scale * ks_cur, 1e-30f);
     bool sixteen = pl.first16, my16 = pl.first16;
+    bool drop = false;  // this row's routing tile is dropped by the threshold skip
     float cscale, tmax, other;
     if (C::SEP16 && pl.two_phase) {
       // The 16-bit S is in Z, issued with the tile.  Look-ahead mode: vote on the 8-bit half-row
@@ -724,8 +727,13 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
         if (!full) apply_mask(j0);
         const float hmax = raw_max();
         const float t8 = (hmax == NEG_INF) ? NEG_INF : hmax * cs8;
+        // vote word: bit 0 recompute (some row within tau of its running max), bit 1 keep (some
+        // row within skip_tau, or without a running max yet); a routing tile whose rows all
+        // miss bit 1 is dropped
         const bool vote = (t8 != NEG_INF) && (t8 >= m_true - p.tau_log2);
-        const uint32_t wv = __any_sync(0xFFFFFFFFu, vote) ? 1u : 0u;
+        const bool keep = (t8 != NEG_INF) && (m_true == NEG_INF || t8 >= m_true - p.skip_log2);
+        const uint32_t wv = (__any_sync(0xFFFFFFFFu, vote) ? 1u : 0u) |
+                            (__any_sync(0xFFFFFFFFu, keep) ? 2u : 0u);
         if (lane == 0) bars.votes[bsel][warp] = wv;
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.vote[bsel]);
@@ -737,15 +745,17 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
         if (!ok) break;
         cvb ^= 1u << bsel;
         const volatile uint32_t* vv = bars.votes[bsel];
-        bool f0, f1;
+        uint32_t v0, v1;
         if (C::STACK) {  // rows 0-63: quadrants 0, 1; rows 64-127: quadrants 2, 3
-          f0 = (vv[0] | vv[1] | vv[4] | vv[5]) != 0;
-          f1 = (vv[2] | vv[3] | vv[6] | vv[7]) != 0;
+          v0 = vv[0] | vv[1] | vv[4] | vv[5];
+          v1 = vv[2] | vv[3] | vv[6] | vv[7];
         } else {
-          f0 = f1 = (vv[0] | vv[1] | vv[2] | vv[3] | vv[4] | vv[5] | vv[6] | vv[7]) != 0;
+          v0 = v1 = vv[0] | vv[1] | vv[2] | vv[3] | vv[4] | vv[5] | vv[6] | vv[7];
         }
-        my16 = hh ? f1 : f0;
-        if (!my16) {  // not flagged: back to the 8-bit scores (still in this tile's S buffer)
+        const uint32_t vw = hh ? v1 : v0;
+        drop = (vw & 2u) == 0;
+        my16 = (vw & 1u) != 0 && !drop;
+        if (!my16 && !drop) {  // not flagged: back to the 8-bit scores (still in this tile's S buffer)
           load_s(bsel * N);
           if (!E4M3) int_to_float();
         }
@@ -768,10 +778,13 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
       if (lane == 0) mbar_arrive(&bars.z_free);
       sixteen = my16;
       cscale = my16 ? p.scale_log2 : cs8;
-      if (!full) apply_mask(j0);
-      tmax = raw_max();
-      if (!(ok = exchange(bsel, tmax, other))) break;
-      tmax = fmaxf(tmax, other);
+      tmax = NEG_INF;
+      if (!drop) {  // (both threads of a row take the same branch)
+        if (!full) apply_mask(j0);
+        tmax = raw_max();
+        if (!(ok = exchange(bsel, tmax, other))) break;
+        tmax = fmaxf(tmax, other);
+      }
     } else {
       load_s(bsel * N);
       cscale = sixteen ? p.scale_log2 : cs8;
@@ -782,10 +795,12 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
       tmax = fmaxf(tmax, other);
     }
     if (!C::SEP16 && pl.two_phase) {
-      if (p.adaptive) {
+      if (p.adaptive) {  // vote word as above: bit 0 recompute, bit 1 keep
         const float t8 = (tmax == NEG_INF) ? NEG_INF : tmax * cscale;
         const bool vote = (t8 != NEG_INF) && (t8 >= m_true - p.tau_log2);
-        const uint32_t wv = __any_sync(0xFFFFFFFFu, vote) ? 1u : 0u;
+        const bool keep = (t8 != NEG_INF) && (m_true == NEG_INF || t8 >= m_true - p.skip_log2);
+        const uint32_t wv = (__any_sync(0xFFFFFFFFu, vote) ? 1u : 0u) |
+                            (__any_sync(0xFFFFFFFFu, keep) ? 2u : 0u);
         if (lane == 0) bars.votes[bsel][warp] = wv;
       }
       tc_fence_before();
@@ -796,18 +811,22 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
       bool f0, f1;
       if (p.adaptive) {
         const volatile uint32_t* vv = bars.votes[bsel];
+        uint32_t v0, v1;
         if (C::STACK) {  // rows 0-63: quadrants 0, 1; rows 64-127: quadrants 2, 3
-          f0 = (vv[0] | vv[1] | vv[4] | vv[5]) != 0;
-          f1 = (vv[2] | vv[3] | vv[6] | vv[7]) != 0;
+          v0 = vv[0] | vv[1] | vv[4] | vv[5];
+          v1 = vv[2] | vv[3] | vv[6] | vv[7];
         } else {
-          f0 = f1 = (vv[0] | vv[1] | vv[2] | vv[3] | vv[4] | vv[5] | vv[6] | vv[7]) != 0;
+          v0 = v1 = vv[0] | vv[1] | vv[2] | vv[3] | vv[4] | vv[5] | vv[6] | vv[7];
         }
+        f0 = (v0 & 1u) != 0;
+        f1 = (v1 & 1u) != 0;
+        drop = ((hh ? v1 : v0) & 2u) == 0;
       } else {
         f0 = pl.live[0] && pl.b16[0];
         f1 = pl.live[1] && pl.b16[1];
       }
       const bool s16 = p.adaptive ? (f0 || f1) : true;
-      my16 = hh ? f1 : f0;
+      my16 = (hh ? f1 : f0) && !drop;
       if (s16) {
         if (!(ok = warp_wait(&bars.s16_full[bsel], (c16b >> bsel) & 1u, wc, W_S16))) break;
         c16b ^= 1u << bsel;
@@ -825,12 +844,12 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
     }
     if (p.route && h == 0 && lane == 0 && (q4 == 0 || (C::STACK && q4 == 2))) {
       if (hh ? pl.live[1] : pl.live[0]) {
-        const uint8_t v = my16 ? (pl.two_phase && p.adaptive ? 3 : 2) : 1;
+        const uint8_t v = drop ? 4 : my16 ? (pl.two_phase && p.adaptive ? 3 : 2) : 1;
         p.route[(static_cast<size_t>(bh_q) * p.nqt + qt_r) * p.nkt + kt] = v;
       }
     }
 
-    const float tl = (tmax == NEG_INF) ? NEG_INF : tmax * cscale;  // log2 units
+    const float tl = (drop || tmax == NEG_INF) ? NEG_INF : tmax * cscale;  // log2 units
     m_true = fmaxf(m_true, tl);
     const bool move = (tl != NEG_INF) && (m_ref == NEG_INF || tl > m_ref + RESCALE_THRESH);
     const float new_ref = move ? tl : m_ref;
@@ -842,50 +861,57 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
     // p = 2^(value * cscale - m_ref); masked entries hold -inf and give 0.  Each 32-column
     // chunk of P (16 packed columns) goes into this tile's S buffer as soon as it is ready: P.V
     // of the tile two steps back, which read that buffer, completed before S was written.
-    const float mu = (m_ref == NEG_INF) ? 0.0f : m_ref;
-    const uint64_t c2 = f2_pack(cscale, cscale);
-    const uint64_t nb2 = f2_pack(-mu, -mu);
-    uint64_t se0 = 0, se1 = 0;
-    float sr0 = 0.f, sr1 = 0.f, sr2 = 0.f, sr3 = 0.f;
+    if (drop) {  // a dropped routing tile: P = 0 for this row, (m, l) unchanged
+      const uint32_t zero[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int c = 0; c < NH; c += 2) {
-      float x0, x1;
-      f2_unpack(f2_fma(f2_pack(__uint_as_float(raw[c]), __uint_as_float(raw[c + 1])), c2, nb2),
-                x0, x1);
-      float p0, p1;
-      if (POLY_EX2 && ((c >> 1) & 7) == 7) {  // one pair in eight on the FMA pipe
-        ex2_poly2(x0, x1, p0, p1);
-      } else {
-        p0 = ex2(x0);
-        p1 = ex2(x1);
+      for (int c = 0; c < NH / 32; ++c)
+        tmem_st16(lane_base + static_cast<uint32_t>(bsel * N + h * NH + c * 16), zero);
+    } else {
+      const float mu = (m_ref == NEG_INF) ? 0.0f : m_ref;
+      const uint64_t c2 = f2_pack(cscale, cscale);
+      const uint64_t nb2 = f2_pack(-mu, -mu);
+      uint64_t se0 = 0, se1 = 0;
+      float sr0 = 0.f, sr1 = 0.f, sr2 = 0.f, sr3 = 0.f;
+#pragma unroll
+      for (int c = 0; c < NH; c += 2) {
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(raw[c]), __uint_as_float(raw[c + 1])), c2, nb2),
+                  x0, x1);
+        float p0, p1;
+        if (POLY_EX2 && ((c >> 1) & 7) == 7) {  // one pair in eight on the FMA pipe
+          ex2_poly2(x0, x1, p0, p1);
+        } else {
+          p0 = ex2(x0);
+          p1 = ex2(x1);
+        }
+        uint32_t pk;
+        if (BF16) {
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+          pk = *reinterpret_cast<uint32_t*>(&h2);
+        } else {
+          __half2 h2 = __floats2half2_rn(p0, p1);
+          pk = *reinterpret_cast<uint32_t*>(&h2);
+        }
+        if (c & 2) {
+          se1 = f2_add(se1, f2_pack(p0, p1));
+          sr2 = add_lo16<BF16>(sr2, pk);
+          sr3 = add_hi16<BF16>(sr3, pk);
+        } else {
+          se0 = f2_add(se0, f2_pack(p0, p1));
+          sr0 = add_lo16<BF16>(sr0, pk);
+          sr1 = add_hi16<BF16>(sr1, pk);
+        }
+        raw[c >> 1] = pk;
+        if ((c & 31) == 30)
+          tmem_st16(lane_base + static_cast<uint32_t>(bsel * N + h * NH + (c >> 5) * 16),
+                    &raw[(c >> 5) * 16]);
       }
-      uint32_t pk;
-      if (BF16) {
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-        pk = *reinterpret_cast<uint32_t*>(&h2);
-      } else {
-        __half2 h2 = __floats2half2_rn(p0, p1);
-        pk = *reinterpret_cast<uint32_t*>(&h2);
+      {
+        float a0, a1;
+        f2_unpack(f2_add(se0, se1), a0, a1);
+        l_ex += a0 + a1;
+        l_rd += (sr0 + sr1) + (sr2 + sr3);
       }
-      if (c & 2) {
-        se1 = f2_add(se1, f2_pack(p0, p1));
-        sr2 = add_lo16<BF16>(sr2, pk);
-        sr3 = add_hi16<BF16>(sr3, pk);
-      } else {
-        se0 = f2_add(se0, f2_pack(p0, p1));
-        sr0 = add_lo16<BF16>(sr0, pk);
-        sr1 = add_hi16<BF16>(sr1, pk);
-      }
-      raw[c >> 1] = pk;
-      if ((c & 31) == 30)
-        tmem_st16(lane_base + static_cast<uint32_t>(bsel * N + h * NH + (c >> 5) * 16),
-                  &raw[(c >> 5) * 16]);
-    }
-    {
-      float a0, a1;
-      f2_unpack(f2_add(se0, se1), a0, a1);
-      l_ex += a0 + a1;
-      l_rd += (sr0 + sr1) + (sr2 + sr3);
     }
 
     // O is rescaled (rarely: lazy reference max) once P.V of the previous tile has completed.

@@ -313,7 +313,7 @@ int attn_q8(const void* q, const void* k, const void* v, const void* q8, const v
             int Hkv, int Lq, int Lk, int D, int causal, int window, float scale,
             const uint64_t* mask_bits, int group_tiles, int mode, float tau, uint8_t* route_out,
             cudaStream_t st, const int* cu_q = nullptr, const int* cu_k = nullptr,
-            int total_q = 0, int total_k = 0) {
+            int total_q = 0, int total_k = 0, float skip_tau = INFINITY) {
   int r = check_sizes(B, H, Hkv, Lq, Lk, D);
   if (r) return r;
   const bool varlen = cu_q != nullptr;
@@ -333,6 +333,9 @@ int attn_q8(const void* q, const void* k, const void* v, const void* q8, const v
   if (!adaptive && group_tiles < 1) return fail(LAMP_ERR_INVALID, "group_tiles must be >= 1");
   if (adaptive && !(tau == tau)) return fail(LAMP_ERR_INVALID, "tau is NaN");
   if (!(scale == scale)) return fail(LAMP_ERR_INVALID, "scale is NaN");
+  const bool skip = !std::isinf(skip_tau) || skip_tau < 0.0f;
+  if (skip && (!adaptive || !(skip_tau >= tau) || !(skip_tau >= 0.0f)))
+    return fail(LAMP_ERR_INVALID, "skip_tau needs look-ahead mode and tau <= skip_tau");
   if ((r = get_encode())) return r;
 
   int bm, bn;
@@ -375,6 +378,7 @@ int attn_q8(const void* q, const void* k, const void* v, const void* q8, const v
   const float log2e = 1.4426950408889634f;
   p.scale_log2 = sc * log2e;
   p.tau_log2 = adaptive ? tau * log2e : 0.0f;
+  p.skip_log2 = skip ? skip_tau * log2e : INFINITY;
   p.adaptive = adaptive ? 1 : 0;
   p.e4m3 = (mode & LAMP_FMT_E4M3) ? 1 : 0;
   p.bf16 = (mode & LAMP_IN_BF16) ? 1 : 0;
@@ -387,7 +391,8 @@ int attn_q8(const void* q, const void* k, const void* v, const void* q8, const v
   if (D == 64) return launch_attn_cfg<Cfg64>(p, static_cast<int>(grid), st);
   // The two-tile kernel keeps two mask words per query tile (128 key groups); wider masks go
   // to the single-tile kernel, which reads any number of words.
-  if (D == 128 && !p.e4m3 && (adaptive || p.mask_words <= 2)) {
+  // (the threshold skip runs on the single-tile kernel)
+  if (D == 128 && !p.e4m3 && !skip && (adaptive || p.mask_words <= 2)) {
     // persistent CTAs: one per SM (the kernel fills the SM's shared and tensor memory), each
     // walking its share of the (batch, head, query-tile pair) work items
     // (work items as in the kernel: query-tile pairs of two heads of one KV group when the
@@ -686,6 +691,18 @@ int lamp_attn_fwd(const void* q, const void* k, const void* v, void* o, float* l
   if ((r = quant_qk(q, k, q8, k8, qs, ks, B, H, Hkv, Lq, Lk, D, mode, st))) return r;
   return attn_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D, causal, window, scale,
                  mask_bits, group_tiles, mode, tau, nullptr, st);
+}
+
+int lamp_attn_fwd_q8_skip(const void* q, const void* k, const void* v, const void* q8,
+                          const void* k8, const float* q_scale, const float* k_scale, void* o,
+                          float* lse, int B, int H, int Hkv, int Lq, int Lk, int D, int causal,
+                          int window, float scale, int mode, float tau, float skip_tau,
+                          uint8_t* route_out, void* stream) {
+  if (!(mode & LAMP_ROUTE_ADAPTIVE)) return fail(LAMP_ERR_INVALID, "the skip needs look-ahead mode");
+  if (!(skip_tau == skip_tau)) return fail(LAMP_ERR_INVALID, "skip_tau is NaN");
+  return attn_q8(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D, causal, window,
+                 scale, nullptr, 1, mode, tau, route_out, static_cast<cudaStream_t>(stream),
+                 nullptr, nullptr, 0, 0, skip_tau);
 }
 
 int lamp_quant_qk_varlen(const void* q, const void* k, void* q8, void* k8, float* q_scale,

@@ -143,3 +143,13 @@ def test_template_calls_reject_bad_arguments_on_host():
                                              ctypes.byref(d)) == mpt.LAMP_ERR_INVALID
     assert L.lamp_template_for_int8_fraction(256, 256, 64, 1, 1, 0, 0.75, None, ctypes.byref(i2),
                                              ctypes.byref(i3), ctypes.byref(d)) == mpt.LAMP_ERR_INVALID
+
+
+def test_skip_call_rejects_bad_arguments_on_host():
+    L = mpt.lib()
+    args = [0x1000] * 7 + [0x2000, 0x3000, 1, 1, 1, 256, 256, 64, 1, 0, 0.0]
+    adaptive = mpt.mode_bits("adaptive")
+    # bitmask mode, skip below tau, NaN threshold
+    assert L.lamp_attn_fwd_q8_skip(*args, mpt.mode_bits("bitmask"), 2.0, 8.0, None, None) == mpt.LAMP_ERR_INVALID
+    assert L.lamp_attn_fwd_q8_skip(*args, adaptive, 4.0, 2.0, None, None) == mpt.LAMP_ERR_INVALID
+    assert L.lamp_attn_fwd_q8_skip(*args, adaptive, 4.0, float("nan"), None, None) == mpt.LAMP_ERR_INVALID

@@ -253,6 +253,59 @@ def test_adaptive_stacked(base):
     parity_case(w, fmt="int8", tau=3.0)
 
 
+# ----------------------------------------------------------------- threshold skip -----
+
+@pytest.mark.parametrize("D,fmt,window,L", [(128, "int8", 0, 1100), (128, "e4m3", 0, 700),
+                                            (64, "int8", 0, 600), (256, "int8", 300, 900)])
+def test_threshold_skip_matches_oracle(D, fmt, window, L):
+    # look-ahead routing with a threshold skip: decisions (within the 1e-3 margin), codes and
+    # outputs against the oracle; the skip must actually drop tiles here
+    bm, bn = mpt.lamp_tile_shape(D)
+    w = small(CONFIGS["adaptive8k"], B=1, H=2, Hkv=1, Lq=L, Lk=L, D=D, bm=bm, bn=bn,
+              window=window, fmt=fmt, tau=2.0)
+    skip = 6.0
+    # inputs whose key tiles sit at seeded offsets along a direction every query shares, so
+    # that whole tiles fall far below the running max (the workload generators rarely do)
+    rng = np.random.default_rng(17)
+    u = rng.standard_normal(D)
+    u *= 0.5 * np.sqrt(D) / np.linalg.norm(u)
+    qf = rng.standard_normal((1, 2, L, D)) + 3.0 * u
+    shift = np.repeat(rng.choice([1.0, 0.0, -1.0, -2.0], size=-(-L // bn)), bn)[:L]
+    kf = rng.standard_normal((1, 1, L, D)) + shift[None, None, :, None] * u
+    vf = rng.standard_normal((1, 1, L, D))
+    q, k, v = (torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).cuda()
+               for x in (qf, kf, vf))
+    t = type("T", (), {})()
+    t.q, t.k, t.v = (x.float().cpu().numpy() for x in (q, k, v))
+    q8, k8, qs, ks = mpt.quantize(q, k, fmt=fmt)
+    o, lse, rmap = mpt.attention_q8(q, k, v, q8, k8, qs, ks, causal=True, window=window,
+                                    route="adaptive", fmt=fmt, tau=w.tau, skip_tau=skip,
+                                    want_route=True)
+    torch.cuda.synchronize()
+    mpt.lamp_check()
+    g = {"o": o.cpu().numpy().astype(np.float64), "lse": lse.cpu().numpy().astype(np.float64),
+         "route": rmap.cpu().numpy()}
+    r = oracle.attention(t.q, t.k, t.v, bm=bm, bn=bn, causal=True, window=window,
+                         route="adaptive", fmt=fmt, tau=w.tau, skip_tau=skip,
+                         route_hint=g["route"], hint_margin=1e-3)
+    assert np.array_equal(g["route"], r["route"])
+    assert (g["route"] == 4).any() and (g["route"] == 3).any()
+    check_outputs(g, r, what=f"skip D={D} {fmt}")
+
+
+def test_threshold_skip_infinite_is_the_look_ahead_rule():
+    w = small(CONFIGS["adaptive8k"], B=1, H=2, Hkv=1, Lq=600, Lk=600, fmt="e4m3", tau=3.0)
+    t = make_workload(w)
+    q, k, v = (to_dev(x, w.dtype) for x in (t.q_bits, t.k_bits, t.v_bits))
+    q8, k8, qs, ks = mpt.quantize(q, k, fmt="e4m3")
+    kw = dict(causal=True, route="adaptive", fmt="e4m3", tau=3.0, want_route=True)
+    a = mpt.attention_q8(q, k, v, q8, k8, qs, ks, **kw)
+    b = mpt.attention_q8(q, k, v, q8, k8, qs, ks, skip_tau=float("inf"), **kw)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
 # ----------------------------------------------------------------- full size, sampled --
 
 @pytest.mark.parametrize("name", ["gqa4k", "gemma_local16k", "long32k"])
