@@ -326,7 +326,7 @@ __device__ void producer_role(const AttnParams& p, const Geo& g, uint8_t* smem, 
 
   // Order of the loads = order in which the MMA warp consumes them: the first S operand of
   // tile t+1 before V of tile t; the 16-bit K of a two-phase tile right behind its 8-bit K
-  // (separate region Z) or after the next tile's first operand (shared columns).
+  // (separate region Z) or, in shared columns, ahead of the next tile's first operand.
   KtPos pos;
   pos.init(p, g.kt_lo);
   Plan cur = make_plan<C>(p, g, pos);
@@ -335,13 +335,13 @@ __device__ void producer_role(const AttnParams& p, const Geo& g, uint8_t* smem, 
   for (int t = 0; ok && t < g.n; ++t) {
     const int kt = g.kt_lo + t;
     Plan nxt;
+    if (!C::SEP16 && cur.two_phase && !(ok = load(1, kt))) break;
     if (t + 1 < g.n) {
       pos.next(p);
       nxt = make_plan<C>(p, g, pos);
       if (!(ok = load(nxt.first16 ? 1 : 0, kt + 1))) break;
       if (C::SEP16 && nxt.two_phase && !(ok = load(1, kt + 1))) break;
     }
-    if (!C::SEP16 && cur.two_phase && !(ok = load(1, kt))) break;
     if (!(ok = load(2, kt))) break;
     cur = nxt;
   }
@@ -461,15 +461,8 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
   for (int t = 0; ok && t < g.n; ++t) {
     const int bsel = t & 1;
     Plan nxt;
-    if (t + 1 < g.n) {
-      pos.next(p);
-      nxt = make_plan<C>(p, g, pos);
-      if (!(ok = take(slot))) break;
-      issue_s(buf(t + 1), nxt.first16, slot);
-      commit(&bars.s_full[(t + 1) & 1]);
-      commit(&bars.empty[slot]);
-      if (C::SEP16 && nxt.two_phase && !(ok = issue_z())) break;
-    }
+    // Shared columns: a two-phase tile's 16-bit S goes ahead of the next tile's first S, so
+    // that the rows waiting for it do not wait for that one too.
     if (!C::SEP16 && cur.two_phase) {
       int slot16;
       if (!(ok = take(slot16))) break;
@@ -493,6 +486,15 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
       } else if (leader) {
         mbar_arrive(&bars.empty[slot16]);
       }
+    }
+    if (t + 1 < g.n) {
+      pos.next(p);
+      nxt = make_plan<C>(p, g, pos);
+      if (!(ok = take(slot))) break;
+      issue_s(buf(t + 1), nxt.first16, slot);
+      commit(&bars.s_full[(t + 1) & 1]);
+      commit(&bars.empty[slot]);
+      if (C::SEP16 && nxt.two_phase && !(ok = issue_z())) break;
     }
     if (!(ok = mbar_wait(&bars.p_full[bsel], static_cast<uint32_t>(t >> 1) & 1u, wc, W_PFULL))) break;
     tc_fence_after();
@@ -606,7 +608,7 @@ __device__ __forceinline__ float add_hi16(float acc, uint32_t pk) {
 // half of the thread's own S columns (each 32-column chunk stored when ready), and keep two
 // partial row sums: of the exact p (for lse) and of the rounded p that the P.V MMA multiplies
 // (for O).  Both threads of a row take identical decisions from identical inputs.
-template <class C, bool BF16, bool E4M3>
+template <class C, bool BF16, bool E4M3, bool SKIP>
 __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars& bars,
                              uint32_t tbase, const WaitCtx wc) {
   constexpr int N = C::BN, NH = C::BN / 2;
@@ -731,9 +733,11 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
         // row within skip_tau, or without a running max yet); a routing tile whose rows all
         // miss bit 1 is dropped
         const bool vote = (t8 != NEG_INF) && (t8 >= m_true - p.tau_log2);
-        const bool keep = (t8 != NEG_INF) && (m_true == NEG_INF || t8 >= m_true - p.skip_log2);
-        const uint32_t wv = (__any_sync(0xFFFFFFFFu, vote) ? 1u : 0u) |
-                            (__any_sync(0xFFFFFFFFu, keep) ? 2u : 0u);
+        uint32_t wv = __any_sync(0xFFFFFFFFu, vote) ? 1u : 0u;
+        if (SKIP) {
+          const bool keep = (t8 != NEG_INF) && (m_true == NEG_INF || t8 >= m_true - p.skip_log2);
+          wv |= __any_sync(0xFFFFFFFFu, keep) ? 2u : 0u;
+        }
         if (lane == 0) bars.votes[bsel][warp] = wv;
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.vote[bsel]);
@@ -753,7 +757,7 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
           v0 = v1 = vv[0] | vv[1] | vv[2] | vv[3] | vv[4] | vv[5] | vv[6] | vv[7];
         }
         const uint32_t vw = hh ? v1 : v0;
-        drop = (vw & 2u) == 0;
+        drop = SKIP && (vw & 2u) == 0;
         my16 = (vw & 1u) != 0 && !drop;
         if (!my16 && !drop) {  // not flagged: back to the 8-bit scores (still in this tile's S buffer)
           load_s(bsel * N);
@@ -798,9 +802,11 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
       if (p.adaptive) {  // vote word as above: bit 0 recompute, bit 1 keep
         const float t8 = (tmax == NEG_INF) ? NEG_INF : tmax * cscale;
         const bool vote = (t8 != NEG_INF) && (t8 >= m_true - p.tau_log2);
-        const bool keep = (t8 != NEG_INF) && (m_true == NEG_INF || t8 >= m_true - p.skip_log2);
-        const uint32_t wv = (__any_sync(0xFFFFFFFFu, vote) ? 1u : 0u) |
-                            (__any_sync(0xFFFFFFFFu, keep) ? 2u : 0u);
+        uint32_t wv = __any_sync(0xFFFFFFFFu, vote) ? 1u : 0u;
+        if (SKIP) {
+          const bool keep = (t8 != NEG_INF) && (m_true == NEG_INF || t8 >= m_true - p.skip_log2);
+          wv |= __any_sync(0xFFFFFFFFu, keep) ? 2u : 0u;
+        }
         if (lane == 0) bars.votes[bsel][warp] = wv;
       }
       tc_fence_before();
@@ -820,7 +826,7 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
         }
         f0 = (v0 & 1u) != 0;
         f1 = (v1 & 1u) != 0;
-        drop = ((hh ? v1 : v0) & 2u) == 0;
+        drop = SKIP && ((hh ? v1 : v0) & 2u) == 0;
       } else {
         f0 = pl.live[0] && pl.b16[0];
         f1 = pl.live[1] && pl.b16[1];
@@ -1013,7 +1019,7 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
 
 // ------------------------------------------------------------------ kernel ------------
 
-template <class C, bool BF16, bool E4M3>
+template <class C, bool BF16, bool E4M3, bool SKIP>
 __global__ void __launch_bounds__(C::THREADS, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023u) != 0) {  // the layouts need a 1024-aligned base
@@ -1059,7 +1065,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) attn_fwd_kernel(const __grid_co
   } else if (warp == 9) {
     if (g.n > 0) mma_role<C, BF16, E4M3>(p, g, smem, bars, tbase, wc);
   } else {
-    softmax_role<C, BF16, E4M3>(p, g, smem, bars, tbase, wc);
+    softmax_role<C, BF16, E4M3, SKIP>(p, g, smem, bars, tbase, wc);
   }
 
   tc_fence_before();

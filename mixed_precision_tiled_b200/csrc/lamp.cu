@@ -253,28 +253,36 @@ int quant_qk(const void* q, const void* k, void* q8, void* k8, float* q_scale, f
   return launch_quant_t<false, false>(jq, jk, D, vec, st);
 }
 
-template <class C, bool BF16, bool E4M3>
+template <class C, bool BF16, bool E4M3, bool SKIP>
 int launch_attn_cfg_t(const lamp::AttnParams& p, int grid, cudaStream_t st) {
   static bool attr_set[64] = {};
   int dev = 0;
   LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    LAMP_CUDA(cudaFuncSetAttribute(lamp::attn_fwd_kernel<C, BF16, E4M3>,
+    LAMP_CUDA(cudaFuncSetAttribute(lamp::attn_fwd_kernel<C, BF16, E4M3, SKIP>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES),
               "cudaFuncSetAttribute");
     attr_set[dev] = true;
   }
-  lamp::attn_fwd_kernel<C, BF16, E4M3><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(p);
+  lamp::attn_fwd_kernel<C, BF16, E4M3, SKIP><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(p);
   LAMP_CUDA(cudaGetLastError(), "attn_fwd_kernel launch");
   return LAMP_OK;
 }
 
 template <class C>
 int launch_attn_cfg(const lamp::AttnParams& p, int grid, cudaStream_t st) {
-  if (p.bf16) return p.e4m3 ? launch_attn_cfg_t<C, true, true>(p, grid, st)
-                            : launch_attn_cfg_t<C, true, false>(p, grid, st);
-  return p.e4m3 ? launch_attn_cfg_t<C, false, true>(p, grid, st)
-                : launch_attn_cfg_t<C, false, false>(p, grid, st);
+  // the threshold skip has its own instantiation, so that the look-ahead path without it keeps
+  // its code
+  if (!std::isinf(p.skip_log2)) {
+    if (p.bf16) return p.e4m3 ? launch_attn_cfg_t<C, true, true, true>(p, grid, st)
+                              : launch_attn_cfg_t<C, true, false, true>(p, grid, st);
+    return p.e4m3 ? launch_attn_cfg_t<C, false, true, true>(p, grid, st)
+                  : launch_attn_cfg_t<C, false, false, true>(p, grid, st);
+  }
+  if (p.bf16) return p.e4m3 ? launch_attn_cfg_t<C, true, true, false>(p, grid, st)
+                            : launch_attn_cfg_t<C, true, false, false>(p, grid, st);
+  return p.e4m3 ? launch_attn_cfg_t<C, false, true, false>(p, grid, st)
+                : launch_attn_cfg_t<C, false, false, false>(p, grid, st);
 }
 
 template <bool BF16, bool ADAPTIVE>
