@@ -116,6 +116,9 @@ __device__ __forceinline__ int pp_item(const AttnParams& p, int r) {
   return j < n_items ? static_cast<int>(j) : -1;
 }
 
+// VARLEN: sequence geometry from the offset arrays (variable-length batches); otherwise the
+// dense layout, with every offset a compile-time zero.
+template <bool VARLEN>
 __device__ __forceinline__ PPGeo pp_geo(const AttnParams& p, int idx) {
   PPGeo g;
   if (pp_head_pairs(p)) {
@@ -142,16 +145,25 @@ __device__ __forceinline__ PPGeo pp_geo(const AttnParams& p, int idx) {
     }
   }
   g.kvh = g.h[0] / (p.H / p.Hkv);
-  for (int x = 0; x < 2; ++x) {
-    const SeqRows sr = seq_rows(p, g.b, g.h[x], g.kvh);
-    g.q_plane[x] = sr.q_plane;
-    if (x == 0) {
-      g.Lq = sr.Lq;
-      g.Lk = sr.Lk;
-      g.q_row0 = sr.q_row0;
-      g.k_row0 = sr.k_row0;
-      g.kv_plane = sr.kv_plane;
+  if (VARLEN) {
+    for (int x = 0; x < 2; ++x) {
+      const SeqRows sr = seq_rows(p, g.b, g.h[x], g.kvh);
+      g.q_plane[x] = sr.q_plane;
+      if (x == 0) {
+        g.Lq = sr.Lq;
+        g.Lk = sr.Lk;
+        g.q_row0 = sr.q_row0;
+        g.k_row0 = sr.k_row0;
+        g.kv_plane = sr.kv_plane;
+      }
     }
+  } else {
+    g.Lq = p.Lq;
+    g.Lk = p.Lk;
+    g.q_row0 = g.k_row0 = 0;
+    g.q_plane[0] = g.b * p.H + g.h[0];
+    g.q_plane[1] = g.b * p.H + g.h[1];
+    g.kv_plane = g.b * p.Hkv + g.kvh;
   }
   int lo_all = 1 << 30, hi_all = -1;
   for (int x = 0; x < 2; ++x) {
@@ -268,6 +280,7 @@ __device__ __forceinline__ PPPlan pp_plan(const AttnParams& p, const PPGeo& g, c
 // item's QK^T MMAs have completed) and the item's routing mask rows, then every key tile's K8,
 // K16 and V in the MMA warp's order of first use within each ring.  The rings run on across
 // items.
+template <bool VARLEN>
 __device__ void pp_producer(const AttnParams& p, uint8_t* smem, PPBars& bars, const WaitCtx wc) {
   using C = PPCfg;
   prefetch_tmap(&p.tm_q16);
@@ -303,7 +316,7 @@ __device__ void pp_producer(const AttnParams& p, uint8_t* smem, PPBars& bars, co
   for (; ok; ++r) {
     const int item = pp_item(p, r);
     if (item < 0) break;
-    const PPGeo g = pp_geo(p, item);
+    const PPGeo g = pp_geo<VARLEN>(p, item);
     pkv = g.kv_plane;
     krow0 = g.k_row0;
     if (!lamp_chk(g.b * p.H + g.h[1] < p.B * p.H && g.b * p.Hkv + g.kvh < p.B * p.Hkv, 3)) {
@@ -354,7 +367,7 @@ __device__ void pp_producer(const AttnParams& p, uint8_t* smem, PPBars& bars, co
 // only MMAs lie between a P tile's arrival and the next QK^T.  Per work item: wait for its Q,
 // and before the first QK^T of a query tile for the previous item's epilogue to have read O;
 // at the end release Q and publish O.
-template <bool BF16, bool ADAPTIVE>
+template <bool BF16, bool ADAPTIVE, bool VARLEN>
 __device__ void pp_mma(const AttnParams& p, uint8_t* smem, PPBars& bars, uint32_t tbase,
                        const WaitCtx wc) {
   using C = PPCfg;
@@ -458,7 +471,7 @@ __device__ void pp_mma(const AttnParams& p, uint8_t* smem, PPBars& bars, uint32_
   for (int r = 0; ok; ++r) {
     const int item = pp_item(p, r);
     if (item < 0) break;
-    const PPGeo g = pp_geo(p, item);
+    const PPGeo g = pp_geo<VARLEN>(p, item);
     const int ms = r & 1;  // mask slot of this item
     const int ra0 = (g.lo[0] <= g.hi[0]) ? g.lo[0] / C::BN : (1 << 30);
     const int rb0 = (g.lo[0] <= g.hi[0]) ? g.hi[0] / C::BN : -1;
@@ -584,7 +597,7 @@ __device__ void pp_mma(const AttnParams& p, uint8_t* smem, PPBars& bars, uint32_
 // One work item of the softmax role (it = the CTA's item count, the parity of its per-item
 // barrier phases).  The phase counters of the per-tile barriers run on across items.  Returns
 // false when a wait gave up.
-template <bool BF16, bool ADAPTIVE>
+template <bool BF16, bool ADAPTIVE, bool VARLEN>
 __device__ __forceinline__ bool pp_softmax_item(const AttnParams& p, const PPGeo& g, PPBars& bars,
                                                 uint32_t tbase, const WaitCtx wc, int it,
                                                 uint32_t& cs, uint32_t& c16, uint32_t& cvv,
@@ -850,21 +863,21 @@ __device__ __forceinline__ bool pp_softmax_item(const AttnParams& p, const PPGeo
 }
 
 // The softmax role: the CTA's work items in turn.
-template <bool BF16, bool ADAPTIVE>
+template <bool BF16, bool ADAPTIVE, bool VARLEN>
 __device__ void pp_softmax(const AttnParams& p, PPBars& bars, uint32_t tbase, const WaitCtx wc) {
   uint32_t cs = 0, c16 = 0, cvv = 0;
   uint32_t raw[PPCfg::BN];
   for (int it = 0;; ++it) {
     const int item = pp_item(p, it);
     if (item < 0) break;
-    const PPGeo g = pp_geo(p, item);
-    if (!pp_softmax_item<BF16, ADAPTIVE>(p, g, bars, tbase, wc, it, cs, c16, cvv, raw)) break;
+    const PPGeo g = pp_geo<VARLEN>(p, item);
+    if (!pp_softmax_item<BF16, ADAPTIVE, VARLEN>(p, g, bars, tbase, wc, it, cs, c16, cvv, raw)) break;
   }
 }
 
 // ------------------------------------------------------------------ kernel ------------
 
-template <bool BF16, bool ADAPTIVE>
+template <bool BF16, bool ADAPTIVE, bool VARLEN>
 __global__ void __launch_bounds__(PPCfg::THREADS, 1)
     attn_fwd_pp_kernel(const __grid_constant__ AttnParams p) {
   using C = PPCfg;
@@ -915,13 +928,13 @@ __global__ void __launch_bounds__(PPCfg::THREADS, 1)
   // itself.
   if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory");
-    pp_softmax<BF16, ADAPTIVE>(p, bars, tbase, wc);
+    pp_softmax<BF16, ADAPTIVE, VARLEN>(p, bars, tbase, wc);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 104;\n" ::: "memory");
     if (warp == 8) {
-      if ((threadIdx.x & 31) == 0) pp_producer(p, smem, bars, wc);
+      if ((threadIdx.x & 31) == 0) pp_producer<VARLEN>(p, smem, bars, wc);
     } else if (warp == 9) {
-      pp_mma<BF16, ADAPTIVE>(p, smem, bars, tbase, wc);
+      pp_mma<BF16, ADAPTIVE, VARLEN>(p, smem, bars, tbase, wc);
     }
   }
   tc_fence_before();

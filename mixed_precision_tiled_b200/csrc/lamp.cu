@@ -285,29 +285,36 @@ int launch_attn_cfg(const lamp::AttnParams& p, int grid, cudaStream_t st) {
                 : launch_attn_cfg_t<C, false, false, false>(p, grid, st);
 }
 
-template <bool BF16, bool ADAPTIVE>
+template <bool BF16, bool ADAPTIVE, bool VARLEN>
 int launch_attn_pp_t(const lamp::AttnParams& p, int grid, cudaStream_t st) {
   static bool attr_set[64] = {};
   int dev = 0;
   LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    LAMP_CUDA(cudaFuncSetAttribute(lamp::attn_fwd_pp_kernel<BF16, ADAPTIVE>,
+    LAMP_CUDA(cudaFuncSetAttribute(lamp::attn_fwd_pp_kernel<BF16, ADAPTIVE, VARLEN>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    lamp::PPCfg::SMEM_BYTES),
               "cudaFuncSetAttribute");
     attr_set[dev] = true;
   }
-  lamp::attn_fwd_pp_kernel<BF16, ADAPTIVE>
+  lamp::attn_fwd_pp_kernel<BF16, ADAPTIVE, VARLEN>
       <<<grid, lamp::PPCfg::THREADS, lamp::PPCfg::SMEM_BYTES, st>>>(p);
   LAMP_CUDA(cudaGetLastError(), "attn_fwd_pp_kernel launch");
   return LAMP_OK;
 }
 
+template <bool VARLEN>
+int launch_attn_pp_v(const lamp::AttnParams& p, int grid, cudaStream_t st) {
+  if (p.bf16) return p.adaptive ? launch_attn_pp_t<true, true, VARLEN>(p, grid, st)
+                                : launch_attn_pp_t<true, false, VARLEN>(p, grid, st);
+  return p.adaptive ? launch_attn_pp_t<false, true, VARLEN>(p, grid, st)
+                    : launch_attn_pp_t<false, false, VARLEN>(p, grid, st);
+}
+
+// Variable-length batches have their own instantiation: the dense one keeps compile-time
+// zero offsets.
 int launch_attn_pp(const lamp::AttnParams& p, int grid, cudaStream_t st) {
-  if (p.bf16) return p.adaptive ? launch_attn_pp_t<true, true>(p, grid, st)
-                                : launch_attn_pp_t<true, false>(p, grid, st);
-  return p.adaptive ? launch_attn_pp_t<false, true>(p, grid, st)
-                    : launch_attn_pp_t<false, false>(p, grid, st);
+  return p.cu_q ? launch_attn_pp_v<true>(p, grid, st) : launch_attn_pp_v<false>(p, grid, st);
 }
 
 using Cfg64 = lamp::AttnCfg<64, 64, true>;
