@@ -62,6 +62,7 @@ class _Args(ctypes.Structure):
         ("q_codes", ctypes.c_void_p), ("q_scales", ctypes.c_void_p),
         ("k_codes", ctypes.c_void_p), ("k_scales", ctypes.c_void_p),
         ("skip_tau", ctypes.c_double),
+        ("k_codes_in", ctypes.c_void_p), ("k_scales_in", ctypes.c_void_p),
     ]
 
 
@@ -159,14 +160,17 @@ def build_mask_template(B: int, H: int, Lq: int, Lk: int, bm: int, bn: int, grou
 
 def attention(q, k, v, *, bm, bn, causal=False, window=0, scale=None, mask=None, group_tiles=1,
               route="bitmask", fmt="int8", tau=0.0, rows=None, threads=0, want_codes=False,
-              route_hint=None, hint_margin=0.0, skip_tau=float("inf")):
+              route_hint=None, hint_margin=0.0, skip_tau=float("inf"), k_codes_in=None,
+              k_scales_in=None):
     """Routed attention on fp32 values of 16-bit inputs.
 
     q [B,H,Lq,D], k/v [B,Hkv,Lk,D].  ``mask`` uint64 [B,H,nQT,W] or None (all 8-bit) in
     bitmask routing.  ``rows`` int64 [B,H,n] (sorted per head) restricts the output rows.
     Returns a dict with o (fp64 [B,H,R,D]), lse (fp64 [B,H,R]), route (uint8 [B,H,nQT,nKT]:
     0 dead, 1 8-bit, 2 16-bit by mask, 3 16-bit flagged, 4 dropped), margin (fp64, adaptive
-    decisions).  ``skip_tau`` (look-ahead mode; LATTE page, low-precision filtering of the keys
+    decisions).  ``k_codes_in`` / ``k_scales_in`` (uint8 [B,Hkv,Lk,D], float32 [B,Hkv,nKT]):
+    an 8-bit key cache used by the 8-bit path instead of quantising ``k`` (decode with an INT8
+    KV cache: TileMix page, section 4).  ``skip_tau`` (look-ahead mode; LATTE page, low-precision filtering of the keys
     far below the row maximum, read per tile): a tile every row of which has t_r < m_r -
     skip_tau is dropped; +inf never drops.
     """
@@ -209,6 +213,11 @@ def attention(q, k, v, *, bm, bn, causal=False, window=0, scale=None, mask=None,
     a.route_hint = _ptr(route_hint)
     a.hint_margin = float(hint_margin)
     a.skip_tau = float(skip_tau)
+    if k_codes_in is not None:  # an 8-bit key cache: codes and scales given, not recomputed
+        k_codes_in = np.ascontiguousarray(k_codes_in, dtype=np.uint8)
+        k_scales_in = np.ascontiguousarray(k_scales_in, dtype=np.float32)
+        assert k_codes_in.shape == k.shape and k_scales_in.shape == (B, Hkv, nkt)
+        a.k_codes_in, a.k_scales_in = _ptr(k_codes_in), _ptr(k_scales_in)
     out = {"o": o, "lse": lse, "route": rmap, "margin": margin}
     if want_codes:
         qc = np.empty(q.shape, np.uint8)

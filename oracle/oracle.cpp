@@ -156,6 +156,11 @@ struct orc_args {
   float* k_scales;         // optional [B,Hkv,nKT]
   double skip_tau;         // look-ahead mode: drop a tile every row of which is this far below
                            // its running max (+inf: never)
+  // optional: 8-bit K given instead of quantised here (an 8-bit key cache, TileMix page,
+  // section 4: INT8 key/value caches for decode); the 8-bit path then uses these codes and
+  // scales, the 16-bit path the values in k
+  const uint8_t* k_codes_in;  // [B,Hkv,Lk,D]
+  const float* k_scales_in;   // [B,Hkv,nKT]
 };
 
 double orc_e4m3_decode(uint8_t c) { return e4m3_decode(c); }
@@ -237,7 +242,12 @@ int orc_attention(const orc_args* a) {
   // Quantise K for every (b, kv head) block of bn rows.
   std::vector<uint8_t> kc((size_t)g.B * g.Hkv * g.Lk * D);
   std::vector<float> ks((size_t)g.B * g.Hkv * nkt);
-  orc_quantize(a->k, g.B * g.Hkv, g.Lk, D, g.bn, a->fmt, kc.data(), ks.data());
+  if (a->k_codes_in && a->k_scales_in) {
+    std::memcpy(kc.data(), a->k_codes_in, kc.size());
+    std::memcpy(ks.data(), a->k_scales_in, ks.size() * sizeof(float));
+  } else {
+    orc_quantize(a->k, g.B * g.Hkv, g.Lk, D, g.bn, a->fmt, kc.data(), ks.data());
+  }
   if (a->k_codes) std::memcpy(a->k_codes, kc.data(), kc.size());
   if (a->k_scales) std::memcpy(a->k_scales, ks.data(), ks.size() * sizeof(float));
   if (a->q_codes || a->q_scales) {

@@ -396,3 +396,36 @@ def test_skip_infinite_threshold_changes_nothing_and_first_tiles_stay():
         live = np.nonzero(c["route"][0, 0, qt])[0]
         assert c["route"][0, 0, qt, live[0]] != 4
     assert np.isfinite(c["lse"]).all()
+
+
+# ---- 8-bit key cache (TileMix page, section 4: INT8 key/value caches for decode) ----------
+
+def test_key_cache_codes_are_used_as_given():
+    # one query row q = 2 * e0 (codes [127, 0, ...], scale fl32(2/127)); a hand-made cache of 4
+    # keys with codes 10, -20, 30, 0 on channel 0 and block scale 0.5: the 8-bit scores are
+    # 127 * c_j * fl32(2/127) * 0.5 (scale 1); v is given as dequantised values
+    D = 16
+    q = np.zeros((1, 1, 1, D), np.float32)
+    q[0, 0, 0, 0] = 2.0
+    codes = np.zeros((1, 1, 4, D), np.uint8)
+    codes[0, 0, :, 0] = np.array([10, -20, 30, 0], np.int8).view(np.uint8)
+    ks = np.array([[[0.5]]], np.float32)
+    k_values = codes.view(np.int8).astype(np.float32) * 0.5  # the cache, dequantised
+    v = np.random.default_rng(3).standard_normal((1, 1, 4, D)).astype(np.float32)
+    r = oracle.attention(q, k_values, v, bm=1, bn=4, scale=1.0, k_codes_in=codes, k_scales_in=ks)
+    sq = float(np.float32(2.0) / np.float32(127.0))
+    s = 127.0 * np.array([10.0, -20.0, 30.0, 0.0]) * sq * 0.5
+    p = np.exp(s - s.max())
+    assert np.allclose(r["o"][0, 0, 0], (p[:, None] * v[0, 0]).sum(0) / p.sum(), atol=1e-12)
+    assert abs(r["lse"][0, 0, 0] - (s.max() + np.log(p.sum()))) < 1e-12
+
+
+def test_key_cache_equal_to_own_quantisation_changes_nothing():
+    rng = np.random.default_rng(9)
+    q, k, v = rand_qkv(rng, 1, 4, 2, 1, 300, 64, scale=1.5)
+    kc, ksc = oracle.quantize(k, 64, "int8")
+    m = oracle.build_mask(1, 4, 1, 5, 1, 0.3, 11)
+    kw = dict(bm=64, bn=64, causal=True, mask=m, group_tiles=1)
+    a = oracle.attention(q, k, v, **kw)
+    b = oracle.attention(q, k, v, k_codes_in=kc, k_scales_in=ksc, **kw)
+    assert np.array_equal(a["o"], b["o"]) and np.array_equal(a["lse"], b["lse"])
