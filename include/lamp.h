@@ -185,6 +185,27 @@ int lamp_attn_fwd_q8_skip(const void* q, const void* k, const void* v, const voi
                           int window, float scale, int mode, float tau, float skip_tau,
                           uint8_t* route_out, void* stream);
 
+/* Decode with an 8-bit key/value cache (TileMix page, section 4: INT8 key/value caches for the
+ * decode phase; GQA).  One new query row per (batch, head) attends to the first len_k[b]
+ * cached keys of its sequence (all max_k when len_k is NULL):
+ *   q: [B][H][D] 16-bit; q8 / q_scale: its 8-bit codes and per-row scales, as lamp_quant_qk
+ *      writes them with Lq = 1 ([B][H][D], [B][H]);
+ *   k8, v8: [B][Hkv][max_k][D] 8-bit cache codes; k_scale, v_scale: [B][Hkv][ceil(max_k/BN)]
+ *      per-block scales (lamp_quant_qk on K, and on V in K's place);
+ *   mask_bits: [B][H][1][W], W = lamp_mask_words(max_k, D, group_tiles), or NULL (every group
+ *      8-bit).  Bit 1: s = (q8 . k8) * sq * sk * scale.  Bit 0 (16-bit route): s =
+ *      (q . k8) * sk * scale, the full-precision query against the dequantised cached key (the
+ *      cache holds no 16-bit keys);
+ *   values v8 * sv; softmax and P.V in fp32; o: [B][H][D] fp32; lse: [B][H] natural log, -inf
+ *      for an empty cache.
+ * mode: LAMP_FMT_*, LAMP_IN_* (bitmask routing, fp32 output; else LAMP_ERR_UNSUPPORTED); at
+ * most 8 query heads per KV head.  Uses the library workspace (B * H * ceil(max_k / 256) *
+ * (D + 2) floats of split partials), like lamp_attn_fwd. */
+int lamp_decode_fwd(const void* q, const void* q8, const float* q_scale, const void* k8,
+                    const float* k_scale, const void* v8, const float* v_scale, const int* len_k,
+                    float* o, float* lse, int B, int H, int Hkv, int max_k, int D, float scale,
+                    const uint64_t* mask_bits, int group_tiles, int mode, void* stream);
+
 /* ---- variable-length batches (TileMix page, section 4: GQA and variable-length batches
  * are supported) --------------------------------------------------------------------------
  * B sequences of different lengths share one launch.  Sequence b owns query rows

@@ -30,7 +30,7 @@ OUT_F32, OUT_INDTYPE = 0x0, 0x8
 
 EXPORTS = ("lamp_tile_shape", "lamp_mask_words", "lamp_quant_qk", "lamp_build_mask",
            "lamp_build_mask_template", "lamp_template_fraction",
-           "lamp_template_for_int8_fraction", "lamp_quant_qk_varlen", "lamp_attn_fwd_q8_varlen", "lamp_attn_fwd_q8_skip",
+           "lamp_template_for_int8_fraction", "lamp_quant_qk_varlen", "lamp_attn_fwd_q8_varlen", "lamp_attn_fwd_q8_skip", "lamp_decode_fwd",
            "lamp_attn_fwd_varlen", "lamp_attn_fwd", "lamp_attn_fwd_q8", "lamp_attn_fwd_noalloc", "lamp_workspace_size",
            "lamp_set_workspace", "lamp_check", "lamp_selftest_timeout", "lamp_mma_probe",
            "lamp_last_error")
@@ -69,6 +69,7 @@ def lib():
                 "lamp_attn_fwd": (_i, [_vp] * 5 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp]),
                 "lamp_quant_qk_varlen": (_i, [_vp] * 8 + [_i] * 9 + [_vp]),
                 "lamp_attn_fwd_q8_skip": (_i, [_vp] * 9 + [_i] * 8 + [_f, _i, _f, _f, _vp, _vp]),
+                "lamp_decode_fwd": (_i, [_vp] * 10 + [_i] * 5 + [_f, _vp, _i, _i, _vp]),
                 "lamp_attn_fwd_q8_varlen": (_i, [_vp] * 11 + [_i] * 10 + [_f, _vp, _i, _i, _f, _vp, _vp]),
                 "lamp_attn_fwd_varlen": (_i, [_vp] * 7 + [_i] * 10 + [_f, _vp, _i, _i, _f, _vp]),
                 "lamp_attn_fwd_q8": (_i, [_vp] * 9 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp, _vp]),
@@ -174,6 +175,14 @@ def lamp_attn_fwd_q8_skip(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, 
                                        Hkv, Lq, Lk, D, int(causal), window, float(scale), mode,
                                        float(tau), float(skip_tau), _ptr(route_out),
                                        _stream(stream)))
+
+
+def lamp_decode_fwd(q, q8, q_scale, k8, k_scale, v8, v_scale, len_k, o, lse, B, H, Hkv, max_k,
+                    D, scale, mask_bits, group_tiles, mode, stream=None):
+    _check(lib().lamp_decode_fwd(_ptr(q), _ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale),
+                                 _ptr(v8), _ptr(v_scale), _ptr(len_k), _ptr(o), _ptr(lse), B, H,
+                                 Hkv, max_k, D, float(scale), _ptr(mask_bits), group_tiles, mode,
+                                 _stream(stream)))
 
 
 def lamp_quant_qk_varlen(q, k, q8, k8, q_scale, k_scale, cu_q, cu_k, B, H, Hkv, max_q, max_k,

@@ -18,6 +18,7 @@
 #include "../../include/lamp.h"
 #include "attn_fwd.cuh"
 #include "attn_fwd_pp.cuh"
+#include "decode.cuh"
 #include "mma_probe.cuh"
 #include "quant.cuh"
 
@@ -503,6 +504,31 @@ bool template_sixteen(long long g, long long gd, int sink, int band, int stride)
 }
 }  // namespace
 
+namespace {
+template <int D>
+int launch_decode(const lamp::DecodeParams& p, cudaStream_t st) {
+  constexpr size_t smem = sizeof(float) * (lamp::DEC_MAX_G * lamp::DEC_CHUNK + lamp::DEC_MAX_G * D +
+                                           lamp::DEC_MAX_G * D / 4 +
+                                           (lamp::DEC_THREADS / 32) * lamp::DEC_MAX_G * D +
+                                           2 * lamp::DEC_MAX_G);
+  static bool attr_set[64] = {};
+  int dev = 0;
+  LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    LAMP_CUDA(cudaFuncSetAttribute(lamp::decode_split_kernel<D>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
+              "cudaFuncSetAttribute");
+    attr_set[dev] = true;
+  }
+  const dim3 grid(p.nsplit, p.B * p.Hkv);
+  lamp::decode_split_kernel<D><<<grid, lamp::DEC_THREADS, smem, st>>>(p);
+  LAMP_CUDA(cudaGetLastError(), "decode_split_kernel launch");
+  lamp::decode_combine_kernel<D><<<p.B * p.H, 128, 0, st>>>(p);
+  LAMP_CUDA(cudaGetLastError(), "decode_combine_kernel launch");
+  return LAMP_OK;
+}
+}  // namespace
+
 extern "C" {
 
 int lamp_tile_shape(int D, int* bm, int* bn) {
@@ -718,6 +744,57 @@ int lamp_attn_fwd_q8_skip(const void* q, const void* k, const void* v, const voi
   return attn_q8(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D, causal, window,
                  scale, nullptr, 1, mode, tau, route_out, static_cast<cudaStream_t>(stream),
                  nullptr, nullptr, 0, 0, skip_tau);
+}
+
+
+int lamp_decode_fwd(const void* q, const void* q8, const float* q_scale, const void* k8,
+                    const float* k_scale, const void* v8, const float* v_scale, const int* len_k,
+                    float* o, float* lse, int B, int H, int Hkv, int max_k, int D, float scale,
+                    const uint64_t* mask_bits, int group_tiles, int mode, void* stream) {
+  int r = check_sizes(B, H, Hkv, 1, max_k, D);
+  if (r) return r;
+  if (!q || !q8 || !q_scale || !k8 || !k_scale || !v8 || !v_scale || !o || !lse)
+    return fail(LAMP_ERR_INVALID, "null pointer");
+  if (!aligned16(k8) || !aligned16(v8) || !aligned16(q8) || !aligned16(q))
+    return fail(LAMP_ERR_INVALID, "q, q8, k8, v8 must be 16-byte aligned");
+  if ((mode & ~0x7u) != 0 || (mode & LAMP_ROUTE_ADAPTIVE))
+    return fail(LAMP_ERR_UNSUPPORTED, "decode takes bitmask routing and fp32 output only");
+  if (H / Hkv > lamp::DEC_MAX_G)
+    return fail(LAMP_ERR_UNSUPPORTED, "more than %d query heads per KV head", lamp::DEC_MAX_G);
+  if (mask_bits && group_tiles < 1) return fail(LAMP_ERR_INVALID, "group_tiles must be >= 1");
+  if (!(scale == scale)) return fail(LAMP_ERR_INVALID, "scale is NaN");
+  int bm, bn;
+  tile_shape(D, &bm, &bn);
+  lamp::DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = static_cast<const uint16_t*>(q);
+  p.q8 = static_cast<const uint8_t*>(q8);
+  p.q_scale = q_scale;
+  p.k8 = static_cast<const uint8_t*>(k8);
+  p.k_scale = k_scale;
+  p.v8 = static_cast<const uint8_t*>(v8);
+  p.v_scale = v_scale;
+  p.len_k = len_k;
+  p.mask = mask_bits;
+  p.o = o;
+  p.lse = lse;
+  p.B = B; p.H = H; p.Hkv = Hkv; p.G = H / Hkv; p.max_k = max_k;
+  p.bn = bn;
+  p.nkt = (max_k + bn - 1) / bn;
+  p.nsplit = (max_k + lamp::DEC_CHUNK - 1) / lamp::DEC_CHUNK;
+  p.group_tiles = mask_bits ? group_tiles : 1;
+  p.mask_words = ((p.nkt + p.group_tiles - 1) / p.group_tiles + 63) / 64;
+  p.scale = (scale > 0.0f) ? scale : 1.0f / std::sqrt(static_cast<float>(D));
+  p.e4m3 = (mode & LAMP_FMT_E4M3) ? 1 : 0;
+  p.bf16 = (mode & LAMP_IN_BF16) ? 1 : 0;
+  const size_t need = static_cast<size_t>(B) * H * p.nsplit * (2 + D) * sizeof(float);
+  void* ws = nullptr;
+  if ((r = get_workspace(need, &ws))) return r;
+  p.part = static_cast<float*>(ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 64) return launch_decode<64>(p, st);
+  if (D == 128) return launch_decode<128>(p, st);
+  return launch_decode<256>(p, st);
 }
 
 int lamp_quant_qk_varlen(const void* q, const void* k, void* q8, void* k8, float* q_scale,
