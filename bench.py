@@ -55,6 +55,10 @@ def parse():
     ap.add_argument("--skip-tau", type=float, default=None,
                     help="look-ahead workloads: drop tiles this far (natural log) below the "
                          "running max (threshold skip)")
+    ap.add_argument("--decode", type=int, default=0,
+                    help="decode step instead of prefill: this many sequences, each with the "
+                         "workload's Lk cached keys in 8 bits (INT8 KV cache), one query row per "
+                         "head")
     ap.add_argument("--varlen", type=int, default=0,
                     help="run the workload's B*L query rows as a variable-length batch of this "
                          "many sequences (seeded lengths), through the packed-layout calls")
@@ -559,6 +563,130 @@ def run_varlen(args, w, mpt, torch, dist, dev, stream, world, rank):
     return 0
 
 
+def run_decode(args, w, mpt, torch, dist, dev, stream, world, rank):
+    """One decode step: args.decode sequences with w.Lk cached keys each (8-bit K and V with
+    per-block scales, the workload's format), one query row per head, bitmask routing with the
+    workload's group size and FP16 fraction.  The kernel reads the cache once: bound by HBM."""
+    B, H, Hkv, D, L = args.decode, w.H, w.Hkv, w.D, w.Lk
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
+    gen = torch.Generator(device="cpu").manual_seed(w.seed)
+    q = torch.randn((B, H, 1, D), generator=gen).to(tdt).to(dev)
+    kv = torch.randn((B, Hkv, L, D), generator=gen).to(tdt).to(dev)
+    nkt = -(-L // w.bn)
+    mode = mpt.mode_bits("bitmask", w.fmt, w.dtype)
+    q8 = torch.empty(q.shape, dtype=torch.uint8, device=dev)
+    qs = torch.empty((B, H, 1), dtype=torch.float32, device=dev)
+    k8 = torch.empty(kv.shape, dtype=torch.uint8, device=dev)
+    v8 = torch.empty(kv.shape, dtype=torch.uint8, device=dev)
+    ks = torch.empty((B, Hkv, nkt), dtype=torch.float32, device=dev)
+    vs = torch.empty((B, Hkv, nkt), dtype=torch.float32, device=dev)
+    mpt.lamp_quant_qk(None, kv, None, k8, None, ks, B, H, Hkv, 1, L, D, mode, stream)
+    kv.copy_(torch.randn(kv.shape, generator=gen).to(tdt))
+    mpt.lamp_quant_qk(None, kv, None, v8, None, vs, B, H, Hkv, 1, L, D, mode, stream)
+    del kv
+    W = mpt.lamp_mask_words(L, D, w.group_tiles)
+    mask = torch.empty((B, H, 1, W), dtype=torch.int64, device=dev)
+    mpt.lamp_build_mask(mask, B, H, 1, L, D, w.group_tiles, w.p_fp16, w.mask_seed, stream)
+    o = torch.empty((B, H, D), dtype=torch.float32, device=dev)
+    lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step(ev_a=None, ev_b=None):
+        mpt.lamp_quant_qk(q, None, q8, None, qs, None, B, H, Hkv, 1, L, D, mode, stream)
+        if ev_a is not None:
+            ev_a.record(stream)
+        mpt.lamp_decode_fwd(q, q8, qs, k8, ks, v8, vs, None, o, lse, B, H, Hkv, L, D, 0.0, mask,
+                            w.group_tiles, mode, stream)
+        if ev_b is not None:
+            ev_b.record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    mpt.lamp_check(stream)
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    if world > 1:
+        dist.barrier()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    with ClockSampler(uuid if rank == 0 else None) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            flush.view(torch.int64).sum()
+            ev[i][0].record(stream)
+            step(ev[i][1], ev[i][2])
+            ev[i][3].record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    mpt.lamp_check(stream)
+    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    tot_ms, d_ms = reduce_max([sum(step_ms), statistics.fmean(dec_ms)], dev, dist)
+    ms_per_step = tot_ms / args.steps
+    F = 4 * D * H * B * L  # one query row per head over L keys
+    cache_bytes = 2 * B * Hkv * L * D + 2 * B * Hkv * nkt * 4
+    peaks = measured_peaks()
+    gbs = cache_bytes / (d_ms * 1e-3) / 1e9
+    # end to end: the query in from pinned host memory, O and lse out
+    hq = torch.empty(q.shape, dtype=tdt, pin_memory=True).copy_(q)
+    ho = torch.empty(o.shape, dtype=torch.float32, pin_memory=True)
+    hl = torch.empty(lse.shape, dtype=torch.float32, pin_memory=True)
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        step()
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    n_e2e = max(3, min(args.steps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms, = reduce_max([e0.elapsed_time(e1) / n_e2e], dev, dist)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(world * F / (ms_per_step * 1e-3) / 1e12, 3),
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": f"int8+{w.dtype}" if w.fmt == "int8" else f"e4m3+{w.dtype}",
+            "data": "synthetic",
+            "config": {"workload": f"decode: {B} sequences x {L} cached keys (8-bit K and V), "
+                                   f"H={H} Hkv={Hkv} D={D}, one query row per head, "
+                                   f"bitmask g={w.group_tiles}, {w.p_fp16:.0%} FP16 groups",
+                       "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "flushed between steps (256 MiB write, then read back); per-step CUDA events exclude the flush"},
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                         "algorithmic_bytes": cache_bytes,
+                         "peak_basis": f"copy bandwidth ({peaks['source']})",
+                         "kernel": "decode_split_kernel + decode_combine_kernel",
+                         "decode_ms": round(d_ms, 4)},
+            "e2e": {"value": round(F * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": q.numel() * q.element_size(),
+                    "d2h_bytes_per_step": o.numel() * 4 + lse.numel() * 4,
+                    "ms_per_step": round(e2e_ms, 4)},
+            "clocks": clk.summary(),
+            "gpu_launches": 3 * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -586,6 +714,8 @@ def main():
         w = w.replace(tau=args.tau)
     if args.varlen > 0:
         return run_varlen(args, w, mpt, torch, dist, dev, stream, world, rank)
+    if args.decode > 0:
+        return run_decode(args, w, mpt, torch, dist, dev, stream, world, rank)
     t = make_workload(w)
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
 

@@ -58,11 +58,12 @@ __device__ __forceinline__ float dec_e4m3(uint32_t c) {
   return (c & 0x80u) ? -mag : mag;
 }
 
-__device__ __forceinline__ float dec_code(uint32_t c, bool e4m3) {
-  return e4m3 ? dec_e4m3(c) : static_cast<float>(static_cast<int8_t>(c));
+template <bool E4M3>
+__device__ __forceinline__ float dec_code(uint32_t c) {
+  return E4M3 ? dec_e4m3(c) : static_cast<float>(static_cast<int8_t>(c));
 }
 
-template <int D>
+template <int D, bool E4M3>
 __global__ void __launch_bounds__(DEC_THREADS, 2) decode_split_kernel(const DecodeParams p) {
   static_assert(D == 64 || D == 128 || D == 256, "head dimension");
   constexpr int NW = DEC_THREADS / 32;
@@ -73,6 +74,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_split_kernel(const Deco
   uint32_t* q8w = reinterpret_cast<uint32_t*>(qf + DEC_MAX_G * D);  // [G][D/4] query codes
   float* red = reinterpret_cast<float*>(q8w + DEC_MAX_G * D / 4);   // [NW][G][D] P.V partials
   float* stat = red + NW * DEC_MAX_G * D;             // [G][2] chunk max and sum
+  // [CHUNK][D] value codes; 16-byte chunk c of row j sits at chunk c ^ (j & SW): the row stores
+  // of consecutive threads and the row reads of a warp are both free of bank conflicts
+  uint8_t* vsm = reinterpret_cast<uint8_t*>(stat + 2 * DEC_MAX_G);
+  constexpr int SW = (D / 16 >= 8) ? 7 : (D / 16 - 1);
 
   const int G = p.G;
   const int split = blockIdx.x, bkv = blockIdx.y;
@@ -80,7 +85,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_split_kernel(const Deco
   const int len = p.len_k ? min(max(__ldg(p.len_k + b), 0), p.max_k) : p.max_k;
   const int c0 = split * DEC_CHUNK;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool e4m3 = p.e4m3 != 0, bf16 = p.bf16 != 0;
+  const bool bf16 = p.bf16 != 0;
   const size_t cache_row0 = static_cast<size_t>(bkv) * p.max_k;  // first row of this KV head
 
   // the G query rows of this KV group: values and codes
@@ -96,73 +101,72 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_split_kernel(const Deco
   }
   __syncthreads();
 
-  // scores: one key per thread, all heads of the group, 16 bytes of the key row at a time
+  // scores: one key per thread, all heads of the group.  The key row stays in registers; the
+  // head loop is not unrolled (the unrolled body of every head overflowed the instruction
+  // cache).
   {
     const int j = c0 + tid;
     const bool live = j < len;
     const int kt = j / p.bn;
     const float sk = live ? __ldg(p.k_scale + static_cast<size_t>(bkv) * p.nkt + kt) : 0.0f;
     const int gi = kt / p.group_tiles;
-    uint32_t eight = (1u << G) - 1u;  // bit g: head g takes the 8-bit route for this key
-    if (p.mask && live) {
-      for (int g = 0; g < G; ++g) {
-        const uint64_t w = __ldg(reinterpret_cast<const unsigned long long*>(p.mask) +
-                                 static_cast<size_t>(b * p.H + kvh * G + g) * p.mask_words +
-                                 (gi >> 6));
-        if (((w >> (gi & 63)) & 1ull) == 0) eight &= ~(1u << g);
-      }
-    }
-    int acc8[DEC_MAX_G];
-    float accf[DEC_MAX_G];
-#pragma unroll
-    for (int g = 0; g < DEC_MAX_G; ++g) {
-      acc8[g] = 0;
-      accf[g] = 0.0f;
-    }
+    // the key and value rows of this thread's key, fetched at once (many loads in flight);
+    // the values go to shared memory for the P.V phase
+    uint32_t kw[D / 4];
     if (live) {
-      const uint4* src = reinterpret_cast<const uint4*>(p.k8 + (cache_row0 + j) * D);
-#pragma unroll 2
+      const uint4* ksrc = reinterpret_cast<const uint4*>(p.k8 + (cache_row0 + j) * D);
+      const uint4* vsrc = reinterpret_cast<const uint4*>(p.v8 + (cache_row0 + j) * D);
+      uint4 vr[D / 16];
+#pragma unroll
       for (int i = 0; i < D / 16; ++i) {
-        const uint4 kr = __ldg(src + i);
-        const uint32_t kw[4] = {kr.x, kr.y, kr.z, kr.w};
-#pragma unroll
-        for (int g = 0; g < DEC_MAX_G; ++g) {
-          if (g >= G) break;
-          if ((eight >> g) & 1u) {
-            const uint32_t* qw = q8w + g * (D / 4) + 4 * i;
-            if (!e4m3) {
-#pragma unroll
-              for (int w = 0; w < 4; ++w)
-                acc8[g] = __dp4a(static_cast<int>(qw[w]), static_cast<int>(kw[w]), acc8[g]);
-            } else {
-#pragma unroll
-              for (int w = 0; w < 4; ++w)
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  accf[g] = fmaf(dec_e4m3((qw[w] >> (8 * e)) & 0xFFu),
-                                 dec_e4m3((kw[w] >> (8 * e)) & 0xFFu), accf[g]);
-            }
-          } else {
-            const float* qv = qf + g * D + 16 * i;
-#pragma unroll
-            for (int w = 0; w < 4; ++w)
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                accf[g] = fmaf(qv[4 * w + e], dec_code((kw[w] >> (8 * e)) & 0xFFu, e4m3), accf[g]);
-          }
-        }
+        const uint4 kr = __ldg(ksrc + i);
+        kw[4 * i] = kr.x;
+        kw[4 * i + 1] = kr.y;
+        kw[4 * i + 2] = kr.z;
+        kw[4 * i + 3] = kr.w;
+        vr[i] = __ldg(vsrc + i);
       }
-    }
 #pragma unroll
-    for (int g = 0; g < DEC_MAX_G; ++g) {
-      if (g >= G) break;
+      for (int i = 0; i < D / 16; ++i)
+        reinterpret_cast<uint4*>(vsm + tid * D)[i ^ (tid & SW)] = vr[i];
+    }
+#pragma unroll 1
+    for (int g = 0; g < G; ++g) {
       float s = -__int_as_float(0x7f800000);
       if (live) {
-        if ((eight >> g) & 1u) {
-          const float sq = __ldg(p.q_scale + b * p.H + kvh * G + g);
-          s = (e4m3 ? accf[g] : static_cast<float>(acc8[g])) * sq * sk * p.scale;
+        const int h = kvh * G + g;
+        bool eight = true;
+        if (p.mask) {
+          const uint64_t w = __ldg(reinterpret_cast<const unsigned long long*>(p.mask) +
+                                   static_cast<size_t>(b * p.H + h) * p.mask_words + (gi >> 6));
+          eight = ((w >> (gi & 63)) & 1ull) != 0;
+        }
+        if (eight) {
+          const uint32_t* qw = q8w + g * (D / 4);
+          const float sq = __ldg(p.q_scale + b * p.H + h);
+          if (!E4M3) {
+            int acc = 0;
+#pragma unroll
+            for (int i = 0; i < D / 4; ++i) acc = __dp4a(static_cast<int>(qw[i]), static_cast<int>(kw[i]), acc);
+            s = static_cast<float>(acc) * sq * sk * p.scale;
+          } else {
+            float acc = 0.0f;
+#pragma unroll
+            for (int i = 0; i < D / 4; ++i)
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                acc = fmaf(dec_e4m3((qw[i] >> (8 * e)) & 0xFFu), dec_e4m3((kw[i] >> (8 * e)) & 0xFFu), acc);
+            s = acc * sq * sk * p.scale;
+          }
         } else {
-          s = accf[g] * sk * p.scale;
+          const float* qv = qf + g * D;
+          float acc = 0.0f;
+#pragma unroll
+          for (int i = 0; i < D / 4; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              acc = fmaf(qv[4 * i + e], dec_code<E4M3>((kw[i] >> (8 * e)) & 0xFFu), acc);
+          s = acc * sk * p.scale;
         }
       }
       sc[g * DEC_CHUNK + tid] = s;
@@ -199,23 +203,31 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_split_kernel(const Deco
 #pragma unroll
     for (int e = 0; e < DL; ++e) acc[g][e] = 0.0f;
   const int jend = min(DEC_CHUNK, len - c0);
+  float vsc[DEC_CHUNK / 64];  // value scales of the chunk's key tiles (BN >= 64)
+#pragma unroll
+  for (int i = 0; i < DEC_CHUNK / 64; ++i) {
+    const int kt = c0 / p.bn + i;
+    vsc[i] = (kt < p.nkt) ? __ldg(p.v_scale + static_cast<size_t>(bkv) * p.nkt + kt) : 0.0f;
+  }
   for (int jj = warp; jj < jend; jj += NW) {
     const int j = c0 + jj;
-    const uint8_t* vrow = p.v8 + (cache_row0 + j) * D + lane * DL;
+    // lane's DL bytes of row jj: logical chunk (lane * DL) / 16, stored at chunk ^ (jj & SW)
+    const int lc = (lane * DL) >> 4;
+    const uint8_t* vrow = vsm + jj * D + ((lc ^ (jj & SW)) << 4) + ((lane * DL) & 15);
     uint32_t vw[(DL + 3) / 4];
     if (DL == 8) {
-      const uint2 t = __ldg(reinterpret_cast<const uint2*>(vrow));
+      const uint2 t = *reinterpret_cast<const uint2*>(vrow);
       vw[0] = t.x;
       vw[1] = t.y;
     } else if (DL == 4) {
-      vw[0] = __ldg(reinterpret_cast<const uint32_t*>(vrow));
+      vw[0] = *reinterpret_cast<const uint32_t*>(vrow);
     } else {
-      vw[0] = __ldg(reinterpret_cast<const uint16_t*>(vrow));
+      vw[0] = *reinterpret_cast<const uint16_t*>(vrow);
     }
-    const float sv = __ldg(p.v_scale + static_cast<size_t>(bkv) * p.nkt + j / p.bn);
+    const float sv = vsc[(j / p.bn) - c0 / p.bn];
     float vv[DL];
 #pragma unroll
-    for (int e = 0; e < DL; ++e) vv[e] = dec_code((vw[e >> 2] >> (8 * (e & 3))) & 0xFFu, e4m3) * sv;
+    for (int e = 0; e < DL; ++e) vv[e] = dec_code<E4M3>((vw[e >> 2] >> (8 * (e & 3))) & 0xFFu) * sv;
 #pragma unroll
     for (int g = 0; g < DEC_MAX_G; ++g) {
       if (g >= G) break;
@@ -249,29 +261,57 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_split_kernel(const Deco
 }
 
 // Merge the partials of one (b, h): M = max m_s, l = sum l_s e^(m_s - M), O = sum O_s e^(m_s - M) / l,
-// lse = M + ln l.  A sequence with no cached key gets O = 0 and lse = -inf.
+// lse = M + ln l.  A sequence with no cached key gets O = 0 and lse = -inf.  The split weights
+// e^(m_s - M) are computed once, in parallel, into shared memory; every thread then sums its
+// channel over the splits with independent, coalesced loads.
+constexpr int DEC_COMBINE_THREADS = 256;
+
 template <int D>
-__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
-  const int bh = blockIdx.x;
+__global__ void __launch_bounds__(DEC_COMBINE_THREADS) decode_combine_kernel(const DecodeParams p) {
+  extern __shared__ __align__(16) float wsm[];  // [nsplit] weights, then [32] reduction scratch
+  float* scratch = wsm + p.nsplit;
+  const int bh = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = DEC_COMBINE_THREADS / 32;
   const float* part = p.part + static_cast<size_t>(bh) * p.nsplit * (2 + D);
   const float NEG_INF = -__int_as_float(0x7f800000);
+  float m = NEG_INF;
+  for (int s = tid; s < p.nsplit; s += DEC_COMBINE_THREADS) m = fmaxf(m, part[s * (2 + D)]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if (lane == 0) scratch[warp] = m;
+  __syncthreads();
   float M = NEG_INF;
-  for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, part[s * (2 + D)]);
+#pragma unroll
+  for (int w = 0; w < NW; ++w) M = fmaxf(M, scratch[w]);
   float l = 0.0f;
-  for (int s = 0; s < p.nsplit; ++s) {
-    const float m = part[s * (2 + D)];
-    if (m != NEG_INF) l += part[s * (2 + D) + 1] * __expf(m - M);
+  for (int s = tid; s < p.nsplit; s += DEC_COMBINE_THREADS) {
+    const float ms = part[s * (2 + D)];
+    const float wt = (ms == NEG_INF) ? 0.0f : __expf(ms - M);
+    wsm[s] = wt;
+    l += part[s * (2 + D) + 1] * wt;
   }
-  const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float o = 0.0f;
-    for (int s = 0; s < p.nsplit; ++s) {
-      const float m = part[s * (2 + D)];
-      if (m != NEG_INF) o += part[s * (2 + D) + 2 + d] * __expf(m - M);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, o);
+  __syncthreads();  // (scratch reused, weights complete)
+  if (lane == 0) scratch[NW + warp] = l;
+  __syncthreads();
+  float L = 0.0f;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) L += scratch[NW + w];
+  const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
+  for (int d = tid; d < D; d += DEC_COMBINE_THREADS) {
+    float o0 = 0.0f, o1 = 0.0f, o2 = 0.0f, o3 = 0.0f;
+    int s = 0;
+    for (; s + 4 <= p.nsplit; s += 4) {
+      o0 = fmaf(part[(s + 0) * (2 + D) + 2 + d], wsm[s + 0], o0);
+      o1 = fmaf(part[(s + 1) * (2 + D) + 2 + d], wsm[s + 1], o1);
+      o2 = fmaf(part[(s + 2) * (2 + D) + 2 + d], wsm[s + 2], o2);
+      o3 = fmaf(part[(s + 3) * (2 + D) + 2 + d], wsm[s + 3], o3);
     }
-    p.o[static_cast<size_t>(bh) * D + d] = o * inv;
+    for (; s < p.nsplit; ++s) o0 = fmaf(part[s * (2 + D) + 2 + d], wsm[s], o0);
+    p.o[static_cast<size_t>(bh) * D + d] = ((o0 + o1) + (o2 + o3)) * inv;
   }
-  if (threadIdx.x == 0) p.lse[bh] = (l > 0.0f) ? M + logf(l) : NEG_INF;
+  if (tid == 0) p.lse[bh] = (L > 0.0f) ? M + logf(L) : NEG_INF;
 }
 
 }  // namespace lamp

@@ -505,27 +505,34 @@ bool template_sixteen(long long g, long long gd, int sink, int band, int stride)
 }  // namespace
 
 namespace {
-template <int D>
-int launch_decode(const lamp::DecodeParams& p, cudaStream_t st) {
+template <int D, bool E4M3>
+int launch_decode_t(const lamp::DecodeParams& p, cudaStream_t st) {
   constexpr size_t smem = sizeof(float) * (lamp::DEC_MAX_G * lamp::DEC_CHUNK + lamp::DEC_MAX_G * D +
                                            lamp::DEC_MAX_G * D / 4 +
                                            (lamp::DEC_THREADS / 32) * lamp::DEC_MAX_G * D +
-                                           2 * lamp::DEC_MAX_G);
+                                           2 * lamp::DEC_MAX_G) +
+                        static_cast<size_t>(lamp::DEC_CHUNK) * D;  // value rows
   static bool attr_set[64] = {};
   int dev = 0;
   LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    LAMP_CUDA(cudaFuncSetAttribute(lamp::decode_split_kernel<D>,
+    LAMP_CUDA(cudaFuncSetAttribute(lamp::decode_split_kernel<D, E4M3>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
               "cudaFuncSetAttribute");
     attr_set[dev] = true;
   }
   const dim3 grid(p.nsplit, p.B * p.Hkv);
-  lamp::decode_split_kernel<D><<<grid, lamp::DEC_THREADS, smem, st>>>(p);
+  lamp::decode_split_kernel<D, E4M3><<<grid, lamp::DEC_THREADS, smem, st>>>(p);
   LAMP_CUDA(cudaGetLastError(), "decode_split_kernel launch");
-  lamp::decode_combine_kernel<D><<<p.B * p.H, 128, 0, st>>>(p);
+  lamp::decode_combine_kernel<D><<<p.B * p.H, lamp::DEC_COMBINE_THREADS,
+                                   (p.nsplit + 64) * sizeof(float), st>>>(p);
   LAMP_CUDA(cudaGetLastError(), "decode_combine_kernel launch");
   return LAMP_OK;
+}
+
+template <int D>
+int launch_decode(const lamp::DecodeParams& p, cudaStream_t st) {
+  return p.e4m3 ? launch_decode_t<D, true>(p, st) : launch_decode_t<D, false>(p, st);
 }
 }  // namespace
 
