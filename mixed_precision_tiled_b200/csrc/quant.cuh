@@ -222,19 +222,26 @@ __device__ __forceinline__ QuantBlock quant_locate(const QuantJob& j0, const Qua
                                                    int D) {
   const bool second = b >= j0.blocks;
   const int id = b - (second ? j0.blocks : 0);
-  const QuantJob& j = second ? j1 : j0;
-  const int o = id / j.nb, bi = id - o * j.nb;
-  const int r0 = bi * j.blk;
-  if (j.cu) {  // rows of sequence o / heads in head plane o % heads, clipped to the tensor
-    const int sb = o / j.heads, h = o - sb * j.heads;
-    const int s0 = min(max(__ldg(j.cu + sb), 0), j.total);
-    const int len = min(max(__ldg(j.cu + sb + 1) - s0, 0), min(j.L, j.total - s0));
-    const int rows = min(max(len - r0, 0), j.blk);
-    const size_t base = (static_cast<size_t>(h) * j.total + s0 + min(r0, len)) * D;
-    return QuantBlock{j.x + base, j.codes + base, j.scales + id, rows * D / 8};
+  // (fields are selected one by one: a reference to a runtime-chosen kernel parameter would
+  // copy both jobs to local memory)
+  const int L = second ? j1.L : j0.L, blk = second ? j1.blk : j0.blk, nb = second ? j1.nb : j0.nb;
+  const uint16_t* x = second ? j1.x : j0.x;
+  uint8_t* codes = second ? j1.codes : j0.codes;
+  float* scales = second ? j1.scales : j0.scales;
+  const int* cu = second ? j1.cu : j0.cu;
+  const int o = id / nb, bi = id - o * nb;
+  const int r0 = bi * blk;
+  if (cu) {  // rows of sequence o / heads in head plane o % heads, clipped to the tensor
+    const int heads = second ? j1.heads : j0.heads, total = second ? j1.total : j0.total;
+    const int sb = o / heads, h = o - sb * heads;
+    const int s0 = min(max(__ldg(cu + sb), 0), total);
+    const int len = min(max(__ldg(cu + sb + 1) - s0, 0), min(L, total - s0));
+    const int rows = min(max(len - r0, 0), blk);
+    const size_t base = (static_cast<size_t>(h) * total + s0 + min(r0, len)) * D;
+    return QuantBlock{x + base, codes + base, scales + id, rows * D / 8};
   }
-  const size_t base = (static_cast<size_t>(o) * j.L + r0) * D;
-  return QuantBlock{j.x + base, j.codes + base, j.scales + id, min(j.blk, j.L - r0) * D / 8};
+  const size_t base = (static_cast<size_t>(o) * L + r0) * D;
+  return QuantBlock{x + base, codes + base, scales + id, min(blk, L - r0) * D / 8};
 }
 
 // Persistent CTAs; CTA c quantises blocks c, c + grid, c + 2 grid, ... of the combined grid
