@@ -10,8 +10,8 @@
 // The work is memory-bound (one pass over the cache), so it runs on the CUDA cores with the
 // cache split across CTAs: CTA (chunk, b * Hkv + kvh) reads CHUNK keys of one KV head once for
 // all G query heads of its group, and writes a partial (m, l, O) per head; a second kernel
-// merges the partials of each (b, h).  Loads are 16-byte (keys, one row per thread) and
-// row-coalesced (values, a warp per key row).
+// merges the partials of each (b, h).  The chunk's key and value rows are loaded cooperatively
+// (coalesced) into XOR-swizzled shared memory; each thread then reads its own key row.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -77,6 +77,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_split_kernel(const Deco
   // [CHUNK][D] value codes; 16-byte chunk c of row j sits at chunk c ^ (j & SW): the row stores
   // of consecutive threads and the row reads of a warp are both free of bank conflicts
   uint8_t* vsm = reinterpret_cast<uint8_t*>(stat + 2 * DEC_MAX_G);
+  uint8_t* ksm = vsm + DEC_CHUNK * D;  // [CHUNK][D] key codes, same swizzle
   constexpr int SW = (D / 16 >= 8) ? 7 : (D / 16 - 1);
 
   const int G = p.G;
@@ -110,25 +111,42 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_split_kernel(const Deco
     const int kt = j / p.bn;
     const float sk = live ? __ldg(p.k_scale + static_cast<size_t>(bkv) * p.nkt + kt) : 0.0f;
     const int gi = kt / p.group_tiles;
-    // the key and value rows of this thread's key, fetched at once (many loads in flight);
-    // the values go to shared memory for the P.V phase
+    // the chunk's key and value rows, loaded cooperatively (a warp reads whole rows: coalesced)
+    // into swizzled shared memory; each thread then reads its own key row from there
+    {
+      constexpr int CPR = D / 16;  // 16-byte chunks per row
+      const int rows = min(DEC_CHUNK, len - c0);
+      const uint4* kbase = reinterpret_cast<const uint4*>(p.k8 + (cache_row0 + c0) * D);
+      const uint4* vbase = reinterpret_cast<const uint4*>(p.v8 + (cache_row0 + c0) * D);
+      uint4 kt_[DEC_CHUNK * CPR / DEC_THREADS], vt_[DEC_CHUNK * CPR / DEC_THREADS];
+#pragma unroll
+      for (int u = 0; u < DEC_CHUNK * CPR / DEC_THREADS; ++u) {
+        const int idx = u * DEC_THREADS + tid, r = idx / CPR;
+        if (r < rows) {
+          kt_[u] = __ldg(kbase + idx);
+          vt_[u] = __ldg(vbase + idx);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < DEC_CHUNK * CPR / DEC_THREADS; ++u) {
+        const int idx = u * DEC_THREADS + tid, r = idx / CPR, c = idx - r * CPR;
+        if (r < rows) {
+          reinterpret_cast<uint4*>(ksm + r * D)[c ^ (r & SW)] = kt_[u];
+          reinterpret_cast<uint4*>(vsm + r * D)[c ^ (r & SW)] = vt_[u];
+        }
+      }
+    }
+    __syncthreads();
     uint32_t kw[D / 4];
     if (live) {
-      const uint4* ksrc = reinterpret_cast<const uint4*>(p.k8 + (cache_row0 + j) * D);
-      const uint4* vsrc = reinterpret_cast<const uint4*>(p.v8 + (cache_row0 + j) * D);
-      uint4 vr[D / 16];
 #pragma unroll
       for (int i = 0; i < D / 16; ++i) {
-        const uint4 kr = __ldg(ksrc + i);
+        const uint4 kr = reinterpret_cast<const uint4*>(ksm + tid * D)[i ^ (tid & SW)];
         kw[4 * i] = kr.x;
         kw[4 * i + 1] = kr.y;
         kw[4 * i + 2] = kr.z;
         kw[4 * i + 3] = kr.w;
-        vr[i] = __ldg(vsrc + i);
       }
-#pragma unroll
-      for (int i = 0; i < D / 16; ++i)
-        reinterpret_cast<uint4*>(vsm + tid * D)[i ^ (tid & SW)] = vr[i];
     }
 #pragma unroll 1
     for (int g = 0; g < G; ++g) {

@@ -511,7 +511,7 @@ int launch_decode_t(const lamp::DecodeParams& p, cudaStream_t st) {
                                            lamp::DEC_MAX_G * D / 4 +
                                            (lamp::DEC_THREADS / 32) * lamp::DEC_MAX_G * D +
                                            2 * lamp::DEC_MAX_G) +
-                        static_cast<size_t>(lamp::DEC_CHUNK) * D;  // value rows
+                        2 * static_cast<size_t>(lamp::DEC_CHUNK) * D;  // value and key rows
   static bool attr_set[64] = {};
   int dev = 0;
   LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
