@@ -308,7 +308,7 @@ def test_threshold_skip_infinite_is_the_look_ahead_rule():
 
 # ----------------------------------------------------------------- full size, sampled --
 
-@pytest.mark.parametrize("name", ["gqa4k", "gemma_local16k", "long32k"])
+@pytest.mark.parametrize("name", ["gqa4k", "gemma_local16k", "long32k", "long64k", "long128k"])
 def test_full_size_bitmask_sampled_rows(name):
     w = CONFIGS[name]
     rows = sample_rows(w, 64)
