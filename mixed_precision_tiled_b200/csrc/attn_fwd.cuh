@@ -47,7 +47,7 @@ namespace lamp {
 // where-codes recorded with a timeout (bits 8..15 of the error word)
 enum : uint32_t {
   W_QFULL = 1, W_EMPTY = 2, W_FULL = 3, W_SFULL = 4, W_S16 = 5, W_VOTE = 6, W_PFULL = 7,
-  W_ODONE = 8, W_DRAIN = 9, W_SELFTEST = 10, W_XCH = 11, W_ZFREE = 12
+  W_ODONE = 8, W_DRAIN = 9, W_SELFTEST = 10, W_XCH = 11, W_ZFREE = 12, W_OSTAGE = 13
 };
 
 struct AttnParams {
@@ -110,6 +110,7 @@ struct AttnCfg {
   static_assert(OFF_Q8 % 1024 == 0 && OFF_SLOTS % 1024 == 0 && SLOT_BYTES % 1024 == 0, "align");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   static_assert(2 * BN + D <= 512, "tmem");
+  static_assert(D != 256 || MT * D * 4 <= OFF_BAR, "O staging");
 };
 
 struct Bars {
@@ -128,6 +129,7 @@ struct Bars {
   uint32_t abort;
   uint32_t votes[2][8];
   uint64_t xbar[4];  // row-pair exchange of lane quadrant q (64 arrivals)
+  uint64_t ostage;   // every softmax warp has put its rows of O into the staging area (8)
 };
 static_assert(sizeof(Bars) <= 512, "barrier block");
 
@@ -971,43 +973,105 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
   constexpr int DH = C::D / 2;
   const size_t orow =
       (static_cast<size_t>(g.s.q_plane) * p.q_rows + g.s.q_row0 + (row_valid ? i : 0)) * C::D + h * DH;
+  // At D = 256 (128 KB of O per tile) O leaves through shared memory; at D <= 128 each thread
+  // stores its own row (measured: staging gains 4% at D = 256 and nothing at D = 128).
+  constexpr bool STAGE_O = C::D == 256;
+  if (STAGE_O && g.n > 0) {
+    // O leaves through shared memory so that every warp store writes whole 128-byte lines (a
+    // thread's own row lies one row pitch away from its neighbours').  Every operand in shared
+    // memory has been consumed (o_final), so Q and the ring hold the staging area: row r of
+    // the tile at r * RB bytes, its 16-byte units XOR-swizzled by r & 7, so that 32 rows
+    // writing the same unit and one warp reading 32 consecutive units hit distinct banks.
+    const uint32_t es = p.out_f32 ? 4u : 2u, RB = C::D * es;
+    const uint32_t stg = smem_u32(smem), rbase = stg + static_cast<uint32_t>(r) * RB;
+    const uint32_t sw = static_cast<uint32_t>(r & 7);
 #pragma unroll 1
-  for (int c = 0; c < DH / 32; ++c) {
-    uint32_t ov[32];
-    if (g.n > 0) {
+    for (int c = 0; c < DH / 32; ++c) {
+      uint32_t ov[32];
       tmem_ld32(lane_base + static_cast<uint32_t>(C::TMEM_O + h * DH + c * 32), ov);
       tmem_wait_ld();
-    } else {
+      auto sc = [&](int e) { return __float_as_uint(__uint_as_float(ov[e]) * inv); };
+      if (p.out_f32) {
+        const uint32_t u0 = static_cast<uint32_t>(h * DH + c * 32) / 4;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) ov[e] = 0u;
-    }
-    if (!row_valid) continue;
-    // 32-byte stores: each thread writes whole sectors of its row
-    auto sc = [&](int e) { return __float_as_uint(__uint_as_float(ov[e]) * inv); };
-    if (p.out_f32) {
-      float* dst = static_cast<float*>(p.o) + orow + c * 32;
+        for (int k = 0; k < 8; ++k)
+          st_shared_v4(rbase + (((u0 + k) ^ sw) << 4), sc(4 * k), sc(4 * k + 1), sc(4 * k + 2),
+                       sc(4 * k + 3));
+      } else {
+        const uint32_t u0 = static_cast<uint32_t>(h * DH + c * 32) / 8;
 #pragma unroll
-      for (int e = 0; e < 32; e += 8)
-        st_global_v8(dst + e, sc(e), sc(e + 1), sc(e + 2), sc(e + 3), sc(e + 4), sc(e + 5), sc(e + 6),
-                     sc(e + 7));
-    } else {
-      uint16_t* dst = static_cast<uint16_t*>(p.o) + orow + c * 32;
+        for (int k = 0; k < 4; ++k) {
+          uint32_t w[4];
 #pragma unroll
-      for (int e = 0; e < 32; e += 16) {
-        uint32_t w[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float a = __uint_as_float(ov[e + 2 * q]) * inv;
-          const float b2 = __uint_as_float(ov[e + 2 * q + 1]) * inv;
-          if (BF16) {
-            __nv_bfloat162 v2 = __floats2bfloat162_rn(a, b2);
-            w[q] = *reinterpret_cast<uint32_t*>(&v2);
-          } else {
-            __half2 v2 = __floats2half2_rn(a, b2);
-            w[q] = *reinterpret_cast<uint32_t*>(&v2);
+          for (int q = 0; q < 4; ++q) {
+            const float a = __uint_as_float(ov[8 * k + 2 * q]) * inv;
+            const float b2 = __uint_as_float(ov[8 * k + 2 * q + 1]) * inv;
+            if (BF16) {
+              __nv_bfloat162 v2 = __floats2bfloat162_rn(a, b2);
+              w[q] = *reinterpret_cast<uint32_t*>(&v2);
+            } else {
+              __half2 v2 = __floats2half2_rn(a, b2);
+              w[q] = *reinterpret_cast<uint32_t*>(&v2);
+            }
           }
+          st_shared_v4(rbase + (((u0 + k) ^ sw) << 4), w[0], w[1], w[2], w[3]);
         }
-        st_global_v8(dst + e, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars.ostage);
+    if (!warp_wait(&bars.ostage, 0, wc, W_OSTAGE)) return;
+    // the eight softmax warps (threads 0-255) copy the tile out, 16 bytes per thread, rows past
+    // the sequence skipped
+    const int UPR = static_cast<int>(RB / 16);
+    const size_t row0 = static_cast<size_t>(g.s.q_plane) * p.q_rows + g.s.q_row0 + g.q0;
+    uint8_t* obase = static_cast<uint8_t*>(p.o);
+    for (int L = static_cast<int>(threadIdx.x); L < C::MT * UPR; L += 256) {
+      const int row = L / UPR, u = L - row * UPR;
+      const uint4 v = ld_shared_v4(stg + static_cast<uint32_t>(row) * RB +
+                                   ((static_cast<uint32_t>(u) ^ static_cast<uint32_t>(row & 7)) << 4));
+      if (g.q0 + row < g.s.Lq)
+        st_global_v4(obase + (row0 + row) * C::D * es + static_cast<size_t>(u) * 16, v);
+    }
+  } else {
+#pragma unroll 1
+    for (int c = 0; c < DH / 32; ++c) {
+      uint32_t ov[32];
+      if (g.n > 0) {
+        tmem_ld32(lane_base + static_cast<uint32_t>(C::TMEM_O + h * DH + c * 32), ov);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) ov[e] = 0u;
+      }
+      if (!row_valid) continue;
+      // 32-byte stores: each thread writes whole sectors of its row
+      auto sc = [&](int e) { return __float_as_uint(__uint_as_float(ov[e]) * inv); };
+      if (p.out_f32) {
+        float* dst = static_cast<float*>(p.o) + orow + c * 32;
+#pragma unroll
+        for (int e = 0; e < 32; e += 8)
+          st_global_v8(dst + e, sc(e), sc(e + 1), sc(e + 2), sc(e + 3), sc(e + 4), sc(e + 5), sc(e + 6),
+                       sc(e + 7));
+      } else {
+        uint16_t* dst = static_cast<uint16_t*>(p.o) + orow + c * 32;
+#pragma unroll
+        for (int e = 0; e < 32; e += 16) {
+          uint32_t w[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float a = __uint_as_float(ov[e + 2 * q]) * inv;
+            const float b2 = __uint_as_float(ov[e + 2 * q + 1]) * inv;
+            if (BF16) {
+              __nv_bfloat162 v2 = __floats2bfloat162_rn(a, b2);
+              w[q] = *reinterpret_cast<uint32_t*>(&v2);
+            } else {
+              __half2 v2 = __floats2half2_rn(a, b2);
+              w[q] = *reinterpret_cast<uint32_t*>(&v2);
+            }
+          }
+          st_global_v8(dst + e, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+        }
       }
     }
   }
@@ -1046,6 +1110,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) attn_fwd_kernel(const __grid_co
     mbar_init(&bars.drain, 1);
     mbar_init(&bars.z_free, 8);
     mbar_init(&bars.o_final, 1);
+    mbar_init(&bars.ostage, 8);
     for (int q = 0; q < 4; ++q) mbar_init(&bars.xbar[q], 64);
     bars.abort = 0;
     fence_mbarrier_init();

@@ -300,6 +300,27 @@ __device__ __forceinline__ void st_global_v8(void* dst, uint32_t a0, uint32_t a1
                : "memory");
 }
 
+// 16-byte vector store and shared-memory copies (32-bit shared addresses, 16-byte aligned).
+__device__ __forceinline__ void st_global_v4(void* dst, uint4 v) {
+  asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a0, uint32_t a1, uint32_t a2,
+                                             uint32_t a3) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a0), "r"(a1), "r"(a2),
+               "r"(a3)
+               : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
 // ------------------------------------------------------------------ math ---------------
 
 // Hardware base-2 exponential (MUFU), flushing subnormal results to zero.
