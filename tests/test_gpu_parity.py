@@ -233,6 +233,14 @@ def test_output_in_input_dtype():
     assert np.abs(g["o"] - r["o"]).max() < 2e-2
 
 
+def test_output_in_input_dtype_d256_ragged():
+    # D = 256 writes O through a shared-memory staging area: 16-bit output, a ragged last
+    # query tile (rows past Lq must not be written) and a sliding window
+    w = small(CONFIGS["gemma_local16k"], B=1, H=2, Hkv=1, Lq=333, Lk=333, window=200)
+    g, r = parity_case(w, p_fp16=0.3, out="in")
+    assert np.abs(g["o"] - r["o"]).max() < 2e-2
+
+
 @pytest.mark.parametrize("fmt", ["int8", "e4m3"])
 @pytest.mark.parametrize("tau", [-1e30, 2.0, 4.0, 8.0])
 def test_adaptive_small(fmt, tau):
