@@ -153,3 +153,53 @@ def test_skip_call_rejects_bad_arguments_on_host():
     assert L.lamp_attn_fwd_q8_skip(*args, mpt.mode_bits("bitmask"), 2.0, 8.0, None, None) == mpt.LAMP_ERR_INVALID
     assert L.lamp_attn_fwd_q8_skip(*args, adaptive, 4.0, 2.0, None, None) == mpt.LAMP_ERR_INVALID
     assert L.lamp_attn_fwd_q8_skip(*args, adaptive, 4.0, float("nan"), None, None) == mpt.LAMP_ERR_INVALID
+
+
+def test_decode_rejects_bad_arguments_on_host():
+    L = mpt.lib()
+    ptrs = [0x1000] * 10  # q, q8, q_scale, k8, k_scale, v8, v_scale, len_k, o, lse
+    bitmask = mpt.mode_bits("bitmask")
+
+    def call(p=ptrs, B=1, H=4, Hkv=1, max_k=256, D=128, scale=0.0, mask=None, gt=1, mode=bitmask):
+        return L.lamp_decode_fwd(*p, B, H, Hkv, max_k, D, scale, mask, gt, mode, None)
+
+    assert call(p=[None] + ptrs[1:]) == mpt.LAMP_ERR_INVALID              # null query
+    assert call(p=ptrs[:3] + [0x1008] + ptrs[4:]) == mpt.LAMP_ERR_INVALID  # k8 not 16-byte aligned
+    assert call(mode=mpt.mode_bits("adaptive")) == mpt.LAMP_ERR_UNSUPPORTED
+    assert call(mode=mpt.mode_bits(out="in")) == mpt.LAMP_ERR_UNSUPPORTED
+    assert call(H=16, Hkv=1) == mpt.LAMP_ERR_UNSUPPORTED                  # 16 query heads per KV head
+    assert call(H=3, Hkv=2) == mpt.LAMP_ERR_INVALID
+    assert call(max_k=0) == mpt.LAMP_ERR_INVALID
+    assert call(D=96) == mpt.LAMP_ERR_UNSUPPORTED
+    assert call(scale=float("nan")) == mpt.LAMP_ERR_INVALID
+    assert call(mask=0x4000, gt=0) == mpt.LAMP_ERR_INVALID
+
+
+def test_varlen_calls_reject_bad_arguments_on_host():
+    L = mpt.lib()
+    m = mpt.mode_bits("bitmask")
+    # quantiser: q set without its offsets, a non-positive total, misaligned input
+    assert L.lamp_quant_qk_varlen(0x1000, None, 0x2000, None, 0x3000, None, None, None,
+                                  1, 2, 1, 256, 256, 256, 256, 128, m, None) == mpt.LAMP_ERR_INVALID
+    assert L.lamp_quant_qk_varlen(0x1000, None, 0x2000, None, 0x3000, None, 0x4000, None,
+                                  1, 2, 1, 256, 256, 0, 256, 128, m, None) == mpt.LAMP_ERR_INVALID
+    assert L.lamp_quant_qk_varlen(0x1008, None, 0x2000, None, 0x3000, None, 0x4000, None,
+                                  1, 2, 1, 256, 256, 256, 256, 128, m, None) == mpt.LAMP_ERR_INVALID
+    # attention on precomputed codes: missing offsets
+    base = [0x1000] * 9
+    assert L.lamp_attn_fwd_q8_varlen(*base, None, 0x5000, 1, 2, 1, 256, 256, 256, 256, 128, 1, 0,
+                                     0.0, None, 1, m, 0.0, None, None) == mpt.LAMP_ERR_INVALID
+    # full call: null operand, non-positive totals, o not 32-byte aligned, unsupported D
+    full = dict(B=1, H=2, Hkv=1, max_q=256, max_k=256, total_q=256, total_k=256, D=128)
+
+    def fwd(q=0x1000, o=0x2000, cu=0x3000, **kw):
+        a = {**full, **kw}
+        return L.lamp_attn_fwd_varlen(q, 0x1000, 0x1000, o, 0x4000, cu, cu, a["B"], a["H"], a["Hkv"],
+                                      a["max_q"], a["max_k"], a["total_q"], a["total_k"], a["D"],
+                                      1, 0, 0.0, None, 1, m, 0.0, None)
+
+    assert fwd(q=None) == mpt.LAMP_ERR_INVALID
+    assert fwd(cu=None) == mpt.LAMP_ERR_INVALID
+    assert fwd(total_q=0) == mpt.LAMP_ERR_INVALID
+    assert fwd(o=0x2010) == mpt.LAMP_ERR_INVALID
+    assert fwd(D=80) == mpt.LAMP_ERR_UNSUPPORTED
