@@ -24,8 +24,8 @@
  *   - q, k, v, q8, k8 must be 16-byte aligned (TMA) and o 32-byte aligned (32-byte stores);
  *     D must be 64, 128 or 256.
  *   - Return value: LAMP_OK or an error code.  Arguments are checked synchronously before
- *     anything is launched; on error nothing is enqueued and lamp_last_error() describes the
- *     problem (thread-local string).  Device-side failures (a bounded wait in a kernel that
+ *     anything is launched or any workspace is touched; on error nothing is enqueued and
+ *     lamp_last_error() describes the problem (thread-local string).  Device-side failures (a bounded wait in a kernel that
  *     gave up) are reported by lamp_check().
  */
 #ifndef LAMP_H
@@ -120,12 +120,18 @@ int lamp_template_for_int8_fraction(int Lq, int Lk, int D, int group_tiles, int 
                                     int* band_groups, int* stride_groups,
                                     double* fp16_fraction);
 
-/* Routed attention forward, end to end: quantises Q and K into the library workspace
- * (lamp_set_workspace, or a cached allocation made on first use with cudaMalloc), then runs
- * the routed attention kernel.  Arguments as lamp_attn_fwd_q8 without the 8-bit operands.
+/* Routed attention forward, end to end: quantises Q and K into the library workspace, then
+ * runs the routed attention kernel.  Arguments as lamp_attn_fwd_q8 without the 8-bit operands.
  * o receives O (fp32, or the input dtype with LAMP_OUT_INDTYPE); lse receives the natural-log
  * row log-sum-exp of the scaled, routed scores (may be NULL).  Rows that see no key get
- * O = 0 and lse = -inf.  Calls that share the library workspace must not overlap on the GPU. */
+ * O = 0 and lse = -inf.
+ * Workspace: the caller's (lamp_set_workspace), else one cached block per device that is
+ * grown in stream order on `stream` (cudaMallocAsync, the old block released with
+ * cudaFreeAsync behind the work already queued there), so growing it never synchronises the
+ * device.  Calls that share the workspace must not overlap on the GPU: calls on different
+ * streams need the caller's ordering (events) between them.
+ * Every argument check of lamp_attn_fwd_q8 runs before the workspace is touched or anything
+ * is enqueued. */
 int lamp_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                   int H, int Hkv, int Lq, int Lk, int D, int causal, int window, float scale,
                   const uint64_t* mask_bits, int group_tiles, int mode, float tau, void* stream);
@@ -159,7 +165,12 @@ int lamp_attn_fwd_q8(const void* q, const void* k, const void* v, const void* q8
  *     process exits.  Problems needing more (lamp_workspace_size(...) > the maximum) are
  *     rejected with LAMP_ERR_INVALID before anything is launched.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.  With CUDA's
+ *     lazy module loading, the first lamp_* call that needs this library's device code on a
+ *     device (a kernel launch, or that lookup) loads the module there, and loading it is when
+ *     the driver places the array and the code in device memory.  Callers that must not see
+ *     any allocation after their set-up make one such call (this one, on a small problem)
+ *     during set-up.
  *   - All calls share the one array and it keeps the last call's contents; every byte a call
  *     reads is written earlier in the same call, so nothing needs clearing.  Calls whose work
  *     overlaps on the GPU (different streams, no ordering between them) race on the array.

@@ -140,7 +140,10 @@ WsLayout ws_layout(int B, int H, int Hkv, int Lq, int Lk, int D, int q_rows = 0,
   return w;
 }
 
-int get_workspace(size_t need, void** out) {
+// The cached workspace of the current device, grown in stream order on `st` (the old block is
+// released with cudaFreeAsync behind the work already queued on `st`, the new one allocated
+// with cudaMallocAsync), so that growing it never synchronises the device.
+int get_workspace(size_t need, cudaStream_t st, void** out) {
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_ws.user) {
     if (g_ws.user_bytes < need)
@@ -152,14 +155,9 @@ int get_workspace(size_t need, void** out) {
   LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
   if (dev < 0 || dev >= 64) return fail(LAMP_ERR_INVALID, "device index out of range");
   if (g_ws.cached_bytes[dev] < need) {
-    if (g_ws.cached[dev]) {
-      LAMP_CUDA(cudaDeviceSynchronize(), "cudaDeviceSynchronize");
-      cudaFree(g_ws.cached[dev]);
-      g_ws.cached[dev] = nullptr;
-      g_ws.cached_bytes[dev] = 0;
-    }
     void* p = nullptr;
-    LAMP_CUDA(cudaMalloc(&p, need), "cudaMalloc(workspace)");
+    LAMP_CUDA(cudaMallocAsync(&p, need, st), "cudaMallocAsync(workspace)");
+    if (g_ws.cached[dev]) cudaFreeAsync(g_ws.cached[dev], st);
     g_ws.cached[dev] = p;
     g_ws.cached_bytes[dev] = need;
   }
@@ -322,23 +320,27 @@ using Cfg64 = lamp::AttnCfg<64, 64, true>;
 using Cfg128 = lamp::AttnCfg<128, 128, false>;
 using Cfg256 = lamp::AttnCfg<256, 128, true>;
 
-// cu_q / cu_k non-null: variable-length batch of B sequences (at most Lq / Lk rows each) packed
-// into [heads][total][D] tensors.
-int attn_q8(const void* q, const void* k, const void* v, const void* q8, const void* k8,
-            const float* q_scale, const float* k_scale, void* o, float* lse, int B, int H,
-            int Hkv, int Lq, int Lk, int D, int causal, int window, float scale,
-            const uint64_t* mask_bits, int group_tiles, int mode, float tau, uint8_t* route_out,
-            cudaStream_t st, const int* cu_q = nullptr, const int* cu_k = nullptr,
-            int total_q = 0, int total_k = 0, float skip_tau = INFINITY) {
+// Host-side checks of a routed-attention call (sizes, operand pointers and alignment, causal /
+// window, mode bits, group size, tau, scale, threshold skip).  Makes no CUDA call and enqueues
+// nothing, so that every entry point can run all of them before it touches the workspace or
+// launches a kernel.  q8 / k8 / q_scale / k_scale are checked only when `codes` is set (the
+// end-to-end entry points place them in the workspace).  cu_q / cu_k non-null: variable-length
+// batch of B sequences (at most Lq / Lk rows each) packed into [heads][total][D] tensors.
+int check_attn(const void* q, const void* k, const void* v, bool codes, const void* q8,
+               const void* k8, const float* q_scale, const float* k_scale, const void* o, int B,
+               int H, int Hkv, int Lq, int Lk, int D, int causal, int window, float scale,
+               int group_tiles, int mode, float tau, const int* cu_q, const int* cu_k,
+               int total_q, int total_k, float skip_tau) {
   int r = check_sizes(B, H, Hkv, Lq, Lk, D);
   if (r) return r;
   const bool varlen = cu_q != nullptr;
   if (varlen && (!cu_k || total_q < 1 || total_k < 1 || total_q > (1 << 30) || total_k > (1 << 30)))
     return fail(LAMP_ERR_INVALID, "variable-length batch needs cu_q, cu_k and positive totals");
-  if (!q || !k || !v || !q8 || !k8 || !q_scale || !k_scale || !o)
-    return fail(LAMP_ERR_INVALID, "null operand pointer");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q8) || !aligned16(k8) ||
-      !aligned32(o))
+  if (!q || !k || !v || !o) return fail(LAMP_ERR_INVALID, "null operand pointer");
+  if (codes && (!q8 || !k8 || !q_scale || !k_scale))
+    return fail(LAMP_ERR_INVALID, "null 8-bit operand or scale pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned32(o) ||
+      (codes && (!aligned16(q8) || !aligned16(k8))))
     return fail(LAMP_ERR_INVALID, "q, k, v, q8, k8 must be 16-byte and o 32-byte aligned");
   if (causal != 0 && causal != 1) return fail(LAMP_ERR_INVALID, "causal must be 0 or 1");
   if (window < 0) return fail(LAMP_ERR_INVALID, "window must be >= 0");
@@ -352,11 +354,37 @@ int attn_q8(const void* q, const void* k, const void* v, const void* q8, const v
   const bool skip = !std::isinf(skip_tau) || skip_tau < 0.0f;
   if (skip && (!adaptive || !(skip_tau >= tau) || !(skip_tau >= 0.0f)))
     return fail(LAMP_ERR_INVALID, "skip_tau needs look-ahead mode and tau <= skip_tau");
-  if ((r = get_encode())) return r;
+  const long long grid = static_cast<long long>(B) * H * ((Lq + 127) / 128);
+  if (grid > 0x7FFFFFFF) return fail(LAMP_ERR_INVALID, "grid too large");
+  return LAMP_OK;
+}
 
+// Which attention kernel runs a prepared call.
+enum AttnKernel { K_CFG64, K_PP, K_CFG128, K_CFG256 };
+
+struct AttnCall {
+  lamp::AttnParams p;
+  AttnKernel kernel;
+  int grid;
+  size_t route_bytes;  // bytes of route_out cleared before the launch (0: none)
+};
+
+// Tensor maps and kernel parameters of a call that passed check_attn (host work only: nothing
+// is enqueued; a failure here leaves the device untouched).
+int prepare_attn(const void* q, const void* k, const void* v, const void* q8, const void* k8,
+                 const float* q_scale, const float* k_scale, void* o, float* lse, int B, int H,
+                 int Hkv, int Lq, int Lk, int D, int causal, int window, float scale,
+                 const uint64_t* mask_bits, int group_tiles, int mode, float tau,
+                 uint8_t* route_out, const int* cu_q, const int* cu_k, int total_q, int total_k,
+                 float skip_tau, AttnCall* call) {
+  int r;
+  if ((r = get_encode())) return r;
+  const bool varlen = cu_q != nullptr;
+  const bool adaptive = (mode & LAMP_ROUTE_ADAPTIVE) != 0;
+  const bool skip = !std::isinf(skip_tau) || skip_tau < 0.0f;
   int bm, bn;
   tile_shape(D, &bm, &bn);
-  lamp::AttnParams p;
+  lamp::AttnParams& p = call->p;
   std::memset(&p, 0, sizeof(p));
   const int BHq = B * H, BHk = B * Hkv;
   // TMA views [planes][rows][D]: dense (B*H planes of L rows) or packed (H planes of total rows)
@@ -400,28 +428,82 @@ int attn_q8(const void* q, const void* k, const void* v, const void* q8, const v
   p.bf16 = (mode & LAMP_IN_BF16) ? 1 : 0;
   p.out_f32 = (mode & LAMP_OUT_INDTYPE) ? 0 : 1;
   p.wait_ns = kWaitUs * 1000ull;
-  const long long grid = static_cast<long long>(BHq) * p.n_ct;
-  if (grid > 0x7FFFFFFF) return fail(LAMP_ERR_INVALID, "grid too large");
-  if (route_out)
-    LAMP_CUDA(cudaMemsetAsync(route_out, 0, static_cast<size_t>(BHq) * nqt * nkt, st), "memset route");
-  if (D == 64) return launch_attn_cfg<Cfg64>(p, static_cast<int>(grid), st);
-  // The two-tile kernel keeps two mask words per query tile (128 key groups); wider masks go
-  // to the single-tile kernel, which reads any number of words.
-  // (the threshold skip runs on the single-tile kernel)
-  if (D == 128 && !p.e4m3 && !skip && (adaptive || p.mask_words <= 2)) {
-    // persistent CTAs: one per SM (the kernel fills the SM's shared and tensor memory), each
-    // walking its share of the (batch, head, query-tile pair) work items
-    // (work items as in the kernel: query-tile pairs of two heads of one KV group when the
-    // group size is even, else pairs of consecutive query tiles of one head)
+  call->route_bytes = route_out ? static_cast<size_t>(BHq) * nqt * nkt : 0;
+  call->grid = BHq * p.n_ct;  // (check_attn bounds it)
+  if (D == 64) {
+    call->kernel = K_CFG64;
+  } else if (D == 128 && !p.e4m3 && !skip && (adaptive || p.mask_words <= 2)) {
+    // The two-tile kernel keeps two mask words per query tile (128 key groups); wider masks go
+    // to the single-tile kernel, which reads any number of words (as does the threshold skip).
+    // Persistent CTAs: one per SM (the kernel fills the SM's shared and tensor memory), each
+    // walking its share of the work items (query-tile pairs of two heads of one KV group when
+    // the group size is even, else pairs of consecutive query tiles of one head).
     const long long items = ((H / Hkv) % 2 == 0) ? static_cast<long long>(B) * (H / 2) * nqt
                                                  : static_cast<long long>(BHq) * ((nqt + 1) / 2);
     int nsm = 0;
-    if (int r = sm_count(&nsm)) return r;
-    const long long pgrid = std::min<long long>(items, nsm);
-    return launch_attn_pp(p, static_cast<int>(pgrid), st);
+    if ((r = sm_count(&nsm))) return r;
+    call->kernel = K_PP;
+    call->grid = static_cast<int>(std::min<long long>(items, nsm));
+  } else {
+    call->kernel = (D == 128) ? K_CFG128 : K_CFG256;
   }
-  if (D == 128) return launch_attn_cfg<Cfg128>(p, static_cast<int>(grid), st);
-  return launch_attn_cfg<Cfg256>(p, static_cast<int>(grid), st);
+  return LAMP_OK;
+}
+
+int launch_attn(const AttnCall& c, cudaStream_t st) {
+  if (c.route_bytes)
+    LAMP_CUDA(cudaMemsetAsync(c.p.route, 0, c.route_bytes, st), "memset route");
+  switch (c.kernel) {
+    case K_CFG64: return launch_attn_cfg<Cfg64>(c.p, c.grid, st);
+    case K_PP: return launch_attn_pp(c.p, c.grid, st);
+    case K_CFG128: return launch_attn_cfg<Cfg128>(c.p, c.grid, st);
+    default: return launch_attn_cfg<Cfg256>(c.p, c.grid, st);
+  }
+}
+
+// The routed attention kernel on already-quantised operands: checks, then prepare, then launch.
+int attn_q8(const void* q, const void* k, const void* v, const void* q8, const void* k8,
+            const float* q_scale, const float* k_scale, void* o, float* lse, int B, int H,
+            int Hkv, int Lq, int Lk, int D, int causal, int window, float scale,
+            const uint64_t* mask_bits, int group_tiles, int mode, float tau, uint8_t* route_out,
+            cudaStream_t st, const int* cu_q = nullptr, const int* cu_k = nullptr,
+            int total_q = 0, int total_k = 0, float skip_tau = INFINITY) {
+  int r = check_attn(q, k, v, true, q8, k8, q_scale, k_scale, o, B, H, Hkv, Lq, Lk, D, causal,
+                     window, scale, group_tiles, mode, tau, cu_q, cu_k, total_q, total_k,
+                     skip_tau);
+  if (r) return r;
+  AttnCall call;
+  if ((r = prepare_attn(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D, causal,
+                        window, scale, mask_bits, group_tiles, mode, tau, route_out, cu_q, cu_k,
+                        total_q, total_k, skip_tau, &call)))
+    return r;
+  return launch_attn(call, st);
+}
+
+// Quantise Q and K into `ws` (laid out as w), then run the routed attention: the end-to-end
+// path shared by lamp_attn_fwd, lamp_attn_fwd_noalloc and lamp_attn_fwd_varlen.  The caller has
+// run check_attn; the tensor maps are built before the quantiser is enqueued, so that a failure
+// there leaves the device untouched too.
+int quant_and_attend(const void* q, const void* k, const void* v, void* o, float* lse,
+                     void* ws, const WsLayout& w, int B, int H, int Hkv, int Lq, int Lk, int D,
+                     int causal, int window, float scale, const uint64_t* mask_bits,
+                     int group_tiles, int mode, float tau, cudaStream_t st,
+                     const int* cu_q = nullptr, const int* cu_k = nullptr, int total_q = 0,
+                     int total_k = 0) {
+  auto* base = static_cast<uint8_t*>(ws);
+  uint8_t* q8 = base + w.q8;
+  uint8_t* k8 = base + w.k8;
+  float* qs = reinterpret_cast<float*>(base + w.qs);
+  float* ks = reinterpret_cast<float*>(base + w.ks);
+  AttnCall call;
+  int r = prepare_attn(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D, causal, window,
+                       scale, mask_bits, group_tiles, mode, tau, nullptr, cu_q, cu_k, total_q,
+                       total_k, INFINITY, &call);
+  if (r) return r;
+  if ((r = quant_qk(q, k, q8, k8, qs, ks, B, H, Hkv, Lq, Lk, D, mode, st, cu_q, cu_k, total_q,
+                    total_k)))
+    return r;
+  return launch_attn(call, st);
 }
 
 }  // namespace
@@ -722,23 +804,16 @@ int lamp_set_workspace(void* ptr, size_t bytes) {
 int lamp_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                   int H, int Hkv, int Lq, int Lk, int D, int causal, int window, float scale,
                   const uint64_t* mask_bits, int group_tiles, int mode, float tau, void* stream) {
-  int r = check_sizes(B, H, Hkv, Lq, Lk, D);
+  int r = check_attn(q, k, v, false, nullptr, nullptr, nullptr, nullptr, o, B, H, Hkv, Lq, Lk,
+                     D, causal, window, scale, group_tiles, mode, tau, nullptr, nullptr, 0, 0,
+                     INFINITY);
   if (r) return r;
-  if (!q || !k || !v || !o) return fail(LAMP_ERR_INVALID, "null operand pointer");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   const WsLayout w = ws_layout(B, H, Hkv, Lq, Lk, D);
   void* ws = nullptr;
-  if ((r = get_workspace(w.total, &ws))) return r;
-  auto* base = static_cast<uint8_t*>(ws);
-  uint8_t* q8 = base + w.q8;
-  uint8_t* k8 = base + w.k8;
-  float* qs = reinterpret_cast<float*>(base + w.qs);
-  float* ks = reinterpret_cast<float*>(base + w.ks);
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned32(o))
-    return fail(LAMP_ERR_INVALID, "q, k, v must be 16-byte and o 32-byte aligned");
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((r = quant_qk(q, k, q8, k8, qs, ks, B, H, Hkv, Lq, Lk, D, mode, st))) return r;
-  return attn_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D, causal, window, scale,
-                 mask_bits, group_tiles, mode, tau, nullptr, st);
+  if ((r = get_workspace(w.total, st, &ws))) return r;
+  return quant_and_attend(q, k, v, o, lse, ws, w, B, H, Hkv, Lq, Lk, D, causal, window, scale,
+                          mask_bits, group_tiles, mode, tau, st);
 }
 
 int lamp_attn_fwd_q8_skip(const void* q, const void* k, const void* v, const void* q8,
@@ -796,9 +871,9 @@ int lamp_decode_fwd(const void* q, const void* q8, const float* q_scale, const v
   p.bf16 = (mode & LAMP_IN_BF16) ? 1 : 0;
   const size_t need = static_cast<size_t>(B) * H * p.nsplit * (2 + D) * sizeof(float);
   void* ws = nullptr;
-  if ((r = get_workspace(need, &ws))) return r;
-  p.part = static_cast<float*>(ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((r = get_workspace(need, st, &ws))) return r;
+  p.part = static_cast<float*>(ws);
   if (D == 64) return launch_decode<64>(p, st);
   if (D == 128) return launch_decode<128>(p, st);
   return launch_decode<256>(p, st);
@@ -840,28 +915,18 @@ int lamp_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, f
                          int max_k, int total_q, int total_k, int D, int causal, int window,
                          float scale, const uint64_t* mask_bits, int group_tiles, int mode,
                          float tau, void* stream) {
-  int r = check_sizes(B, H, Hkv, max_q, max_k, D);
+  if (!cu_q || !cu_k) return fail(LAMP_ERR_INVALID, "null sequence offsets");
+  int r = check_attn(q, k, v, false, nullptr, nullptr, nullptr, nullptr, o, B, H, Hkv, max_q,
+                     max_k, D, causal, window, scale, group_tiles, mode, tau, cu_q, cu_k, total_q,
+                     total_k, INFINITY);
   if (r) return r;
-  if (!q || !k || !v || !o || !cu_q || !cu_k) return fail(LAMP_ERR_INVALID, "null pointer");
-  if (total_q < 1 || total_k < 1 || total_q > (1 << 30) || total_k > (1 << 30))
-    return fail(LAMP_ERR_INVALID, "totals must be positive");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned32(o))
-    return fail(LAMP_ERR_INVALID, "q, k, v must be 16-byte and o 32-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   const WsLayout w = ws_layout(B, H, Hkv, max_q, max_k, D, total_q, total_k);
   void* ws = nullptr;
-  if ((r = get_workspace(w.total, &ws))) return r;
-  auto* base = static_cast<uint8_t*>(ws);
-  uint8_t* q8 = base + w.q8;
-  uint8_t* k8 = base + w.k8;
-  float* qs = reinterpret_cast<float*>(base + w.qs);
-  float* ks = reinterpret_cast<float*>(base + w.ks);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((r = quant_qk(q, k, q8, k8, qs, ks, B, H, Hkv, max_q, max_k, D, mode, st, cu_q, cu_k,
-                    total_q, total_k)))
-    return r;
-  return attn_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, max_q, max_k, D, causal, window,
-                 scale, mask_bits, group_tiles, mode, tau, nullptr, st, cu_q, cu_k, total_q,
-                 total_k);
+  if ((r = get_workspace(w.total, st, &ws))) return r;
+  return quant_and_attend(q, k, v, o, lse, ws, w, B, H, Hkv, max_q, max_k, D, causal, window,
+                          scale, mask_bits, group_tiles, mode, tau, st, cu_q, cu_k, total_q,
+                          total_k);
 }
 
 namespace {
@@ -889,11 +954,10 @@ int lamp_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
                           int B, int H, int Hkv, int Lq, int Lk, int D, int causal, int window,
                           float scale, const uint64_t* mask_bits, int group_tiles, int mode,
                           float tau, void* stream) {
-  int r = check_sizes(B, H, Hkv, Lq, Lk, D);
+  int r = check_attn(q, k, v, false, nullptr, nullptr, nullptr, nullptr, o, B, H, Hkv, Lq, Lk,
+                     D, causal, window, scale, group_tiles, mode, tau, nullptr, nullptr, 0, 0,
+                     INFINITY);
   if (r) return r;
-  if (!q || !k || !v || !o) return fail(LAMP_ERR_INVALID, "null operand pointer");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned32(o))
-    return fail(LAMP_ERR_INVALID, "q, k, v must be 16-byte and o 32-byte aligned");
   const WsLayout w = ws_layout(B, H, Hkv, Lq, Lk, D);
   if (w.total > static_cast<size_t>(LAMP_NOALLOC_MAX_BYTES))
     return fail(LAMP_ERR_INVALID,
@@ -902,17 +966,10 @@ int lamp_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
                 w.total, static_cast<size_t>(LAMP_NOALLOC_MAX_BYTES));
   void* ws = nullptr;
   if ((r = noalloc_base(&ws))) return r;
-  auto* base = static_cast<uint8_t*>(ws);
-  uint8_t* q8 = base + w.q8;
-  uint8_t* k8 = base + w.k8;
-  float* qs = reinterpret_cast<float*>(base + w.qs);
-  float* ks = reinterpret_cast<float*>(base + w.ks);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   // Every byte of the scratch that the attention reads is written first by the quantiser of
   // the same call, so nothing needs clearing between calls.
-  if ((r = quant_qk(q, k, q8, k8, qs, ks, B, H, Hkv, Lq, Lk, D, mode, st))) return r;
-  return attn_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D, causal, window, scale,
-                 mask_bits, group_tiles, mode, tau, nullptr, st);
+  return quant_and_attend(q, k, v, o, lse, ws, w, B, H, Hkv, Lq, Lk, D, causal, window, scale,
+                          mask_bits, group_tiles, mode, tau, static_cast<cudaStream_t>(stream));
 }
 
 int lamp_check(void* stream) {

@@ -67,10 +67,20 @@ def _attn_args(**kw):
     (dict(Lq=0), mpt.LAMP_ERR_INVALID),
     (dict(D=80), mpt.LAMP_ERR_UNSUPPORTED),
     (dict(q=None), mpt.LAMP_ERR_INVALID),
+    # the checks of the attention kernel itself also run before the quantiser is enqueued
+    (dict(q=0x1001), mpt.LAMP_ERR_INVALID),
+    (dict(o=0x5010), mpt.LAMP_ERR_INVALID),
+    (dict(causal=0, window=16), mpt.LAMP_ERR_UNSUPPORTED),
+    (dict(window=-1), mpt.LAMP_ERR_INVALID),
+    (dict(group_tiles=0), mpt.LAMP_ERR_INVALID),
+    (dict(mode=0x30), mpt.LAMP_ERR_INVALID),
+    (dict(mode=1, tau=float("nan")), mpt.LAMP_ERR_INVALID),
+    (dict(scale=float("nan")), mpt.LAMP_ERR_INVALID),
 ])
-def test_attn_fwd_rejects_bad_arguments_on_host(bad, code):
+@pytest.mark.parametrize("entry", ["lamp_attn_fwd", "lamp_attn_fwd_noalloc"])
+def test_attn_fwd_rejects_bad_arguments_on_host(bad, code, entry):
     with pytest.raises(mpt.LampError) as e:
-        mpt.lamp_attn_fwd(**_attn_args(**bad), stream=0)
+        getattr(mpt, entry)(**_attn_args(**bad), stream=0)
     assert e.value.code == code
 
 

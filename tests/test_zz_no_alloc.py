@@ -42,12 +42,21 @@ def test_noalloc_matches_regular_entry_point_twice(name, kw):
             if w.route == "bitmask" else None)
     ref_o, ref_lse = _run(mpt.lamp_attn_fwd, w, t, mask)
     fin = np.isfinite(ref_lse)
-    for _ in range(2):  # the shared scratch keeps the previous call's contents
-        o, lse = _run(mpt.lamp_attn_fwd_noalloc, w, t, mask)
-        assert np.array_equal(np.isfinite(lse), fin)
-        err = np.abs(o - ref_o)
-        assert err.max() <= O_MAX_ABS and err.mean() <= O_MEAN_ABS
-        assert np.abs(lse[fin] - ref_lse[fin]).max() <= LSE_ABS
+    # A caller workspace far too small for this problem: if the allocation-free entry point
+    # fell through to the workspace path (or to an allocation), the call would fail here.
+    tiny = torch.empty(512, dtype=torch.uint8, device="cuda")
+    mpt.lamp_set_workspace((tiny.data_ptr() + 255) & ~255, 256)
+    try:
+        with pytest.raises(mpt.LampError):  # the workspace path does see the small workspace
+            _run(mpt.lamp_attn_fwd, w, t, mask)
+        for _ in range(2):  # the shared scratch keeps the previous call's contents
+            o, lse = _run(mpt.lamp_attn_fwd_noalloc, w, t, mask)
+            assert np.array_equal(np.isfinite(lse), fin)
+            err = np.abs(o - ref_o)
+            assert err.max() <= O_MAX_ABS and err.mean() <= O_MEAN_ABS
+            assert np.abs(lse[fin] - ref_lse[fin]).max() <= LSE_ABS
+    finally:
+        mpt.lamp_set_workspace(None, 0)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
