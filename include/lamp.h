@@ -155,6 +155,36 @@ int lamp_attn_fwd_q8(const void* q, const void* k, const void* v, const void* q8
                      int window, float scale, const uint64_t* mask_bits, int group_tiles,
                      int mode, float tau, uint8_t* route_out, void* stream);
 
+/* Debug capture of the routed attention kernel (parity checks and measurement; the pages have
+ * no counterpart).  Runs the kernel and launch configuration that lamp_attn_fwd_q8 runs for the
+ * same arguments (dense batches, no threshold skip), in an instantiation that also copies raw
+ * score tiles out, and writes o, lse and route_out as lamp_attn_fwd_q8 does:
+ *   tile_slot: device int32 [B][H][nQT][nKT]; a value s in [0, n_slots) selects routing tile
+ *              (b, h, qt, kt) for slot s; any other value leaves the tile out;
+ *   s8_dump:   device 32-bit words [n_slots][BM][BN], or NULL: the tile's 8-bit product as the
+ *              kernel read it from tensor memory, before any scaling or masking -- the int32
+ *              accumulators sum_d cq[i][d] * ck[j][d] (INT8) or their fp32 bits (E4M3) -- for
+ *              every tile scored in 8 bits (route codes 1 and 3: the look-ahead rule's 8-bit
+ *              pass of a recomputed tile included);
+ *   s16_dump:  device fp32 [n_slots][BM][BN], or NULL: the unscaled 16-bit product
+ *              sum_d q[i][d] * k[j][d] of every tile scored in 16 bits (route codes 2 and 3).
+ * Rows i >= Lq and keys j >= Lk of a tile hold the product of the zero padding (0).  Slots of
+ * tiles without such a product are left as they were.  The dump buffers must be 16-byte
+ * aligned; LAMP_ERR_INVALID for a NULL slot map, n_slots < 1 or no dump buffer. */
+int lamp_attn_debug(const void* q, const void* k, const void* v, const void* q8,
+                    const void* k8, const float* q_scale, const float* k_scale, void* o,
+                    float* lse, int B, int H, int Hkv, int Lq, int Lk, int D, int causal,
+                    int window, float scale, const uint64_t* mask_bits, int group_tiles,
+                    int mode, float tau, uint8_t* route_out, const int* tile_slot, int n_slots,
+                    void* s8_dump, void* s16_dump, void* stream);
+
+/* The kernels' exponentials on n inputs (tests and measurement; the pages have no counterpart):
+ * y[i] = 2^x[i] by method 0, the degree-3 polynomial on the FMA pipe that the single-tile
+ * kernel uses for one exponential pair in eight (range reduction to [-1/2, 1/2] with the
+ * round-to-nearest constant 1.5 * 2^23; relative error below 7.7e-5 for x in [-125, 0]; 0 below
+ * -125), or method 1, the hardware approximation ex2.approx.ftz.  x, y: device fp32 arrays. */
+int lamp_exp2_eval(const float* x, float* y, int n, int method, void* stream);
+
 /* Same operation and arguments as lamp_attn_fwd, for callers that cannot allocate device
  * memory: code whose device memory is all owned by another allocator (a framework's caching
  * allocator that has already reserved it), or latency-bound serving loops that must not call

@@ -33,7 +33,7 @@ EXPORTS = ("lamp_tile_shape", "lamp_mask_words", "lamp_quant_qk", "lamp_build_ma
            "lamp_template_for_int8_fraction", "lamp_quant_qk_varlen", "lamp_attn_fwd_q8_varlen", "lamp_attn_fwd_q8_skip", "lamp_decode_fwd",
            "lamp_attn_fwd_varlen", "lamp_attn_fwd", "lamp_attn_fwd_q8", "lamp_attn_fwd_noalloc", "lamp_workspace_size",
            "lamp_set_workspace", "lamp_check", "lamp_selftest_timeout", "lamp_mma_probe",
-           "lamp_last_error")
+           "lamp_attn_debug", "lamp_exp2_eval", "lamp_last_error")
 NOALLOC_MAX_BYTES = 32 << 20  # LAMP_NOALLOC_MAX_BYTES
 
 
@@ -79,6 +79,9 @@ def lib():
                 "lamp_check": (_i, [_vp]),
                 "lamp_selftest_timeout": (_i, [_u64, _vp]),
                 "lamp_mma_probe": (_i, [_i, _i, _i, _vp]),
+                "lamp_attn_debug": (_i, [_vp] * 9 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp, _vp, _i,
+                                                            _vp, _vp, _vp]),
+                "lamp_exp2_eval": (_i, [_vp, _vp, _i, _i, _vp]),
                 "lamp_last_error": (ctypes.c_char_p, []),
             }
             for name, (res, args) in sig.items():
@@ -238,6 +241,21 @@ def lamp_attn_fwd_q8(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, L
                                   _stream(stream)))
 
 
+def lamp_attn_debug(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D, causal,
+                    window, scale, mask_bits, group_tiles, mode, tau, route_out, tile_slot,
+                    n_slots, s8_dump, s16_dump, stream=None):
+    _check(lib().lamp_attn_debug(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(q_scale),
+                                 _ptr(k_scale), _ptr(o), _ptr(lse), B, H, Hkv, Lq, Lk, D,
+                                 int(causal), int(window), float(scale), _ptr(mask_bits),
+                                 int(group_tiles), int(mode), float(tau), _ptr(route_out),
+                                 _ptr(tile_slot), int(n_slots), _ptr(s8_dump), _ptr(s16_dump),
+                                 _stream(stream)))
+
+
+def lamp_exp2_eval(x, y, n, method, stream=None):
+    _check(lib().lamp_exp2_eval(_ptr(x), _ptr(y), int(n), int(method), _stream(stream)))
+
+
 def lamp_workspace_size(B, H, Hkv, Lq, Lk, D, mode=0) -> int:
     return int(lib().lamp_workspace_size(B, H, Hkv, Lq, Lk, D, mode))
 
@@ -338,3 +356,40 @@ def attention_q8(q, k, v, q8, k8, q_scale, k_scale, *, causal=False, window=0, s
         lamp_attn_fwd_q8(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D, causal,
                          window, scale, mask_bits, group_tiles, mode, tau, rmap, stream)
     return (o, lse, rmap) if want_route else (o, lse)
+
+
+def attention_debug(q, k, v, q8, k8, q_scale, k_scale, tiles, *, causal=False, window=0,
+                    scale=0.0, mask_bits=None, group_tiles=1, route="bitmask", fmt="int8",
+                    tau=0.0, stream=None):
+    """lamp_attn_debug on torch tensors: ``tiles`` lists routing tiles (b, h, qt, kt).  Returns
+    (o, lse, route map, s8 [n][BM][BN] int32 words, s16 [n][BM][BN] fp32); slots the kernel did
+    not write keep the fill value 0x7fbadbad (int32) / NaN (fp32)."""
+    import torch
+    B, H, Lq, D = q.shape
+    _, Hkv, Lk, _ = k.shape
+    bm, bn = lamp_tile_shape(D)
+    nqt, nkt = -(-Lq // bm), -(-Lk // bn)
+    dtype = "bf16" if q.dtype == torch.bfloat16 else "fp16"
+    slot = torch.full((B, H, nqt, nkt), -1, dtype=torch.int32)
+    for s_, (b, h, qt, kt) in enumerate(tiles):
+        slot[b, h, qt, kt] = s_
+    slot = slot.to(q.device)
+    n = len(tiles)
+    s8 = torch.full((n, bm, bn), 0x7FBADBAD, dtype=torch.int32, device=q.device)
+    s16 = torch.full((n, bm, bn), float("nan"), dtype=torch.float32, device=q.device)
+    o = torch.empty((B, H, Lq, D), device=q.device, dtype=torch.float32)
+    lse = torch.empty((B, H, Lq), device=q.device, dtype=torch.float32)
+    rmap = torch.empty((B, H, nqt, nkt), device=q.device, dtype=torch.uint8)
+    lamp_attn_debug(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D, causal,
+                    window, scale, mask_bits, group_tiles, mode_bits(route, fmt, dtype), tau,
+                    rmap, slot, n, s8, s16, stream)
+    return o, lse, rmap, s8, s16
+
+
+def exp2_eval(x, method: int, stream=None):
+    """The kernels' 2^x (method 0 polynomial, 1 hardware) on a float32 CUDA tensor."""
+    import torch
+    x = x.contiguous()
+    y = torch.empty_like(x)
+    lamp_exp2_eval(x, y, x.numel(), method, stream)
+    return y

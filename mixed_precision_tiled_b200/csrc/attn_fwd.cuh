@@ -75,6 +75,13 @@ struct AttnParams {
                     // running max (log2 units; +inf: never)
   int adaptive, e4m3, bf16, out_f32;
   uint64_t wait_ns;
+  // Debug capture (lamp_attn_debug only; unused elsewhere): slot map [B][H][nQT][nKT] (slot of
+  // a routing tile, < 0 = not captured), and the raw score tiles [slots][BM][BN]: the 8-bit
+  // product words as read from TMEM (int32 or fp32 bits) and the 16-bit product (fp32).
+  const int* dbg_slot;
+  uint32_t* dbg_s8;
+  uint32_t* dbg_s16;
+  int dbg_nslots;
 };
 
 template <int D_, int BN_, bool STACK_>
@@ -533,6 +540,21 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
+// Debug capture: NCOL words of row `row` of routing tile (bh, qt, kt), starting at column col0,
+// into the caller's slot for that tile, if it has one (base null: that kind is not captured).
+template <int NCOL>
+__device__ __forceinline__ void dbg_dump(const AttnParams& p, uint32_t* base, int bm, int bn,
+                                         int bh, int qt, int kt, int row, int col0,
+                                         const uint32_t* raw) {
+  if (base == nullptr || qt >= p.nqt || kt >= p.nkt) return;
+  const int s = __ldg(p.dbg_slot + (static_cast<size_t>(bh) * p.nqt + qt) * p.nkt + kt);
+  if (s < 0 || s >= p.dbg_nslots) return;
+  uint32_t* dst = base + (static_cast<size_t>(s) * bm + row) * bn + col0;
+#pragma unroll
+  for (int c = 0; c < NCOL; c += 4)
+    st_global_v4(dst + c, make_uint4(raw[c], raw[c + 1], raw[c + 2], raw[c + 3]));
+}
+
 // Packed f32x2 helpers and the mixed-precision adds of the softmax.
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
@@ -610,7 +632,7 @@ __device__ __forceinline__ float add_hi16(float acc, uint32_t pk) {
 // half of the thread's own S columns (each 32-column chunk stored when ready), and keep two
 // partial row sums: of the exact p (for lse) and of the rounded p that the P.V MMA multiplies
 // (for O).  Both threads of a row take identical decisions from identical inputs.
-template <class C, bool BF16, bool E4M3, bool SKIP>
+template <class C, bool BF16, bool E4M3, bool SKIP, bool DBG>
 __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars& bars,
                              uint32_t tbase, const WaitCtx wc) {
   constexpr int N = C::BN, NH = C::BN / 2;
@@ -647,6 +669,15 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
   uint32_t zc = 0;  // uses of the separate 16-bit region Z so far
   bool ok = true;
   uint32_t raw[NH];
+  // debug capture of this thread's half row of a live routing tile's raw S (capture build only)
+  const int row_in_tile = C::STACK ? (r & 63) : r;
+  auto dump = [&](bool s16, bool live, int kt) {
+    if constexpr (DBG) {
+      if (live)
+        dbg_dump<NH>(p, s16 ? p.dbg_s16 : p.dbg_s8, C::BM, N, bh_q, qt_r, kt, row_in_tile,
+                     h * NH, raw);
+    }
+  };
 
   // Publish v in this thread's exchange slot of parity `par` and return the partner's value.
   // The slot's previous value (two key tiles back) has been read: the partner read it before
@@ -725,8 +756,10 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
       // maximum (a row reaches m - tau iff one of its halves does, so the tile vote needs no
       // exchange), read Z while the vote completes, and fall back to the 8-bit S only if the
       // tile is not flagged.  Mixed stacked halves know their precision from the mask.
+      const bool live_mine = hh ? pl.live[1] : pl.live[0];
       if (p.adaptive) {
         load_s(bsel * N);
+        dump(false, live_mine, kt);
         if (!E4M3) int_to_float();
         if (!full) apply_mask(j0);
         const float hmax = raw_max();
@@ -761,6 +794,7 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
         const uint32_t vw = hh ? v1 : v0;
         drop = SKIP && (vw & 2u) == 0;
         my16 = (vw & 1u) != 0 && !drop;
+        if (my16) dump(true, live_mine, kt);  // raw holds the 16-bit S of region Z
         if (!my16 && !drop) {  // not flagged: back to the 8-bit scores (still in this tile's S buffer)
           load_s(bsel * N);
           if (!E4M3) int_to_float();
@@ -771,8 +805,10 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
           if (!(ok = warp_wait(&bars.s16_full[0], zc & 1u, wc, W_S16))) break;
           tc_fence_after();
           load_s(C::TMEM_Z);
+          dump(true, live_mine, kt);
         } else {
           load_s(bsel * N);
+          dump(false, live_mine, kt);
           if (!E4M3) int_to_float();
         }
       }
@@ -793,6 +829,10 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
       }
     } else {
       load_s(bsel * N);
+      // (a two-phase tile here reads its 8-bit S first; in bitmask mode that S belongs to the
+      // 8-bit routing half only)
+      dump(sixteen, (hh ? pl.live[1] : pl.live[0]) &&
+                        (sixteen || p.adaptive || !(hh ? pl.b16[1] : pl.b16[0])), kt);
       cscale = sixteen ? p.scale_log2 : cs8;
       if (!sixteen && !E4M3) int_to_float();
       if (!full) apply_mask(j0);
@@ -841,6 +881,7 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
         tc_fence_after();
         if (my16) {  // (both threads of a row take this branch or neither)
           load_s(bsel * N);
+          dump(true, hh ? pl.live[1] : pl.live[0], kt);
           sixteen = true;
           cscale = p.scale_log2;
           if (!full) apply_mask(j0);
@@ -1083,7 +1124,7 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
 
 // ------------------------------------------------------------------ kernel ------------
 
-template <class C, bool BF16, bool E4M3, bool SKIP>
+template <class C, bool BF16, bool E4M3, bool SKIP, bool DBG>
 __global__ void __launch_bounds__(C::THREADS, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023u) != 0) {  // the layouts need a 1024-aligned base
@@ -1130,7 +1171,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) attn_fwd_kernel(const __grid_co
   } else if (warp == 9) {
     if (g.n > 0) mma_role<C, BF16, E4M3>(p, g, smem, bars, tbase, wc);
   } else {
-    softmax_role<C, BF16, E4M3, SKIP>(p, g, smem, bars, tbase, wc);
+    softmax_role<C, BF16, E4M3, SKIP, DBG>(p, g, smem, bars, tbase, wc);
   }
 
   tc_fence_before();
@@ -1158,6 +1199,23 @@ __global__ void selftest_timeout_kernel(uint64_t wait_ns) {
     mbar_wait(&bar, 0, w, W_SELFTEST);
   }
   __syncthreads();
+}
+
+// Evaluates the kernels' exponentials on a list of inputs (so that they can be checked against
+// the mathematical 2^x): method 0 = ex2_poly2 (the FMA-pipe polynomial), 1 = ex2 (MUFU).
+__global__ void exp2_eval_kernel(const float* x, float* y, int n, int method) {
+  for (int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x); i < n; i += 2 * gridDim.x * blockDim.x) {
+    const float x0 = x[i], x1 = (i + 1 < n) ? x[i + 1] : x[i];
+    float p0, p1;
+    if (method == 0) {
+      ex2_poly2(x0, x1, p0, p1);
+    } else {
+      p0 = ex2(x0);
+      p1 = ex2(x1);
+    }
+    y[i] = p0;
+    if (i + 1 < n) y[i + 1] = p1;
+  }
 }
 
 }  // namespace lamp

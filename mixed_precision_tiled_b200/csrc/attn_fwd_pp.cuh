@@ -597,7 +597,7 @@ __device__ void pp_mma(const AttnParams& p, uint8_t* smem, PPBars& bars, uint32_
 // One work item of the softmax role (it = the CTA's item count, the parity of its per-item
 // barrier phases).  The phase counters of the per-tile barriers run on across items.  Returns
 // false when a wait gave up.
-template <bool BF16, bool ADAPTIVE, bool VARLEN>
+template <bool BF16, bool ADAPTIVE, bool VARLEN, bool DBG>
 __device__ __forceinline__ bool pp_softmax_item(const AttnParams& p, const PPGeo& g, PPBars& bars,
                                                 uint32_t tbase, const WaitCtx wc, int it,
                                                 uint32_t& cs, uint32_t& c16, uint32_t& cvv,
@@ -683,6 +683,8 @@ __device__ __forceinline__ bool pp_softmax_item(const AttnParams& p, const PPGeo
     const int j0 = kt * N;
     const bool full = row_valid && j0 >= lo_r && j0 + N - 1 <= hi_r;
     bool sixteen = !ADAPTIVE && group_b16(p, mrow, gcur);
+    if constexpr (DBG)  // debug capture of the raw S this row read (capture build only)
+      dbg_dump<N>(p, sixteen ? p.dbg_s16 : p.dbg_s8, C::MT, N, bh_q, qt, kt, r, 0, raw);
     // (a zero block scale would turn masked -inf entries into NaN: keep it positive; the
     // scores of an all-zero block are 0 either way)
     float cscale = sixteen ? p.scale_log2 : fmaxf(sq_scale * ks, 1e-30f);
@@ -707,6 +709,7 @@ __device__ __forceinline__ bool pp_softmax_item(const AttnParams& p, const PPGeo
         ++c16;
         tc_fence_after();
         load_s();
+        if constexpr (DBG) dbg_dump<N>(p, p.dbg_s16, C::MT, N, bh_q, qt, kt, r, 0, raw);
         sixteen = true;
         cscale = p.scale_log2;
         if (!full) apply_mask(j0);
@@ -863,7 +866,7 @@ __device__ __forceinline__ bool pp_softmax_item(const AttnParams& p, const PPGeo
 }
 
 // The softmax role: the CTA's work items in turn.
-template <bool BF16, bool ADAPTIVE, bool VARLEN>
+template <bool BF16, bool ADAPTIVE, bool VARLEN, bool DBG>
 __device__ void pp_softmax(const AttnParams& p, PPBars& bars, uint32_t tbase, const WaitCtx wc) {
   uint32_t cs = 0, c16 = 0, cvv = 0;
   uint32_t raw[PPCfg::BN];
@@ -871,13 +874,13 @@ __device__ void pp_softmax(const AttnParams& p, PPBars& bars, uint32_t tbase, co
     const int item = pp_item(p, it);
     if (item < 0) break;
     const PPGeo g = pp_geo<VARLEN>(p, item);
-    if (!pp_softmax_item<BF16, ADAPTIVE, VARLEN>(p, g, bars, tbase, wc, it, cs, c16, cvv, raw)) break;
+    if (!pp_softmax_item<BF16, ADAPTIVE, VARLEN, DBG>(p, g, bars, tbase, wc, it, cs, c16, cvv, raw)) break;
   }
 }
 
 // ------------------------------------------------------------------ kernel ------------
 
-template <bool BF16, bool ADAPTIVE, bool VARLEN>
+template <bool BF16, bool ADAPTIVE, bool VARLEN, bool DBG>
 __global__ void __launch_bounds__(PPCfg::THREADS, 1)
     attn_fwd_pp_kernel(const __grid_constant__ AttnParams p) {
   using C = PPCfg;
@@ -928,7 +931,7 @@ __global__ void __launch_bounds__(PPCfg::THREADS, 1)
   // itself.
   if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory");
-    pp_softmax<BF16, ADAPTIVE, VARLEN>(p, bars, tbase, wc);
+    pp_softmax<BF16, ADAPTIVE, VARLEN, DBG>(p, bars, tbase, wc);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 104;\n" ::: "memory");
     if (warp == 8) {

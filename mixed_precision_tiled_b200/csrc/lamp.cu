@@ -252,24 +252,31 @@ int quant_qk(const void* q, const void* k, void* q8, void* k8, float* q_scale, f
   return launch_quant_t<false, false>(jq, jk, D, vec, st);
 }
 
-template <class C, bool BF16, bool E4M3, bool SKIP>
+template <class C, bool BF16, bool E4M3, bool SKIP, bool DBG = false>
 int launch_attn_cfg_t(const lamp::AttnParams& p, int grid, cudaStream_t st) {
   static bool attr_set[64] = {};
   int dev = 0;
   LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    LAMP_CUDA(cudaFuncSetAttribute(lamp::attn_fwd_kernel<C, BF16, E4M3, SKIP>,
+    LAMP_CUDA(cudaFuncSetAttribute(lamp::attn_fwd_kernel<C, BF16, E4M3, SKIP, DBG>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES),
               "cudaFuncSetAttribute");
     attr_set[dev] = true;
   }
-  lamp::attn_fwd_kernel<C, BF16, E4M3, SKIP><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(p);
+  lamp::attn_fwd_kernel<C, BF16, E4M3, SKIP, DBG><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(p);
   LAMP_CUDA(cudaGetLastError(), "attn_fwd_kernel launch");
   return LAMP_OK;
 }
 
 template <class C>
 int launch_attn_cfg(const lamp::AttnParams& p, int grid, cudaStream_t st) {
+  // the debug capture has its own instantiations (lamp_attn_debug: no threshold skip)
+  if (p.dbg_slot) {
+    if (p.bf16) return p.e4m3 ? launch_attn_cfg_t<C, true, true, false, true>(p, grid, st)
+                              : launch_attn_cfg_t<C, true, false, false, true>(p, grid, st);
+    return p.e4m3 ? launch_attn_cfg_t<C, false, true, false, true>(p, grid, st)
+                  : launch_attn_cfg_t<C, false, false, false, true>(p, grid, st);
+  }
   // the threshold skip has its own instantiation, so that the look-ahead path without it keeps
   // its code
   if (!std::isinf(p.skip_log2)) {
@@ -284,19 +291,19 @@ int launch_attn_cfg(const lamp::AttnParams& p, int grid, cudaStream_t st) {
                 : launch_attn_cfg_t<C, false, false, false>(p, grid, st);
 }
 
-template <bool BF16, bool ADAPTIVE, bool VARLEN>
+template <bool BF16, bool ADAPTIVE, bool VARLEN, bool DBG = false>
 int launch_attn_pp_t(const lamp::AttnParams& p, int grid, cudaStream_t st) {
   static bool attr_set[64] = {};
   int dev = 0;
   LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    LAMP_CUDA(cudaFuncSetAttribute(lamp::attn_fwd_pp_kernel<BF16, ADAPTIVE, VARLEN>,
+    LAMP_CUDA(cudaFuncSetAttribute(lamp::attn_fwd_pp_kernel<BF16, ADAPTIVE, VARLEN, DBG>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    lamp::PPCfg::SMEM_BYTES),
               "cudaFuncSetAttribute");
     attr_set[dev] = true;
   }
-  lamp::attn_fwd_pp_kernel<BF16, ADAPTIVE, VARLEN>
+  lamp::attn_fwd_pp_kernel<BF16, ADAPTIVE, VARLEN, DBG>
       <<<grid, lamp::PPCfg::THREADS, lamp::PPCfg::SMEM_BYTES, st>>>(p);
   LAMP_CUDA(cudaGetLastError(), "attn_fwd_pp_kernel launch");
   return LAMP_OK;
@@ -311,8 +318,14 @@ int launch_attn_pp_v(const lamp::AttnParams& p, int grid, cudaStream_t st) {
 }
 
 // Variable-length batches have their own instantiation: the dense one keeps compile-time
-// zero offsets.
+// zero offsets.  The debug capture (dense batches only) has its own as well.
 int launch_attn_pp(const lamp::AttnParams& p, int grid, cudaStream_t st) {
+  if (p.dbg_slot) {
+    if (p.bf16) return p.adaptive ? launch_attn_pp_t<true, true, false, true>(p, grid, st)
+                                  : launch_attn_pp_t<true, false, false, true>(p, grid, st);
+    return p.adaptive ? launch_attn_pp_t<false, true, false, true>(p, grid, st)
+                      : launch_attn_pp_t<false, false, false, true>(p, grid, st);
+  }
   return p.cu_q ? launch_attn_pp_v<true>(p, grid, st) : launch_attn_pp_v<false>(p, grid, st);
 }
 
@@ -782,6 +795,42 @@ int lamp_attn_fwd_q8(const void* q, const void* k, const void* v, const void* q8
   return attn_q8(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D, causal,
                  window, scale, mask_bits, group_tiles, mode, tau, route_out,
                  static_cast<cudaStream_t>(stream));
+}
+
+int lamp_attn_debug(const void* q, const void* k, const void* v, const void* q8,
+                    const void* k8, const float* q_scale, const float* k_scale, void* o,
+                    float* lse, int B, int H, int Hkv, int Lq, int Lk, int D, int causal,
+                    int window, float scale, const uint64_t* mask_bits, int group_tiles,
+                    int mode, float tau, uint8_t* route_out, const int* tile_slot, int n_slots,
+                    void* s8_dump, void* s16_dump, void* stream) {
+  if (!tile_slot || n_slots < 1) return fail(LAMP_ERR_INVALID, "a slot map and n_slots >= 1 are needed");
+  if (!s8_dump && !s16_dump) return fail(LAMP_ERR_INVALID, "no dump buffer");
+  if (!aligned16(s8_dump) || !aligned16(s16_dump))
+    return fail(LAMP_ERR_INVALID, "dump buffers must be 16-byte aligned");
+  int r = check_attn(q, k, v, true, q8, k8, q_scale, k_scale, o, B, H, Hkv, Lq, Lk, D, causal,
+                     window, scale, group_tiles, mode, tau, nullptr, nullptr, 0, 0, INFINITY);
+  if (r) return r;
+  AttnCall call;
+  if ((r = prepare_attn(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D, causal,
+                        window, scale, mask_bits, group_tiles, mode, tau, route_out, nullptr,
+                        nullptr, 0, 0, INFINITY, &call)))
+    return r;
+  call.p.dbg_slot = tile_slot;
+  call.p.dbg_s8 = static_cast<uint32_t*>(s8_dump);
+  call.p.dbg_s16 = static_cast<uint32_t*>(s16_dump);
+  call.p.dbg_nslots = n_slots;
+  return launch_attn(call, static_cast<cudaStream_t>(stream));
+}
+
+int lamp_exp2_eval(const float* x, float* y, int n, int method, void* stream) {
+  if (!x || !y || n < 0) return fail(LAMP_ERR_INVALID, "null pointer or negative n");
+  if (method != 0 && method != 1) return fail(LAMP_ERR_INVALID, "method must be 0 or 1");
+  if (n == 0) return LAMP_OK;
+  const int pairs = (n + 1) / 2;
+  const int grid = std::min((pairs + 255) / 256, 148 * 8);
+  lamp::exp2_eval_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n, method);
+  LAMP_CUDA(cudaGetLastError(), "exp2_eval_kernel launch");
+  return LAMP_OK;
 }
 
 size_t lamp_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int D, int mode) {

@@ -63,6 +63,7 @@ class _Args(ctypes.Structure):
         ("k_codes", ctypes.c_void_p), ("k_scales", ctypes.c_void_p),
         ("skip_tau", ctypes.c_double),
         ("k_codes_in", ctypes.c_void_p), ("k_scales_in", ctypes.c_void_p),
+        ("hinted", ctypes.c_void_p),
     ]
 
 
@@ -90,6 +91,9 @@ def lib():
             L.orc_build_mask_template.argtypes = [ctypes.c_void_p] + [ctypes.c_int] * 10
             L.orc_attention.restype = ctypes.c_int
             L.orc_attention.argtypes = [ctypes.POINTER(_Args)]
+            L.orc_score_tiles.restype = ctypes.c_int
+            L.orc_score_tiles.argtypes = [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 9 \
+                + [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
             _lib = L
     return _lib
 
@@ -168,7 +172,8 @@ def attention(q, k, v, *, bm, bn, causal=False, window=0, scale=None, mask=None,
     bitmask routing.  ``rows`` int64 [B,H,n] (sorted per head) restricts the output rows.
     Returns a dict with o (fp64 [B,H,R,D]), lse (fp64 [B,H,R]), route (uint8 [B,H,nQT,nKT]:
     0 dead, 1 8-bit, 2 16-bit by mask, 3 16-bit flagged, 4 dropped), margin (fp64, adaptive
-    decisions).  ``k_codes_in`` / ``k_scales_in`` (uint8 [B,Hkv,Lk,D], float32 [B,Hkv,nKT]):
+    decisions), hinted (uint8, 1 where a decision followed ``route_hint`` against the rule's
+    own outcome, which only happens where its margin is below ``hint_margin``).  ``k_codes_in`` / ``k_scales_in`` (uint8 [B,Hkv,Lk,D], float32 [B,Hkv,nKT]):
     an 8-bit key cache used by the 8-bit path instead of quantising ``k`` (decode with an INT8
     KV cache: TileMix page, section 4).  ``skip_tau`` (look-ahead mode; LATTE page, low-precision filtering of the keys
     far below the row maximum, read per tile): a tile every row of which has t_r < m_r -
@@ -218,7 +223,9 @@ def attention(q, k, v, *, bm, bn, causal=False, window=0, scale=None, mask=None,
         k_scales_in = np.ascontiguousarray(k_scales_in, dtype=np.float32)
         assert k_codes_in.shape == k.shape and k_scales_in.shape == (B, Hkv, nkt)
         a.k_codes_in, a.k_scales_in = _ptr(k_codes_in), _ptr(k_scales_in)
-    out = {"o": o, "lse": lse, "route": rmap, "margin": margin}
+    hinted = np.zeros((B, H, nqt, nkt), dtype=np.uint8)
+    a.hinted = _ptr(hinted)
+    out = {"o": o, "lse": lse, "route": rmap, "margin": margin, "hinted": hinted}
     if want_codes:
         qc = np.empty(q.shape, np.uint8)
         qs = np.empty((B, H, nqt), np.float32)
@@ -229,4 +236,26 @@ def attention(q, k, v, *, bm, bn, causal=False, window=0, scale=None, mask=None,
     rc = lib().orc_attention(ctypes.byref(a))
     if rc != 0:
         raise ValueError(f"oracle rejected the arguments (code {rc})")
+    return out
+
+
+def score_tiles(qx, kx, bm: int, bn: int, kind: str, tiles) -> np.ndarray:
+    """Raw (unscaled) score tiles, the reference of the library's debug capture.
+
+    ``tiles``: (b, h, qt, kt) routing tiles.  ``kind``: "int8" / "e4m3" (qx, kx uint8 codes
+    [B,H,Lq,D] / [B,Hkv,Lk,D], exact sums of code products) or "16bit" (fp32 values of the
+    16-bit inputs, fp64 sums).  Rows and keys past the problem count as zero vectors.  Returns
+    fp64 [n, bm, bn] (the INT8 sums are integers, exact in fp64)."""
+    kinds = {"int8": 0, "e4m3": 1, "16bit": 2}
+    dt = np.float32 if kind == "16bit" else np.uint8
+    qx = np.ascontiguousarray(qx, dtype=dt)
+    kx = np.ascontiguousarray(kx, dtype=dt)
+    B, H, Lq, D = qx.shape
+    _, Hkv, Lk, _ = kx.shape
+    t = np.ascontiguousarray(np.asarray(tiles, dtype=np.int32).reshape(-1, 4))
+    out = np.empty((t.shape[0], bm, bn), dtype=np.float64)
+    rc = lib().orc_score_tiles(_ptr(qx), _ptr(kx), B, H, Hkv, Lq, Lk, D, bm, bn, kinds[kind],
+                               _ptr(t), t.shape[0], _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle rejected the tile list")
     return out

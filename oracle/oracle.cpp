@@ -161,6 +161,8 @@ struct orc_args {
   // scales, the 16-bit path the values in k
   const uint8_t* k_codes_in;  // [B,Hkv,Lk,D]
   const float* k_scales_in;   // [B,Hkv,nKT]
+  uint8_t* hinted;            // optional [B,H,nQT,nKT]: 1 where a decision followed route_hint
+                              // against the rule's own outcome (its margin < hint_margin)
 };
 
 double orc_e4m3_decode(uint8_t c) { return e4m3_decode(c); }
@@ -232,6 +234,58 @@ void orc_build_mask_template(uint64_t* mask, int B, int H, int Lq, int Lk, int b
       }
 }
 
+// Raw score tiles (the reference of the library's debug capture).  For each listed routing tile
+// (b, h, qt, kt) -- tiles[4 * t + 0..3] -- the unscaled product over every position of the tile,
+// query row i = qt * bm + r and key j = kt * bn + c, with rows or keys past the problem counting
+// as zero vectors (the 8-bit product is what the scores of TileMix's INT8 path are made of,
+// before the rescale with the two block scales):
+//   kind 0: sum_d cq[i][d] * ck[j][d] over INT8 codes, exact int64;
+//   kind 1: the same over E4M3 codes, each decoded exactly, summed in fp64 (every product is
+//           exact and the sums stay far below 2^53, so the sum is exact);
+//   kind 2: sum_d q[i][d] * k[j][d] over the 16-bit inputs' values, in fp64.
+// qx / kx: uint8 codes (kinds 0, 1) or fp32 values (kind 2), [B][H][Lq][D] and [B][Hkv][Lk][D];
+// query head h reads KV head h / (H / Hkv).  out: fp64 [n][bm][bn].  Returns 1 on bad arguments.
+int orc_score_tiles(const void* qx, const void* kx, int B, int H, int Hkv, int Lq, int Lk, int D,
+                    int bm, int bn, int kind, const int32_t* tiles, int n, double* out) {
+  if (H % Hkv != 0 || kind < 0 || kind > 2) return 1;
+  const int G = H / Hkv;
+  for (int t = 0; t < n; ++t) {
+    const int b = tiles[4 * t], h = tiles[4 * t + 1], qt = tiles[4 * t + 2], kt = tiles[4 * t + 3];
+    if (b < 0 || b >= B || h < 0 || h >= H || qt < 0 || kt < 0) return 1;
+    const int kvh = h / G;
+    for (int r = 0; r < bm; ++r)
+      for (int c = 0; c < bn; ++c) {
+        const long i = (long)qt * bm + r, j = (long)kt * bn + c;
+        double v = 0.0;
+        if (i < Lq && j < Lk) {
+          const size_t qo = (((size_t)b * H + h) * Lq + i) * D;
+          const size_t ko = (((size_t)b * Hkv + kvh) * Lk + j) * D;
+          if (kind == 0) {
+            const uint8_t* cq = static_cast<const uint8_t*>(qx) + qo;
+            const uint8_t* ck = static_cast<const uint8_t*>(kx) + ko;
+            int64_t acc = 0;
+            for (int d = 0; d < D; ++d) acc += (int64_t)(int8_t)cq[d] * (int64_t)(int8_t)ck[d];
+            v = (double)acc;
+          } else if (kind == 1) {
+            const uint8_t* cq = static_cast<const uint8_t*>(qx) + qo;
+            const uint8_t* ck = static_cast<const uint8_t*>(kx) + ko;
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d) acc += e4m3_decode(cq[d]) * e4m3_decode(ck[d]);
+            v = acc;
+          } else {
+            const float* x = static_cast<const float*>(qx) + qo;
+            const float* y = static_cast<const float*>(kx) + ko;
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d) acc += (double)x[d] * (double)y[d];
+            v = acc;
+          }
+        }
+        out[((size_t)t * bm + r) * bn + c] = v;
+      }
+  }
+  return 0;
+}
+
 int orc_attention(const orc_args* a) {
   Geometry g{a->B, a->H, a->Hkv, a->Lq, a->Lk, a->D, a->bm, a->bn, a->causal, a->window};
   if (g.H % g.Hkv != 0 || g.D <= 0 || g.bm <= 0 || g.bn <= 0) return 1;
@@ -281,6 +335,7 @@ int orc_attention(const orc_args* a) {
       }
     }
   if (a->route) std::memset(a->route, 0, (size_t)g.B * g.H * nqt * nkt);
+  if (a->hinted) std::memset(a->hinted, 0, (size_t)g.B * g.H * nqt * nkt);
   if (a->margin)
     for (size_t i = 0; i < (size_t)g.B * g.H * nqt * nkt; ++i) a->margin[i] = INF;
 
@@ -384,8 +439,11 @@ int orc_attention(const orc_args* a) {
               }
             }
             double sm = keep ? keep_margin : drop_margin;
-            if (hint && sm < a->hint_margin && (hint[kt] == 1 || hint[kt] == 3 || hint[kt] == 4))
+            if (hint && sm < a->hint_margin && (hint[kt] == 1 || hint[kt] == 3 || hint[kt] == 4)) {
+              const bool own = keep;
               keep = (hint[kt] != 4);
+              if (a->hinted && keep != own) a->hinted[ti] = 1;
+            }
             if (!keep) {
               tile_route[kt] = 4;
               if (a->margin) a->margin[ti] = sm;
@@ -415,8 +473,11 @@ int orc_attention(const orc_args* a) {
           double margin = flagged ? pass_margin : fail_margin;
           // Where the decision is within `hint_margin` of flipping, two correct
           // implementations may disagree; follow the supplied routing map there.
-          if (hint && margin < a->hint_margin && (hint[kt] == 1 || hint[kt] == 3))
+          if (hint && margin < a->hint_margin && (hint[kt] == 1 || hint[kt] == 3)) {
+            const bool own = flagged;
             flagged = (hint[kt] == 3);
+            if (a->hinted && flagged != own) a->hinted[ti] = 1;
+          }
           tile_route[kt] = flagged ? 3 : 1;
           if (a->margin) a->margin[ti] = std::min(a->margin[ti], margin);
           for (int r = 0; r < rows_in_tile; ++r) {

@@ -213,3 +213,20 @@ def test_varlen_calls_reject_bad_arguments_on_host():
     assert fwd(total_q=0) == mpt.LAMP_ERR_INVALID
     assert fwd(o=0x2010) == mpt.LAMP_ERR_INVALID
     assert fwd(D=80) == mpt.LAMP_ERR_UNSUPPORTED
+
+
+def test_debug_and_exp2_entries_reject_bad_arguments_on_host():
+    L = mpt.lib()
+    base = [0x1000] * 9 + [1, 1, 1, 128, 128, 128, 1, 0, 0.0, None, 1, 0, 0.0, None]
+    # no slot map, n_slots < 1, no dump buffer, misaligned dump buffer
+    assert L.lamp_attn_debug(*base, None, 1, 0x2000, None, None) == mpt.LAMP_ERR_INVALID
+    assert L.lamp_attn_debug(*base, 0x3000, 0, 0x2000, None, None) == mpt.LAMP_ERR_INVALID
+    assert L.lamp_attn_debug(*base, 0x3000, 1, None, None, None) == mpt.LAMP_ERR_INVALID
+    assert L.lamp_attn_debug(*base, 0x3000, 1, 0x2004, None, None) == mpt.LAMP_ERR_INVALID
+    # the attention checks apply too (window without causal)
+    bad = list(base)
+    bad[15], bad[16] = 0, 16
+    assert L.lamp_attn_debug(*bad, 0x3000, 1, 0x2000, None, None) == mpt.LAMP_ERR_UNSUPPORTED
+    assert L.lamp_exp2_eval(None, 0x1000, 4, 0, None) == mpt.LAMP_ERR_INVALID
+    assert L.lamp_exp2_eval(0x1000, 0x1000, 4, 2, None) == mpt.LAMP_ERR_INVALID
+    assert L.lamp_exp2_eval(0x1000, 0x1000, -1, 0, None) == mpt.LAMP_ERR_INVALID
