@@ -11,7 +11,16 @@ all of P.V), with P16 the measured dense bf16 peak and P8 = 2 * P16 (the nominal
 ratio of the part).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lamp|reference]
-                    [--workload gqa4k] [--p-fp16 P] [--tau T] [--no-sweep]
+                    [--workload long128k] [--p-fp16 P] [--tau T] [--no-sweep] [--no-extras]
+
+The default workload is the largest single-GPU configuration, long-context prefill at
+L = 131072 (B=1, H=32, Hkv=8, D=128, causal, 25% FP16 groups, swept over 0-100%).  The same
+run then measures the attention kernel on the other workloads at L >= 8192 (adaptive8k with
+its tau x 8-bit-format sweep, gemma_local16k, long32k, long64k) and reports them under
+"other_workloads_L_ge_8192".  Each roofline fraction is given on the ruled basis (P16 = the
+measured bf16 burst, P8 = 2 x P16) and, as "frac_other_bases", against the vendor library's
+measured 8-bit GEMM rate (torch._int_mm / torch._scaled_mm at 8192^3) and against the rates of
+the tcgen05 MMA shapes the kernel issues (the probe).
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own copy of the workload (independent
 problems, no data-path collective: weak scaling); the timed region is bracketed by a barrier and
@@ -41,15 +50,19 @@ KERNEL_SOURCES = ["mixed_precision_tiled_b200/csrc/attn_fwd.cuh",
                   "mixed_precision_tiled_b200/csrc/attn_fwd_pp.cuh",
                   "mixed_precision_tiled_b200/csrc/ptx.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
+# The headline is the largest single-GPU workload (long-context prefill at L = 131072); the
+# other workloads at L >= 8192 are measured in the same run as extra keys.
+DEFAULT_WORKLOAD = "long128k"
+EXTRA_WORKLOADS = ["adaptive8k", "gemma_local16k", "long32k", "long64k"]
 
 
 def parse():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["lamp", "reference"], default="lamp")
-    ap.add_argument("--workload", default="gqa4k", choices=sorted(CONFIGS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(CONFIGS))
     ap.add_argument("--p-fp16", type=float, default=None)
     ap.add_argument("--tau", type=float, default=None)
     ap.add_argument("--skip-tau", type=float, default=None,
@@ -67,6 +80,8 @@ def parse():
                          "default) or the structured sink/band/stride template whose INT8 share "
                          "is 1 - FP16 fraction (--p-fp16 0.25 = SpTrans75)")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other L >= 8192 workloads measured after the default one")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -325,7 +340,9 @@ def cpu_baseline(w, mask_np, t, seconds_target=15.0):
     flops = row_flops(w, rows)
     whole = rows.shape[-1] >= w.Lq
     what = (f"the whole workload {w.name}" if whole else
-            f"{rows.shape[-1]} seeded query rows per (batch, head) of {w.name}")
+            f"{rows.shape[-1]} seeded query rows per (batch, head) of {w.name}; the rate is "
+            f"measured on this sample, a whole run of the workload would take "
+            f"{w.flops() / (flops / dt) / 3600:.1f} h at it (extrapolated)")
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"{what} ({rows.size} rows, {flops / 1e9:.1f} GFLOP, {dt:.1f} s)",
             "seconds": dt}
@@ -341,7 +358,7 @@ def head_problem(w, t, mask, b, h):
     return sub, t.q[b:b + 1, h:h + 1], t.k[b:b + 1, kv:kv + 1], t.v[b:b + 1, kv:kv + 1], m
 
 
-def run_reference(args, budget_s=150.0):
+def run_reference(args, budget_s=90.0):
     """The oracle as it stands, timed on the host cores, on the CUDA arm's workload and metric.
 
     Each step runs the oracle on one seeded (batch, head) and a seeded sample of its query rows
@@ -687,6 +704,215 @@ def run_decode(args, w, mpt, torch, dist, dev, stream, world, rank):
     return 0
 
 
+def library_peaks(torch, dev, n=8192, reps=10):
+    """Dense 8-bit GEMM rates of the vendor library at n^3 (best of `reps`, CUDA events): INT8
+    by torch._int_mm, FP8 E4M3 by torch._scaled_mm (bf16 output, unit scales), and bf16 by
+    torch.matmul, in TOP/s / TFLOP/s (2 n^3 operations).  These are denominators only."""
+    out = {}
+    g = torch.Generator(device=dev).manual_seed(0)
+
+    def best(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return round(2.0 * n ** 3 / (min(ts) * 1e-3) / 1e12, 1)
+
+    try:
+        a = torch.randint(-127, 128, (n, n), device=dev, dtype=torch.int8, generator=g)
+        b = torch.randint(-127, 128, (n, n), device=dev, dtype=torch.int8, generator=g)
+        out["int8_int_mm"] = best(lambda: torch._int_mm(a, b))
+        del a, b
+    except Exception as e:  # noqa: BLE001  (report, do not fail the bench)
+        out["int8_int_mm_error"] = str(e)[:200]
+    try:
+        a = torch.randn((n, n), device=dev, generator=g).to(torch.float8_e4m3fn)
+        b = torch.randn((n, n), device=dev, generator=g).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device=dev, dtype=torch.float32)
+        out["e4m3_scaled_mm"] = best(lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one,
+                                                               out_dtype=torch.bfloat16))
+        del a, b
+    except Exception as e:  # noqa: BLE001
+        out["e4m3_scaled_mm_error"] = str(e)[:200]
+    a = torch.randn((n, n), device=dev, generator=g, dtype=torch.bfloat16)
+    b = torch.randn((n, n), device=dev, generator=g, dtype=torch.bfloat16)
+    out["bf16_matmul"] = best(lambda: torch.matmul(a, b))
+    del a, b
+    torch.cuda.empty_cache()
+    return out
+
+
+def roofline_fracs(F8, F16, attn_ms, peaks, fmt, lib=None, probe=None):
+    """Blended-roofline fractions of one attention launch: T_roof / measured time, with
+    T_roof = F8 / P8 + F16 / P16 on three bases: the ruled one (P16 = the measured bf16 burst,
+    P8 = 2 x P16), the vendor library's measured 8-bit GEMM rate for P8 (bf16 unchanged), and
+    the tcgen05 probe's rates for both (the MMA shapes the kernel issues)."""
+    t = attn_ms * 1e-3
+    P16 = peaks["bf16"] * 1e12
+    out = {"ruled": (F8 / (2.0 * P16) + F16 / P16) / t}
+    key = "int8_int_mm" if fmt == "int8" else "e4m3_scaled_mm"
+    if lib and key in lib:
+        out["library_8bit"] = (F8 / (lib[key] * 1e12) + F16 / P16) / t
+    if probe and "i8_ss_n128" in probe and "bf16_ss_n128" in probe:
+        # (no E4M3 probe kind: kind::f8f6f4 and kind::i8 have the same dense rate on this part)
+        out["tcgen05_probe"] = (F8 / (probe["i8_ss_n128"] * 1e12)
+                                + F16 / (probe["bf16_ss_n128"] * 1e12)) / t
+    return {k: round(v, 4) for k, v in out.items()}
+
+
+def traffic_record(w):
+    try:
+        with open(TRAFFIC_FILE) as f:
+            tr = json.load(f)
+        rec = tr.get("records", {}).get(w.name)
+        if rec and tr.get("kernel_hash") == kernel_hash():
+            return rec.get("traffic_bytes_per_launch")
+    except (OSError, ValueError):
+        pass
+    return None
+
+
+class Prefill:
+    """One workload on the device: inputs resident in HBM, the step (quantiser, routing mask,
+    attention kernel), its timing and the route map behind the blended roofline."""
+
+    def __init__(self, args, w, mpt, torch, dev, stream, t=None):
+        self.args, self.w, self.mpt, self.torch, self.dev, self.stream = args, w, mpt, torch, dev, stream
+        self.t = make_workload(w) if t is None else t
+        tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
+        self.tdt = tdt
+
+        def dev16(bits):
+            return torch.from_numpy(bits.view(np.int16)).view(tdt).to(dev)
+
+        self.q, self.k, self.v = dev16(self.t.q_bits), dev16(self.t.k_bits), dev16(self.t.v_bits)
+        B, H, Hkv = w.B, w.H, w.Hkv
+        self.mode = mpt.mode_bits(w.route, w.fmt, w.dtype)
+        self.q8 = torch.empty(self.q.shape, dtype=torch.uint8, device=dev)
+        self.k8 = torch.empty(self.k.shape, dtype=torch.uint8, device=dev)
+        self.qs = torch.empty((B, H, w.nqt), dtype=torch.float32, device=dev)
+        self.ks = torch.empty((B, Hkv, w.nkt), dtype=torch.float32, device=dev)
+        W = mpt.lamp_mask_words(w.Lk, w.D, w.group_tiles)
+        self.mask = torch.empty((B, H, w.nqt, W), dtype=torch.int64, device=dev)
+        self.o = torch.empty((B, H, w.Lq, w.D), dtype=torch.float32, device=dev)
+        self.lse = torch.empty((B, H, w.Lq), dtype=torch.float32, device=dev)
+        self.rmap = torch.empty((B, H, w.nqt, w.nkt), dtype=torch.uint8, device=dev)
+        self.flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 256 MiB > 126 MB L2
+        self.bitmask = w.route == "bitmask"
+        self.skip = args.skip_tau is not None and not self.bitmask
+        self.tparams = {}
+        self.launches_per_step = 1 + (1 if self.bitmask else 0) + 1  # quantiser, mask, attention
+
+    def flush_l2(self):
+        """Evict the previous step's lines: write 256 MiB, then read it back so that L2 holds
+        clean lines only (no write-back of the flush lands in the next timed step)."""
+        self.flush.zero_()
+        self.flush.view(self.torch.int64).sum()
+
+    def build_mask(self, pf):
+        w, mpt = self.w, self.mpt
+        if self.args.template == "sptrans":
+            if pf not in self.tparams:
+                self.tparams[pf] = template_params(mpt, w, pf)
+            mpt.lamp_build_mask_template(self.mask, w.B, w.H, w.Lq, w.Lk, w.D, w.group_tiles,
+                                         *self.tparams[pf], self.stream)
+        else:
+            mpt.lamp_build_mask(self.mask, w.B, w.H, w.Lq, w.Lk, w.D, w.group_tiles, pf,
+                                w.mask_seed, self.stream)
+
+    def attn(self, md, tu, route_out=None):
+        w, mpt = self.w, self.mpt
+        if self.skip:
+            mpt.lamp_attn_fwd_q8_skip(self.q, self.k, self.v, self.q8, self.k8, self.qs, self.ks,
+                                      self.o, self.lse, w.B, w.H, w.Hkv, w.Lq, w.Lk, w.D,
+                                      int(w.causal), w.window, 0.0, md, tu, self.args.skip_tau,
+                                      route_out, self.stream)
+        else:
+            mpt.lamp_attn_fwd_q8(self.q, self.k, self.v, self.q8, self.k8, self.qs, self.ks,
+                                 self.o, self.lse, w.B, w.H, w.Hkv, w.Lq, w.Lk, w.D,
+                                 int(w.causal), w.window, 0.0,
+                                 self.mask if self.bitmask else None, w.group_tiles, md, tu,
+                                 route_out, self.stream)
+
+    def step(self, ev_a=None, ev_b=None, p_fp16=None, mode_=None, tau_=None):
+        w = self.w
+        md = self.mode if mode_ is None else mode_
+        tu = w.tau if tau_ is None else tau_
+        self.mpt.lamp_quant_qk(self.q, self.k, self.q8, self.k8, self.qs, self.ks, w.B, w.H,
+                               w.Hkv, w.Lq, w.Lk, w.D, md, self.stream)
+        if self.bitmask:
+            self.build_mask(w.p_fp16 if p_fp16 is None else p_fp16)
+        if ev_a is not None:
+            ev_a.record(self.stream)
+        self.attn(md, tu)
+        if ev_b is not None:
+            ev_b.record(self.stream)
+
+    def timed(self, n, **kw):
+        """Per-step and attention-kernel device times (ms) over n steps, L2 flushed between."""
+        torch = self.torch
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+        for i in range(n):
+            self.flush_l2()
+            ev[i][0].record(self.stream)
+            self.step(ev[i][1], ev[i][2], **kw)
+            ev[i][3].record(self.stream)
+        torch.cuda.synchronize()
+        return ([ev[i][0].elapsed_time(ev[i][3]) for i in range(n)],
+                [ev[i][1].elapsed_time(ev[i][2]) for i in range(n)])
+
+    def route_flops(self, p_fp16=None, mode_=None, tau_=None):
+        """(F8, F16, F, 16-bit fraction, route map) of the configuration (one untimed call)."""
+        w = self.w
+        self.step(p_fp16=p_fp16, mode_=mode_, tau_=tau_)
+        self.attn(self.mode if mode_ is None else mode_, w.tau if tau_ is None else tau_,
+                  self.rmap)
+        self.torch.cuda.synchronize()
+        rm = self.rmap.cpu().numpy()
+        return (*blended_flops(w, rm), rm)
+
+    def sweep(self, peaks, lib, probe):
+        """FP16-fraction sweep (bitmask) or tau x 8-bit-format sweep with the rerouted fraction
+        (look-ahead), each point timed on its own."""
+        w, mpt, out = self.w, self.mpt, {}
+        n = 10 if w.flops() > 5e12 else max(20, self.args.steps // 10)
+        if self.bitmask:
+            for pf in (0.0, 0.1, 0.25, 0.5, 1.0):
+                f8, f16, ff, fr, _ = self.route_flops(p_fp16=pf)
+                _, at = self.timed(n, p_fp16=pf)
+                a = float(statistics.fmean(at))
+                out[f"{pf:g}"] = {"fp16_fraction_realised": round(fr, 4),
+                                  "attn_tflops": round(ff / (a * 1e-3) / 1e12, 1),
+                                  "roofline_frac": roofline_fracs(f8, f16, a, peaks, w.fmt, lib,
+                                                                  probe)["ruled"]}
+        else:
+            for fmt in ("int8", "e4m3"):
+                md = mpt.mode_bits(w.route, fmt, w.dtype)
+                for tau in (0.5, 1.0, 2.0, 4.0, 8.0):
+                    f8, f16, ff, fr, _ = self.route_flops(mode_=md, tau_=tau)
+                    _, at = self.timed(n, mode_=md, tau_=tau)
+                    a = float(statistics.fmean(at))
+                    out[f"{fmt} tau={tau:g}"] = {
+                        "rerouted_fraction": round(fr, 4),
+                        "attn_tflops": round(ff / (a * 1e-3) / 1e12, 1),
+                        "roofline_frac": roofline_fracs(f8, f16, a, peaks, fmt, lib, probe)["ruled"],
+                        "kernel": attn_kernel_name(w.replace(fmt=fmt))}
+        self.step()  # restore the configured mask / format / tau
+        self.torch.cuda.synchronize()
+        return out
+
+    def release(self):
+        for name in ("q", "k", "v", "q8", "k8", "qs", "ks", "mask", "o", "lse", "rmap", "flush"):
+            setattr(self, name, None)
+        self.torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -716,107 +942,27 @@ def main():
         return run_varlen(args, w, mpt, torch, dist, dev, stream, world, rank)
     if args.decode > 0:
         return run_decode(args, w, mpt, torch, dist, dev, stream, world, rank)
-    t = make_workload(w)
-    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
-
-    def dev16(bits):
-        return torch.from_numpy(bits.view(np.int16)).view(tdt).to(dev)
-
-    q, k, v = dev16(t.q_bits), dev16(t.k_bits), dev16(t.v_bits)
-    B, H, Hkv, Lq, Lk, D = w.B, w.H, w.Hkv, w.Lq, w.Lk, w.D
-    mode = mpt.mode_bits(w.route, w.fmt, w.dtype)
-    q8 = torch.empty(q.shape, dtype=torch.uint8, device=dev)
-    k8 = torch.empty(k.shape, dtype=torch.uint8, device=dev)
-    qs = torch.empty((B, H, w.nqt), dtype=torch.float32, device=dev)
-    ks = torch.empty((B, Hkv, w.nkt), dtype=torch.float32, device=dev)
-    W = mpt.lamp_mask_words(Lk, D, w.group_tiles)
-    mask = torch.empty((B, H, w.nqt, W), dtype=torch.int64, device=dev)
-    o = torch.empty((B, H, Lq, D), dtype=torch.float32, device=dev)
-    lse = torch.empty((B, H, Lq), dtype=torch.float32, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 256 MiB > 126 MB L2
-
-    def flush_l2():
-        """Evict the previous step's lines: write 256 MiB, then read it back so that L2 holds
-        clean lines only (no write-back of the flush lands in the next timed step)."""
-        flush.zero_()
-        flush.view(torch.int64).sum()
-    bitmask = w.route == "bitmask"
-
-    tparams = {}
-
-    def build_mask(pf):
-        if args.template == "sptrans":
-            if pf not in tparams:
-                tparams[pf] = template_params(mpt, w, pf)
-            mpt.lamp_build_mask_template(mask, B, H, Lq, Lk, D, w.group_tiles, *tparams[pf],
-                                         stream)
-        else:
-            mpt.lamp_build_mask(mask, B, H, Lq, Lk, D, w.group_tiles, pf, w.mask_seed, stream)
-
-    def step(ev_a=None, ev_b=None, p_fp16=None, mode_=None, tau_=None):
-        md = mode if mode_ is None else mode_
-        tu = w.tau if tau_ is None else tau_
-        mpt.lamp_quant_qk(q, k, q8, k8, qs, ks, B, H, Hkv, Lq, Lk, D, md, stream)
-        if bitmask:
-            build_mask(w.p_fp16 if p_fp16 is None else p_fp16)
-        if ev_a is not None:
-            ev_a.record(stream)
-        if args.skip_tau is not None and not bitmask:
-            mpt.lamp_attn_fwd_q8_skip(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D,
-                                      int(w.causal), w.window, 0.0, md, tu, args.skip_tau, None,
-                                      stream)
-        else:
-            mpt.lamp_attn_fwd_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D,
-                                 int(w.causal), w.window, 0.0, mask if bitmask else None,
-                                 w.group_tiles, md, tu, None, stream)
-        if ev_b is not None:
-            ev_b.record(stream)
-
-    launches_per_step = 1 + (1 if bitmask else 0) + 1  # quantiser (Q and K), mask, attention
-
-    def timed(n, **kw):
-        """Per-step and attention-kernel device times (ms) over n steps, L2 flushed between."""
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
-        for i in range(n):
-            flush_l2()
-            ev[i][0].record(stream)
-            step(ev[i][1], ev[i][2], **kw)
-            ev[i][3].record(stream)
-        torch.cuda.synchronize()
-        st = [ev[i][0].elapsed_time(ev[i][3]) for i in range(n)]
-        at = [ev[i][1].elapsed_time(ev[i][2]) for i in range(n)]
-        return st, at
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    mpt.lamp_check(stream)
-
-    # routing map of this configuration (untimed) -> blended-roofline FLOP split
-    rmap = torch.empty((B, H, w.nqt, w.nkt), dtype=torch.uint8, device=dev)
-    if args.skip_tau is not None and not bitmask:
-        mpt.lamp_attn_fwd_q8_skip(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D,
-                                  int(w.causal), w.window, 0.0, mode, w.tau, args.skip_tau, rmap,
-                                  stream)
-    else:
-        mpt.lamp_attn_fwd_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D,
-                             int(w.causal), w.window, 0.0, mask if bitmask else None,
-                             w.group_tiles, mode, w.tau, rmap, stream)
-    torch.cuda.synchronize()
-    rm = rmap.cpu().numpy()
-    F8, F16, F, frac16 = blended_flops(w, rm)
 
     uuid = None
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
         pass
+    peaks = measured_peaks()
+    P = Prefill(args, w, mpt, torch, dev, stream)
+    B, H, Hkv, Lq, Lk, D = w.B, w.H, w.Hkv, w.Lq, w.Lk, w.D
+
+    for _ in range(args.warmup):
+        P.step()
+    torch.cuda.synchronize()
+    mpt.lamp_check(stream)
+    F8, F16, F, frac16, rm = P.route_flops()
 
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(uuid if rank == 0 else None) as clk:
-        step_ms, attn_ms = timed(args.steps)
+        step_ms, attn_ms = P.timed(args.steps)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
@@ -826,23 +972,24 @@ def main():
     value = world * F / (ms_per_step * 1e-3) / 1e12
 
     # end-to-end through the public C-ABI call with pinned host buffers
-    hq = torch.empty(q.shape, dtype=tdt, pin_memory=True).copy_(q)
-    hk = torch.empty(k.shape, dtype=tdt, pin_memory=True).copy_(k)
-    hv = torch.empty(v.shape, dtype=tdt, pin_memory=True).copy_(v)
-    ho = torch.empty(o.shape, dtype=torch.float32, pin_memory=True)
-    hl = torch.empty(lse.shape, dtype=torch.float32, pin_memory=True)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    tdt = P.tdt
+    hq = torch.empty(P.q.shape, dtype=tdt, pin_memory=True).copy_(P.q)
+    hk = torch.empty(P.k.shape, dtype=tdt, pin_memory=True).copy_(P.k)
+    hv = torch.empty(P.v.shape, dtype=tdt, pin_memory=True).copy_(P.v)
+    ho = torch.empty(P.o.shape, dtype=torch.float32, pin_memory=True)
+    hl = torch.empty(P.lse.shape, dtype=torch.float32, pin_memory=True)
+    dq, dk, dv = torch.empty_like(P.q), torch.empty_like(P.k), torch.empty_like(P.v)
 
     def e2e_step():
         dq.copy_(hq, non_blocking=True)
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
-        if bitmask:
-            build_mask(w.p_fp16)
-        mpt.lamp_attn_fwd(dq, dk, dv, o, lse, B, H, Hkv, Lq, Lk, D, int(w.causal), w.window,
-                          0.0, mask if bitmask else None, w.group_tiles, mode, w.tau, stream)
-        ho.copy_(o, non_blocking=True)
-        hl.copy_(lse, non_blocking=True)
+        if P.bitmask:
+            P.build_mask(w.p_fp16)
+        mpt.lamp_attn_fwd(dq, dk, dv, P.o, P.lse, B, H, Hkv, Lq, Lk, D, int(w.causal), w.window,
+                          0.0, P.mask if P.bitmask else None, w.group_tiles, P.mode, w.tau, stream)
+        ho.copy_(P.o, non_blocking=True)
+        hl.copy_(P.lse, non_blocking=True)
 
     n_e2e = max(3, min(args.steps, 30))
     for _ in range(3):
@@ -858,105 +1005,101 @@ def main():
     torch.cuda.synchronize()
     e2e_ms, = reduce_max([e0.elapsed_time(e1) / n_e2e], dev, dist)
     mpt.lamp_check(stream)
-    h2d = (q.numel() + k.numel() + v.numel()) * q.element_size()
-    d2h = o.numel() * 4 + lse.numel() * 4
+    h2d = (P.q.numel() + P.k.numel() + P.v.numel()) * P.q.element_size()
+    d2h = P.o.numel() * 4 + P.lse.numel() * 4
+    del hq, hk, hv, ho, hl, dq, dk, dv
 
-    # FP16-fraction sweep (bitmask workloads): TFLOP/s and roofline fraction per point
-    peaks = measured_peaks()
-    P16 = peaks["bf16"] * 1e12
-    P8 = 2.0 * P16
-    sweep = {}
-    if bitmask and not args.no_sweep:
-        for pf in (0.0, 0.1, 0.25, 0.5, 1.0):
-            step(p_fp16=pf)
-            mpt.lamp_attn_fwd_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D,
-                                 int(w.causal), w.window, 0.0, mask, w.group_tiles, mode, w.tau,
-                                 rmap, stream)
-            torch.cuda.synchronize()
-            f8, f16, ff, fr = blended_flops(w, rmap.cpu().numpy())
-            n = max(20, args.steps // 10)
-            _, at = timed(n, p_fp16=pf)
-            a = float(statistics.fmean(at))
-            sweep[f"{pf:g}"] = {"fp16_fraction_realised": round(fr, 4),
-                                "attn_tflops": round(ff / (a * 1e-3) / 1e12, 1),
-                                "roofline_frac": round((f8 / P8 + f16 / P16) / (a * 1e-3), 3)}
-        step()  # restore the configured mask
-        torch.cuda.synchronize()
-    # look-ahead workloads: tau x 8-bit format, with the rerouted (recomputed) tile fraction
-    if not bitmask and not args.no_sweep:
-        for fmt in ("int8", "e4m3"):
-            md = mpt.mode_bits(w.route, fmt, w.dtype)
-            for tau in (2.0, 4.0, 8.0):
-                step(mode_=md, tau_=tau)
-                mpt.lamp_attn_fwd_q8(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D,
-                                     int(w.causal), w.window, 0.0, None, w.group_tiles, md, tau,
-                                     rmap, stream)
-                torch.cuda.synchronize()
-                f8, f16, ff, fr = blended_flops(w, rmap.cpu().numpy())
-                n = max(10, args.steps // 10)
-                _, at = timed(n, mode_=md, tau_=tau)
-                a = float(statistics.fmean(at))
-                sweep[f"{fmt} tau={tau:g}"] = {
-                    "rerouted_fraction": round(fr, 4),
-                    "attn_tflops": round(ff / (a * 1e-3) / 1e12, 1),
-                    "roofline_frac": round((f8 / P8 + f16 / P16) / (a * 1e-3), 3)}
-        step()  # restore the configured format and tau
-        torch.cuda.synchronize()
-
-    quant = quantiser_bandwidth(mpt, torch, dev, stream, peaks) if not args.no_sweep else None
+    lib = library_peaks(torch, dev) if not args.no_sweep else None
     probe = tensor_probe(mpt, torch, stream) if not args.no_sweep else None
+    sweep = P.sweep(peaks, lib, probe) if not args.no_sweep else {}
+    quant = quantiser_bandwidth(mpt, torch, dev, stream, peaks) if not args.no_sweep else None
 
-    T_roof = F8 / P8 + F16 / P16
+    fr = roofline_fracs(F8, F16, att_ms, peaks, w.fmt, lib, probe)
     achieved = F / (att_ms * 1e-3) / 1e12
-    peak_blend = F / T_roof / 1e12
-    traffic = None
-    try:
-        with open(TRAFFIC_FILE) as f:
-            tr = json.load(f)
-        rec = tr.get("records", {}).get(w.name)
-        if rec and tr.get("kernel_hash") == kernel_hash():
-            traffic = rec.get("traffic_bytes_per_launch")
-    except (OSError, ValueError):
-        pass
+    T_roof = F8 / (2.0 * peaks["bf16"] * 1e12) + F16 / (peaks["bf16"] * 1e12)
+    mask_np = P.mask.cpu().numpy().view(np.uint64) if P.bitmask else None
+    dropped = round(float((tile_pairs(w)[None, None] * (rm == 4)).sum()) / max(1, F // (4 * w.D)), 4)
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": f"int8+{w.dtype}" if w.fmt == "int8" else f"e4m3+{w.dtype}",
+        "data": "synthetic",
+        "config": {"workload": describe(w, args.template, P.tparams.get(w.p_fp16))
+                               + (f", threshold skip {args.skip_tau}" if P.skip else ""),
+                   "fp16_fraction_realised": round(frac16, 4),
+                   "dropped_fraction": dropped,
+                   "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed between steps (256 MiB write, then read back); per-step CUDA "
+                         "events exclude the flush"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
+                     "peak": round(F / T_roof / 1e12, 1), "unit": "TFLOP/s",
+                     "frac": fr["ruled"], "traffic": traffic_record(w),
+                     "peak_basis": f"blended: F8/P8 + F16/P16, P16 = {peaks['bf16']} TFLOP/s bf16 "
+                                   f"burst ({peaks['source']}), P8 = 2 x P16 (nominal ratio)",
+                     "frac_other_bases": {k: v for k, v in fr.items() if k != "ruled"},
+                     "kernel": attn_kernel_name(w, args.skip_tau is not None),
+                     "attn_ms": round(att_ms, 4)},
+        "e2e": {"value": round(F * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 4)},
+        "clocks": clocks,
+        "gpu_launches": P.launches_per_step * args.steps,
+    }
+    if clocks.get("sm_mhz") and clocks.get("sm_max_mhz"):
+        # the same fraction against the peaks scaled to the SM clock seen under load (a kernel
+        # running under the power cap cannot reach the burst-clock peak)
+        line["roofline"]["frac_at_observed_clock"] = round(
+            fr["ruled"] * clocks["sm_max_mhz"] / clocks["sm_mhz"], 4)
+    if sweep:
+        line["sweep_fp16_fraction" if P.bitmask else "sweep_tau_format"] = sweep
+    if quant:
+        line["quantiser"] = quant
+    if probe:
+        line["tensor_probe_tflops"] = probe
+    if lib:
+        line["library_gemm_tflops"] = lib
+    t_host = P.t
+    P.release()
+
+    # the other workloads at L >= 8192 (the target's configurations), kernel-level, same run
+    if not args.no_extras and args.workload == DEFAULT_WORKLOAD and args.varlen == 0:
+        extras = {}
+        for name in EXTRA_WORKLOADS:
+            we = CONFIGS[name]
+            X = Prefill(args, we, mpt, torch, dev, stream)
+            for _ in range(max(3, min(args.warmup, 5))):
+                X.step()
+            torch.cuda.synchronize()
+            f8, f16, ff, fr16, rme = X.route_flops()
+            n = max(3, min(args.steps, 20))
+            with ClockSampler(uuid if rank == 0 else None) as clk_e:
+                st_ms, at_ms = X.timed(n)
+            mpt.lamp_check(stream)
+            a = float(statistics.fmean(at_ms))
+            s_ms = float(statistics.fmean(st_ms))
+            fre = roofline_fracs(f8, f16, a, peaks, we.fmt, lib, probe)
+            ex = {"workload": describe(we), "steps": n,
+                  "step_tflops": round(ff / (s_ms * 1e-3) / 1e12, 1),
+                  "attn_tflops": round(ff / (a * 1e-3) / 1e12, 1), "attn_ms": round(a, 4),
+                  ("fp16_fraction_realised" if we.route == "bitmask" else "rerouted_fraction"):
+                      round(fr16, 4),
+                  "roofline_frac": fre["ruled"],
+                  "frac_other_bases": {k: v for k, v in fre.items() if k != "ruled"},
+                  "kernel": attn_kernel_name(we), "traffic": traffic_record(we),
+                  "clocks": clk_e.summary()}
+            if not args.no_sweep:
+                ex["sweep_fp16_fraction" if X.bitmask else "sweep_tau_format"] = X.sweep(peaks, lib, probe)
+            extras[name] = ex
+            X.release()
+            del X
+        line["other_workloads_L_ge_8192"] = extras
 
     if rank == 0:
-        line = {
-            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": f"int8+{w.dtype}" if w.fmt == "int8" else f"e4m3+{w.dtype}",
-            "data": "synthetic",
-            "config": {"workload": describe(w, args.template, tparams.get(w.p_fp16))
-                                   + (f", threshold skip {args.skip_tau}"
-                                      if args.skip_tau is not None and not bitmask else ""),
-                       "fp16_fraction_realised": round(frac16, 4),
-                       "dropped_fraction": round(float((tile_pairs(w)[None, None]
-                                                        * (rm == 4)).sum()) / max(1, F // (4 * w.D)), 4),
-                       "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "flushed between steps (256 MiB write, then read back); per-step CUDA events exclude the flush"},
-            "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
-                         "peak": round(peak_blend, 1), "unit": "TFLOP/s",
-                         "frac": round(achieved / peak_blend, 4), "traffic": traffic,
-                         "peak_basis": f"blended: F8/P8 + F16/P16, P16 = {peaks['bf16']} TFLOP/s "
-                                       f"bf16 burst ({peaks['source']}), P8 = 2 x P16 (nominal ratio)",
-                         "kernel": attn_kernel_name(w, args.skip_tau is not None),
-                         "attn_ms": round(att_ms, 4)},
-            "e2e": {"value": round(F * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": round(e2e_ms, 4)},
-            "clocks": clk.summary(),
-            "gpu_launches": launches_per_step * args.steps,
-        }
-        if sweep:
-            line["sweep_fp16_fraction" if bitmask else "sweep_tau_format"] = sweep
-        if quant:
-            line["quantiser"] = quant
-        if probe:
-            line["tensor_probe_tflops"] = probe
         if world == 1 and not args.no_cpu_baseline:
             import oracle  # noqa: F401  (CPU baseline leg only)
-            mask_np = mask.cpu().numpy().view(np.uint64) if bitmask else None
-            line["cpu_baseline"] = cpu_baseline(w, mask_np, t)
+            line["cpu_baseline"] = cpu_baseline(w, mask_np, t_host)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

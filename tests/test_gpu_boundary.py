@@ -121,11 +121,13 @@ def test_valid_call_still_runs(entry):
     cu = torch.tensor([0, L], dtype=torch.int32, device="cuda")
     stream = torch.cuda.Stream()
     o_buf, lse = _outputs()
+    torch.cuda.synchronize()  # inputs were made on the default stream
     assert _call(entry, q, k, v, o_buf, lse, cu, stream) == mpt.LAMP_OK, mpt.lamp_last_error()
     mpt.lamp_check(stream)
     o = o_buf[:B * H * L * D]
     assert torch.isfinite(o).all() and not torch.any(lse == SENT)
     ref_o, ref_lse = _outputs()
+    torch.cuda.synchronize()
     assert _call("fwd", q, k, v, ref_o, ref_lse, cu, stream) == mpt.LAMP_OK
     mpt.lamp_check(stream)
     assert torch.equal(o, ref_o[:B * H * L * D]) and torch.equal(lse, ref_lse)
@@ -141,6 +143,7 @@ def test_workspace_grows_in_stream_order():
         q = torch.randn((1, 2, Lx, D), generator=g).to(torch.bfloat16).cuda()
         k = torch.randn((1, 1, Lx, D), generator=g).to(torch.bfloat16).cuda()
         v = torch.randn((1, 1, Lx, D), generator=g).to(torch.bfloat16).cuda()
+        stream.wait_stream(torch.cuda.current_stream())
         o, lse = mpt.attention(q, k, v, causal=True, stream=stream)
         q8, k8, qs, ks = mpt.quantize(q, k, stream=stream)
         o2, lse2 = mpt.attention_q8(q, k, v, q8, k8, qs, ks, causal=True, stream=stream)

@@ -132,15 +132,41 @@ def config_by_name(name: str) -> Workload:
     return CONFIGS[name]
 
 
+def _chunked(fn, n: int, chunk: int = 1 << 24):
+    """Runs fn(lo, hi) over [0, n) in chunks on a thread pool (numpy's element-wise kernels
+    release the GIL); the result does not depend on the chunking."""
+    if n <= chunk:
+        fn(0, n)
+        return
+    from concurrent.futures import ThreadPoolExecutor
+    import os
+    with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+        list(ex.map(lambda lo: fn(lo, min(n, lo + chunk)), range(0, n, chunk)))
+
+
 def _round_bf16(x: np.ndarray) -> np.ndarray:
     """fp32 -> bf16 bit patterns (uint16), round to nearest even (finite inputs)."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
-    r = ((u >> np.uint32(16)) & np.uint32(1)) + np.uint32(0x7FFF)
-    return ((u + r) >> np.uint32(16)).astype(np.uint16)
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).reshape(-1)
+    out = np.empty(u.shape, dtype=np.uint16)
+
+    def part(lo, hi):
+        v = u[lo:hi]
+        r = ((v >> np.uint32(16)) & np.uint32(1)) + np.uint32(0x7FFF)
+        out[lo:hi] = (v + r) >> np.uint32(16)
+
+    _chunked(part, u.size)
+    return out.reshape(x.shape)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
-    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32)
+    flat = np.ascontiguousarray(b).reshape(-1)
+    out = np.empty(flat.shape, dtype=np.uint32)
+
+    def part(lo, hi):
+        out[lo:hi] = flat[lo:hi].astype(np.uint32) << np.uint32(16)
+
+    _chunked(part, flat.size)
+    return out.view(np.float32).reshape(b.shape)
 
 
 def to_16bit(x: np.ndarray, dtype: str):
