@@ -240,8 +240,8 @@ int lamp_attn_fwd_q8_skip(const void* q, const void* k, const void* v, const voi
  *   values v8 * sv; softmax and P.V in fp32; o: [B][H][D] fp32; lse: [B][H] natural log, -inf
  *      for an empty cache.
  * mode: LAMP_FMT_*, LAMP_IN_* (bitmask routing, fp32 output; else LAMP_ERR_UNSUPPORTED); at
- * most 8 query heads per KV head.  Uses the library workspace (B * H * ceil(max_k / 256) *
- * (D + 2) floats of split partials), like lamp_attn_fwd. */
+ * most 8 query heads per KV head.  Uses the library workspace (B * H * ceil(max_k / 1024) *
+ * (D + 2) floats of split partials: one per run of 8 chunks of 128 keys), like lamp_attn_fwd. */
 int lamp_decode_fwd(const void* q, const void* q8, const float* q_scale, const void* k8,
                     const float* k_scale, const void* v8, const float* v_scale, const int* len_k,
                     float* o, float* lse, int B, int H, int Hkv, int max_k, int D, float scale,

@@ -74,6 +74,9 @@ struct AttnParams {
   float skip_log2;  // look-ahead mode: drop a tile every row of which is this far below its
                     // running max (log2 units; +inf: never)
   int adaptive, e4m3, bf16, out_f32;
+  // single-tile kernel: KV planes (b * Hkv + kvh) per chunk of the CTA order (a divisor of
+  // B * Hkv); the CTAs of one chunk run before the next chunk's, longest query tile first
+  int chunk_kv;
   uint64_t wait_ns;
   // Debug capture (lamp_attn_debug only; unused elsewhere): slot map [B][H][nQT][nKT] (slot of
   // a routing tile, < 0 = not captured), and the raw score tiles [slots][BM][BN]: the 8-bit
@@ -198,16 +201,25 @@ __device__ __forceinline__ void visible_range(const AttnParams& p, int Lq, int L
   lo = (p.window > 0) ? max(0, i + off - p.window + 1) : 0;
 }
 
+// CTA order: the KV planes are taken in chunks of p.chunk_kv, so that the K / V tiles of the
+// CTAs in flight stay resident in L2 while Q and O stream through it; within a chunk, the
+// longest query tiles go first (causal), all query heads of the chunk's KV planes side by side.
 template <class C>
 __device__ __forceinline__ Geo make_geo(const AttnParams& p) {
   Geo g;
-  const int BH = p.B * p.H;
+  const int G = p.H / p.Hkv;
+  const int per_ct = p.chunk_kv * G;         // CTAs of one chunk at one query tile
+  const int per_chunk = per_ct * p.n_ct;
   const int idx = blockIdx.x;
-  g.ct = p.n_ct - 1 - idx / BH;  // longest-first for causal workloads
-  const int bh = idx - (idx / BH) * BH;
-  g.b = bh / p.H;
-  g.h = bh - g.b * p.H;
-  g.kvh = g.h / (p.H / p.Hkv);
+  const int chunk = idx / per_chunk;
+  int rem = idx - chunk * per_chunk;
+  const int ctr = rem / per_ct;
+  rem -= ctr * per_ct;
+  g.ct = p.n_ct - 1 - ctr;                   // longest-first for causal workloads
+  const int kvp = chunk * p.chunk_kv + rem / G;  // KV plane b * Hkv + kvh
+  g.b = kvp / p.Hkv;
+  g.kvh = kvp - g.b * p.Hkv;
+  g.h = g.kvh * G + (rem - (rem / G) * G);
   g.q0 = g.ct * C::MT;
   g.s = seq_rows(p, g.b, g.h, g.kvh);
   const int nh = C::STACK ? 2 : 1;
@@ -555,30 +567,7 @@ __device__ __forceinline__ void dbg_dump(const AttnParams& p, uint32_t* base, in
     st_global_v4(dst + c, make_uint4(raw[c], raw[c + 1], raw[c + 2], raw[c + 3]));
 }
 
-// Packed f32x2 helpers and the mixed-precision adds of the softmax.
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
+// (packed f32x2 helpers: ptx.cuh)
 // 2^x for a pair on the FMA and ALU pipes instead of the MUFU: 2^x = 2^n * 2^f with n = rint(x)
 // (magic-number rounding) and f = x - n in [-1/2, 1/2], 2^f from a degree-3 polynomial fitted
 // to it for least relative error on that interval (max 7.7e-5, below the 16-bit rounding of

@@ -246,7 +246,8 @@ __device__ __forceinline__ bool group_b16(const AttnParams& p, const MaskRow& m,
 }
 // As above, with the mask row of query tile x read from shared memory (it costs the issuing
 // warps no registers).
-__device__ __forceinline__ bool group_b16(const AttnParams& p, const PPBars& bars, int slot, int x,
+template <class BarsT>
+__device__ __forceinline__ bool group_b16(const AttnParams& p, const BarsT& bars, int slot, int x,
                                           int gi) {
   if (p.adaptive) return false;
   const uint64_t w = bars.mask[slot][x][(gi >> 6) & 1];
@@ -258,7 +259,8 @@ struct PPPlan {
   bool live0, live1, b16_0, b16_1, need8, need16;
 };
 
-__device__ __forceinline__ PPPlan pp_plan(const AttnParams& p, const PPGeo& g, const PPBars& bars,
+template <class BarsT>
+__device__ __forceinline__ PPPlan pp_plan(const AttnParams& p, const PPGeo& g, const BarsT& bars,
                                           int slot, const KtCursor& c) {
   PPPlan pl;
   pl.live0 = tile_live(g, p, 0, c.kt);
@@ -280,8 +282,8 @@ __device__ __forceinline__ PPPlan pp_plan(const AttnParams& p, const PPGeo& g, c
 // item's QK^T MMAs have completed) and the item's routing mask rows, then every key tile's K8,
 // K16 and V in the MMA warp's order of first use within each ring.  The rings run on across
 // items.
-template <bool VARLEN>
-__device__ void pp_producer(const AttnParams& p, uint8_t* smem, PPBars& bars, const WaitCtx wc) {
+template <bool VARLEN, class BarsT>
+__device__ void pp_producer(const AttnParams& p, uint8_t* smem, BarsT& bars, const WaitCtx wc) {
   using C = PPCfg;
   prefetch_tmap(&p.tm_q16);
   prefetch_tmap(&p.tm_k16);

@@ -7,11 +7,17 @@
 //                                                     dequantised key: no 16-bit key is cached),
 // values v = v8 * sv, softmax and P.V in fp32.
 //
-// The work is memory-bound (one pass over the cache), so it runs on the CUDA cores with the
-// cache split across CTAs: CTA (chunk, b * Hkv + kvh) reads CHUNK keys of one KV head once for
-// all G query heads of its group, and writes a partial (m, l, O) per head; a second kernel
-// merges the partials of each (b, h).  The chunk's key and value rows are loaded cooperatively
-// (coalesced) into XOR-swizzled shared memory; each thread then reads its own key row.
+// The work is memory-bound (one pass over the cache), so it runs on the CUDA cores.  CTA
+// (split, b * Hkv + kvh) serves all G query heads of one KV head from one read of its cache and
+// walks a run of DEC_SPLIT_CHUNKS chunks of DEC_CHUNK keys: the chunks stream through a ring of
+// shared-memory stages filled by bulk asynchronous copies (one thread issues them, an mbarrier
+// per stage counts the bytes), so the next chunks' loads overlap the current chunk's
+// arithmetic.  An online softmax per head runs across the CTA's chunks; the CTA writes one
+// partial (m, l, O) per head and a second kernel merges the partials of each (b, h).
+// Per chunk: scores with one thread per key (the key row read from shared memory in a rotated
+// 16-byte order, free of bank conflicts), the chunk's softmax update with one warp per head, and
+// P.V with the warps over keys and the lanes over channels, so that each value code is
+// converted once for all heads of the group.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -22,9 +28,12 @@
 
 namespace lamp {
 
-constexpr int DEC_THREADS = 256;
-constexpr int DEC_CHUNK = 256;  // keys per CTA (one per thread in the score phase)
-constexpr int DEC_MAX_G = 8;    // query heads per KV head
+// threads of the split kernel: 8 warps, 16 at D = 256 (whose CTA is alone on its SM)
+__host__ __device__ constexpr int dec_threads(int D) { return D == 256 ? 512 : 256; }
+constexpr int DEC_CHUNK = 128;        // keys per pipeline stage
+constexpr int DEC_STAGES = 2;         // stages of the shared-memory ring
+constexpr int DEC_SPLIT_CHUNKS = 8;   // chunks per CTA (the split of the cache)
+constexpr int DEC_MAX_G = 8;          // query heads per KV head
 
 struct DecodeParams {
   const uint16_t* q;      // [B][H][D] 16-bit
@@ -42,6 +51,7 @@ struct DecodeParams {
   int B, H, Hkv, G, max_k, nkt, bn, nsplit, mask_words, group_tiles;
   float scale;            // natural-log units
   int e4m3, bf16;
+  uint32_t wait_us;       // limit of one bounded wait
 };
 
 __device__ __forceinline__ float dec_h16(uint16_t bits, bool bf16) {
@@ -58,212 +68,370 @@ __device__ __forceinline__ float dec_e4m3(uint32_t c) {
   return (c & 0x80u) ? -mag : mag;
 }
 
+// Two codes (bits 0-7 and 8-15 of c) -> two floats: E4M3 through the hardware conversion to a
+// half pair (exact: every E4M3 value is an fp16 value), INT8 by sign-extending conversions.
+template <bool E4M3>
+__device__ __forceinline__ float2 dec_pair(uint32_t c) {
+  if (E4M3) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 lo;\n\tcvt.u16.u32 lo, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}"
+        : "=r"(h2) : "r"(c & 0xFFFFu));
+    return __half22float2(*reinterpret_cast<__half2*>(&h2));
+  }
+  return make_float2(static_cast<float>(static_cast<int8_t>(c & 0xFFu)),
+                     static_cast<float>(static_cast<int8_t>((c >> 8) & 0xFFu)));
+}
+
 template <bool E4M3>
 __device__ __forceinline__ float dec_code(uint32_t c) {
   return E4M3 ? dec_e4m3(c) : static_cast<float>(static_cast<int8_t>(c));
 }
 
-template <int D, bool E4M3>
-__global__ void __launch_bounds__(DEC_THREADS, 2) decode_split_kernel(const DecodeParams p) {
+// Shared-memory plan of the split kernel (bytes): the ring of key and value stages, then the
+// query of every head (codes and values), scores, the scaled probabilities and the stage
+// barriers.  At the end of the split the ring holds the cross-warp reduction of O.
+template <int D>
+struct DecSmem {
+  static constexpr int STAGE = DEC_CHUNK * D;                         // one chunk of codes
+  static constexpr int OFF_K = 0;                                     // + stage * STAGE
+  static constexpr int OFF_V = DEC_STAGES * STAGE;                    // + stage * STAGE
+  static constexpr int OFF_Q8 = 2 * DEC_STAGES * STAGE;               // [G][D] codes
+  static constexpr int OFF_QF = OFF_Q8 + DEC_MAX_G * D;               // [G][D] fp32
+  static constexpr int OFF_QE = OFF_QF + DEC_MAX_G * D * 4;           // [G][D] decoded E4M3 codes
+  static constexpr int OFF_S = OFF_QE + DEC_MAX_G * D * 4;            // [G][CHUNK] fp32
+  static constexpr int OFF_P = OFF_S + DEC_MAX_G * DEC_CHUNK * 4;     // [G][CHUNK] (p, p) pairs
+  static constexpr int OFF_A = OFF_P + DEC_CHUNK * DEC_MAX_G * 8;     // [G] rescale factors
+  static constexpr int OFF_ML = OFF_A + DEC_MAX_G * 4;                // [G][2] running m, l
+  static constexpr int OFF_BAR = (OFF_ML + DEC_MAX_G * 8 + 7) & ~7;   // [STAGES] mbarriers
+  static constexpr int BYTES = OFF_BAR + DEC_STAGES * 8;
+  static_assert((dec_threads(D) / 32) * DEC_MAX_G * D * 4 <= 2 * DEC_STAGES * STAGE,
+                "O reduction fits the ring");
+  static_assert(STAGE % 16 == 0 && OFF_Q8 % 16 == 0 && OFF_QF % 16 == 0, "alignment");
+};
+
+// GM: the group size rounded up to a power of two (1, 2, 4 or 8), the compile-time bound of
+// every per-head loop (the heads past G are skipped at run time)
+template <int D, bool E4M3, int GM>
+__global__ void __launch_bounds__(dec_threads(D)) decode_split_kernel(const DecodeParams p) {
   static_assert(D == 64 || D == 128 || D == 256, "head dimension");
-  constexpr int NW = DEC_THREADS / 32;
-  constexpr int DL = D / 32;  // channels per lane in the P.V phase
-  extern __shared__ __align__(16) float dsm[];
-  float* sc = dsm;                                    // [G][CHUNK] scores, then probabilities
-  float* qf = sc + DEC_MAX_G * DEC_CHUNK;             // [G][D] query values
-  uint32_t* q8w = reinterpret_cast<uint32_t*>(qf + DEC_MAX_G * D);  // [G][D/4] query codes
-  float* red = reinterpret_cast<float*>(q8w + DEC_MAX_G * D / 4);   // [NW][G][D] P.V partials
-  float* stat = red + NW * DEC_MAX_G * D;             // [G][2] chunk max and sum
-  // [CHUNK][D] value codes; 16-byte chunk c of row j sits at chunk c ^ (j & SW): the row stores
-  // of consecutive threads and the row reads of a warp are both free of bank conflicts
-  uint8_t* vsm = reinterpret_cast<uint8_t*>(stat + 2 * DEC_MAX_G);
-  uint8_t* ksm = vsm + DEC_CHUNK * D;  // [CHUNK][D] key codes, same swizzle
-  constexpr int SW = (D / 16 >= 8) ? 7 : (D / 16 - 1);
+  static_assert(GM == 1 || GM == 2 || GM == 4 || GM == 8, "group bound");
+  constexpr int NT = dec_threads(D);
+  constexpr int NHG = NT / DEC_CHUNK;           // head groups of the score phase
+  constexpr int GH = (GM + NHG - 1) / NHG;      // heads per thread in the score phase
+  using S = DecSmem<D>;
+  constexpr int NW = NT / 32;
+  constexpr int CPL = D / 32;            // channels per lane in the P.V phase
+  constexpr int KPW = DEC_CHUNK / NW;    // keys per warp in the P.V phase
+  constexpr int CPR = D / 16;            // 16-byte pieces per code row
+  extern __shared__ __align__(16) uint8_t dsm[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(dsm + S::OFF_BAR);
+  float* sc = reinterpret_cast<float*>(dsm + S::OFF_S);
+  float2* pw = reinterpret_cast<float2*>(dsm + S::OFF_P);
+  float* al = reinterpret_cast<float*>(dsm + S::OFF_A);
+  float* ml = reinterpret_cast<float*>(dsm + S::OFF_ML);
+  const float* qf = reinterpret_cast<const float*>(dsm + S::OFF_QF);
+  const float* qe = reinterpret_cast<const float*>(dsm + S::OFF_QE);
+  const uint32_t* q8w = reinterpret_cast<const uint32_t*>(dsm + S::OFF_Q8);
 
   const int G = p.G;
   const int split = blockIdx.x, bkv = blockIdx.y;
   const int b = bkv / p.Hkv, kvh = bkv - b * p.Hkv;
   const int len = p.len_k ? min(max(__ldg(p.len_k + b), 0), p.max_k) : p.max_k;
-  const int c0 = split * DEC_CHUNK;
+  const int nchunk = (len + DEC_CHUNK - 1) / DEC_CHUNK;
+  const int cbeg = split * DEC_SPLIT_CHUNKS;
+  const int cend = min(nchunk, cbeg + DEC_SPLIT_CHUNKS);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool bf16 = p.bf16 != 0;
-  const size_t cache_row0 = static_cast<size_t>(bkv) * p.max_k;  // first row of this KV head
+  const size_t row0 = static_cast<size_t>(bkv) * p.max_k;  // first cache row of this KV head
+  const float NEG_INF = -__int_as_float(0x7f800000);
+  const WaitCtx wc{0u, p.wait_us};
 
-  // the G query rows of this KV group: values and codes
-  for (int i = tid; i < G * D; i += DEC_THREADS) {
+  // stage s holds chunk cbeg + s + k * STAGES; thread 0 issues the copies
+  auto issue = [&](int c) {
+    const int st = (c - cbeg) % DEC_STAGES;
+    const int c0 = c * DEC_CHUNK;
+    const uint32_t rows = static_cast<uint32_t>(min(DEC_CHUNK, p.max_k - c0));
+    const uint32_t bytes = rows * D;
+    mbar_arrive_expect_tx(&full[st], 2u * bytes);
+    bulk_load(smem_u32(dsm + S::OFF_K + st * S::STAGE), p.k8 + (row0 + c0) * D, bytes, &full[st]);
+    bulk_load(smem_u32(dsm + S::OFF_V + st * S::STAGE), p.v8 + (row0 + c0) * D, bytes, &full[st]);
+  };
+  if (tid == 0) {
+    for (int s = 0; s < DEC_STAGES; ++s) mbar_init(&full[s], 1);
+    fence_mbarrier_init();
+    for (int c = cbeg; c < min(cend, cbeg + DEC_STAGES); ++c) issue(c);
+  }
+  // the G query rows of this KV group: values and codes; running max and sum per head
+  for (int i = tid; i < G * D; i += NT) {
     const int g = i / D, d = i - g * D;
     const size_t qi = static_cast<size_t>(b * p.H + kvh * G + g) * D + d;
-    qf[g * D + d] = dec_h16(p.q[qi], bf16);
+    reinterpret_cast<float*>(dsm + S::OFF_QF)[g * D + d] = dec_h16(p.q[qi], bf16);
   }
-  for (int i = tid; i < G * D / 4; i += DEC_THREADS) {
+  for (int i = tid; i < G * D / 4; i += NT) {
     const int g = i / (D / 4), w = i - g * (D / 4);
-    q8w[g * (D / 4) + w] = __ldg(reinterpret_cast<const uint32_t*>(
-        p.q8 + static_cast<size_t>(b * p.H + kvh * G + g) * D) + w);
+    const uint32_t word = __ldg(
+        reinterpret_cast<const uint32_t*>(p.q8 + static_cast<size_t>(b * p.H + kvh * G + g) * D) + w);
+    reinterpret_cast<uint32_t*>(dsm + S::OFF_Q8)[g * (D / 4) + w] = word;
+    if (E4M3) {
+      float* qd = reinterpret_cast<float*>(dsm + S::OFF_QE) + g * D + 4 * w;
+      const float2 a = dec_pair<true>(word), c = dec_pair<true>(word >> 16);
+      qd[0] = a.x; qd[1] = a.y; qd[2] = c.x; qd[3] = c.y;
+    }
   }
+  if (tid < G) {
+    ml[2 * tid] = NEG_INF;
+    ml[2 * tid + 1] = 0.0f;
+  }
+  // the scores of this thread's key: heads g = hh, hh + NHG, ... (hh = tid / 128)
+  const int hh = tid / DEC_CHUNK, jl = tid - hh * DEC_CHUNK;
+  float sqh[GH];
+#pragma unroll
+  for (int k = 0; k < GH; ++k) {
+    const int g = hh + NHG * k;
+    sqh[k] = (g < G) ? __ldg(p.q_scale + b * p.H + kvh * G + g) : 0.0f;
+  }
+  uint64_t acc[GM][CPL / 2];  // O accumulators of this lane's channels, as f32x2 pairs
+#pragma unroll
+  for (int g = 0; g < GM; ++g)
+#pragma unroll
+    for (int e = 0; e < CPL / 2; ++e) acc[g][e] = 0ull;
   __syncthreads();
 
-  // scores: one key per thread, all heads of the group.  The key row stays in registers; the
-  // head loop is not unrolled (the unrolled body of every head overflowed the instruction
-  // cache).
-  {
-    const int j = c0 + tid;
-    const bool live = j < len;
-    const int kt = j / p.bn;
-    const float sk = live ? __ldg(p.k_scale + static_cast<size_t>(bkv) * p.nkt + kt) : 0.0f;
-    const int gi = kt / p.group_tiles;
-    // the chunk's key and value rows, loaded cooperatively (a warp reads whole rows: coalesced)
-    // into swizzled shared memory; each thread then reads its own key row from there
+  bool ok = true;
+  for (int c = cbeg; c < cend; ++c) {
+    const int st = (c - cbeg) % DEC_STAGES;
+    const uint32_t par = static_cast<uint32_t>((c - cbeg) / DEC_STAGES) & 1u;
+    const int c0 = c * DEC_CHUNK;
+    const int rows = min(DEC_CHUNK, len - c0);  // keys of this chunk in the sequence
+    if (!mbar_wait(&full[st], par, wc, W_FULL)) ok = false;
+    const uint8_t* ksm = dsm + S::OFF_K + st * S::STAGE;
+    const uint8_t* vsm = dsm + S::OFF_V + st * S::STAGE;
+
+    // ---- scores
     {
-      constexpr int CPR = D / 16;  // 16-byte chunks per row
-      const int rows = min(DEC_CHUNK, len - c0);
-      const uint4* kbase = reinterpret_cast<const uint4*>(p.k8 + (cache_row0 + c0) * D);
-      const uint4* vbase = reinterpret_cast<const uint4*>(p.v8 + (cache_row0 + c0) * D);
-      uint4 kt_[DEC_CHUNK * CPR / DEC_THREADS], vt_[DEC_CHUNK * CPR / DEC_THREADS];
+      const int j = c0 + jl;
+      const bool live = ok && jl < rows;
+      const int kt = j / p.bn;
+      const float sk = live ? __ldg(p.k_scale + static_cast<size_t>(bkv) * p.nkt + kt) : 0.0f;
+      const int gi = kt / p.group_tiles;
+      // routing word of each of this thread's heads (loaded ahead of the dot products)
+      uint64_t mw[GH];
 #pragma unroll
-      for (int u = 0; u < DEC_CHUNK * CPR / DEC_THREADS; ++u) {
-        const int idx = u * DEC_THREADS + tid, r = idx / CPR;
-        if (r < rows) {
-          kt_[u] = __ldg(kbase + idx);
-          vt_[u] = __ldg(vbase + idx);
+      for (int k = 0; k < GH; ++k) {
+        const int g = hh + NHG * k;
+        mw[k] = ~0ull;
+        if (live && p.mask && g < G)
+          mw[k] = __ldg(reinterpret_cast<const unsigned long long*>(p.mask) +
+                        static_cast<size_t>(b * p.H + kvh * G + g) * p.mask_words + (gi >> 6));
+      }
+      // heads scored from the INT8 codes (dp4a) and heads scored in floats: the 16-bit route
+      // (full-precision query, dequantised key) and the E4M3 8-bit route (decoded codes)
+      bool eight[GH];
+      bool any_float = false;
+#pragma unroll
+      for (int k = 0; k < GH; ++k) {
+        eight[k] = ((mw[k] >> (gi & 63)) & 1ull) != 0;
+        any_float = any_float || ((hh + NHG * k) < G && (E4M3 || !eight[k]));
+      }
+      int ia[GH];
+      uint64_t fa[GH];  // float-path dot products as f32x2 partial sums (even, odd channels)
+#pragma unroll
+      for (int k = 0; k < GH; ++k) {
+        ia[k] = 0;
+        fa[k] = 0ull;
+      }
+      if (live) {
+        // the key row's 16-byte pieces are read in a rotated order (piece (i + jl) % CPR at step
+        // i) so that a warp's lanes hit distinct banks, and the query at the matching channels
+        const uint4* krow = reinterpret_cast<const uint4*>(ksm + jl * D);
+        // float heads (16-bit route, E4M3 codes): piece i converted once for all of them
+        auto float_piece = [&](int i, const uint4& kq) {
+          const int ci = (i + jl) & (CPR - 1);
+          uint64_t kf[8];  // the piece's 16 codes as f32x2 pairs
+          const uint32_t ka[4] = {kq.x, kq.y, kq.z, kq.w};
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const float2 f0 = dec_pair<E4M3>(ka[w]), f1 = dec_pair<E4M3>(ka[w] >> 16);
+            kf[2 * w] = f2_pack(f0.x, f0.y);
+            kf[2 * w + 1] = f2_pack(f1.x, f1.y);
+          }
+#pragma unroll
+          for (int k = 0; k < GH; ++k) {
+            const int g = hh + NHG * k;
+            if (g >= G) break;
+            if (!E4M3 && eight[k]) continue;
+            const ulonglong2* q4 =
+                reinterpret_cast<const ulonglong2*>((eight[k] ? qe : qf) + g * D + 16 * ci);
+            uint64_t f = fa[k];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const ulonglong2 qq = q4[w];
+              f = f2_fma(qq.x, kf[2 * w], f);
+              f = f2_fma(qq.y, kf[2 * w + 1], f);
+            }
+            fa[k] = f;
+          }
+        };
+        // INT8 heads: four dp4a per piece
+        auto int_piece = [&](int i, const uint4& kq, int k, int g) {
+          const uint4 qq = reinterpret_cast<const uint4*>(q8w + g * (D / 4))[(i + jl) & (CPR - 1)];
+          ia[k] = __dp4a(static_cast<int>(qq.x), static_cast<int>(kq.x), ia[k]);
+          ia[k] = __dp4a(static_cast<int>(qq.y), static_cast<int>(kq.y), ia[k]);
+          ia[k] = __dp4a(static_cast<int>(qq.z), static_cast<int>(kq.z), ia[k]);
+          ia[k] = __dp4a(static_cast<int>(qq.w), static_cast<int>(kq.w), ia[k]);
+        };
+        if constexpr (D <= 128) {
+          // the whole row in registers; the dp4a chains of each head fully unrolled
+          uint4 kr[CPR];
+#pragma unroll
+          for (int i = 0; i < CPR; ++i) kr[i] = krow[(i + jl) & (CPR - 1)];
+          if (!E4M3) {
+#pragma unroll
+            for (int k = 0; k < GH; ++k) {
+              const int g = hh + NHG * k;
+              if (g >= G) break;
+              if (!eight[k]) continue;
+#pragma unroll
+              for (int i = 0; i < CPR; ++i) int_piece(i, kr[i], k, g);
+            }
+          }
+          if (any_float) {
+#pragma unroll
+            for (int i = 0; i < CPR; ++i) float_piece(i, kr[i]);
+          }
+        } else {
+          // D = 256: piece by piece (the row would not fit the register budget of 512 threads)
+#pragma unroll 2
+          for (int i = 0; i < CPR; ++i) {
+            const uint4 kq = krow[(i + jl) & (CPR - 1)];
+            if (!E4M3) {
+#pragma unroll
+              for (int k = 0; k < GH; ++k) {
+                const int g = hh + NHG * k;
+                if (g >= G) break;
+                if (eight[k]) int_piece(i, kq, k, g);
+              }
+            }
+            if (any_float) float_piece(i, kq);
+          }
         }
       }
 #pragma unroll
-      for (int u = 0; u < DEC_CHUNK * CPR / DEC_THREADS; ++u) {
-        const int idx = u * DEC_THREADS + tid, r = idx / CPR, c = idx - r * CPR;
-        if (r < rows) {
-          reinterpret_cast<uint4*>(ksm + r * D)[c ^ (r & SW)] = kt_[u];
-          reinterpret_cast<uint4*>(vsm + r * D)[c ^ (r & SW)] = vt_[u];
+      for (int k = 0; k < GH; ++k) {
+        const int g = hh + NHG * k;
+        if (g >= G) break;
+        float s = NEG_INF;
+        if (live) {
+          float f0, f1;
+          f2_unpack(fa[k], f0, f1);
+          if (eight[k])
+            s = (E4M3 ? f0 + f1 : static_cast<float>(ia[k])) * sqh[k] * sk * p.scale;
+          else
+            s = (f0 + f1) * sk * p.scale;
         }
+        sc[g * DEC_CHUNK + jl] = s;
       }
     }
     __syncthreads();
-    uint32_t kw[D / 4];
-    if (live) {
+
+    // ---- softmax update, warp g for head g: chunk max, rescale factor, p * v_scale
+    if (warp < G) {
+      const int g = warp;
+      // value scales of the chunk's key blocks (a chunk spans one block of 128 keys or two of
+      // 64), read before the reduction so that their latency overlaps it
+      const int kt0 = c0 / p.bn;
+      const float vs0 = __ldg(p.v_scale + static_cast<size_t>(bkv) * p.nkt + kt0);
+      const float vs1 = (p.bn < DEC_CHUNK && kt0 + 1 < p.nkt)
+                            ? __ldg(p.v_scale + static_cast<size_t>(bkv) * p.nkt + kt0 + 1) : 0.0f;
+      float m = ml[2 * g], l = ml[2 * g + 1];
+      float sv[DEC_CHUNK / 32];
+      float cm = NEG_INF;
 #pragma unroll
-      for (int i = 0; i < D / 16; ++i) {
-        const uint4 kr = reinterpret_cast<const uint4*>(ksm + tid * D)[i ^ (tid & SW)];
-        kw[4 * i] = kr.x;
-        kw[4 * i + 1] = kr.y;
-        kw[4 * i + 2] = kr.z;
-        kw[4 * i + 3] = kr.w;
+      for (int k = 0; k < DEC_CHUNK / 32; ++k) {
+        sv[k] = sc[g * DEC_CHUNK + k * 32 + lane];
+        cm = fmaxf(cm, sv[k]);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, o));
+      const float mn = fmaxf(m, cm);
+      const float a = (m == NEG_INF) ? 0.0f : __expf(m - mn);
+      float ls = 0.0f;
+#pragma unroll
+      for (int k = 0; k < DEC_CHUNK / 32; ++k) {
+        const int jj = k * 32 + lane;
+        const float pr = (sv[k] == NEG_INF) ? 0.0f : __expf(sv[k] - mn);
+        ls += pr;
+        const float pv = pr * ((jj < p.bn) ? vs0 : vs1);
+        pw[g * DEC_CHUNK + jj] = make_float2(pv, pv);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xFFFFFFFFu, ls, o);
+      if (lane == 0) {
+        al[g] = a;
+        ml[2 * g] = mn;
+        ml[2 * g + 1] = l * a + ls;
       }
     }
-#pragma unroll 1
-    for (int g = 0; g < G; ++g) {
-      float s = -__int_as_float(0x7f800000);
-      if (live) {
-        const int h = kvh * G + g;
-        bool eight = true;
-        if (p.mask) {
-          const uint64_t w = __ldg(reinterpret_cast<const unsigned long long*>(p.mask) +
-                                   static_cast<size_t>(b * p.H + h) * p.mask_words + (gi >> 6));
-          eight = ((w >> (gi & 63)) & 1ull) != 0;
-        }
-        if (eight) {
-          const uint32_t* qw = q8w + g * (D / 4);
-          const float sq = __ldg(p.q_scale + b * p.H + h);
-          if (!E4M3) {
-            int acc = 0;
+    __syncthreads();
+
+    // ---- P.V: warp w takes keys w * KPW .. + KPW of the chunk, lane l channels l * CPL ..
+    // (f32x2 FMAs: each weight is stored as a (p, p) pair, the channels go in pairs)
+    {
 #pragma unroll
-            for (int i = 0; i < D / 4; ++i) acc = __dp4a(static_cast<int>(qw[i]), static_cast<int>(kw[i]), acc);
-            s = static_cast<float>(acc) * sq * sk * p.scale;
-          } else {
-            float acc = 0.0f;
+      for (int g = 0; g < GM; ++g) {
+        if (g >= G) break;
+        const uint64_t a2 = f2_pack(al[g], al[g]);
 #pragma unroll
-            for (int i = 0; i < D / 4; ++i)
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                acc = fmaf(dec_e4m3((qw[i] >> (8 * e)) & 0xFFu), dec_e4m3((kw[i] >> (8 * e)) & 0xFFu), acc);
-            s = acc * sq * sk * p.scale;
-          }
+        for (int e = 0; e < CPL / 2; ++e) acc[g][e] = f2_fma(acc[g][e], a2, 0ull);
+      }
+      const int jb = warp * KPW, je = min(jb + KPW, rows);
+      for (int jj = jb; jj < je; ++jj) {
+        const uint8_t* vrow = vsm + jj * D + lane * CPL;
+        uint32_t vw[(CPL + 3) / 4];
+        if (CPL == 8) {
+          const uint2 t = *reinterpret_cast<const uint2*>(vrow);
+          vw[0] = t.x;
+          vw[1] = t.y;
+        } else if (CPL == 4) {
+          vw[0] = *reinterpret_cast<const uint32_t*>(vrow);
         } else {
-          const float* qv = qf + g * D;
-          float acc = 0.0f;
+          vw[0] = *reinterpret_cast<const uint16_t*>(vrow);
+        }
+        uint64_t vv[CPL / 2];
 #pragma unroll
-          for (int i = 0; i < D / 4; ++i)
+        for (int e = 0; e < CPL; e += 2) {
+          const float2 f = dec_pair<E4M3>(vw[e >> 2] >> (8 * (e & 3)));
+          vv[e / 2] = f2_pack(f.x, f.y);
+        }
+        const uint64_t* pcol = reinterpret_cast<const uint64_t*>(pw + jj);
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              acc = fmaf(qv[4 * i + e], dec_code<E4M3>((kw[i] >> (8 * e)) & 0xFFu), acc);
-          s = acc * sk * p.scale;
+        for (int g = 0; g < GM; ++g) {
+          if (g >= G) break;
+          const uint64_t pg = pcol[g * DEC_CHUNK];  // (the whole warp reads one address)
+#pragma unroll
+          for (int e = 0; e < CPL / 2; ++e) acc[g][e] = f2_fma(pg, vv[e], acc[g][e]);
         }
       }
-      sc[g * DEC_CHUNK + tid] = s;
     }
+    __syncthreads();  // every thread is done with this stage and with the scores / weights
+    if (tid == 0 && c + DEC_STAGES < cend) issue(c + DEC_STAGES);
   }
-  __syncthreads();
 
-  // per head: chunk max, probabilities p = e^(s - m), their sum (warp g takes head g)
-  for (int g = warp; g < G; g += NW) {
-    float m = -__int_as_float(0x7f800000);
-    for (int i = lane; i < DEC_CHUNK; i += 32) m = fmaxf(m, sc[g * DEC_CHUNK + i]);
+  // ---- the partial of each head: m, l and O summed over the warps (in the ring's space)
+  float* red = reinterpret_cast<float*>(dsm);  // [NW][G][D]
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    float l = 0.0f;
-    for (int i = lane; i < DEC_CHUNK; i += 32) {
-      const float s = sc[g * DEC_CHUNK + i];
-      const float pr = (s == -__int_as_float(0x7f800000)) ? 0.0f : __expf(s - m);
-      sc[g * DEC_CHUNK + i] = pr;
-      l += pr;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, o);
-    if (lane == 0) {
-      stat[2 * g] = m;
-      stat[2 * g + 1] = l;
-    }
-  }
-  __syncthreads();
-
-  // P.V: warp w takes keys w, w + NW, ...; lane l holds channels [l * DL, l * DL + DL)
-  float acc[DEC_MAX_G][DL];
-#pragma unroll
-  for (int g = 0; g < DEC_MAX_G; ++g)
-#pragma unroll
-    for (int e = 0; e < DL; ++e) acc[g][e] = 0.0f;
-  const int jend = min(DEC_CHUNK, len - c0);
-  float vsc[DEC_CHUNK / 64];  // value scales of the chunk's key tiles (BN >= 64)
-#pragma unroll
-  for (int i = 0; i < DEC_CHUNK / 64; ++i) {
-    const int kt = c0 / p.bn + i;
-    vsc[i] = (kt < p.nkt) ? __ldg(p.v_scale + static_cast<size_t>(bkv) * p.nkt + kt) : 0.0f;
-  }
-  for (int jj = warp; jj < jend; jj += NW) {
-    const int j = c0 + jj;
-    // lane's DL bytes of row jj: logical chunk (lane * DL) / 16, stored at chunk ^ (jj & SW)
-    const int lc = (lane * DL) >> 4;
-    const uint8_t* vrow = vsm + jj * D + ((lc ^ (jj & SW)) << 4) + ((lane * DL) & 15);
-    uint32_t vw[(DL + 3) / 4];
-    if (DL == 8) {
-      const uint2 t = *reinterpret_cast<const uint2*>(vrow);
-      vw[0] = t.x;
-      vw[1] = t.y;
-    } else if (DL == 4) {
-      vw[0] = *reinterpret_cast<const uint32_t*>(vrow);
-    } else {
-      vw[0] = *reinterpret_cast<const uint16_t*>(vrow);
-    }
-    const float sv = vsc[(j / p.bn) - c0 / p.bn];
-    float vv[DL];
-#pragma unroll
-    for (int e = 0; e < DL; ++e) vv[e] = dec_code<E4M3>((vw[e >> 2] >> (8 * (e & 3))) & 0xFFu) * sv;
-#pragma unroll
-    for (int g = 0; g < DEC_MAX_G; ++g) {
-      if (g >= G) break;
-      const float pr = sc[g * DEC_CHUNK + jj];
-#pragma unroll
-      for (int e = 0; e < DL; ++e) acc[g][e] = fmaf(pr, vv[e], acc[g][e]);
-    }
-  }
-#pragma unroll
-  for (int g = 0; g < DEC_MAX_G; ++g) {
+  for (int g = 0; g < GM; ++g) {
     if (g >= G) break;
 #pragma unroll
-    for (int e = 0; e < DL; ++e) red[(warp * DEC_MAX_G + g) * D + lane * DL + e] = acc[g][e];
+    for (int e = 0; e < CPL / 2; ++e) {
+      float lo, hi;
+      f2_unpack(acc[g][e], lo, hi);
+      red[(warp * DEC_MAX_G + g) * D + lane * CPL + 2 * e] = lo;
+      red[(warp * DEC_MAX_G + g) * D + lane * CPL + 2 * e + 1] = hi;
+    }
   }
   __syncthreads();
-
-  // the partial of each head: m, l, O = sum over the warps
-  for (int i = tid; i < G * D; i += DEC_THREADS) {
+  for (int i = tid; i < G * D; i += NT) {
     const int g = i / D, d = i - g * D;
     float s = 0.0f;
 #pragma unroll
@@ -272,8 +440,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_split_kernel(const Deco
     float* out = p.part + (static_cast<size_t>(b * p.H + h) * p.nsplit + split) * (2 + D);
     out[2 + d] = s;
     if (d == 0) {
-      out[0] = stat[2 * g];
-      out[1] = stat[2 * g + 1];
+      out[0] = ml[2 * g];
+      out[1] = ml[2 * g + 1];
     }
   }
 }

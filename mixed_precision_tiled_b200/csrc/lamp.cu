@@ -460,6 +460,20 @@ int prepare_attn(const void* q, const void* k, const void* v, const void* q8, co
   } else {
     call->kernel = (D == 128) ? K_CFG128 : K_CFG256;
   }
+  // Chunks of KV planes for the single-tile kernel's CTA order: the largest divisor of B * Hkv
+  // whose K16, V and K8 tiles (5 bytes per element) fit in 40 MB of L2.  A sliding window
+  // already keeps the CTAs of one query tile on one band of keys, and a variable-length batch
+  // has its own lengths: one chunk there.
+  const int nkv = BHk;
+  p.chunk_kv = nkv;
+  if (window == 0 && !varlen) {
+    const double plane = 5.0 * static_cast<double>(Lk) * D;
+    for (int d = nkv; d >= 1; --d)
+      if (nkv % d == 0 && (d == 1 || d * plane <= 40e6)) {
+        p.chunk_kv = d;
+        break;
+      }
+  }
   return LAMP_OK;
 }
 
@@ -600,24 +614,20 @@ bool template_sixteen(long long g, long long gd, int sink, int band, int stride)
 }  // namespace
 
 namespace {
-template <int D, bool E4M3>
+template <int D, bool E4M3, int GM>
 int launch_decode_t(const lamp::DecodeParams& p, cudaStream_t st) {
-  constexpr size_t smem = sizeof(float) * (lamp::DEC_MAX_G * lamp::DEC_CHUNK + lamp::DEC_MAX_G * D +
-                                           lamp::DEC_MAX_G * D / 4 +
-                                           (lamp::DEC_THREADS / 32) * lamp::DEC_MAX_G * D +
-                                           2 * lamp::DEC_MAX_G) +
-                        2 * static_cast<size_t>(lamp::DEC_CHUNK) * D;  // value and key rows
+  constexpr int smem = lamp::DecSmem<D>::BYTES;
   static bool attr_set[64] = {};
   int dev = 0;
   LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    LAMP_CUDA(cudaFuncSetAttribute(lamp::decode_split_kernel<D, E4M3>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
+    LAMP_CUDA(cudaFuncSetAttribute(lamp::decode_split_kernel<D, E4M3, GM>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
               "cudaFuncSetAttribute");
     attr_set[dev] = true;
   }
   const dim3 grid(p.nsplit, p.B * p.Hkv);
-  lamp::decode_split_kernel<D, E4M3><<<grid, lamp::DEC_THREADS, smem, st>>>(p);
+  lamp::decode_split_kernel<D, E4M3, GM><<<grid, lamp::dec_threads(D), smem, st>>>(p);
   LAMP_CUDA(cudaGetLastError(), "decode_split_kernel launch");
   lamp::decode_combine_kernel<D><<<p.B * p.H, lamp::DEC_COMBINE_THREADS,
                                    (p.nsplit + 64) * sizeof(float), st>>>(p);
@@ -625,9 +635,18 @@ int launch_decode_t(const lamp::DecodeParams& p, cudaStream_t st) {
   return LAMP_OK;
 }
 
+// per-head loops bounded by the group size rounded up to a power of two
+template <int D, bool E4M3>
+int launch_decode_g(const lamp::DecodeParams& p, cudaStream_t st) {
+  if (p.G <= 1) return launch_decode_t<D, E4M3, 1>(p, st);
+  if (p.G <= 2) return launch_decode_t<D, E4M3, 2>(p, st);
+  if (p.G <= 4) return launch_decode_t<D, E4M3, 4>(p, st);
+  return launch_decode_t<D, E4M3, 8>(p, st);
+}
+
 template <int D>
 int launch_decode(const lamp::DecodeParams& p, cudaStream_t st) {
-  return p.e4m3 ? launch_decode_t<D, true>(p, st) : launch_decode_t<D, false>(p, st);
+  return p.e4m3 ? launch_decode_g<D, true>(p, st) : launch_decode_g<D, false>(p, st);
 }
 }  // namespace
 
@@ -912,7 +931,9 @@ int lamp_decode_fwd(const void* q, const void* q8, const float* q_scale, const v
   p.B = B; p.H = H; p.Hkv = Hkv; p.G = H / Hkv; p.max_k = max_k;
   p.bn = bn;
   p.nkt = (max_k + bn - 1) / bn;
-  p.nsplit = (max_k + lamp::DEC_CHUNK - 1) / lamp::DEC_CHUNK;
+  const int nchunk = (max_k + lamp::DEC_CHUNK - 1) / lamp::DEC_CHUNK;
+  p.nsplit = (nchunk + lamp::DEC_SPLIT_CHUNKS - 1) / lamp::DEC_SPLIT_CHUNKS;
+  p.wait_us = kWaitUs;
   p.group_tiles = mask_bits ? group_tiles : 1;
   p.mask_words = ((p.nkt + p.group_tiles - 1) / p.group_tiles + 63) / 64;
   p.scale = (scale > 0.0f) ? scale : 1.0f / std::sqrt(static_cast<float>(D));

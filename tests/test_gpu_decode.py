@@ -30,6 +30,10 @@ def dequant(codes, scales, bn, fmt):
     (64, 4, 2, [300, 0, 129], "e4m3", None, 1),
     (256, 8, 4, [700, 1024], "int8", 0.5, 2),
     (128, 32, 8, [4096], "e4m3", 0.2, 4),
+    # long caches: many 128-key chunks and several splits of 8 chunks per CTA, ragged ends
+    (128, 32, 8, [20000, 9001], "int8", 0.25, 8),
+    (64, 8, 1, [3000, 1025], "e4m3", 0.5, 1),
+    (256, 16, 2, [5000], "int8", 0.3, 2),
 ])
 def test_decode_matches_oracle(D, H, Hkv, lens, fmt, p16, g):
     B, max_k = len(lens), max(lens)
