@@ -294,7 +294,10 @@ int lamp_set_workspace(void* ptr, size_t bytes);
 
 /* Synchronises `stream`, then reports and clears the device-side error word: LAMP_OK, or
  * LAMP_ERR_TIMEOUT when a kernel's bounded wait gave up since the last check (the kernel
- * then stopped early and its outputs are undefined), or LAMP_ERR_CUDA. */
+ * then stopped early and its outputs are undefined), or LAMP_ERR_CUDA.  After a timeout it
+ * also synchronises the device and returns the attention kernel's work-item counters to
+ * idle (a launch that gave up may have left one held), so call it while no other call of
+ * the library is running on the device. */
 int lamp_check(void* stream);
 
 /* Launches a one-block kernel that waits, with a limit of `wait_ns` nanoseconds, on a

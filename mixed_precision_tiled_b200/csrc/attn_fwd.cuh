@@ -47,7 +47,8 @@ namespace lamp {
 // where-codes recorded with a timeout (bits 8..15 of the error word)
 enum : uint32_t {
   W_QFULL = 1, W_EMPTY = 2, W_FULL = 3, W_SFULL = 4, W_S16 = 5, W_VOTE = 6, W_PFULL = 7,
-  W_ODONE = 8, W_DRAIN = 9, W_SELFTEST = 10, W_XCH = 11, W_ZFREE = 12, W_OSTAGE = 13
+  W_ODONE = 8, W_DRAIN = 9, W_SELFTEST = 10, W_XCH = 11, W_ZFREE = 12, W_OSTAGE = 13,
+  W_ITEM = 14, W_CLAIM = 15
 };
 
 struct AttnParams {
@@ -74,9 +75,12 @@ struct AttnParams {
   float skip_log2;  // look-ahead mode: drop a tile every row of which is this far below its
                     // running max (log2 units; +inf: never)
   int adaptive, e4m3, bf16, out_f32;
-  // single-tile kernel: KV planes (b * Hkv + kvh) per chunk of the CTA order (a divisor of
-  // B * Hkv); the CTAs of one chunk run before the next chunk's, longest query tile first
+  // KV planes (b * Hkv + kvh) per chunk of the CTA / work-item order (a divisor of B * Hkv):
+  // the work of one chunk runs before the next chunk's, longest query tiles first
   int chunk_kv;
+  // two-tile kernel: its scheduler slot (work-item ticket counter) and the launch's nonzero tag
+  unsigned long long* sched;
+  uint32_t sched_tag;
   uint64_t wait_ns;
   // Debug capture (lamp_attn_debug only; unused elsewhere): slot map [B][H][nQT][nKT] (slot of
   // a routing tile, < 0 = not captured), and the raw score tiles [slots][BM][BN]: the 8-bit

@@ -6,7 +6,9 @@
 // score tiles chosen per tile, one shared online softmax; LampAttention abstract: 8-bit
 // products, look-ahead recomputation of sensitive tiles in 16 bits), organised for B200 so
 // that the tensor core works on one query tile while the softmax works on the other:
-//   * persistent CTAs (one per SM) walk a list of work items, longest first, in a snake order;
+//   * persistent CTAs (one per SM) walk the work items longest first, in a fixed snake
+//     order, or (when the KV planes exceed L2) take them from a launch-wide ticket counter in
+//     an order that keeps the K/V planes in flight within L2;
 //     an item is two 128-row query tiles X = 0, 1 that read the same K/V: the same query tile
 //     of two heads of one KV group (grouped-query attention with an even group), otherwise two
 //     query tiles of one head.  Each key tile is streamed through shared memory once for both:
@@ -78,6 +80,9 @@ struct PPBars {
   uint64_t o_done[2];
   uint64_t o_free[2];  // the epilogue has read O of query tile X: the next item may overwrite it
   uint64_t drain;
+  uint64_t item_full[2];   // the producer has published work item r in slot r & 1
+  uint64_t item_empty[2];  // the MMA warp and the 8 softmax warps have read it
+  int item[2];             // item index, -1: no item left (or the claim of the counter failed)
   uint32_t tmem_base;
   uint32_t abort;
   uint32_t votes[2][4];
@@ -107,21 +112,80 @@ __device__ __forceinline__ long long pp_n_items(const AttnParams& p) {
                           : static_cast<long long>(p.B) * p.H * ((p.nqt + 1) / 2);
 }
 
-// Persistent CTAs: round r gives CTA c the item r * G + c (r even) or r * G + G - 1 - c (r odd),
-// a snake that keeps the CTAs' total work close.  -1: no item left.
-__device__ __forceinline__ int pp_item(const AttnParams& p, int r) {
+// Work distribution (when the KV planes exceed L2; otherwise the fixed order below): a
+// launch-wide ticket counter in a scheduler slot (one 64-bit word in
+// global memory, 0 when the slot is idle): the launch's tag in the high 32 bits, the next
+// ticket in the low 32 bits.  CTA c runs item c first; ticket t gives item gridDim.x + t, so
+// that tickets go to whichever CTA asks first and the CTAs' work balances itself whatever the
+// items' costs.  Each CTA's producer claims the slot as it starts (idle -> tag, or already
+// holding this launch's tag; a slot still held by another launch is waited for, bounded) and
+// takes tickets until one is past the last item.  Every CTA takes exactly one such ticket, so
+// the CTA that takes ticket n_items - 1 is the last to use the counter: it returns the slot to
+// idle, and the next launch given the same slot (a later call, or a replay of a captured
+// graph) finds it idle.
+constexpr int SCHED_SLOTS = 1024;
+__device__ unsigned long long g_lamp_sched[SCHED_SLOTS];
+
+__device__ __forceinline__ bool sched_owned(const AttnParams& p, unsigned long long prev) {
+  return prev == 0ull || static_cast<uint32_t>(prev >> 32) == p.sched_tag;
+}
+
+__device__ __forceinline__ unsigned long long sched_try_claim(const AttnParams& p) {
+  return atomicCAS(p.sched, 0ull, static_cast<unsigned long long>(p.sched_tag) << 32);
+}
+
+// The slot held by another launch: wait (bounded) until it is idle and claim it.
+__device__ bool sched_claim_wait(const AttnParams& p, const WaitCtx wc) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (sched_owned(p, sched_try_claim(p))) return true;
+    __nanosleep(1000);
+    if ((it & 7u) == 7u) {
+      if (wc.abort && lds_u32(wc.abort)) return false;
+      if (globaltimer_ns() - t0 > static_cast<uint64_t>(wc.limit_us) * 1000ull) {
+        if (wc.abort) sts_u32(wc.abort, 1u);
+        atomicOr(&g_lamp_error, 1u | (W_CLAIM << 8));
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ int sched_ticket(const AttnParams& p) {
+  return static_cast<int>(atomicAdd(p.sched, 1ull) & 0x7FFFFFFFull);
+}
+
+// The fixed order (no ticket counter): round r gives CTA c the item r * G + c (r even) or
+// r * G + G - 1 - c (r odd), a snake that keeps the CTAs' total work close on the
+// longest-first items.  -1: no item left.
+__device__ __forceinline__ int pp_item_fixed(const AttnParams& p, int r) {
   const long long n_items = pp_n_items(p);
   const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
   const long long j = static_cast<long long>(r) * G + ((r & 1) ? G - 1 - c : c);
   return j < n_items ? static_cast<int>(j) : -1;
 }
 
+// With the ticket counter, a consumer warp (all lanes) takes work item r from the producer's
+// two-slot ring: the item's index, -1 when none is left, -2 when the wait gave up.
+__device__ __forceinline__ int pp_take_item(PPBars& bars, int r, const WaitCtx wc) {
+  const int s = r & 1;
+  if (!mbar_wait(&bars.item_full[s], static_cast<uint32_t>(r >> 1) & 1u, wc, W_ITEM)) return -2;
+  const int item = *reinterpret_cast<volatile int*>(&bars.item[s]);
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(&bars.item_empty[s]);
+  return item;
+}
+
 // VARLEN: sequence geometry from the offset arrays (variable-length batches); otherwise the
 // dense layout, with every offset a compile-time zero.
-template <bool VARLEN>
+// Item order: longest first, all heads side by side; with the ticket counter (TK) the KV planes
+// (b * Hkv + kvh) are taken in chunks of p.chunk_kv, so that the K / V tiles the CTAs in flight
+// stream stay in L2 while Q and O pass through it, longest first within a chunk.
+template <bool VARLEN, bool TK>
 __device__ __forceinline__ PPGeo pp_geo(const AttnParams& p, int idx) {
   PPGeo g;
-  if (pp_head_pairs(p)) {
+  const int G = p.H / p.Hkv;
+  if (!TK && pp_head_pairs(p)) {
     const int BH2 = p.B * (p.H / 2);
     const int qt = p.nqt - 1 - idx / BH2;  // longest-first
     const int bhp = idx - (idx / BH2) * BH2;
@@ -132,7 +196,7 @@ __device__ __forceinline__ PPGeo pp_geo(const AttnParams& p, int idx) {
       g.q0[x] = qt * PPCfg::MT;
       g.qt[x] = qt;
     }
-  } else {
+  } else if (!TK) {
     const int BH = p.B * p.H;
     const int n_pairs = (p.nqt + 1) / 2;
     const int pair = n_pairs - 1 - idx / BH;  // longest-first
@@ -140,6 +204,39 @@ __device__ __forceinline__ PPGeo pp_geo(const AttnParams& p, int idx) {
     g.b = bh / p.H;
     for (int x = 0; x < 2; ++x) {
       g.h[x] = bh - g.b * p.H;
+      g.q0[x] = (2 * pair + x) * PPCfg::MT;
+      g.qt[x] = 2 * pair + x;
+    }
+  } else if (pp_head_pairs(p)) {
+    const int per_qt = p.chunk_kv * (G / 2);  // items of one chunk at one query tile
+    const int per_chunk = per_qt * p.nqt;
+    const int chunk = idx / per_chunk;
+    int rem = idx - chunk * per_chunk;
+    const int qr = rem / per_qt;
+    rem -= qr * per_qt;
+    const int qt = p.nqt - 1 - qr;  // longest-first
+    const int kvp = chunk * p.chunk_kv + rem / (G / 2);  // KV plane b * Hkv + kvh
+    g.b = kvp / p.Hkv;
+    const int hp = (kvp - g.b * p.Hkv) * (G / 2) + (rem - (rem / (G / 2)) * (G / 2));
+    for (int x = 0; x < 2; ++x) {
+      g.h[x] = 2 * hp + x;
+      g.q0[x] = qt * PPCfg::MT;
+      g.qt[x] = qt;
+    }
+  } else {
+    const int n_pairs = (p.nqt + 1) / 2;
+    const int per_pr = p.chunk_kv * G;  // items of one chunk at one query-tile pair
+    const int per_chunk = per_pr * n_pairs;
+    const int chunk = idx / per_chunk;
+    int rem = idx - chunk * per_chunk;
+    const int pr = rem / per_pr;
+    rem -= pr * per_pr;
+    const int pair = n_pairs - 1 - pr;  // longest-first
+    const int kvp = chunk * p.chunk_kv + rem / G;
+    g.b = kvp / p.Hkv;
+    const int h = (kvp - g.b * p.Hkv) * G + (rem - (rem / G) * G);
+    for (int x = 0; x < 2; ++x) {
+      g.h[x] = h;
       g.q0[x] = (2 * pair + x) * PPCfg::MT;
       g.qt[x] = 2 * pair + x;
     }
@@ -282,7 +379,7 @@ __device__ __forceinline__ PPPlan pp_plan(const AttnParams& p, const PPGeo& g, c
 // item's QK^T MMAs have completed) and the item's routing mask rows, then every key tile's K8,
 // K16 and V in the MMA warp's order of first use within each ring.  The rings run on across
 // items.
-template <bool VARLEN, class BarsT>
+template <bool VARLEN, bool TK, class BarsT>
 __device__ void pp_producer(const AttnParams& p, uint8_t* smem, BarsT& bars, const WaitCtx wc) {
   using C = PPCfg;
   prefetch_tmap(&p.tm_q16);
@@ -313,12 +410,39 @@ __device__ void pp_producer(const AttnParams& p, uint8_t* smem, BarsT& bars, con
     ++n16;
     return true;
   };
+  const int n_items = static_cast<int>(pp_n_items(p));
+  const int grid = static_cast<int>(gridDim.x);
+  // the claim is issued now and its answer read when the first ticket is taken
+  const unsigned long long claim0 = TK ? sched_try_claim(p) : 0ull;
+  bool claimed = false;
   bool ok = true;
+  int next = static_cast<int>(blockIdx.x);  // the first item (the grid never exceeds the items)
+  auto take_ticket = [&]() {
+    if (!claimed) {
+      ok = claimed = sched_owned(p, claim0) || sched_claim_wait(p, wc);
+      if (!ok) return;
+    }
+    next = grid + sched_ticket(p);
+  };
   int r = 0;
   for (; ok; ++r) {
-    const int item = pp_item(p, r);
+    int item;
+    if constexpr (TK) {
+      // ticket n_items - 1 is the last any CTA takes: return the slot to idle
+      if (next == n_items - 1 + grid) atomicExch(p.sched, 0ull);
+      // publish item r (or the end) to the consumers
+      item = (next < n_items) ? next : -1;
+      const int is = r & 1;
+      if (r >= 2 && !(ok = mbar_wait(&bars.item_empty[is],
+                                     static_cast<uint32_t>((r >> 1) - 1) & 1u, wc, W_ITEM)))
+        break;
+      bars.item[is] = item;
+      mbar_arrive(&bars.item_full[is]);
+    } else {
+      item = pp_item_fixed(p, r);  // every role computes the fixed order itself
+    }
     if (item < 0) break;
-    const PPGeo g = pp_geo<VARLEN>(p, item);
+    const PPGeo g = pp_geo<VARLEN, TK>(p, item);
     pkv = g.kv_plane;
     krow0 = g.k_row0;
     if (!lamp_chk(g.b * p.H + g.h[1] < p.B * p.H && g.b * p.Hkv + g.kvh < p.B * p.Hkv, 3)) {
@@ -341,13 +465,23 @@ __device__ void pp_producer(const AttnParams& p, uint8_t* smem, BarsT& bars, con
                     &bars.q_full, c * 64, row, pq);
       tma_load_3d(smem + C::OFF_Q8 + x * C::Q8_BYTES, &p.tm_q8, &bars.q_full, 0, row, pq);
     }
+    // The next item's ticket is taken before the loads of the item's second-last key tile,
+    // a few key tiles before the CTA is done with the item: late enough that the CTAs which
+    // finish first take the next items, early enough that the round trip is over (behind the
+    // ring waits of the last two tiles) before the next item is published.
+    const int t_ticket = g.n > 2 ? g.n - 2 : 0;
     KtCursor cur = kt_first(p, g.kt_lo);
     for (int t = 0; ok && t < g.n; ++t, kt_next(p, cur)) {
+      if (TK && t == t_ticket) {
+        take_ticket();
+        if (!ok) break;
+      }
       const PPPlan pl = pp_plan(p, g, bars, r & 1, cur);
       if (pl.need8 && !(ok = load8(cur.kt))) break;
       if (pl.need16 && !(ok = load16(&p.tm_k16, cur.kt))) break;
       if (!(ok = load16(&p.tm_v, cur.kt))) break;
     }
+    if (TK && ok && g.n == 0) take_ticket();
   }
   // Drain: every slot's most recent load must have landed before the CTA may exit.
   const WaitCtx drain{0u, 50000u};  // no abort word: in-flight work always completes
@@ -369,7 +503,7 @@ __device__ void pp_producer(const AttnParams& p, uint8_t* smem, BarsT& bars, con
 // only MMAs lie between a P tile's arrival and the next QK^T.  Per work item: wait for its Q,
 // and before the first QK^T of a query tile for the previous item's epilogue to have read O;
 // at the end release Q and publish O.
-template <bool BF16, bool ADAPTIVE, bool VARLEN>
+template <bool BF16, bool ADAPTIVE, bool VARLEN, bool TK>
 __device__ void pp_mma(const AttnParams& p, uint8_t* smem, PPBars& bars, uint32_t tbase,
                        const WaitCtx wc) {
   using C = PPCfg;
@@ -471,9 +605,9 @@ __device__ void pp_mma(const AttnParams& p, uint8_t* smem, PPBars& bars, uint32_
   };
 
   for (int r = 0; ok; ++r) {
-    const int item = pp_item(p, r);
+    const int item = TK ? pp_take_item(bars, r, wc) : pp_item_fixed(p, r);
     if (item < 0) break;
-    const PPGeo g = pp_geo<VARLEN>(p, item);
+    const PPGeo g = pp_geo<VARLEN, TK>(p, item);
     const int ms = r & 1;  // mask slot of this item
     const int ra0 = (g.lo[0] <= g.hi[0]) ? g.lo[0] / C::BN : (1 << 30);
     const int rb0 = (g.lo[0] <= g.hi[0]) ? g.hi[0] / C::BN : -1;
@@ -868,21 +1002,21 @@ __device__ __forceinline__ bool pp_softmax_item(const AttnParams& p, const PPGeo
 }
 
 // The softmax role: the CTA's work items in turn.
-template <bool BF16, bool ADAPTIVE, bool VARLEN, bool DBG>
+template <bool BF16, bool ADAPTIVE, bool VARLEN, bool DBG, bool TK>
 __device__ void pp_softmax(const AttnParams& p, PPBars& bars, uint32_t tbase, const WaitCtx wc) {
   uint32_t cs = 0, c16 = 0, cvv = 0;
   uint32_t raw[PPCfg::BN];
   for (int it = 0;; ++it) {
-    const int item = pp_item(p, it);
+    const int item = TK ? pp_take_item(bars, it, wc) : pp_item_fixed(p, it);
     if (item < 0) break;
-    const PPGeo g = pp_geo<VARLEN>(p, item);
+    const PPGeo g = pp_geo<VARLEN, TK>(p, item);
     if (!pp_softmax_item<BF16, ADAPTIVE, VARLEN, DBG>(p, g, bars, tbase, wc, it, cs, c16, cvv, raw)) break;
   }
 }
 
 // ------------------------------------------------------------------ kernel ------------
 
-template <bool BF16, bool ADAPTIVE, bool VARLEN, bool DBG>
+template <bool BF16, bool ADAPTIVE, bool VARLEN, bool DBG, bool TK>
 __global__ void __launch_bounds__(PPCfg::THREADS, 1)
     attn_fwd_pp_kernel(const __grid_constant__ AttnParams p) {
   using C = PPCfg;
@@ -914,6 +1048,10 @@ __global__ void __launch_bounds__(PPCfg::THREADS, 1)
       mbar_init(&bars.o_free[x], 4);
     }
     mbar_init(&bars.drain, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.item_full[i], 1);
+      mbar_init(&bars.item_empty[i], 9);  // the MMA warp and the 8 softmax warps
+    }
     bars.abort = 0;
     fence_mbarrier_init();
   }
@@ -929,17 +1067,17 @@ __global__ void __launch_bounds__(PPCfg::THREADS, 1)
   // Register split within the launch allotment of 384 x 168: the control warpgroup gives
   // back to 104 per thread, the two softmax warpgroups grow to 200
   // (128 * 104 + 256 * 200 = 64512 = 384 * 168).
-  // Every role walks the same sequence of work items (pp_item) and derives each item's geometry
-  // itself.
+  // Every role derives each item's geometry itself; with the ticket counter the producer
+  // takes the tickets and publishes each item to the other roles.
   if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory");
-    pp_softmax<BF16, ADAPTIVE, VARLEN, DBG>(p, bars, tbase, wc);
+    pp_softmax<BF16, ADAPTIVE, VARLEN, DBG, TK>(p, bars, tbase, wc);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 104;\n" ::: "memory");
     if (warp == 8) {
-      if ((threadIdx.x & 31) == 0) pp_producer<VARLEN>(p, smem, bars, wc);
+      if ((threadIdx.x & 31) == 0) pp_producer<VARLEN, TK>(p, smem, bars, wc);
     } else if (warp == 9) {
-      pp_mma<BF16, ADAPTIVE, VARLEN>(p, smem, bars, tbase, wc);
+      pp_mma<BF16, ADAPTIVE, VARLEN, TK>(p, smem, bars, tbase, wc);
     }
   }
   tc_fence_before();

@@ -291,19 +291,19 @@ int launch_attn_cfg(const lamp::AttnParams& p, int grid, cudaStream_t st) {
                 : launch_attn_cfg_t<C, false, false, false>(p, grid, st);
 }
 
-template <bool BF16, bool ADAPTIVE, bool VARLEN, bool DBG = false>
+template <bool BF16, bool ADAPTIVE, bool VARLEN, bool DBG = false, bool TK = false>
 int launch_attn_pp_t(const lamp::AttnParams& p, int grid, cudaStream_t st) {
   static bool attr_set[64] = {};
   int dev = 0;
   LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    LAMP_CUDA(cudaFuncSetAttribute(lamp::attn_fwd_pp_kernel<BF16, ADAPTIVE, VARLEN, DBG>,
+    LAMP_CUDA(cudaFuncSetAttribute(lamp::attn_fwd_pp_kernel<BF16, ADAPTIVE, VARLEN, DBG, TK>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    lamp::PPCfg::SMEM_BYTES),
               "cudaFuncSetAttribute");
     attr_set[dev] = true;
   }
-  lamp::attn_fwd_pp_kernel<BF16, ADAPTIVE, VARLEN, DBG>
+  lamp::attn_fwd_pp_kernel<BF16, ADAPTIVE, VARLEN, DBG, TK>
       <<<grid, lamp::PPCfg::THREADS, lamp::PPCfg::SMEM_BYTES, st>>>(p);
   LAMP_CUDA(cudaGetLastError(), "attn_fwd_pp_kernel launch");
   return LAMP_OK;
@@ -317,16 +317,60 @@ int launch_attn_pp_v(const lamp::AttnParams& p, int grid, cudaStream_t st) {
                     : launch_attn_pp_t<false, false, VARLEN>(p, grid, st);
 }
 
+// Scheduler slots of the two-tile kernel, handed out round-robin per device.  A launch's tag
+// is the number of earlier launches given the same slot, plus one: distinct among the launches
+// that share a slot (and never 0, the idle value).
+std::mutex g_sched_mu;
+unsigned long long* g_sched_base[64] = {};
+uint32_t g_sched_seq[64] = {};
+
+int sched_base(unsigned long long** out) {
+  int dev = 0;
+  LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(LAMP_ERR_INVALID, "device index out of range");
+  if (!g_sched_base[dev]) {
+    void* a = nullptr;
+    LAMP_CUDA(cudaGetSymbolAddress(&a, lamp::g_lamp_sched), "cudaGetSymbolAddress(sched)");
+    if (!a) return fail(LAMP_ERR_CUDA, "scheduler slots have no device address");
+    g_sched_base[dev] = static_cast<unsigned long long*>(a);
+  }
+  *out = g_sched_base[dev];
+  return LAMP_OK;
+}
+
+int sched_slot(unsigned long long** slot, uint32_t* tag) {
+  int dev = 0;
+  LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(g_sched_mu);
+  unsigned long long* base = nullptr;
+  if (int r = sched_base(&base)) return r;
+  const uint32_t s = g_sched_seq[dev]++;
+  *slot = base + (s % lamp::SCHED_SLOTS);
+  *tag = s / lamp::SCHED_SLOTS + 1u;
+  return LAMP_OK;
+}
+
 // Variable-length batches have their own instantiation: the dense one keeps compile-time
-// zero offsets.  The debug capture (dense batches only) has its own as well.
-int launch_attn_pp(const lamp::AttnParams& p, int grid, cudaStream_t st) {
+// zero offsets.  The debug capture (dense batches only) has its own as well, and so has the
+// ticket counter (dense batches only).  The debug capture always takes the fixed order (its
+// outputs do not depend on the order).
+int launch_attn_pp(const lamp::AttnParams& p0, int grid, bool dynamic, cudaStream_t st) {
+  lamp::AttnParams p = p0;
+  p.sched = nullptr;
+  p.sched_tag = 0;
   if (p.dbg_slot) {
     if (p.bf16) return p.adaptive ? launch_attn_pp_t<true, true, false, true>(p, grid, st)
                                   : launch_attn_pp_t<true, false, false, true>(p, grid, st);
     return p.adaptive ? launch_attn_pp_t<false, true, false, true>(p, grid, st)
                       : launch_attn_pp_t<false, false, false, true>(p, grid, st);
   }
-  return p.cu_q ? launch_attn_pp_v<true>(p, grid, st) : launch_attn_pp_v<false>(p, grid, st);
+  if (p.cu_q) return launch_attn_pp_v<true>(p, grid, st);
+  if (!dynamic) return launch_attn_pp_v<false>(p, grid, st);
+  if (int r = sched_slot(&p.sched, &p.sched_tag)) return r;
+  if (p.bf16) return p.adaptive ? launch_attn_pp_t<true, true, false, false, true>(p, grid, st)
+                                : launch_attn_pp_t<true, false, false, false, true>(p, grid, st);
+  return p.adaptive ? launch_attn_pp_t<false, true, false, false, true>(p, grid, st)
+                    : launch_attn_pp_t<false, false, false, false, true>(p, grid, st);
 }
 
 using Cfg64 = lamp::AttnCfg<64, 64, true>;
@@ -378,6 +422,7 @@ enum AttnKernel { K_CFG64, K_PP, K_CFG128, K_CFG256 };
 struct AttnCall {
   lamp::AttnParams p;
   AttnKernel kernel;
+  bool pp_dynamic;  // two-tile kernel: work items from a ticket counter (else a fixed order)
   int grid;
   size_t route_bytes;  // bytes of route_out cleared before the launch (0: none)
 };
@@ -460,19 +505,30 @@ int prepare_attn(const void* q, const void* k, const void* v, const void* q8, co
   } else {
     call->kernel = (D == 128) ? K_CFG128 : K_CFG256;
   }
-  // Chunks of KV planes for the single-tile kernel's CTA order: the largest divisor of B * Hkv
-  // whose K16, V and K8 tiles (5 bytes per element) fit in 40 MB of L2.  A sliding window
-  // already keeps the CTAs of one query tile on one band of keys, and a variable-length batch
-  // has its own lengths: one chunk there.
+  // Chunks of KV planes for the kernels' work order: the largest divisor of B * Hkv whose K16,
+  // V and K8 tiles (5 bytes per element) fit in 40 MB of L2 (one plane at least), so that the
+  // work in flight streams one chunk's keys from L2 while Q and O pass through it.  A sliding
+  // window already keeps the CTAs of one query tile on one band of keys, and a
+  // variable-length batch has its own lengths: one chunk there.  The two-tile kernel, whose
+  // persistent CTAs take items in turn, uses the chunked order (with items from a ticket
+  // counter, which keeps its CTAs' work even across the chunks) only when all KV planes
+  // together exceed L2 (more than 100 MB); below that every key stays in L2 anyway, and the
+  // fixed snake order over the longest-first items measured faster (no atomics on the
+  // producer's path).
   const int nkv = BHk;
+  const double plane = 5.0 * static_cast<double>(Lk) * D;
   p.chunk_kv = nkv;
+  call->pp_dynamic = false;
   if (window == 0 && !varlen) {
-    const double plane = 5.0 * static_cast<double>(Lk) * D;
     for (int d = nkv; d >= 1; --d)
       if (nkv % d == 0 && (d == 1 || d * plane <= 40e6)) {
         p.chunk_kv = d;
         break;
       }
+    if (call->kernel == K_PP) {
+      call->pp_dynamic = nkv * plane > 100e6;
+      if (!call->pp_dynamic) p.chunk_kv = nkv;
+    }
   }
   return LAMP_OK;
 }
@@ -482,7 +538,7 @@ int launch_attn(const AttnCall& c, cudaStream_t st) {
     LAMP_CUDA(cudaMemsetAsync(c.p.route, 0, c.route_bytes, st), "memset route");
   switch (c.kernel) {
     case K_CFG64: return launch_attn_cfg<Cfg64>(c.p, c.grid, st);
-    case K_PP: return launch_attn_pp(c.p, c.grid, st);
+    case K_PP: return launch_attn_pp(c.p, c.grid, c.pp_dynamic, st);
     case K_CFG128: return launch_attn_cfg<Cfg128>(c.p, c.grid, st);
     default: return launch_attn_cfg<Cfg256>(c.p, c.grid, st);
   }
@@ -1049,6 +1105,15 @@ int lamp_check(void* stream) {
   if (v) {
     const uint32_t zero = 0;
     LAMP_CUDA(cudaMemcpyToSymbol(lamp::g_lamp_error, &zero, sizeof(zero)), "clear error word");
+    // A launch that gave up may leave its work-item counter held: wait for the device, then
+    // return every scheduler slot of this device to idle.
+    LAMP_CUDA(cudaDeviceSynchronize(), "cudaDeviceSynchronize");
+    {
+      std::lock_guard<std::mutex> lk(g_sched_mu);
+      unsigned long long* base = nullptr;
+      if (int r = sched_base(&base)) return r;
+      LAMP_CUDA(cudaMemset(base, 0, sizeof(lamp::g_lamp_sched)), "reset scheduler slots");
+    }
     return fail(LAMP_ERR_TIMEOUT, "a device wait gave up (error word 0x%x, site %u)", v, (v >> 8) & 0xFFu);
   }
   return LAMP_OK;
