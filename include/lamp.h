@@ -211,6 +211,29 @@ int lamp_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
                           float scale, const uint64_t* mask_bits, int group_tiles, int mode,
                           float tau, void* stream);
 
+/* lamp_attn_fwd on HOST buffers, with the host-device copies pipelined against the compute
+ * (no counterpart in the pages: a runtime entry point for callers whose Q, K, V live in host
+ * memory and who want O back there).  q, k, v: host [B][H|Hkv][L][D] 16-bit; o: host
+ * [B][H][Lq][D] (fp32, or the input dtype with LAMP_OUT_INDTYPE); lse: host [B][H][Lq] fp32 or
+ * NULL; host buffers need no alignment, and only page-locked (pinned) ones let the copies
+ * overlap the compute.  mask_bits stays a DEVICE buffer (as for lamp_attn_fwd).  Every other
+ * argument, every check and every result bit is as lamp_attn_fwd's.
+ * The B * Hkv KV planes (each KV head with its H / Hkv query heads: independent problems) are
+ * cut into n_chunks chunks of consecutive planes (0: about 256 MB of copies per chunk, at most
+ * 8; clamped to [1, B * Hkv]).  Per chunk: Q, K, V are copied in on a library copy stream,
+ * quantised and attended on `stream`, and O, lse copied out on a second copy stream, through
+ * two device buffer slots in the library workspace (two chunks' inputs and outputs plus one
+ * chunk's 8-bit codes), so that chunk c + 1 is copied in and chunk c - 1 copied out while
+ * chunk c computes.  The copy streams start behind the work queued on `stream` before the
+ * call, and `stream` continues only once every copy of the call has completed; the host
+ * buffers must stay valid until then.  Calls on different streams share the workspace and
+ * the copy streams: they need the caller's ordering between them.  Argument errors return
+ * before anything is enqueued. */
+int lamp_attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int H, int Hkv, int Lq, int Lk, int D, int causal, int window,
+                       float scale, const uint64_t* mask_bits, int group_tiles, int mode,
+                       float tau, int n_chunks, void* stream);
+
 /* Look-ahead routing with a threshold skip (LampAttention abstract: 8-bit products decide which
  * sub-blocks need 16 bits; LATTE page: low-precision dot products filter out the keys far below
  * the row maximum).  As lamp_attn_fwd_q8 in look-ahead mode (mode must hold

@@ -31,7 +31,8 @@ OUT_F32, OUT_INDTYPE = 0x0, 0x8
 EXPORTS = ("lamp_tile_shape", "lamp_mask_words", "lamp_quant_qk", "lamp_build_mask",
            "lamp_build_mask_template", "lamp_template_fraction",
            "lamp_template_for_int8_fraction", "lamp_quant_qk_varlen", "lamp_attn_fwd_q8_varlen", "lamp_attn_fwd_q8_skip", "lamp_decode_fwd",
-           "lamp_attn_fwd_varlen", "lamp_attn_fwd", "lamp_attn_fwd_q8", "lamp_attn_fwd_noalloc", "lamp_workspace_size",
+           "lamp_attn_fwd_varlen", "lamp_attn_fwd", "lamp_attn_fwd_q8", "lamp_attn_fwd_noalloc", "lamp_attn_fwd_host",
+           "lamp_workspace_size",
            "lamp_set_workspace", "lamp_check", "lamp_selftest_timeout", "lamp_mma_probe",
            "lamp_attn_debug", "lamp_exp2_eval", "lamp_last_error")
 NOALLOC_MAX_BYTES = 32 << 20  # LAMP_NOALLOC_MAX_BYTES
@@ -74,6 +75,7 @@ def lib():
                 "lamp_attn_fwd_varlen": (_i, [_vp] * 7 + [_i] * 10 + [_f, _vp, _i, _i, _f, _vp]),
                 "lamp_attn_fwd_q8": (_i, [_vp] * 9 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp, _vp]),
                 "lamp_attn_fwd_noalloc": (_i, [_vp] * 5 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp]),
+                "lamp_attn_fwd_host": (_i, [_vp] * 5 + [_i] * 8 + [_f, _vp, _i, _i, _f, _i, _vp]),
                 "lamp_workspace_size": (_sz, [_i] * 7),
                 "lamp_set_workspace": (_i, [_vp, _sz]),
                 "lamp_check": (_i, [_vp]),
@@ -229,6 +231,16 @@ def lamp_attn_fwd_noalloc(q, k, v, o, lse, B, H, Hkv, Lq, Lk, D, causal, window,
                                        Lq, Lk, D, int(causal), int(window), float(scale),
                                        _ptr(mask_bits), int(group_tiles), int(mode), float(tau),
                                        _stream(stream)))
+
+
+def lamp_attn_fwd_host(q, k, v, o, lse, B, H, Hkv, Lq, Lk, D, causal, window, scale, mask_bits,
+                       group_tiles, mode, tau, n_chunks=0, stream=None):
+    """lamp_attn_fwd on host buffers (q, k, v, o, lse: pinned CPU tensors or host addresses),
+    the copies pipelined against the compute; mask_bits stays on the device."""
+    _check(lib().lamp_attn_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Lq,
+                                    Lk, D, int(causal), int(window), float(scale),
+                                    _ptr(mask_bits), int(group_tiles), int(mode), float(tau),
+                                    int(n_chunks), _stream(stream)))
 
 
 def lamp_attn_fwd_q8(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D, causal,

@@ -940,6 +940,134 @@ int lamp_attn_fwd(const void* q, const void* k, const void* v, void* o, float* l
                           mask_bits, group_tiles, mode, tau, st);
 }
 
+namespace {
+// Per-device resources of lamp_attn_fwd_host: a host-to-device and a device-to-host copy stream
+// and the events of two buffer slots, created on first use and kept for the process.
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t fork = nullptr, join_in = nullptr, join_out = nullptr;
+  cudaEvent_t in_done[2] = {}, cmp_done[2] = {}, out_done[2] = {};
+};
+HostPipe g_pipe[64];
+std::mutex g_pipe_mu;
+
+int host_pipe(HostPipe** out) {
+  int dev = 0;
+  LAMP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(LAMP_ERR_INVALID, "device index out of range");
+  HostPipe& hp = g_pipe[dev];
+  if (!hp.ready) {
+    LAMP_CUDA(cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking), "cudaStreamCreate(in)");
+    LAMP_CUDA(cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking), "cudaStreamCreate(out)");
+    cudaEvent_t* evs[] = {&hp.fork, &hp.join_in, &hp.join_out, &hp.in_done[0], &hp.in_done[1],
+                          &hp.cmp_done[0], &hp.cmp_done[1], &hp.out_done[0], &hp.out_done[1]};
+    for (cudaEvent_t* e : evs)
+      LAMP_CUDA(cudaEventCreateWithFlags(e, cudaEventDisableTiming), "cudaEventCreate");
+    hp.ready = true;
+  }
+  *out = &hp;
+  return LAMP_OK;
+}
+}  // namespace
+
+int lamp_attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int H, int Hkv, int Lq, int Lk, int D, int causal, int window,
+                       float scale, const uint64_t* mask_bits, int group_tiles, int mode,
+                       float tau, int n_chunks, void* stream) {
+  if (!q || !k || !v || !o) return fail(LAMP_ERR_INVALID, "null operand pointer");
+  if (n_chunks < 0) return fail(LAMP_ERR_INVALID, "n_chunks must be >= 0");
+  // The host buffers need no alignment: the kernels' operands are the device chunks.  Every
+  // other check of lamp_attn_fwd runs here, on stand-in aligned addresses.
+  alignas(256) static const char kStandIn[256] = {};
+  int r = check_attn(kStandIn, kStandIn, kStandIn, false, nullptr, nullptr, nullptr, nullptr,
+                     kStandIn, B, H, Hkv, Lq, Lk, D, causal, window, scale, group_tiles, mode,
+                     tau, nullptr, nullptr, 0, 0, INFINITY);
+  if (r) return r;
+  const int G = H / Hkv;
+  const int planes = B * Hkv;  // (b, kvh): G query heads and one KV head, an independent problem
+  const size_t eb = 2, ob = (mode & LAMP_OUT_INDTYPE) ? 2 : 4;
+  const size_t q_pl = static_cast<size_t>(G) * Lq * D * eb;   // bytes of one plane's Q
+  const size_t kv_pl = static_cast<size_t>(Lk) * D * eb;      // ... of its K (and of its V)
+  const size_t o_pl = static_cast<size_t>(G) * Lq * D * ob;   // ... of its O
+  const size_t l_pl = static_cast<size_t>(G) * Lq * sizeof(float);
+  if (n_chunks == 0) {  // about 256 MB of copies per chunk, at most 8 chunks
+    const double bytes = static_cast<double>(planes) * (q_pl + 2 * kv_pl + o_pl + l_pl);
+    n_chunks = static_cast<int>(std::max(1.0, std::min(8.0, std::floor(bytes / 256e6))));
+  }
+  n_chunks = std::min(n_chunks, planes);
+  const int per = (planes + n_chunks - 1) / n_chunks;  // planes per chunk (the last may be short)
+  n_chunks = (planes + per - 1) / per;
+  // workspace: the quantiser's codes and scales for one chunk, then two slots of device chunks
+  const WsLayout wq = ws_layout(per, G, 1, Lq, Lk, D);
+  const size_t s_q = 0, s_k = align256(per * q_pl), s_v = s_k + align256(per * kv_pl),
+               s_o = s_v + align256(per * kv_pl), s_l = s_o + align256(per * o_pl),
+               slot = s_l + align256(per * l_pl);
+  const size_t need = align256(wq.total) + 2 * slot;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lk(g_pipe_mu);
+  HostPipe* hp = nullptr;
+  if ((r = host_pipe(&hp))) return r;
+  void* ws = nullptr;
+  if ((r = get_workspace(need, st, &ws))) return r;
+  auto* base = static_cast<uint8_t*>(ws);
+  uint8_t* slots = base + align256(wq.total);
+  int bm = 0, bn = 0;
+  tile_shape(D, &bm, &bn);
+  const size_t mask_pl = mask_bits ? static_cast<size_t>(G) * ((Lq + bm - 1) / bm) *
+                                         lamp_mask_words(Lk, D, group_tiles)
+                                   : 0;  // mask words of one plane
+  const auto* hq = static_cast<const uint8_t*>(q);
+  const auto* hk = static_cast<const uint8_t*>(k);
+  const auto* hv = static_cast<const uint8_t*>(v);
+  auto* ho = static_cast<uint8_t*>(o);
+  auto* hl = reinterpret_cast<uint8_t*>(lse);
+  // fork: the copy streams start behind the work already queued on `stream`
+  LAMP_CUDA(cudaEventRecord(hp->fork, st), "cudaEventRecord");
+  LAMP_CUDA(cudaStreamWaitEvent(hp->in, hp->fork, 0), "cudaStreamWaitEvent");
+  LAMP_CUDA(cudaStreamWaitEvent(hp->out, hp->fork, 0), "cudaStreamWaitEvent");
+  for (int c = 0; c < n_chunks; ++c) {
+    const int s = c & 1;
+    const int p0 = c * per, np = std::min(per, planes - p0);
+    uint8_t* d = slots + s * slot;
+    // in: chunk c's Q, K, V, once chunk c - 2 (same slot) has been computed
+    if (c >= 2) LAMP_CUDA(cudaStreamWaitEvent(hp->in, hp->cmp_done[s], 0), "cudaStreamWaitEvent");
+    LAMP_CUDA(cudaMemcpyAsync(d + s_q, hq + p0 * q_pl, np * q_pl, cudaMemcpyHostToDevice, hp->in),
+              "copy Q to the device");
+    LAMP_CUDA(cudaMemcpyAsync(d + s_k, hk + p0 * kv_pl, np * kv_pl, cudaMemcpyHostToDevice, hp->in),
+              "copy K to the device");
+    LAMP_CUDA(cudaMemcpyAsync(d + s_v, hv + p0 * kv_pl, np * kv_pl, cudaMemcpyHostToDevice, hp->in),
+              "copy V to the device");
+    LAMP_CUDA(cudaEventRecord(hp->in_done[s], hp->in), "cudaEventRecord");
+    // compute on `stream`: chunk c as B = np problems of G query heads and one KV head, once
+    // its inputs are in and chunk c - 2's outputs have been copied out
+    LAMP_CUDA(cudaStreamWaitEvent(st, hp->in_done[s], 0), "cudaStreamWaitEvent");
+    if (c >= 2) LAMP_CUDA(cudaStreamWaitEvent(st, hp->out_done[s], 0), "cudaStreamWaitEvent");
+    if ((r = quant_and_attend(d + s_q, d + s_k, d + s_v, d + s_o,
+                              lse ? reinterpret_cast<float*>(d + s_l) : nullptr, base, wq, np, G,
+                              1, Lq, Lk, D, causal, window, scale,
+                              mask_bits ? mask_bits + p0 * mask_pl : nullptr, group_tiles, mode,
+                              tau, st)))
+      return r;
+    LAMP_CUDA(cudaEventRecord(hp->cmp_done[s], st), "cudaEventRecord");
+    // out: chunk c's O and lse
+    LAMP_CUDA(cudaStreamWaitEvent(hp->out, hp->cmp_done[s], 0), "cudaStreamWaitEvent");
+    LAMP_CUDA(cudaMemcpyAsync(ho + p0 * o_pl, d + s_o, np * o_pl, cudaMemcpyDeviceToHost, hp->out),
+              "copy O to the host");
+    if (lse)
+      LAMP_CUDA(cudaMemcpyAsync(hl + p0 * l_pl, d + s_l, np * l_pl, cudaMemcpyDeviceToHost,
+                                hp->out),
+                "copy lse to the host");
+    LAMP_CUDA(cudaEventRecord(hp->out_done[s], hp->out), "cudaEventRecord");
+  }
+  // join: `stream` continues once every copy has completed
+  LAMP_CUDA(cudaEventRecord(hp->join_in, hp->in), "cudaEventRecord");
+  LAMP_CUDA(cudaEventRecord(hp->join_out, hp->out), "cudaEventRecord");
+  LAMP_CUDA(cudaStreamWaitEvent(st, hp->join_in, 0), "cudaStreamWaitEvent");
+  LAMP_CUDA(cudaStreamWaitEvent(st, hp->join_out, 0), "cudaStreamWaitEvent");
+  return LAMP_OK;
+}
+
 int lamp_attn_fwd_q8_skip(const void* q, const void* k, const void* v, const void* q8,
                           const void* k8, const float* q_scale, const float* k_scale, void* o,
                           float* lse, int B, int H, int Hkv, int Lq, int Lk, int D, int causal,

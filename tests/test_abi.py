@@ -85,6 +85,28 @@ def test_attn_fwd_rejects_bad_arguments_on_host(bad, code, entry):
 
 
 @pytest.mark.parametrize("bad,code", [
+    (dict(H=3, Hkv=2), mpt.LAMP_ERR_INVALID),
+    (dict(B=0), mpt.LAMP_ERR_INVALID),
+    (dict(D=80), mpt.LAMP_ERR_UNSUPPORTED),
+    (dict(q=None), mpt.LAMP_ERR_INVALID),
+    (dict(o=None), mpt.LAMP_ERR_INVALID),
+    (dict(causal=0, window=16), mpt.LAMP_ERR_UNSUPPORTED),
+    (dict(group_tiles=0), mpt.LAMP_ERR_INVALID),
+    (dict(mode=0x30), mpt.LAMP_ERR_INVALID),
+    (dict(scale=float("nan")), mpt.LAMP_ERR_INVALID),
+    (dict(n_chunks=-1), mpt.LAMP_ERR_INVALID),
+])
+def test_attn_fwd_host_rejects_bad_arguments_on_host(bad, code):
+    # host buffers need no alignment, so an odd host address alone is no error; everything else
+    # lamp_attn_fwd checks is checked before anything is enqueued
+    n_chunks = bad.pop("n_chunks", 0)
+    a = _attn_args(**bad)
+    with pytest.raises(mpt.LampError) as e:
+        mpt.lamp_attn_fwd_host(**a, n_chunks=n_chunks, stream=0)
+    assert e.value.code == code
+
+
+@pytest.mark.parametrize("bad,code", [
     (dict(q=0x1001), mpt.LAMP_ERR_INVALID),            # misaligned
     (dict(o=0x5010), mpt.LAMP_ERR_INVALID),            # O written with 32-byte stores
     (dict(causal=0, window=16), mpt.LAMP_ERR_UNSUPPORTED),
