@@ -14,7 +14,9 @@ What it computes, with the pages' passages it follows:
                          4, "static, data-free structured templates"; section 3, "SpTrans75").
   * ``attention``     -- routed scores, shared softmax and 16-bit-routed tiles (TileMix page,
                          section 2, "The Dual-Path Engine"; LampAttention abstract for the
-                         adaptive 8-bit -> 16-bit recomputation).
+                         adaptive 8-bit -> 16-bit recomputation, and, with ``pv8``, for
+                         exponentials and P.V in 8-bit formats).
+  * ``quantize_v``, ``e4m3_round_pos`` -- the 8-bit V and the rounding of the 8-bit p.
 Every function is pinned by CPU tests against closed forms, brute force and invariants.
 """
 from __future__ import annotations
@@ -64,6 +66,8 @@ class _Args(ctypes.Structure):
         ("skip_tau", ctypes.c_double),
         ("k_codes_in", ctypes.c_void_p), ("k_scales_in", ctypes.c_void_p),
         ("hinted", ctypes.c_void_p),
+        ("pv8", ctypes.c_int), ("v_codes", ctypes.c_void_p), ("v_scales", ctypes.c_void_p),
+        ("pv8_margin", ctypes.c_void_p),
     ]
 
 
@@ -91,6 +95,11 @@ def lib():
             L.orc_build_mask_template.argtypes = [ctypes.c_void_p] + [ctypes.c_int] * 10
             L.orc_attention.restype = ctypes.c_int
             L.orc_attention.argtypes = [ctypes.POINTER(_Args)]
+            L.orc_e4m3_round_pos.restype = ctypes.c_double
+            L.orc_e4m3_round_pos.argtypes = [ctypes.c_double, ctypes.POINTER(ctypes.c_double)]
+            L.orc_quantize_v.restype = None
+            L.orc_quantize_v.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
             L.orc_score_tiles.restype = ctypes.c_int
             L.orc_score_tiles.argtypes = [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 9 \
                 + [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
@@ -111,6 +120,27 @@ def e4m3_decode(code: int) -> float:
 
 def e4m3_encode(x: float) -> int:
     return int(lib().orc_e4m3_encode(float(x)))
+
+
+def e4m3_round_pos(p: float):
+    """(nearest e4m3 value of p >= 0, relative distance of p from the nearest rounding
+    midpoint) -- the rounding of the 8-bit exponentials."""
+    d = ctypes.c_double()
+    r = lib().orc_e4m3_round_pos(float(p), ctypes.byref(d))
+    return r, d.value
+
+
+def quantize_v(x: np.ndarray):
+    """Per-channel E4M3 V of x [..., Lk, D] (one scale per leading index and channel over all
+    keys; LampAttention abstract, 8-bit formats, read for V).  Returns (codes uint8
+    [..., D, Lk] channel-major, scales float32 [..., D])."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    *lead, L, D = x.shape
+    outer = int(np.prod(lead)) if lead else 1
+    codes = np.empty((*lead, D, L), dtype=np.uint8)
+    scales = np.empty((*lead, D), dtype=np.float32)
+    lib().orc_quantize_v(_ptr(x), outer, L, D, _ptr(codes), _ptr(scales))
+    return codes, scales
 
 
 def splitmix64_next(state: int) -> int:
@@ -165,7 +195,7 @@ def build_mask_template(B: int, H: int, Lq: int, Lk: int, bm: int, bn: int, grou
 def attention(q, k, v, *, bm, bn, causal=False, window=0, scale=None, mask=None, group_tiles=1,
               route="bitmask", fmt="int8", tau=0.0, rows=None, threads=0, want_codes=False,
               route_hint=None, hint_margin=0.0, skip_tau=float("inf"), k_codes_in=None,
-              k_scales_in=None):
+              k_scales_in=None, pv8=False):
     """Routed attention on fp32 values of 16-bit inputs.
 
     q [B,H,Lq,D], k/v [B,Hkv,Lk,D].  ``mask`` uint64 [B,H,nQT,W] or None (all 8-bit) in
@@ -177,7 +207,12 @@ def attention(q, k, v, *, bm, bn, causal=False, window=0, scale=None, mask=None,
     an 8-bit key cache used by the 8-bit path instead of quantising ``k`` (decode with an INT8
     KV cache: TileMix page, section 4).  ``skip_tau`` (look-ahead mode; LATTE page, low-precision filtering of the keys
     far below the row maximum, read per tile): a tile every row of which has t_r < m_r -
-    skip_tau is dropped; +inf never drops.
+    skip_tau is dropped; +inf never drops.  ``pv8``: 8-bit exponentials and an 8-bit P.V
+    (LampAttention abstract): V in per-channel E4M3 (``quantize_v``), each p = e^(s - m_t)
+    * 2^8 rounded to E4M3 against the running max m_t after its key tile (ascending tiles), O =
+    sv * sum p8 v8 / sum p8 over the tiles rescaled to the final max; adds v_codes, v_scales and
+    pv8_margin (per output row, the smallest relative distance of one of its p from an E4M3
+    rounding midpoint).  lse stays the exact softmax's.
     """
     q = np.ascontiguousarray(q, dtype=np.float32)
     k = np.ascontiguousarray(k, dtype=np.float32)
@@ -226,6 +261,12 @@ def attention(q, k, v, *, bm, bn, causal=False, window=0, scale=None, mask=None,
     hinted = np.zeros((B, H, nqt, nkt), dtype=np.uint8)
     a.hinted = _ptr(hinted)
     out = {"o": o, "lse": lse, "route": rmap, "margin": margin, "hinted": hinted}
+    if pv8:
+        vcodes = np.empty((B, Hkv, D, Lk), np.uint8)
+        vscales = np.empty((B, Hkv, D), np.float32)
+        pmargin = np.empty((B, H, R), np.float64)
+        a.pv8, a.v_codes, a.v_scales, a.pv8_margin = 1, _ptr(vcodes), _ptr(vscales), _ptr(pmargin)
+        out.update(v_codes=vcodes, v_scales=vscales, pv8_margin=pmargin)
     if want_codes:
         qc = np.empty(q.shape, np.uint8)
         qs = np.empty((B, H, nqt), np.float32)

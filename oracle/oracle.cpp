@@ -98,6 +98,53 @@ void quantize_block(const float* x, int rows, int D, int fmt, uint8_t* codes, fl
     }
 }
 
+// ---------------------------------------------------------------------------------------
+// 8-bit exponentials and 8-bit P.V (LampAttention page, abstract: the exponentials are
+// evaluated in 8-bit formats; the pages fix no format, so the reading is E4M3 for both P and
+// V).
+//
+// V: one scale per (batch, KV head, channel) over all keys of the plane (the pages give no V
+// block; a per-channel scale commutes with the sum over keys, so it applies to O once):
+// a = max_j |v_jd|, s = fl32(a / 448), code = E4M3(fl32(v / s)) rounded to nearest even,
+// saturating; a = 0 gives s = 0 and zero codes.  Codes are laid out [D][Lk] (channel-major).
+// ---------------------------------------------------------------------------------------
+void quantize_v_plane(const float* v, int Lk, int D, uint8_t* codes_t, float* scales) {
+  for (int d = 0; d < D; ++d) {
+    float a = 0.0f;
+    for (int j = 0; j < Lk; ++j) a = std::fmax(a, std::fabs(v[(size_t)j * D + d]));
+    const float s = a / 448.0f;  // IEEE fp32 divide
+    scales[d] = (a == 0.0f) ? 0.0f : s;
+    for (int j = 0; j < Lk; ++j)
+      codes_t[(size_t)d * Lk + j] = (a == 0.0f) ? 0 : e4m3_encode(v[(size_t)j * D + d] / s);
+  }
+}
+
+// P: the nearest E4M3 value of a non-negative p <= 448 (ties to even), computed from the
+// format's grid (a step of 2^-9 below 2^-6, else 2^(e-3) on [2^e, 2^(e+1))), and the relative
+// distance of p from the nearest rounding midpoint: how far p is from rounding the other way.
+double e4m3_round_pos(double p, double* midpoint_dist) {
+  if (!(p > 0.0)) {
+    if (midpoint_dist) *midpoint_dist = std::numeric_limits<double>::infinity();
+    return 0.0;
+  }
+  double step;
+  if (p < 0.015625) {
+    step = 0.001953125;
+  } else {
+    int E;
+    std::frexp(p, &E);  // p in [2^(E-1), 2^E)
+    step = std::ldexp(1.0, E - 1 - 3);
+  }
+  const double q = p / step;  // exact: step is a power of two
+  const double fl = std::floor(q), frac = q - fl;
+  double n;
+  if (frac > 0.5) n = fl + 1.0;
+  else if (frac < 0.5) n = fl;
+  else n = (std::fmod(fl, 2.0) == 0.0) ? fl : fl + 1.0;
+  if (midpoint_dist) *midpoint_dist = std::fabs(frac - 0.5) * step / p;
+  return n * step;
+}
+
 // SplitMix64 (Steele, Lea and Flood, OOPSLA 2014): one step of the generator from state x:
 // add the golden gamma, then the variant-13 finaliser.
 uint64_t splitmix64_next(uint64_t x) {
@@ -163,9 +210,25 @@ struct orc_args {
   const float* k_scales_in;   // [B,Hkv,nKT]
   uint8_t* hinted;            // optional [B,H,nQT,nKT]: 1 where a decision followed route_hint
                               // against the rule's own outcome (its margin < hint_margin)
+  // 8-bit exponentials and 8-bit P.V (see e4m3_round_pos and quantize_v_plane): O of a row is
+  // sv * sum_t 2^(m_t - m) sum_{j in t} p8_j v8_j / sum_t 2^(m_t - m) sum_{j in t} p8_j, with
+  // key tiles t in ascending order, m_t the row's running max of the routed scores after tile
+  // t, m the final one, and p8_j = E4M3(e^(s_j - m_t) * 2^8) (the largest p is 256 < 448).
+  // lse stays the exact softmax's.
+  int pv8;
+  uint8_t* v_codes;           // optional [B,Hkv,D,Lk] output of the V quantiser
+  float* v_scales;            // optional [B,Hkv,D]
+  double* pv8_margin;         // optional [B,H,R]: the row's smallest midpoint distance of a p
 };
 
 double orc_e4m3_decode(uint8_t c) { return e4m3_decode(c); }
+double orc_e4m3_round_pos(double p, double* midpoint_dist) { return e4m3_round_pos(p, midpoint_dist); }
+// Per-channel 8-bit V of x [outer, Lk, D]: codes [outer, D, Lk], scales [outer, D].
+void orc_quantize_v(const float* x, int outer, int Lk, int D, uint8_t* codes_t, float* scales) {
+  for (int o = 0; o < outer; ++o)
+    quantize_v_plane(x + (size_t)o * Lk * D, Lk, D, codes_t + (size_t)o * D * Lk,
+                     scales + (size_t)o * D);
+}
 uint8_t orc_e4m3_encode(float x) { return e4m3_encode(x); }
 uint64_t orc_splitmix64_next(uint64_t x) { return splitmix64_next(x); }
 
@@ -301,6 +364,18 @@ int orc_attention(const orc_args* a) {
     std::memcpy(ks.data(), a->k_scales_in, ks.size() * sizeof(float));
   } else {
     orc_quantize(a->k, g.B * g.Hkv, g.Lk, D, g.bn, a->fmt, kc.data(), ks.data());
+  }
+  // 8-bit V, per channel (8-bit P.V only)
+  std::vector<uint8_t> vc;
+  std::vector<float> vs;
+  if (a->pv8) {
+    vc.resize((size_t)g.B * g.Hkv * D * g.Lk);
+    vs.resize((size_t)g.B * g.Hkv * D);
+    for (int p = 0; p < g.B * g.Hkv; ++p)
+      quantize_v_plane(a->v + (size_t)p * g.Lk * D, g.Lk, D, vc.data() + (size_t)p * D * g.Lk,
+                       vs.data() + (size_t)p * D);
+    if (a->v_codes) std::memcpy(a->v_codes, vc.data(), vc.size());
+    if (a->v_scales) std::memcpy(a->v_scales, vs.data(), vs.size() * sizeof(float));
   }
   if (a->k_codes) std::memcpy(a->k_codes, kc.data(), kc.size());
   if (a->k_scales) std::memcpy(a->k_scales, ks.data(), ks.size() * sizeof(float));
@@ -525,6 +600,38 @@ int orc_attention(const orc_args* a) {
         }
         for (int d = 0; d < D; ++d) orow[d] /= l;
         *lrow = M + std::log(l);
+        if (a->pv8) {
+          // 8-bit exponentials against the running max, ascending key tiles, and an 8-bit P.V
+          const size_t plane = (size_t)b * g.Hkv + kvh;
+          const uint8_t* vct = vc.data() + plane * D * g.Lk;
+          const float* vsc = vs.data() + plane * D;
+          double m = NEG_INF, l8 = 0.0, mind = INF;
+          for (int d = 0; d < D; ++d) orow[d] = 0.0;
+          for (long kt = jl / g.bn; kt <= jh / g.bn; ++kt) {
+            const long c0 = std::max(jl, kt * g.bn), c1 = std::min(jh, kt * g.bn + g.bn - 1);
+            double tmax = NEG_INF;
+            for (long j = c0; j <= c1; ++j) tmax = std::max(tmax, srow[j]);
+            if (tmax == NEG_INF) continue;
+            if (tmax > m) {
+              if (m != NEG_INF) {
+                const double f = std::exp(m - tmax);
+                l8 *= f;
+                for (int d = 0; d < D; ++d) orow[d] *= f;
+              }
+              m = tmax;
+            }
+            for (long j = c0; j <= c1; ++j) {
+              if (srow[j] == NEG_INF) continue;
+              double md;
+              const double p8 = e4m3_round_pos(std::exp(srow[j] - m) * 256.0, &md);
+              mind = std::min(mind, md);
+              l8 += p8;
+              for (int d = 0; d < D; ++d) orow[d] += p8 * e4m3_decode(vct[(size_t)d * g.Lk + j]);
+            }
+          }
+          for (int d = 0; d < D; ++d) orow[d] = (double)vsc[d] * orow[d] / l8;
+          if (a->pv8_margin) a->pv8_margin[((size_t)b * g.H + h) * R + s] = mind;
+        }
       }
     }
   };
