@@ -55,6 +55,7 @@ enum {
 #define LAMP_IN_BF16 0x4u        /* bit 2: q, k, v are bf16                               */
 #define LAMP_OUT_F32 0x0u        /* bit 3: o is fp32                                      */
 #define LAMP_OUT_INDTYPE 0x8u    /* bit 3: o has the input dtype                          */
+#define LAMP_PV_E4M3 0x10u       /* bit 4: 8-bit exponentials and an 8-bit P.V (below)     */
 
 /* Routing tile (BM x BN) for head dimension D: 64 -> 64x64, 128 -> 128x128, 256 -> 64x128
  * (TileMix "The Tile Architecture": hardware-aligned score tiles of 128x128 or 64x64).
@@ -77,6 +78,17 @@ int lamp_mask_words(int Lk, int D, int group_tiles);
 int lamp_quant_qk(const void* q, const void* k, void* q8, void* k8, float* q_scale,
                   float* k_scale, int B, int H, int Hkv, int Lq, int Lk, int D, int mode,
                   void* stream);
+
+/* 8-bit V for the 8-bit P.V mode (LampAttention abstract: the exponentials are evaluated in
+ * 8-bit formats; the pages fix no format, and this library reads it as E4M3 for both P and V).
+ * One scale per (batch, KV head, channel) over all Lk keys: a = max_j |v_jd|, v_scale =
+ * fl32(a / 448), code = E4M3(fl32(v / v_scale)) rounded to nearest even (a = 0: scale 0 and
+ * zero codes).  v: [B][Hkv][Lk][D] 16-bit (mode: LAMP_IN_*); v8t: [B][Hkv][D][Lk16] E4M3
+ * codes, channel-major, Lk16 = Lk rounded up to a multiple of 16 (the padding written as
+ * zero), 16-byte aligned; v_scale: [B][Hkv][D] fp32.  D: 64, 128 or 256.  Three kernels (channel
+ * maxima into v_scale, codes, maxima -> scales) on `stream`. */
+int lamp_quant_v(const void* v, void* v8t, float* v_scale, int B, int Hkv, int Lk, int D,
+                 int mode, void* stream);
 
 /* Seeded routing template (TileMix: routing policies are static, data-free templates; the
  * template's shape is not given, so each group bit is an independent draw).  Bit g of the
@@ -233,6 +245,20 @@ int lamp_attn_fwd_host(const void* q, const void* k, const void* v, void* o, flo
                        int H, int Hkv, int Lq, int Lk, int D, int causal, int window,
                        float scale, const uint64_t* mask_bits, int group_tiles, int mode,
                        float tau, int n_chunks, void* stream);
+
+/* The routed attention kernel with 8-bit exponentials and an 8-bit P.V (mode must include
+ * LAMP_PV_E4M3; D = 128; dense batches; no threshold skip).  As lamp_attn_fwd_q8, except that
+ * V is given as lamp_quant_v's v8t / v_scale (no 16-bit V).  Per row, in ascending key tiles:
+ * the running max m_t after tile t (of the routed scores, as in the 16-bit P mode), each
+ * p = 2^(x - m_t) * 2^8 rounded to E4M3 (the row max's p is 256), P.V = the E4M3 MMA of P and
+ * V's codes, and O = v_scale * sum p8 v8 / sum p8 (the tiles rescaled to the final max); lse
+ * is that of the exact p.  Runs on the single-tile kernel. */
+int lamp_attn_fwd_q8_pv8(const void* q, const void* k, const void* q8, const void* k8,
+                         const float* q_scale, const float* k_scale, const void* v8t,
+                         const float* v_scale, void* o, float* lse, int B, int H, int Hkv,
+                         int Lq, int Lk, int D, int causal, int window, float scale,
+                         const uint64_t* mask_bits, int group_tiles, int mode, float tau,
+                         void* stream);
 
 /* Look-ahead routing with a threshold skip (LampAttention abstract: 8-bit products decide which
  * sub-blocks need 16 bits; LATTE page: low-precision dot products filter out the keys far below

@@ -27,11 +27,13 @@ ROUTE_BITMASK, ROUTE_ADAPTIVE = 0x0, 0x1
 FMT_INT8, FMT_E4M3 = 0x0, 0x2
 IN_FP16, IN_BF16 = 0x0, 0x4
 OUT_F32, OUT_INDTYPE = 0x0, 0x8
+PV_E4M3 = 0x10  # 8-bit exponentials and an 8-bit P.V
 
 EXPORTS = ("lamp_tile_shape", "lamp_mask_words", "lamp_quant_qk", "lamp_build_mask",
            "lamp_build_mask_template", "lamp_template_fraction",
            "lamp_template_for_int8_fraction", "lamp_quant_qk_varlen", "lamp_attn_fwd_q8_varlen", "lamp_attn_fwd_q8_skip", "lamp_decode_fwd",
            "lamp_attn_fwd_varlen", "lamp_attn_fwd", "lamp_attn_fwd_q8", "lamp_attn_fwd_noalloc", "lamp_attn_fwd_host",
+           "lamp_quant_v", "lamp_attn_fwd_q8_pv8",
            "lamp_workspace_size",
            "lamp_set_workspace", "lamp_check", "lamp_selftest_timeout", "lamp_mma_probe",
            "lamp_attn_debug", "lamp_exp2_eval", "lamp_last_error")
@@ -76,6 +78,8 @@ def lib():
                 "lamp_attn_fwd_q8": (_i, [_vp] * 9 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp, _vp]),
                 "lamp_attn_fwd_noalloc": (_i, [_vp] * 5 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp]),
                 "lamp_attn_fwd_host": (_i, [_vp] * 5 + [_i] * 8 + [_f, _vp, _i, _i, _f, _i, _vp]),
+                "lamp_quant_v": (_i, [_vp] * 3 + [_i] * 5 + [_vp]),
+                "lamp_attn_fwd_q8_pv8": (_i, [_vp] * 10 + [_i] * 8 + [_f, _vp, _i, _i, _f, _vp]),
                 "lamp_workspace_size": (_sz, [_i] * 7),
                 "lamp_set_workspace": (_i, [_vp, _sz]),
                 "lamp_check": (_i, [_vp]),
@@ -115,11 +119,12 @@ def _check(code: int):
         raise LampError(code, lib().lamp_last_error().decode())
 
 
-def mode_bits(route="bitmask", fmt="int8", dtype="bf16", out="f32") -> int:
+def mode_bits(route="bitmask", fmt="int8", dtype="bf16", out="f32", pv8=False) -> int:
     return ((ROUTE_ADAPTIVE if route == "adaptive" else ROUTE_BITMASK)
             | (FMT_E4M3 if fmt == "e4m3" else FMT_INT8)
             | (IN_BF16 if dtype == "bf16" else IN_FP16)
-            | (OUT_INDTYPE if out == "in" else OUT_F32))
+            | (OUT_INDTYPE if out == "in" else OUT_F32)
+            | (PV_E4M3 if pv8 else 0))
 
 
 # ------------------------------------------------------------ C-ABI wrappers ----------
@@ -243,6 +248,20 @@ def lamp_attn_fwd_host(q, k, v, o, lse, B, H, Hkv, Lq, Lk, D, causal, window, sc
                                     int(n_chunks), _stream(stream)))
 
 
+def lamp_quant_v(v, v8t, v_scale, B, Hkv, Lk, D, mode, stream=None):
+    _check(lib().lamp_quant_v(_ptr(v), _ptr(v8t), _ptr(v_scale), B, Hkv, Lk, D, int(mode),
+                              _stream(stream)))
+
+
+def lamp_attn_fwd_q8_pv8(q, k, q8, k8, q_scale, k_scale, v8t, v_scale, o, lse, B, H, Hkv, Lq, Lk,
+                         D, causal, window, scale, mask_bits, group_tiles, mode, tau, stream=None):
+    _check(lib().lamp_attn_fwd_q8_pv8(_ptr(q), _ptr(k), _ptr(q8), _ptr(k8), _ptr(q_scale),
+                                      _ptr(k_scale), _ptr(v8t), _ptr(v_scale), _ptr(o), _ptr(lse),
+                                      B, H, Hkv, Lq, Lk, D, int(causal), int(window), float(scale),
+                                      _ptr(mask_bits), int(group_tiles), int(mode), float(tau),
+                                      _stream(stream)))
+
+
 def lamp_attn_fwd_q8(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D, causal,
                      window, scale, mask_bits, group_tiles, mode, tau, route_out=None,
                      stream=None):
@@ -297,8 +316,9 @@ def lamp_last_error() -> str:
 # stays in the library.
 
 def attention(q, k, v, *, causal=False, window=0, scale=0.0, mask_bits=None, group_tiles=1,
-              route="bitmask", fmt="int8", tau=0.0, out="f32", stream=None):
-    """O, lse for q [B,H,Lq,D], k/v [B,Hkv,Lk,D] (fp16/bf16 CUDA tensors)."""
+              route="bitmask", fmt="int8", tau=0.0, out="f32", pv8=False, stream=None):
+    """O, lse for q [B,H,Lq,D], k/v [B,Hkv,Lk,D] (fp16/bf16 CUDA tensors); ``pv8``: 8-bit
+    exponentials and an 8-bit P.V (D = 128)."""
     import torch
     B, H, Lq, D = q.shape
     _, Hkv, Lk, _ = k.shape
@@ -307,7 +327,36 @@ def attention(q, k, v, *, causal=False, window=0, scale=0.0, mask_bits=None, gro
                     dtype=torch.float32 if out == "f32" else q.dtype)
     lse = torch.empty((B, H, Lq), device=q.device, dtype=torch.float32)
     lamp_attn_fwd(q, k, v, o, lse, B, H, Hkv, Lq, Lk, D, causal, window, scale, mask_bits,
-                  group_tiles, mode_bits(route, fmt, dtype, out), tau, stream)
+                  group_tiles, mode_bits(route, fmt, dtype, out, pv8), tau, stream)
+    return o, lse
+
+
+def quantize_v(v, *, stream=None):
+    """(v8t uint8 [B,Hkv,D,Lk16] channel-major E4M3 codes, v_scale float32 [B,Hkv,D]) for v
+    [B,Hkv,Lk,D]; Lk16 = Lk rounded up to 16."""
+    import torch
+    B, Hkv, Lk, D = v.shape
+    v8t = torch.empty((B, Hkv, D, (Lk + 15) // 16 * 16), device=v.device, dtype=torch.uint8)
+    vs = torch.empty((B, Hkv, D), device=v.device, dtype=torch.float32)
+    dtype = "bf16" if v.dtype == torch.bfloat16 else "fp16"
+    lamp_quant_v(v, v8t, vs, B, Hkv, Lk, D, mode_bits(dtype=dtype), stream)
+    return v8t, vs
+
+
+def attention_q8_pv8(q, k, q8, k8, q_scale, k_scale, v8t, v_scale, *, causal=False, window=0,
+                     scale=0.0, mask_bits=None, group_tiles=1, route="bitmask", fmt="int8",
+                     tau=0.0, out="f32", stream=None):
+    """The 8-bit P.V kernel alone on quantised Q, K (``quantize``) and V (``quantize_v``)."""
+    import torch
+    B, H, Lq, D = q.shape
+    _, Hkv, Lk, _ = k.shape
+    dtype = "bf16" if q.dtype == torch.bfloat16 else "fp16"
+    o = torch.empty((B, H, Lq, D), device=q.device,
+                    dtype=torch.float32 if out == "f32" else q.dtype)
+    lse = torch.empty((B, H, Lq), device=q.device, dtype=torch.float32)
+    lamp_attn_fwd_q8_pv8(q, k, q8, k8, q_scale, k_scale, v8t, v_scale, o, lse, B, H, Hkv, Lq, Lk,
+                         D, causal, window, scale, mask_bits, group_tiles,
+                         mode_bits(route, fmt, dtype, out, True), tau, stream)
     return o, lse
 
 

@@ -57,6 +57,10 @@ struct AttnParams {
   CUtensorMap tm_v;    // [B*Hkv][Lk][D] 16-bit, box 64 x BN x 1, 128B swizzle
   CUtensorMap tm_q8;   // [B*H][Lq][D] 8-bit, box min(D,128) x 128 x 1
   CUtensorMap tm_k8;   // [B*Hkv][Lk][D] 8-bit, box min(D,128) x BN x 1
+  // 8-bit P.V mode: V in E4M3, channel-major [B*Hkv][D][Lk rounded up to 16], box BN x D x 1,
+  // 128B swizzle, and its per-channel scales [B*Hkv][D]
+  CUtensorMap tm_v8;
+  const float* v_scale;
   const float* q_scale;  // [B][H][nQT]
   const float* k_scale;  // [B][Hkv][nKT]
   const uint64_t* mask;  // [B][H][nQT][W] or null
@@ -91,17 +95,20 @@ struct AttnParams {
   int dbg_nslots;
 };
 
-template <int D_, int BN_, bool STACK_>
+template <int D_, int BN_, bool STACK_, bool PV8_ = false>
 struct AttnCfg {
   static constexpr int D = D_;
   static constexpr int BN = BN_;
   static constexpr bool STACK = STACK_;        // routing tiles of 64 rows, two per MMA tile
+  // 8-bit exponentials and 8-bit P.V: P goes to shared memory in E4M3 (one 16 KB buffer per S
+  // buffer) and P.V is the SS-form E4M3 MMA with V channel-major in the ring
+  static constexpr bool PV8 = PV8_;
   static constexpr int BM = STACK ? 64 : 128;  // routing tile rows
   static constexpr int MT = 128;               // MMA tile rows
   static constexpr int Q16_BYTES = MT * D * 2;
   static constexpr int Q8_BYTES = MT * D;
   static constexpr int SLOT_BYTES = BN * D * 2;
-  static constexpr int NS = (D == 64) ? 8 : (D == 128 ? 5 : 2);
+  static constexpr int NS = PV8 ? 4 : (D == 64) ? 8 : (D == 128 ? 5 : 2);
   static constexpr bool Q8_SW64 = (D == 64);  // 64-byte rows of 8-bit codes
   static constexpr int C16 = D / 64;           // 128-byte chunks of a 16-bit row
   static constexpr int C8 = (D == 64) ? 1 : D / 128;
@@ -116,7 +123,9 @@ struct AttnCfg {
   static constexpr int OFF_Q16 = 0;
   static constexpr int OFF_Q8 = Q16_BYTES;
   static constexpr int OFF_SLOTS = Q16_BYTES + Q8_BYTES;
-  static constexpr int OFF_BAR = OFF_SLOTS + NS * SLOT_BYTES;
+  static constexpr int OFF_P8 = OFF_SLOTS + NS * SLOT_BYTES;  // [2][MT rows][BN bytes], PV8
+  static constexpr int P8_BYTES = MT * BN;
+  static constexpr int OFF_BAR = OFF_P8 + (PV8 ? 2 * P8_BYTES : 0);
   static constexpr int BAR_BYTES = 512;
   static constexpr int OFF_XCH = OFF_BAR + BAR_BYTES;  // row-pair exchange: float [2][2][MT]
   static constexpr int SMEM_BYTES = OFF_XCH + 2 * 2 * MT * 4;  // dynamic base is 1024-aligned
@@ -125,6 +134,7 @@ struct AttnCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   static_assert(2 * BN + D <= 512, "tmem");
   static_assert(D != 256 || MT * D * 4 <= OFF_BAR, "O staging");
+  static_assert(!PV8 || (D == 128 && BN == 128 && !STACK), "8-bit P.V: D = 128, one routing tile");
 };
 
 struct Bars {
@@ -316,7 +326,7 @@ __device__ void producer_role(const AttnParams& p, const Geo& g, uint8_t* smem, 
 
   prefetch_tmap(&p.tm_q16);
   prefetch_tmap(&p.tm_k16);
-  prefetch_tmap(&p.tm_v);
+  prefetch_tmap(C::PV8 ? &p.tm_v8 : &p.tm_v);
   prefetch_tmap(&p.tm_q8);
   prefetch_tmap(&p.tm_k8);
 
@@ -339,6 +349,9 @@ __device__ void producer_role(const AttnParams& p, const Geo& g, uint8_t* smem, 
       mbar_arrive_expect_tx(&bars.full[slot], C::BN * C::D);
       for (int c = 0; c < C::C8; ++c)
         tma_load_3d(dst + c * C::BN * 128, &p.tm_k8, &bars.full[slot], c * 128, row, pkv);
+    } else if (C::PV8 && kind == 2) {  // V8: D channel rows of the tile's BN key bytes
+      mbar_arrive_expect_tx(&bars.full[slot], C::BN * C::D);
+      tma_load_3d(dst, &p.tm_v8, &bars.full[slot], row, 0, pkv);
     } else {
       const CUtensorMap* tm = (kind == 1) ? &p.tm_k16 : &p.tm_v;
       mbar_arrive_expect_tx(&bars.full[slot], C::BN * C::D * 2);
@@ -401,6 +414,8 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
   const uint64_t d_q8 = C::Q8_SW64 ? sdesc(sQ8, 16, 512, SWZ_64B) : sdesc(sQ8, 16, 1024, SWZ_128B);
   const uint64_t d_k8 = C::Q8_SW64 ? sdesc(slots, 16, 512, SWZ_64B) : sdesc(slots, 16, 1024, SWZ_128B);
   const uint64_t d_v = sdesc(slots, C::BN * 128, 1024, SWZ_128B);
+  const uint64_t d_p8 = sdesc(smem_u32(smem + C::OFF_P8), 16, 1024, SWZ_128B);
+  constexpr uint32_t id_pv8 = idesc(1, 0, 0, 0, 0, C::D, 128);  // E4M3 x E4M3, both K-major
   constexpr uint64_t SLOT_D = C::SLOT_BYTES >> 4;
 
   uint32_t item = 0;
@@ -525,16 +540,30 @@ __device__ void mma_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars&
     tc_fence_after();
     int slotv;
     if (!(ok = take(slotv))) break;
-    const uint64_t vb = d_v + slotv * SLOT_D;
-    const uint32_t pt = tbase + static_cast<uint32_t>(bsel * C::BN);
-    // P (16-bit pairs): each softmax column half packs its keys into the first half of its own
-    // S columns, so keys [BN/2 * h, BN/2 * (h + 1)) sit at columns BN/2 * h + [0, BN/4)
-    constexpr int SPH = C::BN / 32;  // K steps of 16 keys per column half
-    if (leader) {
+    if constexpr (C::PV8) {
+      // P8 [128 rows][128 key bytes] and V8 [D rows][128 key bytes], both K-major with 128-byte
+      // rows: the operand layout of the E4M3 QK^T; K steps of 32 keys
+      const uint64_t pb = d_p8 + static_cast<uint64_t>(bsel * (C::P8_BYTES >> 4));
+      const uint64_t vb8 = d_k8 + slotv * SLOT_D;
+      if (leader) {
 #pragma unroll
-      for (int s = 0; s < C::BN / 16; ++s)
-        mma_f16_ts(tbase + C::TMEM_O, pt + (s / SPH) * (C::BN / 2) + (s % SPH) * 8,
-                   vb + static_cast<uint64_t>(s * ((16 * 128) >> 4)), id_pv, (t > 0 || s > 0) ? 1u : 0u);
+        for (int s = 0; s < C::BN / 32; ++s)
+          mma_f8_ss(tbase + C::TMEM_O, pb + static_cast<uint64_t>(s * 2),
+                    vb8 + static_cast<uint64_t>(s * 2), id_pv8, (t > 0 || s > 0) ? 1u : 0u);
+      }
+    } else {
+      const uint64_t vb = d_v + slotv * SLOT_D;
+      const uint32_t pt = tbase + static_cast<uint32_t>(bsel * C::BN);
+      // P (16-bit pairs): each softmax column half packs its keys into the first half of its
+      // own S columns, so keys [BN/2 * h, BN/2 * (h + 1)) sit at columns BN/2 * h + [0, BN/4)
+      constexpr int SPH = C::BN / 32;  // K steps of 16 keys per column half
+      if (leader) {
+#pragma unroll
+        for (int s = 0; s < C::BN / 16; ++s)
+          mma_f16_ts(tbase + C::TMEM_O, pt + (s / SPH) * (C::BN / 2) + (s % SPH) * 8,
+                     vb + static_cast<uint64_t>(s * ((16 * 128) >> 4)), id_pv,
+                     (t > 0 || s > 0) ? 1u : 0u);
+      }
     }
     commit(&bars.o_done);
     commit(&bars.empty[slotv]);
@@ -629,7 +658,10 @@ template <class C, bool BF16, bool E4M3, bool SKIP, bool DBG>
 __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, Bars& bars,
                              uint32_t tbase, const WaitCtx wc) {
   constexpr int N = C::BN, NH = C::BN / 2;
-  constexpr float RESCALE_THRESH = 8.0f;
+  // lazy reference max (the O rescale only when a row max passes it by 8); the 8-bit P.V mode
+  // takes its exponentials against the exact running max (the rounding of p to E4M3 is defined
+  // against it)
+  constexpr float RESCALE_THRESH = C::PV8 ? 0.0f : 8.0f;
   // At D = 128 the two partner warps of a row run their exponentials in lock step on one SM
   // sub-partition's MUFU; moving one pair in eight to the FMA pipe shortens that phase (at
   // D = 256 the tensor core sets the pace and the extra instructions cost more than they save).
@@ -903,7 +935,53 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
     // p = 2^(value * cscale - m_ref); masked entries hold -inf and give 0.  Each 32-column
     // chunk of P (16 packed columns) goes into this tile's S buffer as soon as it is ready: P.V
     // of the tile two steps back, which read that buffer, completed before S was written.
-    if (drop) {  // a dropped routing tile: P = 0 for this row, (m, l) unchanged
+    if constexpr (C::PV8) {
+      // 8-bit P: p * 2^8 rounded to E4M3 (the running max's own p is 256 < 448), into this
+      // tile's P8 buffer, row r, keys [NH * h, NH * h + NH) = 16-byte units 4h .. 4h + 3,
+      // XOR-swizzled by r & 7 (the 128-byte swizzle of a K-major operand).  P.V of the tile two
+      // steps back, which read this buffer, completed before S(t) was written.
+      const uint32_t prow = smem_u32(smem + C::OFF_P8) + static_cast<uint32_t>(bsel * C::P8_BYTES) +
+                            static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128);
+      const float mu = (m_ref == NEG_INF) ? 0.0f : m_ref;
+      const uint64_t c2 = f2_pack(cscale, cscale);
+      const uint64_t nb2 = f2_pack(-mu, -mu);
+      uint64_t se0 = 0, se1 = 0;
+      float sr0 = 0.f, sr1 = 0.f, sr2 = 0.f, sr3 = 0.f;
+      uint32_t w[4];
+#pragma unroll
+      for (int c = 0; c < NH; c += 4) {
+        float x0, x1, x2, x3, p0, p1, p2, p3;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(raw[c]), __uint_as_float(raw[c + 1])), c2, nb2),
+                  x0, x1);
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(raw[c + 2]), __uint_as_float(raw[c + 3])), c2, nb2),
+                  x2, x3);
+        p0 = drop ? 0.0f : ex2(x0);
+        p1 = drop ? 0.0f : ex2(x1);
+        p2 = drop ? 0.0f : ex2(x2);
+        p3 = drop ? 0.0f : ex2(x3);
+        se0 = f2_add(se0, f2_pack(p0, p1));
+        se1 = f2_add(se1, f2_pack(p2, p3));
+        const uint32_t lo = e4m3x2(p0 * 256.0f, p1 * 256.0f), hi = e4m3x2(p2 * 256.0f, p3 * 256.0f);
+        const uint32_t flo = e4m3x2_to_f16x2(lo), fhi = e4m3x2_to_f16x2(hi);
+        sr0 = add_lo16<false>(sr0, flo);
+        sr1 = add_hi16<false>(sr1, flo);
+        sr2 = add_lo16<false>(sr2, fhi);
+        sr3 = add_hi16<false>(sr3, fhi);
+        w[(c >> 2) & 3] = lo | (hi << 16);
+        if ((c & 15) == 12) {
+          const uint32_t u = static_cast<uint32_t>(4 * h + (c >> 4));
+          st_shared_v4(prow + ((u ^ static_cast<uint32_t>(r & 7)) << 4), w[0], w[1], w[2], w[3]);
+        }
+      }
+      if (!drop) {
+        float a0, a1;
+        f2_unpack(f2_add(se0, se1), a0, a1);
+        l_ex += a0 + a1;
+        // the rounded p carry the factor 2^8; O is divided by this sum, so it cancels
+        l_rd += (sr0 + sr1) + (sr2 + sr3);
+      }
+      fence_proxy_async_smem();  // the P.V MMA reads P8 through the async proxy
+    } else if (drop) {  // a dropped routing tile: P = 0 for this row, (m, l) unchanged
       const uint32_t zero[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
       for (int c = 0; c < NH / 32; ++c)
@@ -1068,6 +1146,8 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
         st_global_v4(obase + (row0 + row) * C::D * es + static_cast<size_t>(u) * 16, v);
     }
   } else {
+    // 8-bit P.V: O carries V's per-channel scale, applied here
+    const float* svp = C::PV8 ? p.v_scale + static_cast<size_t>(g.s.kv_plane) * C::D + h * DH : nullptr;
 #pragma unroll 1
     for (int c = 0; c < DH / 32; ++c) {
       uint32_t ov[32];
@@ -1079,6 +1159,11 @@ __device__ void softmax_role(const AttnParams& p, const Geo& g, uint8_t* smem, B
         for (int e = 0; e < 32; ++e) ov[e] = 0u;
       }
       if (!row_valid) continue;
+      if constexpr (C::PV8) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          ov[e] = __float_as_uint(__uint_as_float(ov[e]) * __ldg(svp + c * 32 + e));
+      }
       // 32-byte stores: each thread writes whole sectors of its row
       auto sc = [&](int e) { return __float_as_uint(__uint_as_float(ov[e]) * inv); };
       if (p.out_f32) {

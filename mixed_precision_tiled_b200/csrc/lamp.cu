@@ -108,6 +108,26 @@ int make_map(CUtensorMap* m, const void* base, int ebytes, int D, int L, int out
   return LAMP_OK;
 }
 
+// 3-D map over 8-bit [outer][rows][inner] with a row pitch of `pitch` bytes (>= inner, a
+// multiple of 16); box (box_inner, box_rows, 1).
+int make_map_pitch(CUtensorMap* m, const void* base, int inner, int pitch, int rows, int outer,
+                   int box_inner, int box_rows, CUtensorMapSwizzle swz) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(pitch),
+                           static_cast<cuuint64_t>(pitch) * static_cast<cuuint64_t>(rows)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LAMP_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return LAMP_OK;
+}
+
+// Row pitch of the channel-major 8-bit V: keys rounded up to 16 bytes.
+int v8_pitch(int Lk) { return (Lk + 15) & ~15; }
+
 // ---------------------------------------------------------------- workspace -----------
 
 struct Workspace {
@@ -121,11 +141,12 @@ Workspace g_ws;
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct WsLayout {
-  size_t q8, k8, qs, ks, total;
+  size_t q8, k8, qs, ks, v8, vs, total;  // v8, vs: the 8-bit P.V mode's V codes and scales
 };
 
 // q_rows / k_rows: rows per head plane of a variable-length batch (0: dense, B * L).
-WsLayout ws_layout(int B, int H, int Hkv, int Lq, int Lk, int D, int q_rows = 0, int k_rows = 0) {
+WsLayout ws_layout(int B, int H, int Hkv, int Lq, int Lk, int D, int q_rows = 0, int k_rows = 0,
+                   bool pv8 = false) {
   int bm, bn;
   tile_shape(D, &bm, &bn);
   const size_t nqt = (Lq + bm - 1) / bm, nkt = (Lk + bn - 1) / bn;
@@ -136,7 +157,9 @@ WsLayout ws_layout(int B, int H, int Hkv, int Lq, int Lk, int D, int q_rows = 0,
   w.k8 = align256(qr * H * D);
   w.qs = w.k8 + align256(kr * Hkv * D);
   w.ks = w.qs + align256(static_cast<size_t>(B) * H * nqt * sizeof(float));
-  w.total = w.ks + align256(static_cast<size_t>(B) * Hkv * nkt * sizeof(float));
+  w.v8 = w.ks + align256(static_cast<size_t>(B) * Hkv * nkt * sizeof(float));
+  w.vs = w.v8 + (pv8 ? align256(static_cast<size_t>(B) * Hkv * D * v8_pitch(Lk)) : 0);
+  w.total = w.vs + (pv8 ? align256(static_cast<size_t>(B) * Hkv * D * sizeof(float)) : 0);
   return w;
 }
 
@@ -250,6 +273,31 @@ int quant_qk(const void* q, const void* k, void* q8, void* k8, float* q_scale, f
   if (bf16) return launch_quant_t<true, false>(jq, jk, D, vec, st);
   if (e4m3) return launch_quant_t<false, true>(jq, jk, D, vec, st);
   return launch_quant_t<false, false>(jq, jk, D, vec, st);
+}
+
+// Per-channel 8-bit V (the 8-bit P.V mode): maxima into v_scale (as bits), codes, scales.
+int quant_v(const void* v, void* v8t, float* v_scale, int B, int Hkv, int Lk, int D, int mode,
+            cudaStream_t st) {
+  const int planes = B * Hkv;
+  const bool bf16 = (mode & LAMP_IN_BF16) != 0;
+  auto* amax = reinterpret_cast<uint32_t*>(v_scale);
+  const auto* src = static_cast<const uint16_t*>(v);
+  auto* dst = static_cast<uint8_t*>(v8t);
+  LAMP_CUDA(cudaMemsetAsync(amax, 0, static_cast<size_t>(planes) * D * sizeof(float), st),
+            "memset V maxima");
+  const dim3 g1((Lk + lamp::VQ_KEYS - 1) / lamp::VQ_KEYS, planes);
+  if (bf16) lamp::vmax_kernel<true><<<g1, D, 0, st>>>(src, amax, Lk, D);
+  else lamp::vmax_kernel<false><<<g1, D, 0, st>>>(src, amax, Lk, D);
+  LAMP_CUDA(cudaGetLastError(), "vmax_kernel launch");
+  const int pitch = v8_pitch(Lk);
+  const dim3 g2((pitch + 127) / 128, planes);
+  if (bf16) lamp::vquant_kernel<true><<<g2, 256, 0, st>>>(src, amax, dst, Lk, pitch, D);
+  else lamp::vquant_kernel<false><<<g2, 256, 0, st>>>(src, amax, dst, Lk, pitch, D);
+  LAMP_CUDA(cudaGetLastError(), "vquant_kernel launch");
+  const int n = planes * D;
+  lamp::vscale_kernel<<<(n + 255) / 256, 256, 0, st>>>(amax, n);
+  LAMP_CUDA(cudaGetLastError(), "vscale_kernel launch");
+  return LAMP_OK;
 }
 
 template <class C, bool BF16, bool E4M3, bool SKIP, bool DBG = false>
@@ -376,6 +424,14 @@ int launch_attn_pp(const lamp::AttnParams& p0, int grid, bool dynamic, cudaStrea
 using Cfg64 = lamp::AttnCfg<64, 64, true>;
 using Cfg128 = lamp::AttnCfg<128, 128, false>;
 using Cfg256 = lamp::AttnCfg<256, 128, true>;
+using Cfg128P8 = lamp::AttnCfg<128, 128, false, true>;  // 8-bit exponentials and P.V
+
+int launch_attn_pv8(const lamp::AttnParams& p, int grid, cudaStream_t st) {
+  if (p.bf16) return p.e4m3 ? launch_attn_cfg_t<Cfg128P8, true, true, false>(p, grid, st)
+                            : launch_attn_cfg_t<Cfg128P8, true, false, false>(p, grid, st);
+  return p.e4m3 ? launch_attn_cfg_t<Cfg128P8, false, true, false>(p, grid, st)
+                : launch_attn_cfg_t<Cfg128P8, false, false, false>(p, grid, st);
+}
 
 // Host-side checks of a routed-attention call (sizes, operand pointers and alignment, causal /
 // window, mode bits, group size, tau, scale, threshold skip).  Makes no CUDA call and enqueues
@@ -403,7 +459,7 @@ int check_attn(const void* q, const void* k, const void* v, bool codes, const vo
   if (window < 0) return fail(LAMP_ERR_INVALID, "window must be >= 0");
   if (window > 0 && !causal)
     return fail(LAMP_ERR_UNSUPPORTED, "a sliding window needs causal = 1");
-  if ((mode & ~0xFu) != 0) return fail(LAMP_ERR_INVALID, "unknown mode bits 0x%x", mode);
+  if ((mode & ~0x1Fu) != 0) return fail(LAMP_ERR_INVALID, "unknown mode bits 0x%x", mode);
   const bool adaptive = (mode & LAMP_ROUTE_ADAPTIVE) != 0;
   if (!adaptive && group_tiles < 1) return fail(LAMP_ERR_INVALID, "group_tiles must be >= 1");
   if (adaptive && !(tau == tau)) return fail(LAMP_ERR_INVALID, "tau is NaN");
@@ -411,13 +467,16 @@ int check_attn(const void* q, const void* k, const void* v, bool codes, const vo
   const bool skip = !std::isinf(skip_tau) || skip_tau < 0.0f;
   if (skip && (!adaptive || !(skip_tau >= tau) || !(skip_tau >= 0.0f)))
     return fail(LAMP_ERR_INVALID, "skip_tau needs look-ahead mode and tau <= skip_tau");
+  if ((mode & LAMP_PV_E4M3) && (D != 128 || varlen || skip))
+    return fail(LAMP_ERR_UNSUPPORTED,
+                "8-bit P.V: D = 128, dense batches and no threshold skip only");
   const long long grid = static_cast<long long>(B) * H * ((Lq + 127) / 128);
   if (grid > 0x7FFFFFFF) return fail(LAMP_ERR_INVALID, "grid too large");
   return LAMP_OK;
 }
 
 // Which attention kernel runs a prepared call.
-enum AttnKernel { K_CFG64, K_PP, K_CFG128, K_CFG256 };
+enum AttnKernel { K_CFG64, K_PP, K_CFG128, K_CFG256, K_CFG128P8 };
 
 struct AttnCall {
   lamp::AttnParams p;
@@ -434,9 +493,10 @@ int prepare_attn(const void* q, const void* k, const void* v, const void* q8, co
                  int Hkv, int Lq, int Lk, int D, int causal, int window, float scale,
                  const uint64_t* mask_bits, int group_tiles, int mode, float tau,
                  uint8_t* route_out, const int* cu_q, const int* cu_k, int total_q, int total_k,
-                 float skip_tau, AttnCall* call) {
+                 float skip_tau, AttnCall* call, const float* v_scale = nullptr) {
   int r;
   if ((r = get_encode())) return r;
+  const bool pv8 = (mode & LAMP_PV_E4M3) != 0;  // v is then the channel-major 8-bit V
   const bool varlen = cu_q != nullptr;
   const bool adaptive = (mode & LAMP_ROUTE_ADAPTIVE) != 0;
   const bool skip = !std::isinf(skip_tau) || skip_tau < 0.0f;
@@ -450,7 +510,14 @@ int prepare_attn(const void* q, const void* k, const void* v, const void* q8, co
   const int qpl = varlen ? H : BHq, kpl = varlen ? Hkv : BHk;
   if ((r = make_map(&p.tm_q16, q, 2, D, qr, qpl, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))) return r;
   if ((r = make_map(&p.tm_k16, k, 2, D, kr, kpl, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B))) return r;
-  if ((r = make_map(&p.tm_v, v, 2, D, kr, kpl, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B))) return r;
+  if (pv8) {
+    if ((r = make_map_pitch(&p.tm_v8, v, Lk, v8_pitch(Lk), D, kpl, bn, D,
+                            CU_TENSOR_MAP_SWIZZLE_128B)))
+      return r;
+    p.v_scale = v_scale;
+  } else if ((r = make_map(&p.tm_v, v, 2, D, kr, kpl, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B))) {
+    return r;
+  }
   const CUtensorMapSwizzle sw8 = (D == 64) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   const int in8 = (D == 64) ? 64 : 128;
   if ((r = make_map(&p.tm_q8, q8, 1, D, qr, qpl, in8, 128, sw8))) return r;
@@ -488,7 +555,9 @@ int prepare_attn(const void* q, const void* k, const void* v, const void* q8, co
   p.wait_ns = kWaitUs * 1000ull;
   call->route_bytes = route_out ? static_cast<size_t>(BHq) * nqt * nkt : 0;
   call->grid = BHq * p.n_ct;  // (check_attn bounds it)
-  if (D == 64) {
+  if (pv8) {
+    call->kernel = K_CFG128P8;  // (check_attn: D = 128)
+  } else if (D == 64) {
     call->kernel = K_CFG64;
   } else if (D == 128 && !p.e4m3 && !skip && (adaptive || p.mask_words <= 2)) {
     // The two-tile kernel keeps two mask words per query tile (128 key groups); wider masks go
@@ -540,6 +609,7 @@ int launch_attn(const AttnCall& c, cudaStream_t st) {
     case K_CFG64: return launch_attn_cfg<Cfg64>(c.p, c.grid, st);
     case K_PP: return launch_attn_pp(c.p, c.grid, c.pp_dynamic, st);
     case K_CFG128: return launch_attn_cfg<Cfg128>(c.p, c.grid, st);
+    case K_CFG128P8: return launch_attn_pv8(c.p, c.grid, st);
     default: return launch_attn_cfg<Cfg256>(c.p, c.grid, st);
   }
 }
@@ -578,14 +648,19 @@ int quant_and_attend(const void* q, const void* k, const void* v, void* o, float
   uint8_t* k8 = base + w.k8;
   float* qs = reinterpret_cast<float*>(base + w.qs);
   float* ks = reinterpret_cast<float*>(base + w.ks);
+  const bool pv8 = (mode & LAMP_PV_E4M3) != 0;  // (dense batches only: check_attn)
+  uint8_t* v8 = base + w.v8;
+  float* vs = reinterpret_cast<float*>(base + w.vs);
   AttnCall call;
-  int r = prepare_attn(q, k, v, q8, k8, qs, ks, o, lse, B, H, Hkv, Lq, Lk, D, causal, window,
-                       scale, mask_bits, group_tiles, mode, tau, nullptr, cu_q, cu_k, total_q,
-                       total_k, INFINITY, &call);
+  int r = prepare_attn(q, k, pv8 ? static_cast<const void*>(v8) : v, q8, k8, qs, ks, o, lse, B, H,
+                       Hkv, Lq, Lk, D, causal, window, scale, mask_bits, group_tiles, mode, tau,
+                       nullptr, cu_q, cu_k, total_q, total_k, INFINITY, &call,
+                       pv8 ? vs : nullptr);
   if (r) return r;
   if ((r = quant_qk(q, k, q8, k8, qs, ks, B, H, Hkv, Lq, Lk, D, mode, st, cu_q, cu_k, total_q,
                     total_k)))
     return r;
+  if (pv8 && (r = quant_v(v, v8, vs, B, Hkv, Lk, D, mode, st))) return r;
   return launch_attn(call, st);
 }
 
@@ -867,9 +942,41 @@ int lamp_attn_fwd_q8(const void* q, const void* k, const void* v, const void* q8
                      float* lse, int B, int H, int Hkv, int Lq, int Lk, int D, int causal,
                      int window, float scale, const uint64_t* mask_bits, int group_tiles,
                      int mode, float tau, uint8_t* route_out, void* stream) {
+  if ((mode & ~0x1Fu) == 0 && (mode & LAMP_PV_E4M3))  // (unknown bits: check_attn's error)
+    return fail(LAMP_ERR_UNSUPPORTED, "8-bit P.V takes the 8-bit V: lamp_attn_fwd_q8_pv8");
   return attn_q8(q, k, v, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D, causal,
                  window, scale, mask_bits, group_tiles, mode, tau, route_out,
                  static_cast<cudaStream_t>(stream));
+}
+
+int lamp_attn_fwd_q8_pv8(const void* q, const void* k, const void* q8, const void* k8,
+                         const float* q_scale, const float* k_scale, const void* v8t,
+                         const float* v_scale, void* o, float* lse, int B, int H, int Hkv,
+                         int Lq, int Lk, int D, int causal, int window, float scale,
+                         const uint64_t* mask_bits, int group_tiles, int mode, float tau,
+                         void* stream) {
+  if (!(mode & LAMP_PV_E4M3)) return fail(LAMP_ERR_INVALID, "mode must include LAMP_PV_E4M3");
+  if (!v_scale) return fail(LAMP_ERR_INVALID, "null v_scale");
+  int r = check_attn(q, k, v8t, true, q8, k8, q_scale, k_scale, o, B, H, Hkv, Lq, Lk, D, causal,
+                     window, scale, group_tiles, mode, tau, nullptr, nullptr, 0, 0, INFINITY);
+  if (r) return r;
+  AttnCall call;
+  if ((r = prepare_attn(q, k, v8t, q8, k8, q_scale, k_scale, o, lse, B, H, Hkv, Lq, Lk, D,
+                        causal, window, scale, mask_bits, group_tiles, mode, tau, nullptr,
+                        nullptr, nullptr, 0, 0, INFINITY, &call, v_scale)))
+    return r;
+  return launch_attn(call, static_cast<cudaStream_t>(stream));
+}
+
+int lamp_quant_v(const void* v, void* v8t, float* v_scale, int B, int Hkv, int Lk, int D,
+                 int mode, void* stream) {
+  int r = check_sizes(B, Hkv, Hkv, 1, Lk, D);
+  if (r) return r;
+  if (!v || !v8t || !v_scale) return fail(LAMP_ERR_INVALID, "null pointer");
+  if (!aligned16(v8t)) return fail(LAMP_ERR_INVALID, "v8t must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(v) & 1u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u))
+    return fail(LAMP_ERR_INVALID, "v and v_scale must be aligned to their elements");
+  return quant_v(v, v8t, v_scale, B, Hkv, Lk, D, mode, static_cast<cudaStream_t>(stream));
 }
 
 int lamp_attn_debug(const void* q, const void* k, const void* v, const void* q8,
@@ -878,6 +985,8 @@ int lamp_attn_debug(const void* q, const void* k, const void* v, const void* q8,
                     int window, float scale, const uint64_t* mask_bits, int group_tiles,
                     int mode, float tau, uint8_t* route_out, const int* tile_slot, int n_slots,
                     void* s8_dump, void* s16_dump, void* stream) {
+  if ((mode & ~0x1Fu) == 0 && (mode & LAMP_PV_E4M3))
+    return fail(LAMP_ERR_UNSUPPORTED, "no debug capture of the 8-bit P.V mode");
   if (!tile_slot || n_slots < 1) return fail(LAMP_ERR_INVALID, "a slot map and n_slots >= 1 are needed");
   if (!s8_dump && !s16_dump) return fail(LAMP_ERR_INVALID, "no dump buffer");
   if (!aligned16(s8_dump) || !aligned16(s16_dump))
@@ -909,11 +1018,10 @@ int lamp_exp2_eval(const float* x, float* y, int n, int method, void* stream) {
 }
 
 size_t lamp_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int D, int mode) {
-  (void)mode;
   int bm, bn;
   if (B < 1 || H < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || tile_shape(D, &bm, &bn) != LAMP_OK)
     return 0;
-  return ws_layout(B, H, Hkv, Lq, Lk, D).total;
+  return ws_layout(B, H, Hkv, Lq, Lk, D, 0, 0, (mode & LAMP_PV_E4M3) != 0).total;
 }
 
 int lamp_set_workspace(void* ptr, size_t bytes) {
@@ -933,7 +1041,7 @@ int lamp_attn_fwd(const void* q, const void* k, const void* v, void* o, float* l
                      INFINITY);
   if (r) return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const WsLayout w = ws_layout(B, H, Hkv, Lq, Lk, D);
+  const WsLayout w = ws_layout(B, H, Hkv, Lq, Lk, D, 0, 0, (mode & LAMP_PV_E4M3) != 0);
   void* ws = nullptr;
   if ((r = get_workspace(w.total, st, &ws))) return r;
   return quant_and_attend(q, k, v, o, lse, ws, w, B, H, Hkv, Lq, Lk, D, causal, window, scale,
@@ -999,7 +1107,7 @@ int lamp_attn_fwd_host(const void* q, const void* k, const void* v, void* o, flo
   const int per = (planes + n_chunks - 1) / n_chunks;  // planes per chunk (the last may be short)
   n_chunks = (planes + per - 1) / per;
   // workspace: the quantiser's codes and scales for one chunk, then two slots of device chunks
-  const WsLayout wq = ws_layout(per, G, 1, Lq, Lk, D);
+  const WsLayout wq = ws_layout(per, G, 1, Lq, Lk, D, 0, 0, (mode & LAMP_PV_E4M3) != 0);
   const size_t s_q = 0, s_k = align256(per * q_pl), s_v = s_k + align256(per * kv_pl),
                s_o = s_v + align256(per * kv_pl), s_l = s_o + align256(per * o_pl),
                slot = s_l + align256(per * l_pl);
@@ -1212,7 +1320,7 @@ int lamp_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
                      D, causal, window, scale, group_tiles, mode, tau, nullptr, nullptr, 0, 0,
                      INFINITY);
   if (r) return r;
-  const WsLayout w = ws_layout(B, H, Hkv, Lq, Lk, D);
+  const WsLayout w = ws_layout(B, H, Hkv, Lq, Lk, D, 0, 0, (mode & LAMP_PV_E4M3) != 0);
   if (w.total > static_cast<size_t>(LAMP_NOALLOC_MAX_BYTES))
     return fail(LAMP_ERR_INVALID,
                 "problem needs %zu bytes of scratch; lamp_attn_fwd_noalloc holds at most %zu "

@@ -323,6 +323,21 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
 
 // ------------------------------------------------------------------ math ---------------
 
+// Two fp32 values -> two E4M3 codes (round to nearest even, saturating to +-448): lo in bits
+// 0-7, hi in bits 8-15.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// Two E4M3 codes (bits 0-15) -> the same values as an f16x2 pair (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t c2) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo;\n\tcvt.u16.u32 lo, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}"
+      : "=r"(r) : "r"(c2));
+  return r;
+}
+
 // Packed f32x2 arithmetic (two fp32 lanes in one 64-bit register pair).
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;

@@ -43,12 +43,6 @@ __device__ __forceinline__ float h16_to_f32(uint32_t bits, bool bf16) {
   return __half2float(__ushort_as_half(static_cast<unsigned short>(bits)));
 }
 
-__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
 // Lane-wise max(|a|, |b|) of two pairs of 16-bit floats (the sign bits of the result are
 // meaningless; NaN lanes lose against numbers, as fmax does).
 template <bool BF16>
@@ -342,6 +336,73 @@ __device__ __forceinline__ uint64_t splitmix64_step(uint64_t x) {
   z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
   z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
   return z ^ (z >> 31);
+}
+
+// ------------------------------------------------------------------ 8-bit V -----------
+// Per-channel E4M3 V for the 8-bit P.V mode (LampAttention abstract, exponentials in 8-bit
+// formats; the pages give no V format): one scale per (batch, KV head, channel) over all keys,
+// s = fl32(a / 448) with a the channel's absolute maximum, code = E4M3(fl32(v / s)) rounded to
+// nearest even; a = 0 gives s = 0 and zero codes.  Codes channel-major [planes][D][Lk_pad]
+// (keys contiguous, Lk_pad = Lk rounded up to 16, the padding zero), so that a tile of 128
+// keys is a K-major operand of the P.V MMA.
+//
+// Pass 1: the channel maxima, folded into amax[planes][D] as bit patterns (non-negative floats
+// order as their bits; the array starts at zero).  Block = D threads (thread = channel),
+// grid = (key chunks of VQ_KEYS, planes).
+constexpr int VQ_KEYS = 256;
+
+template <bool BF16>
+__global__ void vmax_kernel(const uint16_t* __restrict__ v, uint32_t* __restrict__ amax, int Lk,
+                            int D) {
+  const int d = threadIdx.x, plane = blockIdx.y;
+  const int j0 = blockIdx.x * VQ_KEYS, j1 = min(Lk, j0 + VQ_KEYS);
+  const uint16_t* src = v + static_cast<size_t>(plane) * Lk * D + d;
+  float a = 0.0f;
+  for (int j = j0; j < j1; ++j) a = fmaxf(a, fabsf(h16_to_f32(src[static_cast<size_t>(j) * D], BF16)));
+  atomicMax(amax + static_cast<size_t>(plane) * D + d, __float_as_uint(a));
+}
+
+// Pass 2: codes of 128 keys x D channels per CTA (256 threads), transposed through shared
+// memory (words of 4 keys, rows padded to 33 words) and written as 128-byte channel rows.
+template <bool BF16>
+__global__ void vquant_kernel(const uint16_t* __restrict__ v, const uint32_t* __restrict__ amax,
+                              uint8_t* __restrict__ v8t, int Lk, int Lk_pad, int D) {
+  __shared__ uint32_t tw[256 * 33];  // [D][32 words] (+1 pad), D <= 256
+  const int plane = blockIdx.y, j0 = blockIdx.x * 128;
+  const uint16_t* src = v + static_cast<size_t>(plane) * Lk * D;
+  for (int idx = threadIdx.x; idx < D * 32; idx += blockDim.x) {
+    const int d = idx % D, wq = idx / D;  // channel, word of 4 keys
+    const float a = __uint_as_float(__ldg(amax + static_cast<size_t>(plane) * D + d));
+    const float sc = __fdiv_rn(a, 448.0f);
+    uint32_t word = 0;
+    if (a > 0.0f) {
+      float x[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = j0 + 4 * wq + e;
+        x[e] = (j < Lk) ? __fdiv_rn(h16_to_f32(src[static_cast<size_t>(j) * D + d], BF16), sc) : 0.0f;
+      }
+      word = e4m3x2(x[0], x[1]) | (e4m3x2(x[2], x[3]) << 16);
+    }
+    tw[d * 33 + wq] = word;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int d = warp; d < D; d += blockDim.x >> 5) {
+    const int j = j0 + 4 * lane;
+    if (j < Lk_pad)
+      *reinterpret_cast<uint32_t*>(v8t + (static_cast<size_t>(plane) * D + d) * Lk_pad + j) =
+          tw[d * 33 + lane];
+  }
+}
+
+// Pass 3: the maxima become the scales (in place).
+__global__ void vscale_kernel(uint32_t* __restrict__ amax_to_scale, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    const float a = __uint_as_float(amax_to_scale[i]);
+    amax_to_scale[i] = __float_as_uint(a > 0.0f ? __fdiv_rn(a, 448.0f) : 0.0f);
+  }
 }
 
 // One thread per mask word: rows = B*H*nQT mask rows of W words each.

@@ -84,6 +84,44 @@ def test_attn_fwd_rejects_bad_arguments_on_host(bad, code, entry):
     assert e.value.code == code
 
 
+def test_pv8_entries_reject_bad_arguments_on_host():
+    pv8 = mpt.mode_bits(pv8=True)
+    a = _attn_args()
+    args = lambda **kw: {**a, **kw}
+    # the 8-bit P.V mode: D = 128, dense, no skip; the q8 entry points route it to the pv8 one
+    for D, code in ((64, mpt.LAMP_ERR_UNSUPPORTED), (256, mpt.LAMP_ERR_UNSUPPORTED)):
+        with pytest.raises(mpt.LampError) as e:
+            mpt.lamp_attn_fwd(**args(D=D, mode=pv8), stream=0)
+        assert e.value.code == code
+    x = args(mode=pv8)
+    with pytest.raises(mpt.LampError) as e:
+        mpt.lamp_attn_fwd_q8(x["q"], x["k"], x["v"], 0x6000, 0x7000, 0x8000, 0x9000, x["o"],
+                             x["lse"], x["B"], x["H"], x["Hkv"], x["Lq"], x["Lk"], x["D"],
+                             x["causal"], x["window"], x["scale"], x["mask_bits"],
+                             x["group_tiles"], x["mode"], x["tau"], None, stream=0)
+    assert e.value.code == mpt.LAMP_ERR_UNSUPPORTED
+    def q8pv8(**kw):
+        y = args(**kw)
+        mpt.lamp_attn_fwd_q8_pv8(y["q"], y["k"], 0x6000, 0x7000, 0x8000, 0x9000, y["v"],
+                                 kw.get("v_scale", 0xA000), y["o"], y["lse"], y["B"], y["H"],
+                                 y["Hkv"], y["Lq"], y["Lk"], y["D"], y["causal"], y["window"],
+                                 y["scale"], y["mask_bits"], y["group_tiles"], y["mode"], y["tau"],
+                                 stream=0)
+    for kw, code in ((dict(mode=0), mpt.LAMP_ERR_INVALID),            # the bit is required
+                     (dict(mode=pv8, v_scale=None), mpt.LAMP_ERR_INVALID),
+                     (dict(mode=pv8, D=64), mpt.LAMP_ERR_UNSUPPORTED),
+                     (dict(mode=pv8, v=0x1008), mpt.LAMP_ERR_INVALID)):  # V codes 16-byte aligned
+        with pytest.raises(mpt.LampError) as e:
+            q8pv8(**kw)
+        assert e.value.code == code, kw
+    for kw in (dict(v=None), dict(v8t=0x1008), dict(D=80), dict(Lk=0)):
+        call = dict(v=0x1000, v8t=0x2000, v_scale=0x3000, B=1, Hkv=2, Lk=64, D=128, mode=0)
+        call.update(kw)
+        with pytest.raises(mpt.LampError):
+            mpt.lamp_quant_v(call["v"], call["v8t"], call["v_scale"], call["B"], call["Hkv"],
+                             call["Lk"], call["D"], call["mode"], stream=0)
+
+
 @pytest.mark.parametrize("bad,code", [
     (dict(H=3, Hkv=2), mpt.LAMP_ERR_INVALID),
     (dict(B=0), mpt.LAMP_ERR_INVALID),
