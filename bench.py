@@ -68,6 +68,9 @@ def parse():
     ap.add_argument("--skip-tau", type=float, default=None,
                     help="look-ahead workloads: drop tiles this far (natural log) below the "
                          "running max (threshold skip)")
+    ap.add_argument("--pv8", action="store_true",
+                    help="8-bit exponentials and an 8-bit P.V (E4M3 P and per-channel E4M3 V; "
+                         "D = 128, the single-tile kernel); V's quantiser joins the step")
     ap.add_argument("--decode", type=int, default=0,
                     help="decode step instead of prefill: this many sequences, each with the "
                          "workload's Lk cached keys in 8 bits (INT8 KV cache), one query row per "
@@ -127,20 +130,20 @@ def tile_pairs(w) -> np.ndarray:
     return out
 
 
-def blended_flops(w, route_map: np.ndarray):
+def blended_flops(w, route_map: np.ndarray, pv8: bool = False):
     """(F8, F16, F_total, 16-bit fraction): FLOPs of 8-bit QK tiles, of 16-bit QK tiles + P.V,
     the metric's FLOPs, and the fraction of visible pairs scored in 16 bits.  Route codes: 1
     8-bit, 2 16-bit by the mask, 3 recomputed by the look-ahead rule, 4 dropped by the
     threshold skip; a recomputed or dropped tile counts its 8-bit pass (the rules need the
     8-bit tile max of every tile to decide), a dropped tile has no P.V.  The metric's FLOPs
-    count every visible pair."""
+    count every visible pair.  ``pv8``: P.V runs in 8 bits and counts in F8."""
     pairs = tile_pairs(w)[None, None]  # broadcast over B, H
     p8 = int((pairs * ((route_map == 1) | (route_map == 3) | (route_map == 4))).sum())
     p16 = int((pairs * ((route_map == 2) | (route_map == 3))).sum())
     total = int((pairs * (route_map != 0)).sum())
     kept = int((pairs * ((route_map != 0) & (route_map != 4))).sum())  # P.V of kept tiles
-    F8 = 2 * w.D * p8
-    F16 = 2 * w.D * p16 + 2 * w.D * kept
+    F8 = 2 * w.D * p8 + (2 * w.D * kept if pv8 else 0)
+    F16 = 2 * w.D * p16 + (0 if pv8 else 2 * w.D * kept)
     return F8, F16, 4 * w.D * total, (p16 / total if total else 0.0)
 
 
@@ -290,8 +293,10 @@ def tensor_probe(mpt, torch, stream, iters=4096):
     return out
 
 
-def attn_kernel_name(w, skip=False):
+def attn_kernel_name(w, skip=False, pv8=False):
     """The attention kernel the library dispatches for this workload."""
+    if pv8:
+        return "attn_fwd_kernel (8-bit P.V)"
     wide_mask = w.route == "bitmask" and -(-w.nkt // w.group_tiles) > 128  # more than 2 words
     skip = skip and w.route == "adaptive"
     return ("attn_fwd_pp_kernel" if (w.D == 128 and w.fmt == "int8" and not wide_mask and not skip)
@@ -808,6 +813,13 @@ class Prefill:
         self.skip = args.skip_tau is not None and not self.bitmask
         self.tparams = {}
         self.launches_per_step = 1 + (1 if self.bitmask else 0) + 1  # quantiser, mask, attention
+        self.pv8 = bool(getattr(args, "pv8", False))
+        if self.pv8:  # V's quantiser (three kernels) joins the step
+            self.mode |= mpt.PV_E4M3
+            self.v8t = torch.empty((B, Hkv, w.D, (w.Lk + 15) // 16 * 16), dtype=torch.uint8,
+                                   device=dev)
+            self.vs = torch.empty((B, Hkv, w.D), dtype=torch.float32, device=dev)
+            self.launches_per_step += 3
 
     def flush_l2(self):
         """Evict the previous step's lines: write 256 MiB, then read it back so that L2 holds
@@ -828,6 +840,14 @@ class Prefill:
 
     def attn(self, md, tu, route_out=None):
         w, mpt = self.w, self.mpt
+        if self.pv8 and route_out is None:
+            mpt.lamp_attn_fwd_q8_pv8(self.q, self.k, self.q8, self.k8, self.qs, self.ks, self.v8t,
+                                     self.vs, self.o, self.lse, w.B, w.H, w.Hkv, w.Lq, w.Lk, w.D,
+                                     int(w.causal), w.window, 0.0,
+                                     self.mask if self.bitmask else None, w.group_tiles,
+                                     md | mpt.PV_E4M3, tu, self.stream)
+            return
+        md &= ~mpt.PV_E4M3  # the route map comes from the 16-bit P kernel: the same decisions
         if self.skip:
             mpt.lamp_attn_fwd_q8_skip(self.q, self.k, self.v, self.q8, self.k8, self.qs, self.ks,
                                       self.o, self.lse, w.B, w.H, w.Hkv, w.Lq, w.Lk, w.D,
@@ -846,6 +866,8 @@ class Prefill:
         tu = w.tau if tau_ is None else tau_
         self.mpt.lamp_quant_qk(self.q, self.k, self.q8, self.k8, self.qs, self.ks, w.B, w.H,
                                w.Hkv, w.Lq, w.Lk, w.D, md, self.stream)
+        if self.pv8:
+            self.mpt.lamp_quant_v(self.v, self.v8t, self.vs, w.B, w.Hkv, w.Lk, w.D, md, self.stream)
         if self.bitmask:
             self.build_mask(w.p_fp16 if p_fp16 is None else p_fp16)
         if ev_a is not None:
@@ -875,7 +897,7 @@ class Prefill:
                   self.rmap)
         self.torch.cuda.synchronize()
         rm = self.rmap.cpu().numpy()
-        return (*blended_flops(w, rm), rm)
+        return (*blended_flops(w, rm, self.pv8), rm)
 
     def sweep(self, peaks, lib, probe):
         """FP16-fraction sweep (bitmask) or tau x 8-bit-format sweep with the rerouted fraction
@@ -893,7 +915,7 @@ class Prefill:
                                                                   probe)["ruled"]}
         else:
             for fmt in ("int8", "e4m3"):
-                md = mpt.mode_bits(w.route, fmt, w.dtype)
+                md = mpt.mode_bits(w.route, fmt, w.dtype, pv8=self.pv8)
                 for tau in (0.5, 1.0, 2.0, 4.0, 8.0):
                     f8, f16, ff, fr, _ = self.route_flops(mode_=md, tau_=tau)
                     _, at = self.timed(n, mode_=md, tau_=tau)
@@ -902,13 +924,14 @@ class Prefill:
                         "rerouted_fraction": round(fr, 4),
                         "attn_tflops": round(ff / (a * 1e-3) / 1e12, 1),
                         "roofline_frac": roofline_fracs(f8, f16, a, peaks, fmt, lib, probe)["ruled"],
-                        "kernel": attn_kernel_name(w.replace(fmt=fmt))}
+                        "kernel": attn_kernel_name(w.replace(fmt=fmt), pv8=self.pv8)}
         self.step()  # restore the configured mask / format / tau
         self.torch.cuda.synchronize()
         return out
 
     def release(self):
-        for name in ("q", "k", "v", "q8", "k8", "qs", "ks", "mask", "o", "lse", "rmap", "flush"):
+        for name in ("q", "k", "v", "q8", "k8", "qs", "ks", "mask", "o", "lse", "rmap", "flush",
+                     "v8t", "vs"):
             setattr(self, name, None)
         self.torch.cuda.empty_cache()
 
@@ -1032,11 +1055,12 @@ def main():
                          "events exclude the flush"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
                      "peak": round(F / T_roof / 1e12, 1), "unit": "TFLOP/s",
-                     "frac": fr["ruled"], "traffic": traffic_record(w),
+                     "frac": fr["ruled"], "traffic": None if P.pv8 else traffic_record(w),
                      "peak_basis": f"blended: F8/P8 + F16/P16, P16 = {peaks['bf16']} TFLOP/s bf16 "
-                                   f"burst ({peaks['source']}), P8 = 2 x P16 (nominal ratio)",
+                                   f"burst ({peaks['source']}), P8 = 2 x P16 (nominal ratio)"
+                                   + ("; P.V counted in F8" if P.pv8 else ""),
                      "frac_other_bases": {k: v for k, v in fr.items() if k != "ruled"},
-                     "kernel": attn_kernel_name(w, args.skip_tau is not None),
+                     "kernel": attn_kernel_name(w, args.skip_tau is not None, P.pv8),
                      "attn_ms": round(att_ms, 4)},
         "e2e": {"value": round(F * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -1061,7 +1085,8 @@ def main():
     P.release()
 
     # the other workloads at L >= 8192 (the target's configurations), kernel-level, same run
-    if not args.no_extras and args.workload == DEFAULT_WORKLOAD and args.varlen == 0:
+    if (not args.no_extras and args.workload == DEFAULT_WORKLOAD and args.varlen == 0
+            and not args.pv8):
         extras = {}
         for name in EXTRA_WORKLOADS:
             we = CONFIGS[name]

@@ -98,3 +98,27 @@ def test_pv8_attention_matches_oracle(B, H, Hkv, Lq, Lk, causal, window, route, 
     # and within the E4M3 rounding bound of the 16-bit P result on the same inputs
     o16, _ = mpt.attention(dq, dk, dv, **kw)
     assert (o16 - o).abs().max().item() <= 2 * 2.0 ** -4 * vmax
+
+
+def test_pv8_through_the_allocation_free_and_host_buffer_entries():
+    # both quantise V themselves in this mode: bit-identical to lamp_attn_fwd
+    B, H, Hkv, L, D = 2, 4, 2, 600, 128
+    q, k, v = _inputs(B, H, Hkv, L, L, D, torch.bfloat16, seed=3)
+    dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
+    mask = mpt.build_mask(B, H, L, L, D, 2, 0.3, 5)
+    mode = mpt.mode_bits("bitmask", "int8", "bf16", pv8=True)
+    o = torch.empty((B, H, L, D), device="cuda", dtype=torch.float32)
+    lse = torch.empty((B, H, L), device="cuda", dtype=torch.float32)
+    mpt.lamp_attn_fwd(dq, dk, dv, o, lse, B, H, Hkv, L, L, D, 1, 0, 0.0, mask, 2, mode, 0.0)
+    o2, lse2 = torch.empty_like(o), torch.empty_like(lse)
+    mpt.lamp_attn_fwd_noalloc(dq, dk, dv, o2, lse2, B, H, Hkv, L, L, D, 1, 0, 0.0, mask, 2, mode,
+                              0.0)
+    hin = [x.pin_memory() for x in (q, k, v)]
+    ho = torch.empty((B, H, L, D), dtype=torch.float32).pin_memory()
+    hl = torch.empty((B, H, L), dtype=torch.float32).pin_memory()
+    mpt.lamp_attn_fwd_host(*hin, ho, hl, B, H, Hkv, L, L, D, 1, 0, 0.0, mask, 2, mode, 0.0,
+                           n_chunks=3)
+    torch.cuda.synchronize()
+    mpt.lamp_check()
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)
+    assert torch.equal(ho, o.cpu()) and torch.equal(hl, lse.cpu())
