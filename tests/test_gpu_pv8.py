@@ -122,3 +122,40 @@ def test_pv8_through_the_allocation_free_and_host_buffer_entries():
     mpt.lamp_check()
     assert torch.equal(o, o2) and torch.equal(lse, lse2)
     assert torch.equal(ho, o.cpu()) and torch.equal(hl, lse.cpu())
+
+
+@pytest.mark.parametrize("out", ["f32", "in"])
+def test_pv8_full_size_gqa4k_sampled_rows(out):
+    # the gqa4k workload's shape and inputs (B=1 H=32 Hkv=8 L=4096, INT8, structured values) in
+    # the 8-bit P.V mode, 64 seeded rows per head against the oracle; O in fp32 and in bf16.
+    # Every tile 8-bit: the scores are exact integers times one fp32 constant on both sides, so
+    # the GPU's p stays within ~1e-6 of the oracle's and the 1e-5 midpoint margin holds for
+    # 4096-key rows (16-bit tiles, whose fp32 tensor-core sums add their own error, are covered
+    # by the smaller cases above)
+    from workloads import CONFIGS, make_workload, sample_rows
+    w = CONFIGS["gqa4k"].replace(p_fp16=0.0)
+    t = make_workload(w)
+    dq, dk, dv = (torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).cuda()
+                  for b in (t.q_bits, t.k_bits, t.v_bits))
+    mask = mpt.build_mask(w.B, w.H, w.Lq, w.Lk, w.D, w.group_tiles, w.p_fp16, w.mask_seed)
+    o, lse = mpt.attention(dq, dk, dv, causal=True, mask_bits=mask, group_tiles=w.group_tiles,
+                           fmt=w.fmt, out=out, pv8=True)
+    torch.cuda.synchronize()
+    mpt.lamp_check()
+    rows = sample_rows(w, 64, seed=21)
+    ref = oracle.attention(t.q, t.k, t.v, bm=w.bm, bn=w.bn, causal=True,
+                           mask=mask.cpu().numpy().view(np.uint64), group_tiles=w.group_tiles,
+                           fmt=w.fmt, rows=rows, pv8=True)
+    go = o.float().cpu().numpy().astype(np.float64)
+    gl = lse.cpu().numpy().astype(np.float64)
+    go = np.stack([np.stack([go[0, h, rows[0, h]] for h in range(w.H)])])
+    gl = np.stack([np.stack([gl[0, h, rows[0, h]] for h in range(w.H)])])
+    vmax = float(np.abs(t.v).max())
+    # bf16 output adds its own rounding: half an ulp of |O| <= vmax
+    tol = 2e-4 * vmax + (0.0 if out == "f32" else vmax * 2.0 ** -8)
+    err = np.abs(go - ref["o"]).max(axis=-1)
+    sure = ref["pv8_margin"] >= MARGIN
+    assert sure.mean() > 0.5, sure.mean()
+    assert err[sure].max() <= tol, (err[sure].max(), tol)
+    assert err[~sure].max(initial=0.0) <= 0.25 * vmax
+    assert np.abs(gl - ref["lse"]).max() <= 1e-3
