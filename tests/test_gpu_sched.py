@@ -26,12 +26,14 @@ D = 128
 L_BIG = 19600
 
 
-def _case(B, H, Hkv, L, seed, g=2, p16=0.3):
+def _case(B, H, Hkv, L, seed, g=2, p16=0.3, route="bitmask", dt=torch.bfloat16):
     gen = torch.Generator(device="cpu").manual_seed(seed)
-    q = torch.randn((B, H, L, D), generator=gen).to(torch.bfloat16).cuda()
-    k = torch.randn((B, Hkv, L, D), generator=gen).to(torch.bfloat16).cuda()
-    v = torch.randn((B, Hkv, L, D), generator=gen).to(torch.bfloat16).cuda()
+    q = torch.randn((B, H, L, D), generator=gen).to(dt).cuda()
+    k = torch.randn((B, Hkv, L, D), generator=gen).to(dt).cuda()
+    v = torch.randn((B, Hkv, L, D), generator=gen).to(dt).cuda()
     q8, k8, qs, ks = mpt.quantize(q, k)
+    if route == "adaptive":
+        return [q, k, v, q8, k8, qs, ks], dict(causal=True, route="adaptive", tau=4.0)
     mask = mpt.build_mask(B, H, L, L, D, g, p16, seed)
     return [q, k, v, q8, k8, qs, ks], dict(causal=True, mask_bits=mask, group_tiles=g)
 
@@ -44,14 +46,18 @@ def _head_slice(args, kw, h0, h1, kv0, kv1):
     q, k, v, q8, k8, qs, ks = args
     sub = [q[:, h0:h1], k[:, kv0:kv1], v[:, kv0:kv1], q8[:, h0:h1], k8[:, kv0:kv1],
            qs[:, h0:h1], ks[:, kv0:kv1]]
-    kw2 = dict(kw, mask_bits=kw["mask_bits"][:, h0:h1])
+    kw2 = dict(kw, mask_bits=kw["mask_bits"][:, h0:h1]) if "mask_bits" in kw else dict(kw)
     return [x.contiguous() for x in sub], kw2
 
 
-@pytest.mark.parametrize("H,Hkv", [(16, 8), (8, 8)])
-def test_ticket_order_equals_fixed_order_on_head_slices(H, Hkv):
-    # (16, 8): items are one query tile of two heads; (8, 8): two query tiles of one head
-    args, kw = _case(1, H, Hkv, L_BIG, 11)
+@pytest.mark.parametrize("H,Hkv,route,dt", [(16, 8, "bitmask", torch.bfloat16),
+                                            (8, 8, "bitmask", torch.bfloat16),
+                                            (16, 8, "adaptive", torch.bfloat16),
+                                            (16, 8, "bitmask", torch.float16)])
+def test_ticket_order_equals_fixed_order_on_head_slices(H, Hkv, route, dt):
+    # (16, 8): items are one query tile of two heads; (8, 8): two query tiles of one head; the
+    # look-ahead and fp16 instantiations of the ticket order too
+    args, kw = _case(1, H, Hkv, L_BIG, 11, route=route, dt=dt)
     o, lse = _run(args, kw)
     torch.cuda.synchronize()
     mpt.lamp_check()
