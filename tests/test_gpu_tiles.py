@@ -8,7 +8,7 @@ compared here with ``oracle.score_tiles`` on the GPU's own codes (which the quan
 tests pin to the oracle's):
   * INT8 8-bit tiles: bit-exact (int32);
   * E4M3 8-bit tiles and 16-bit tiles: fp32 accumulation on the tensor core, whose internal
-    order and width are not documented (E4M3 is "parity unpinned" bit-wise): every product
+    order and width are not documented, so E4M3 tiles are compared with a tolerance: every product
     is exact in fp32, so the sum of D products is within D * 2^-24 * sum |products| of the
     exact fp64 sum; the test allows 1e-5 * sum |products|;
 and, tile by tile, the dump holds a product exactly when the route map says the tile used it
